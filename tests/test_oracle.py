@@ -1,0 +1,344 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: the OCP E4M3
+definition points, torch's independent float8_e4m3fn codec, hand-worked
+fixtures, closed forms, integer special cases that reduce to a plain matmul,
+and algebraic invariants (swap symmetry, grouping consistency, the relation
+between block and token scales).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def torch_decode(codes: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def torch_encode(values: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(values, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+ALL_CODES = np.arange(256, dtype=np.uint8)
+FINITE_CODES = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+
+
+# ---------------------------------------------------------------- e4m3 codec
+
+def test_decode_matches_ocp_definition_points():
+    path = os.path.join(GOLDEN, "e4m3_ocp_points.txt")
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        code_s, val_s = line.split()
+        code = int(code_s, 16)
+        got = float(oracle.e4m3_decode(np.array([code], np.uint8))[0])
+        if val_s == "nan":
+            assert math.isnan(got), hex(code)
+        else:
+            want = float(val_s)
+            assert got == want and math.copysign(1, got) == math.copysign(1, want), hex(code)
+
+
+def test_decode_all_codes_match_torch():
+    ours = oracle.e4m3_decode(ALL_CODES)
+    ref = torch_decode(ALL_CODES)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))
+
+
+def test_encode_decode_roundtrip_every_finite_code():
+    vals = oracle.e4m3_decode(FINITE_CODES).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(vals), FINITE_CODES)
+
+
+def test_encode_ties_go_to_even_code():
+    pos = np.arange(0, 0x7F, dtype=np.uint8)  # 0x00 .. 0x7E, increasing values
+    v = oracle.e4m3_decode(pos)
+    mid = ((v[:-1] + v[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (v[:-1] + v[1:]) / 2)  # exact in fp32
+    got = oracle.e4m3_encode(mid)
+    lo = pos[:-1]
+    even = np.where(lo % 2 == 0, lo, lo + 1).astype(np.uint8)
+    assert np.array_equal(got, even)
+    assert np.array_equal(oracle.e4m3_encode(-mid), even | 0x80)
+
+
+def test_encode_matches_torch_on_random_values():
+    rng = np.random.default_rng(123)
+    # log-uniform magnitudes from deep subnormal to the saturation midpoint
+    mag = np.exp(rng.uniform(np.log(1e-5), np.log(463.9), size=200000)).astype(np.float32)
+    sgn = np.where(rng.random(mag.size) < 0.5, -1, 1).astype(np.float32)
+    vals = np.concatenate([mag * sgn, np.float32([0.0, -0.0, 464.0, -464.0])])
+    assert np.array_equal(oracle.e4m3_encode(vals), torch_encode(vals))
+
+
+def test_encode_saturates_at_448():
+    vals = np.float32([448.0, 449.0, 464.0, 465.0, 1e6, 3e38, -500.0, -1e30])
+    got = oracle.e4m3_encode(vals)
+    assert np.array_equal(got, np.uint8([0x7E] * 6 + [0xFE] * 2))
+    assert oracle.e4m3_encode(np.float32([np.nan]))[0] == 0x7F
+
+
+# ---------------------------------------------------------------- quantizers
+
+def _ulp_e4m3(v: np.ndarray) -> np.ndarray:
+    a = np.abs(v)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    return np.where(a < 2.0 ** -6, 2.0 ** -9, 2.0 ** (e - 3))
+
+
+def test_per_token_worked_example():
+    path = os.path.join(GOLDEN, "per_token_worked_example.txt")
+    x = np.zeros(128, np.float32)
+    x[:4] = [3.5, -1.75, 0.5, 0.001]
+    q, s = oracle.per_token_cast(workloads.bf16_bits(x)[None, :])
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        a, b = line.split()
+        if a == "scale":
+            assert s[0, 0] == np.float32(float(b))
+        else:
+            assert q[0, int(a)] == int(b, 16), a
+
+
+def test_per_token_invariants():
+    rng = np.random.default_rng(7)
+    M, K = 37, 512
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    x[3] *= 30.0
+    x[5, 128:256] = 0.0                      # an all-zero slice
+    x[6, :128] *= 1e-6                       # a slice far below 1e-4 amax
+    bits = workloads.bf16_bits(x)
+    xf = workloads.bf16_to_f32(bits).astype(np.float64)
+    q, s = oracle.per_token_cast(bits)
+    assert q.shape == (M, K) and s.shape == (M, K // 128)
+    deq = oracle.e4m3_decode(q).reshape(M, K // 128, 128)
+    xs = xf.reshape(M, K // 128, 128)
+    amax = np.abs(xs).max(axis=2)
+    live = amax >= 1e-4
+    # the scale is amax/448 (one fp32 rounding), floored at 1e-4/448
+    np.testing.assert_allclose(s[live].astype(np.float64) * 448.0, amax[live], rtol=2 ** -23)
+    assert np.all(s[~live] == np.float32(1e-4) / np.float32(448.0))
+    # the element holding the slice's amax lands on +-448
+    idx = np.abs(xs).argmax(axis=2)
+    top = np.take_along_axis(deq, idx[..., None], axis=2)[..., 0]
+    assert np.all(np.abs(top[live]) == 448.0)
+    # reconstruction error: at most half an e4m3 ulp of x/s (plus fp32 slop)
+    y = xs / s[..., None].astype(np.float64)
+    err = np.abs(y - deq)
+    assert np.all(err <= 0.5 * _ulp_e4m3(y) * (1 + 1e-6) + 1e-9)
+    # the all-zero slice encodes to zero codes
+    assert np.all(q[5, 128:256] == 0)
+
+
+def test_per_token_power_of_two_slices_are_exact():
+    K = 256
+    j = np.arange(-14, 2)                          # 16 powers of two, max 2
+    vals = np.concatenate([2.0 ** j, -(2.0 ** j)]).astype(np.float32)
+    x = np.tile(vals, K // vals.size + 1)[:K][None, :]
+    q, s = oracle.per_token_cast(workloads.bf16_bits(x))
+    want = 448.0 * x[0].astype(np.float64) / 2.0     # amax = 2 in every slice
+    assert np.array_equal(oracle.e4m3_decode(q[0]), want)
+
+
+def test_per_block_relates_to_per_token():
+    """The block scale is the max of the 128 row scales of that block (amax is
+    a max and the scale map is monotone); N tail blocks use only their rows."""
+    rng = np.random.default_rng(11)
+    for N in (256, 192, 64, 130):
+        K = 384
+        x = workloads.bf16_bits(rng.standard_normal((N, K), dtype=np.float32) * 0.02)
+        qb, sb = oracle.per_block_cast(x)
+        _, st = oracle.per_token_cast(x)
+        NB = -(-N // 128)
+        assert sb.shape == (NB, K // 128)
+        for nb in range(NB):
+            rows = st[nb * 128:min(N, nb * 128 + 128)]
+            assert np.array_equal(sb[nb], rows.max(axis=0))
+        # a tail block quantizes exactly like a stand-alone matrix of its rows
+        if N % 128:
+            q2, s2 = oracle.per_block_cast(x[(NB - 1) * 128:])
+            assert np.array_equal(q2, qb[(NB - 1) * 128:])
+            assert np.array_equal(s2[0], sb[NB - 1])
+
+
+def test_per_block_invariants_and_groups():
+    rng = np.random.default_rng(5)
+    G, N, K = 3, 256, 256
+    x = workloads.bf16_bits(rng.standard_normal((G, N, K), dtype=np.float32) * 0.02)
+    q, s = oracle.per_block_cast(x)
+    for g in range(G):
+        qg, sg = oracle.per_block_cast(x[g])
+        assert np.array_equal(qg, q[g]) and np.array_equal(sg, s[g])
+    xf = workloads.bf16_to_f32(x).astype(np.float64).reshape(G, 2, 128, 2, 128)
+    amax = np.abs(xf).max(axis=(2, 4))
+    np.testing.assert_allclose(s.astype(np.float64) * 448.0, amax, rtol=2 ** -23)
+    deq = oracle.e4m3_decode(q).reshape(G, 2, 128, 2, 128)
+    y = xf / s[:, :, None, :, None].astype(np.float64)
+    assert np.all(np.abs(y - deq) <= 0.5 * _ulp_e4m3(y) * (1 + 1e-6) + 1e-9)
+
+
+# ---------------------------------------------------------------- GEMM
+
+def _expand_sa(sa):       # [M][KB] -> [M][K]
+    return np.repeat(sa.astype(np.float64), 128, axis=1)
+
+
+def _expand_sb(sb, N):    # [NB][KB] -> [N][K]
+    return np.repeat(np.repeat(sb.astype(np.float64), 128, axis=0)[:N], 128, axis=1)
+
+
+def _small_int_codes(rng, shape):
+    vals = rng.integers(-2, 3, size=shape).astype(np.float32)
+    return torch_encode(vals), vals.astype(np.int64)
+
+
+def test_gemm_integer_case_unit_scales_is_integer_matmul():
+    rng = np.random.default_rng(1)
+    M, N, K = 40, 200, 256
+    qa, ia = _small_int_codes(rng, (M, K))
+    qb, ib = _small_int_codes(rng, (N, K))
+    sa = np.ones((M, 2), np.float32)
+    sb = np.ones((2, 2), np.float32)
+    got = oracle.gemm_nt(qa, sa, qb, sb)
+    assert np.array_equal(got, (ia @ ib.T).astype(np.float64))
+
+
+def test_gemm_integer_case_power_of_two_scales_exact():
+    rng = np.random.default_rng(2)
+    M, N, K = 33, 160, 256
+    qa, ia = _small_int_codes(rng, (M, K))
+    qb, ib = _small_int_codes(rng, (N, K))
+    sa = (2.0 ** rng.integers(-3, 3, size=(M, 2))).astype(np.float32)
+    sb = (2.0 ** rng.integers(-3, 3, size=(2, 2))).astype(np.float32)
+    got = oracle.gemm_nt(qa, sa, qb, sb)
+    ref = (ia * _expand_sa(sa)) @ (ib * _expand_sb(sb, N)).T
+    assert np.array_equal(got, ref)
+
+
+def test_gemm_closed_form_all_ones():
+    M, N, K = 5, 300, 640
+    qa = np.full((M, K), 0x38, np.uint8)     # 1.0
+    qb = np.full((N, K), 0x38, np.uint8)
+    sa = np.full((M, K // 128), 0.375, np.float32)
+    sb = np.full((3, K // 128), 0.0625, np.float32)
+    got = oracle.gemm_nt(qa, sa, qb, sb)
+    assert np.all(got == K * 0.375 * 0.0625)
+
+
+def test_gemm_random_matches_scaled_operand_product():
+    """The blocked definition equals one fp64 matmul of the scaled, dequantized
+    operands (decoded by torch); a wrong block index or operand fails it."""
+    rng = np.random.default_rng(3)
+    M, N, K = 70, 300, 512
+    xa = workloads.bf16_bits(rng.standard_normal((M, K), dtype=np.float32))
+    xb = workloads.bf16_bits(rng.standard_normal((N, K), dtype=np.float32) * 0.02)
+    qa, sa = oracle.per_token_cast(xa)
+    qb, sb = oracle.per_block_cast(xb)
+    got = oracle.gemm_nt(qa, sa, qb, sb)
+    ref = (torch_decode(qa) * _expand_sa(sa)) @ (torch_decode(qb) * _expand_sb(sb, N)).T
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_gemm_brute_force_long_double_tiny():
+    rng = np.random.default_rng(4)
+    M, N, K = 6, 9, 256
+    qa = rng.integers(0, 256, size=(M, K)).astype(np.uint8)
+    qb = rng.integers(0, 256, size=(N, K)).astype(np.uint8)
+    qa[(qa & 0x7F) == 0x7F] = 0x3F
+    qb[(qb & 0x7F) == 0x7F] = 0x3F
+    sa = rng.uniform(0.001, 0.01, size=(M, 2)).astype(np.float32)
+    sb = rng.uniform(1e-4, 1e-3, size=(1, 2)).astype(np.float32)
+    da = torch_decode(qa).astype(np.longdouble)
+    db = torch_decode(qb).astype(np.longdouble)
+    ref = np.zeros((M, N), np.longdouble)
+    for m in range(M):
+        for n in range(N):
+            tot = np.longdouble(0)
+            for k in range(K):
+                tot += (da[m, k] * np.longdouble(sa[m, k // 128])) * (db[n, k] * np.longdouble(sb[n // 128, k // 128]))
+            ref[m, n] = tot
+    got = oracle.gemm_nt(qa, sa, qb, sb)
+    np.testing.assert_allclose(got, ref.astype(np.float64), rtol=1e-13, atol=1e-300)
+
+
+def test_gemm_swap_symmetry():
+    """With activation scales constant over 128-row groups, gemm(A,B)^T equals
+    gemm(B,A) with the two scale roles exchanged (the identity swapAB uses)."""
+    rng = np.random.default_rng(6)
+    M, N, K = 256, 384, 384
+    qa = torch_encode(rng.standard_normal((M, K)).astype(np.float32) * 8)
+    qb = torch_encode(rng.standard_normal((N, K)).astype(np.float32) * 8)
+    sa_blk = rng.uniform(0.01, 0.02, size=(M // 128, K // 128)).astype(np.float32)
+    sb = rng.uniform(0.001, 0.002, size=(N // 128, K // 128)).astype(np.float32)
+    sa = np.repeat(sa_blk, 128, axis=0)
+    sb_rows = np.repeat(sb, 128, axis=0)
+    d = oracle.gemm_nt(qa, sa, qb, sb)
+    dt = oracle.gemm_nt(qb, sb_rows, qa, sa_blk)
+    assert np.array_equal(d.T, dt)
+
+
+def test_grouped_forms_equal_per_expert_dense():
+    rng = np.random.default_rng(8)
+    N, K = 192, 256
+    counts = np.array([130, 0, 5, 128])
+    inp = workloads.contiguous(N, K, counts=counts, seed=3)
+    qa, sa = oracle.per_token_cast(inp.a)
+    qb, sb = oracle.per_block_cast(inp.b)
+    out = oracle.grouped_contiguous(qa, sa, qb, sb, inp.m_indices)
+    assert out.shape == (inp.M_total, N)
+    assert np.all(np.isnan(out[inp.m_indices < 0]))
+    for g in range(len(counts)):
+        rows = np.nonzero(inp.m_indices == g)[0]
+        if rows.size == 0:
+            continue
+        ref = oracle.gemm_nt(qa[rows], sa[rows], qb[g], sb[g])
+        assert np.array_equal(out[rows], ref)
+
+    G, M_max = 3, 80
+    minp = workloads.masked(G, M_max, N, K, seed=4, masked_m=np.array([0, 80, 17]))
+    qa3, sa3 = oracle.per_token_cast(minp.a)
+    qb3, sb3 = oracle.per_block_cast(minp.b)
+    out3 = oracle.grouped_masked(qa3, sa3, qb3, sb3, minp.masked_m)
+    for e in range(G):
+        mv = int(minp.masked_m[e])
+        assert np.all(np.isnan(out3[e, mv:]))
+        if mv:
+            ref = oracle.gemm_nt(qa3[e, :mv], sa3[e, :mv], qb3[e], sb3[e])
+            assert np.array_equal(out3[e, :mv], ref)
+
+
+def test_points_equal_full_gemm():
+    rng = np.random.default_rng(9)
+    M, N, K, G = 50, 130, 384, 2
+    xa = workloads.bf16_bits(rng.standard_normal((M, K), dtype=np.float32))
+    xb = workloads.bf16_bits(rng.standard_normal((G, N, K), dtype=np.float32) * 0.02)
+    qa, sa = oracle.per_token_cast(xa)
+    qb, sb = oracle.per_block_cast(xb)
+    r = rng.integers(0, M, 300)
+    e = rng.integers(0, G, 300)
+    n = rng.integers(0, N, 300)
+    pts = oracle.gemm_points(qa, sa, qb, sb, r, e, n)
+    full = [oracle.gemm_nt(qa, sa, qb[g], sb[g]) for g in range(G)]
+    assert np.array_equal(pts, np.array([full[ei][ri, ni] for ri, ei, ni in zip(r, e, n)]))
+
+
+def test_oracle_rejects_bad_sizes():
+    with pytest.raises(ValueError):
+        oracle.per_token_cast(np.zeros((4, 100), np.uint16))

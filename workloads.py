@@ -1,0 +1,204 @@
+"""Seeded synthetic inputs for the FP8 block-scaled GEMM workloads.
+
+This module is shared by the CPU oracle's tests, the CUDA path's tests and the
+benchmark. It holds none of the method's arithmetic: no quantization, no
+scales, no products. It only draws random numbers, rounds them to the bf16
+input format and lays them out in the shapes the workloads use.
+
+Workloads (sizes from the DeepGEMM pages' serving scenarios: dense prefill and
+decode shapes of DeepSeek-V3/R1, MoE grouped GEMM in contiguous and masked
+layouts; the pages print no shape list, so these stand in for "all V3/R1
+inference shapes"):
+
+  dense_128x256x512        A ~ N(0,1), B ~ N(0,0.02)
+  decode_64x4096x7168      A ~ N(0,1) with 1% of its rows (at least one) x30
+  prefill_4096x7168x2048   A ~ N(0,1), B ~ N(0,0.02)
+  prefill_4096x2112x7168   same, N not a multiple of 128
+  contiguous_8x4096x7168   8 experts, token counts from top-8 routing of 4096
+                           tokens over 256 experts (Gumbel-top-k on Zipf
+                           s=1.1 weights over expert ids), experts 0..7,
+                           each group padded to a multiple of 128, padding
+                           rows zero, m_indices = -1 on padding rows
+  masked_32x256x4096x7168  32 experts, capacity 256, masked_m ~ U{0..256}
+
+Seeds: every tensor draws from its own ``numpy.random.default_rng(seed + i)``
+with i = 0 for A, 1 for B, 2 for the routing and 3 for masked_m.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+ALIGN_M = 128  # contiguous layout: each expert group starts on a 128-row boundary
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (round to nearest, ties to even).
+
+    Returns the raw 16-bit patterns as uint16. Inputs must be finite.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    u = (u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
+    return u.astype(np.uint16)
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bfloat16 bit patterns to float32."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32)
+
+
+def normal_bf16(rng: np.random.Generator, shape, std: float = 1.0) -> np.ndarray:
+    """bf16 bits of N(0, std^2) samples drawn in float32."""
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    return bf16_bits(x)
+
+
+def zipf_top8_counts(seed: int, tokens: int = 4096, experts: int = 256,
+                     topk: int = 8, s: float = 1.1) -> np.ndarray:
+    """Per-expert token counts of top-k routing over Zipf(s) expert weights.
+
+    Each token picks ``topk`` distinct experts by Gumbel-top-k on log weights
+    w_i = (i+1)^-s (sampling without replacement proportionally to w).
+    Returns counts for all ``experts`` experts.
+    """
+    rng = np.random.default_rng(seed + 2)
+    logw = -s * np.log(np.arange(1, experts + 1, dtype=np.float64))
+    g = rng.gumbel(size=(tokens, experts)) + logw[None, :]
+    top = np.argpartition(-g, topk - 1, axis=1)[:, :topk]
+    return np.bincount(top.ravel(), minlength=experts).astype(np.int64)
+
+
+@dataclasses.dataclass
+class DenseInputs:
+    a: np.ndarray  # bf16 bits [M][K]
+    b: np.ndarray  # bf16 bits [N][K]
+    M: int
+    N: int
+    K: int
+
+
+@dataclasses.dataclass
+class ContiguousInputs:
+    a: np.ndarray          # bf16 bits [M_total][K], padding rows zero
+    b: np.ndarray          # bf16 bits [G][N][K]
+    m_indices: np.ndarray  # int32 [M_total], expert id or -1 on padding rows
+    counts: np.ndarray     # int64 [G] valid rows per expert
+    M_total: int
+    N: int
+    K: int
+    G: int
+
+
+@dataclasses.dataclass
+class MaskedInputs:
+    a: np.ndarray         # bf16 bits [G][M_max][K]
+    b: np.ndarray         # bf16 bits [G][N][K]
+    masked_m: np.ndarray  # int32 [G]
+    G: int
+    M_max: int
+    N: int
+    K: int
+
+
+def dense(M: int, N: int, K: int, seed: int = 0, outlier_frac: float = 0.0,
+          outlier_scale: float = 30.0, a_std: float = 1.0,
+          b_std: float = 0.02) -> DenseInputs:
+    rng_a = np.random.default_rng(seed + 0)
+    x = rng_a.standard_normal(size=(M, K), dtype=np.float32) * np.float32(a_std)
+    if outlier_frac > 0.0 and M > 0:
+        n_out = max(1, int(np.ceil(outlier_frac * M)))
+        rows = rng_a.choice(M, size=n_out, replace=False)
+        x[rows] *= np.float32(outlier_scale)
+    a = bf16_bits(x)
+    b = normal_bf16(np.random.default_rng(seed + 1), (N, K), b_std)
+    return DenseInputs(a=a, b=b, M=M, N=N, K=K)
+
+
+def contiguous_layout(counts: np.ndarray, align: int = ALIGN_M):
+    """m_indices for groups stacked along M, each padded to ``align`` rows."""
+    padded = [int(-(-int(c) // align) * align) for c in counts]
+    M_total = int(sum(padded))
+    m_indices = np.full(M_total, -1, dtype=np.int32)
+    row = 0
+    for g, (c, p) in enumerate(zip(counts, padded)):
+        m_indices[row:row + int(c)] = g
+        row += p
+    return m_indices, M_total
+
+
+def contiguous(N: int, K: int, counts: Optional[np.ndarray] = None, G: int = 8,
+               seed: int = 0, a_std: float = 1.0, b_std: float = 0.02) -> ContiguousInputs:
+    if counts is None:
+        counts = zipf_top8_counts(seed)[:G]
+    counts = np.asarray(counts, dtype=np.int64)
+    G = len(counts)
+    m_indices, M_total = contiguous_layout(counts)
+    rng_a = np.random.default_rng(seed + 0)
+    M_valid = int(counts.sum())
+    xv = rng_a.standard_normal(size=(M_valid, K), dtype=np.float32) * np.float32(a_std)
+    a = np.zeros((M_total, K), dtype=np.uint16)
+    a[m_indices >= 0] = bf16_bits(xv)
+    b = normal_bf16(np.random.default_rng(seed + 1), (G, N, K), b_std)
+    return ContiguousInputs(a=a, b=b, m_indices=m_indices, counts=counts,
+                            M_total=M_total, N=N, K=K, G=G)
+
+
+def masked(G: int, M_max: int, N: int, K: int, seed: int = 0,
+           masked_m: Optional[np.ndarray] = None, a_std: float = 1.0,
+           b_std: float = 0.02) -> MaskedInputs:
+    a = normal_bf16(np.random.default_rng(seed + 0), (G, M_max, K), a_std)
+    b = normal_bf16(np.random.default_rng(seed + 1), (G, N, K), b_std)
+    if masked_m is None:
+        masked_m = np.random.default_rng(seed + 3).integers(0, M_max + 1, size=G)
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    return MaskedInputs(a=a, b=b, masked_m=masked_m, G=G, M_max=M_max, N=N, K=K)
+
+
+# Named workloads: name -> (kind, constructor kwargs)
+WORKLOADS = {
+    "dense_128x256x512": ("dense", dict(M=128, N=256, K=512)),
+    "decode_64x4096x7168": ("dense", dict(M=64, N=4096, K=7168, outlier_frac=0.01)),
+    "prefill_4096x7168x2048": ("dense", dict(M=4096, N=7168, K=2048)),
+    "prefill_4096x2112x7168": ("dense", dict(M=4096, N=2112, K=7168)),
+    "contiguous_8x4096x7168": ("contiguous", dict(N=4096, K=7168, G=8)),
+    "masked_32x256x4096x7168": ("masked", dict(G=32, M_max=256, N=4096, K=7168)),
+}
+
+
+def make(name: str, seed: int = 0):
+    kind, kw = WORKLOADS[name]
+    if kind == "dense":
+        return dense(seed=seed, **kw)
+    if kind == "contiguous":
+        return contiguous(seed=seed, **kw)
+    return masked(seed=seed, **kw)
+
+
+def flops_and_bytes(kind: str, inp) -> tuple:
+    """Algorithmic FLOPs and HBM bytes of one GEMM call (valid rows only).
+
+    FLOPs = 2 * M_valid * N * K. Bytes = A (1 B/elt) + its fp32 scales (one per
+    128 elements) + B (1 B/elt) and its fp32 scales (one per 128x128 block) for
+    every expert with at least one valid row + D (2 B/elt) over valid rows.
+    """
+    N, K = inp.N, inp.K
+    nb = -(-N // 128)
+    kb = K // 128
+    if kind == "dense":
+        mv, experts = inp.M, 1
+    elif kind == "contiguous":
+        mv = int(inp.counts.sum())
+        experts = int((inp.counts > 0).sum())
+    else:
+        mv = int(inp.masked_m.sum())
+        experts = int((inp.masked_m > 0).sum())
+    flops = 2.0 * mv * N * K
+    byts = mv * K + 4 * mv * kb + experts * (N * K + 4 * nb * kb) + 2 * mv * N
+    return flops, float(byts)
