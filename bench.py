@@ -1,0 +1,479 @@
+"""Benchmark of the FP8 block-scaled GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the per-call hot path over one batch of synthetic
+input: the activation quantizer (per token, per 128 channels) followed by the
+GEMM (dense, contiguous-grouped or masked-grouped, per the workload). Weights
+are quantized once before timing, as inference stores them (pass
+--with-weight-quant to quantize them inside every step as well).
+
+The default workload is decode_64x4096x7168 (the swapped-product decode
+shape). Inputs are resident in HBM when the timed region starts; L2 is flushed
+(a 256 MiB write) before every timed step and the flush is outside the step's
+CUDA events. `value` is FLOPs (2*M_valid*N*K) per step time; `roofline` covers
+the GEMM kernel against the measured HBM bandwidth or FP8 tensor peak; `e2e`
+repeats the step through the public API from pinned host buffers with the
+host<->device copies inside the timed region; `cpu_baseline` times the CPU
+oracle on a bounded sample of the same workload.
+
+Multi-GPU (torchrun, one process per GPU): the path does not shard across
+GPUs within one call, so every rank runs an independent replica (weak
+scaling); the timed region is bracketed by a barrier and the reported time is
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOPS (device-timed) and % of B200 FP8/HBM roofline"
+L2_FLUSH_BYTES = 256 << 20
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_64x4096x7168", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--with-weight-quant", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_grouped_gemm_04_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per GEMM launch from a committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- CPU legs
+
+def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
+    """Oracle on a bounded sample of the workload: quantize the sampled A rows
+    and compute their outputs against all N columns (weights are quantized
+    outside the timed part, as on the GPU side). Returns
+    (flops_per_second, description, seconds)."""
+    import oracle
+
+    K, N = inp.K, inp.N
+    if kind == "dense":
+        a_rows, experts = inp.a, np.zeros(inp.M, np.int64)
+    elif kind == "contiguous":
+        valid = np.nonzero(inp.m_indices >= 0)[0]
+        a_rows, experts = inp.a[valid], inp.m_indices[valid].astype(np.int64)
+    else:
+        sel = [(e, m) for e in range(inp.G) for m in range(int(inp.masked_m[e]))]
+        a_rows = np.stack([inp.a[e, m] for e, m in sel]) if sel else inp.a[0, :0]
+        experts = np.array([e for e, _ in sel], np.int64)
+
+    def weights(e):
+        if e not in cache:
+            b = inp.b if kind == "dense" else inp.b[e]
+            cache[e] = oracle.per_block_cast(b, threads=threads)
+        return cache[e]
+
+    order = np.random.default_rng(0).permutation(len(a_rows))
+    rows = cache.get("rows", 1)
+    while True:
+        take = order[:min(rows, len(order))]
+        for e in np.unique(experts[take]):
+            weights(int(e))
+        t0 = time.perf_counter()
+        qa, sa = oracle.per_token_cast(a_rows[take], threads=threads)
+        for e in np.unique(experts[take]):
+            sub = np.nonzero(experts[take] == e)[0]
+            qb, sb = weights(int(e))
+            oracle.gemm_nt(qa[sub], sa[sub], qb, sb, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or len(take) >= len(order):
+            break
+        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9))
+    cache["rows"] = rows
+    done = len(take)
+    flops = 2.0 * done * N * K
+    desc = "%d of %d valid A rows x all %d columns, K=%d (activation quantization + GEMM)" % (
+        done, len(order), N, K)
+    return flops / dt, desc, dt
+
+
+# ---------------------------------------------------------------------- GPU leg
+
+class Step:
+    """Device buffers and the launches of one step."""
+
+    def __init__(self, fg, torch, kind, inp, with_weight_quant: bool):
+        self.fg, self.torch, self.kind, self.inp = fg, torch, kind, inp
+        self.with_wq = with_weight_quant
+        dev = "cuda"
+        K, N = inp.K, inp.N
+
+        def bf16(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+        self.x = bf16(inp.a)
+        self.w = bf16(inp.b)
+        if kind == "dense":
+            self.G, self.M = 1, inp.M
+            self.A = torch.empty((inp.M, K), dtype=torch.uint8, device=dev)
+            self.B = torch.empty((N, K), dtype=torch.uint8, device=dev)
+            self.D = torch.empty((inp.M, N), dtype=torch.bfloat16, device=dev)
+            Gw = 1
+        elif kind == "contiguous":
+            self.G, self.M = 1, inp.M_total
+            self.A = torch.empty((inp.M_total, K), dtype=torch.uint8, device=dev)
+            self.B = torch.empty((inp.G, N, K), dtype=torch.uint8, device=dev)
+            self.D = torch.empty((inp.M_total, N), dtype=torch.bfloat16, device=dev)
+            self.mi = torch.from_numpy(inp.m_indices).to(dev)
+            Gw = inp.G
+        else:
+            self.G, self.M = inp.G, inp.M_max
+            self.A = torch.empty((inp.G, inp.M_max, K), dtype=torch.uint8, device=dev)
+            self.B = torch.empty((inp.G, N, K), dtype=torch.uint8, device=dev)
+            self.D = torch.empty((inp.G, inp.M_max, N), dtype=torch.bfloat16, device=dev)
+            self.mm = torch.from_numpy(inp.masked_m).to(dev)
+            self.expected_m = max(1, int(round(float(np.mean(inp.masked_m)))))
+            Gw = inp.G
+        self.SA = fg.empty_sfa(self.G, self.M, K, dev)
+        self.SB = fg.empty_sfb(Gw, N, K, dev)
+        self.quant_weights()
+
+    def quant_weights(self):
+        self.fg.per_block_cast_to_fp8(self.w, self.B, self.SB)
+
+    def quant_acts(self):
+        self.fg.per_token_cast_to_fp8(self.x, self.A, self.SA)
+
+    def gemm(self):
+        fg = self.fg
+        if self.kind == "dense":
+            fg.fp8_gemm_nt(self.A, self.SA, self.B, self.SB, self.D)
+        elif self.kind == "contiguous":
+            fg.fp8_grouped_gemm_contiguous(self.A, self.SA, self.B, self.SB, self.D, self.mi)
+        else:
+            fg.fp8_grouped_gemm_masked(self.A, self.SA, self.B, self.SB, self.D, self.mm,
+                                       self.expected_m)
+
+    def launches_per_step(self):
+        return 2 + (1 if self.with_wq else 0)
+
+    def run(self, ev=None):
+        if self.with_wq:
+            self.quant_weights()
+        self.quant_acts()
+        if ev is not None:
+            ev[0].record()
+        self.gemm()
+        if ev is not None:
+            ev[1].record()
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import moe_grouped_gemm_04_b200 as fg
+
+    torch.cuda.set_device(local_rank)
+    fg.load_library()
+    kind = workloads.WORKLOADS[args.workload][0]
+    inp = workloads.make(args.workload, seed=0)
+    flops, alg_bytes = workloads.flops_and_bytes(kind, inp)
+    step = Step(fg, torch, kind, inp, args.with_weight_quant)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+    assert fg.get_device_status() == 0
+
+    K = args.steps
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_gemm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)  # let the sampler see the timed region from its start
+    for i in range(K):
+        flush.zero_()
+        ev_step[i][0].record(stream)
+        step.run(ev_gemm[i])
+        ev_step[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    assert fg.get_device_status() == 0
+    step_ms = [a.elapsed_time(b) for a, b in ev_step]
+    gemm_ms = [a.elapsed_time(b) for a, b in ev_gemm]
+    ms = float(np.mean(step_ms))
+    gms = float(np.mean(gemm_ms))
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        xh = step.x.cpu().pin_memory()
+        dh = torch.empty(step.D.shape, dtype=step.D.dtype).pin_memory()
+        for _ in range(max(1, args.warmup)):
+            step.x.copy_(xh, non_blocking=True)
+            step.run()
+            dh.copy_(step.D, non_blocking=True)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step.x.copy_(xh, non_blocking=True)
+            step.run()
+            dh.copy_(step.D, non_blocking=True)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        e2e = {"ms": e2e_ms, "h2d": xh.numel() * xh.element_size(), "d2h": dh.numel() * dh.element_size()}
+
+    # max over ranks
+    if dist is not None:
+        t = torch.tensor([ms, gms, e2e["ms"] if e2e else 0.0], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, gms = float(t[0]), float(t[1])
+        if e2e:
+            e2e["ms"] = float(t[2])
+
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    tensor_bound = flops / alg_bytes > (2 * peaks.get("bf16_tflops", 1590.0) * 1e12) / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        peak = FP8_OVER_BF16 * peaks["bf16_tflops"]
+        achieved = flops / (gms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+        peak_note = "FP8 = %.1f x %s bf16 burst %.1f TFLOP/s (%s)" % (
+            FP8_OVER_BF16, peak_src, peaks["bf16_tflops"], "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
+    else:
+        peak = peaks["hbm_gbs"]
+        achieved = alg_bytes / (gms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak}
+        peak_note = "%s HBM copy bandwidth (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
+    roof["traffic"] = traffic_for(args.workload)
+    roof["kernel"] = "fp8_gemm_kernel"
+    roof["algorithmic_per_launch"] = {"flops": flops, "bytes": alg_bytes}
+    roof["kernel_ms"] = gms
+    roof["peak_source"] = peak_note
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        threads = oracle.hardware_threads()
+        fps, desc, secs = cpu_sample(inp, kind, args.cpu_seconds, threads, {})
+        cpu = {"value": fps / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "seconds": secs}
+
+    value = world * flops / (ms * 1e-3) / 1e12
+    cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K,
+           "l2": "flushed before every timed step (256 MiB write, outside the step events)",
+           "weights": "quantized inside every step" if args.with_weight_quant else "quantized once before timing",
+           "parallelism": "replicas" if world > 1 else "single GPU"}
+    if kind == "dense":
+        cfg["M"] = inp.M
+    elif kind == "contiguous":
+        cfg.update(G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
+    else:
+        cfg.update(G=inp.G, M_max=inp.M_max, M_valid=int(inp.masked_m.sum()))
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic (seeded numpy, random weights)",
+        "config": cfg, "roofline": roof, "cpu_baseline": cpu,
+        "gpu_launches": step.launches_per_step() * K,
+        "clocks": clocks,
+    }
+    if e2e:
+        out["e2e"] = {"value": world * flops / (e2e["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                      "ms_per_step": e2e["ms"]}
+    return out
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm, on rank 0 only."""
+    if rank != 0:
+        return None
+    import oracle
+    kind = workloads.WORKLOADS[args.workload][0]
+    inp = workloads.make(args.workload, seed=0)
+    threads = oracle.hardware_threads()
+    per_step = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    cache = {}
+    for _ in range(args.warmup):
+        cpu_sample(inp, kind, per_step, threads, cache)
+    vals, descs, secs = [], [], []
+    for _ in range(args.steps):
+        fps, desc, s = cpu_sample(inp, kind, per_step, threads, cache)
+        vals.append(fps)
+        descs.append(desc)
+        secs.append(s)
+    value = float(np.mean(vals)) / 1e12
+    ms = float(np.mean(secs)) * 1e3
+    cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K}
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy)",
+        "config": cfg,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": descs[-1] if descs else ""},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            out = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

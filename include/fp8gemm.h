@@ -1,0 +1,177 @@
+/*
+ * fp8gemm.h - C ABI of the B200 (sm_100a) FP8 block-scaled GEMM library.
+ *
+ * The library computes D[bf16] = (A * sa)(B * sb)^T where A and B hold FP8
+ * e4m3 codes, A carries one fp32 scale per token per 128-channel slice and B
+ * one fp32 scale per 128x128 block, with two-level accumulation: the FP8
+ * products of each 128-wide K block are summed on the tensor cores and then
+ * promoted into an fp32 accumulator with both scales applied.
+ *
+ * Sources for the operation:
+ *   - "DeepGEMM" overview (zixun.chuxinyishu.com/article/345.html), section
+ *     "FP8与细粒度缩放": FP8 operands, activations scaled per slice, weights
+ *     per matrix block, higher-precision accumulation; section "约300行JIT核心"
+ *     paragraph on contiguous and masked MoE layouts (grouping along M, the
+ *     masked layout meeting the communication library); section "swapAB与
+ *     Mega MoE": computing the transposed product for thin M.
+ *   - "一文看懂 DeepSeek 開源項目第三彈" (animattoys.com), sections
+ *     "為現代 AI 計算而造" and "DeepGEMM 部署指南": normal and MoE grouped
+ *     GEMM, two-level accumulation (promotion) because FP8 tensor-core
+ *     accumulation is imprecise.
+ *   - DeepSeek-V3 review "28.5 倍压缩 + 1/10 成本"
+ *     (developer.cloud.tencent.cn/article/2686109), "创新之处" item 4: one
+ *     scale per 128 elements, 128x128 block scaling; "风险与不足" item 6: the
+ *     448.0 FP8 bound used by the quantizer.
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are DEVICE pointers allocated and owned by the caller.
+ *     The library never allocates, frees or retains them.
+ *   - Every data pointer must be 16-byte aligned (TMA requirement).
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream). The
+ *     host returns after the launch; nothing synchronises the host.
+ *   - e4m3 payloads are bytes (OCP E4M3 "fn": bias 7, no infinities, max 448).
+ *     bf16 tensors are passed as their 16-bit patterns. Scales are fp32.
+ *   - Argument errors are reported synchronously (FG_ERR_INVALID_ARG or
+ *     FG_ERR_UNSUPPORTED) and then nothing is launched. Launch failures
+ *     return FG_ERR_CUDA. Faults detected on the device (a bounded wait that
+ *     gave up, masked_m outside [0, M_max], an m_indices entry >= G) set a
+ *     device status word read by fg_get_device_status(); the kernels never
+ *     trap and never wait without a bound.
+ *   - fg_last_error() returns a human-readable detail of the last failing
+ *     call on the calling host thread.
+ *
+ * Scale layouts:
+ *   - Activation scales (SFA) are "MN-major": for each K block kb the scales
+ *     of all M rows are contiguous, with a row stride of fg_sfa_stride(M) =
+ *     round_up(M, 4) floats so that every K block starts 16-byte aligned:
+ *       sfa[(g * (K/128) + kb) * fg_sfa_stride(M) + m]
+ *     (g = group of a batched quantizer call / expert of the masked layout;
+ *     0 otherwise). Entries m in [M, stride) are padding and never read.
+ *   - Weight scales (SFB): sfb[(g * ceil(N/128) + nb) * (K/128) + kb].
+ */
+#ifndef FP8GEMM_H_
+#define FP8GEMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t. */
+struct CUstream_st;
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum {
+  FG_OK = 0,
+  FG_ERR_INVALID_ARG = 1,  /* bad size, null or misaligned pointer */
+  FG_ERR_UNSUPPORTED = 2,  /* valid request this build does not cover */
+  FG_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  FG_ERR_DEVICE = 4        /* device status word set (see fg_get_device_status) */
+} fg_status;
+
+/* Device status word values (returned through fg_get_device_status). */
+#define FG_DEVICE_OK 0
+#define FG_DEVICE_WAIT_TIMEOUT 1   /* a bounded pipeline wait gave up */
+#define FG_DEVICE_BAD_MASKED_M 2   /* masked_m[e] < 0 or > M_max (clamped) */
+#define FG_DEVICE_BAD_M_INDEX 3    /* m_indices entry >= G (tile skipped) */
+
+/* Row stride (in floats) of the MN-major activation-scale layout. */
+int fg_sfa_stride(int M);
+
+/*
+ * Activation quantizer (per token, per 128-channel slice).
+ * For every group g < num_groups, row m < M and K block kb:
+ *   amax  = max |x[g][m][kb*128 .. kb*128+127]|  (bf16 widened exactly)
+ *   amx   = max(amax, 1e-4f)
+ *   sfa   = amx / 448.0f                         (fp32, IEEE division)
+ *   q[..] = e4m3_rne_satfinite(x[..] * (448.0f / amx))  (fp32 product)
+ * x: bf16 [num_groups][M][K]; q: e4m3 [num_groups][M][K];
+ * sfa: fp32, MN-major layout above, num_groups * (K/128) * fg_sfa_stride(M)
+ * floats. K % 128 == 0, M >= 0, num_groups >= 1. The masked layout's A is
+ * one call with num_groups = G, M = M_max; the dense and contiguous A is one
+ * call with num_groups = 1.
+ */
+fg_status per_token_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfa, int num_groups,
+                                int M, int K, cudaStream_t stream);
+
+/*
+ * Weight quantizer (per 128x128 block). Same arithmetic with amax over each
+ * block of 128 rows x 128 columns; a last block along N that has fewer than
+ * 128 rows uses only its valid rows.
+ * x: bf16 [num_groups][N][K]; q: e4m3 [num_groups][N][K];
+ * sfb: fp32 [num_groups][ceil(N/128)][K/128]. K % 128 == 0, N >= 1.
+ */
+fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int num_groups,
+                                int N, int K, cudaStream_t stream);
+
+/*
+ * Dense FP8 GEMM, "NT": D[m][n] = sum_kb sa[m][kb] * sb[n/128][kb] *
+ *   sum_{k in kb} e4m3(A[m][k]) * e4m3(B[n][k]), rounded once to bf16.
+ * A: e4m3 [M][K] (row-major, K contiguous); sfa: MN-major [K/128][stride(M)];
+ * B: e4m3 [N][K]; sfb: [ceil(N/128)][K/128]; D: bf16 [M][N] row-major.
+ * M >= 0, N >= 16 with N % 16 == 0, K % 128 == 0.
+ * For M <= 64 the library uses the swapped product D^T = B * A^T so that the
+ * thin token dimension lands on the tensor-core instruction's N side, and
+ * when that leaves most SMs idle it splits K across the 2 or 4 CTAs of a
+ * thread-block cluster, which sum their partials through distributed shared
+ * memory in a fixed order (deterministic; no scratch memory is used).
+ */
+fg_status fp8_gemm_nt(const uint8_t* A, const float* sfa, const uint8_t* B, const float* sfb,
+                      uint16_t* D, int M, int N, int K, cudaStream_t stream);
+
+/*
+ * MoE grouped FP8 GEMM, contiguous layout: the token groups of G experts are
+ * stacked along M, each group starting on a 128-row boundary and padded to a
+ * multiple of 128 rows. Row m uses expert m_indices[m]'s weights; padding
+ * rows carry m_indices[m] = -1 (their A rows should be zero).
+ * A: e4m3 [M_total][K]; sfa: MN-major [K/128][stride(M_total)];
+ * B: e4m3 [G][N][K]; sfb: [G][ceil(N/128)][K/128]; D: bf16 [M_total][N];
+ * m_indices: int32 [M_total], device memory.
+ * Contract: all valid rows of a 128-row block share one expert and come
+ * before its padding rows. D rows with m_indices[m] = -1 are not written.
+ * M_total % 128 == 0, G >= 1, N % 16 == 0, K % 128 == 0.
+ */
+fg_status fp8_grouped_gemm_contiguous(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                      const float* sfb, uint16_t* D, const int32_t* m_indices,
+                                      int M_total, int N, int K, int G, cudaStream_t stream);
+
+/*
+ * MoE grouped FP8 GEMM, masked layout: expert e owns an M_max-row slab of A
+ * and D, of which the first masked_m[e] rows are valid. masked_m stays on the
+ * device and is never read by the host, so the call does not synchronise.
+ * A: e4m3 [G][M_max][K]; sfa: MN-major [G][K/128][stride(M_max)];
+ * B: e4m3 [G][N][K]; sfb: [G][ceil(N/128)][K/128]; D: bf16 [G][M_max][N];
+ * masked_m: int32 [G], device memory. expected_m: host-side hint of the
+ * typical masked_m (selects the tile shape; any value is correct).
+ * D rows m >= masked_m[e] are not written and the kernel does not read the
+ * A rows past masked_m[e] into any stored output.
+ * G >= 1, M_max >= 1, N % 16 == 0, K % 128 == 0.
+ */
+fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                  const float* sfb, uint16_t* D, const int32_t* masked_m, int G,
+                                  int M_max, int N, int K, int expected_m, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device. Returns FG_OK when it was clear, FG_ERR_DEVICE otherwise
+ * (the detail is in fg_last_error and *code, which may be NULL).
+ */
+fg_status fg_get_device_status(cudaStream_t stream, int* code);
+
+/*
+ * Self-test of the bounded wait used by every pipeline barrier: launches one
+ * CTA that waits on a barrier nobody arrives at, for at most timeout_us
+ * microseconds, after which it sets FG_DEVICE_WAIT_TIMEOUT and returns.
+ */
+fg_status fg_selftest_wait_timeout(int timeout_us, cudaStream_t stream);
+
+const char* fg_status_string(fg_status s);
+const char* fg_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8GEMM_H_ */

@@ -1,0 +1,196 @@
+"""Python binding of libfp8gemm.so, the B200 FP8 block-scaled GEMM library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/fp8gemm.h. Tensors are torch
+tensors used as device memory; the calls run on the current torch CUDA stream
+(or the stream passed in) and never synchronise the host. There is no CPU
+fallback: if the library is missing or the device is not sm_100a, every call
+raises.
+
+The functions carry the C names:
+  per_token_cast_to_fp8, per_block_cast_to_fp8, fp8_gemm_nt,
+  fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked
+plus allocation helpers that return tensors in the layouts the kernels use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8gemm.so")
+
+FG_OK = 0
+FG_ERR_INVALID_ARG = 1
+FG_ERR_UNSUPPORTED = 2
+FG_ERR_CUDA = 3
+FG_ERR_DEVICE = 4
+
+EXPORTED = (
+    "fg_sfa_stride", "per_token_cast_to_fp8", "per_block_cast_to_fp8", "fp8_gemm_nt",
+    "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
+)
+
+
+class FP8GemmError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("%s: %s" % (_status_name(status), message))
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libfp8gemm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise FP8GemmError(FG_ERR_UNSUPPORTED,
+                           "%s is missing; build it with moe_grouped_gemm_04_b200/build.py" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.fg_sfa_stride.argtypes = [I]
+    lib.fg_sfa_stride.restype = I
+    lib.per_token_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
+    lib.per_block_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
+    lib.fp8_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, P]
+    lib.fp8_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+    lib.fp8_grouped_gemm_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+    lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
+    lib.fg_selftest_wait_timeout.argtypes = [I, P]
+    lib.fg_status_string.argtypes = [I]
+    lib.fg_status_string.restype = ctypes.c_char_p
+    lib.fg_last_error.argtypes = []
+    lib.fg_last_error.restype = ctypes.c_char_p
+    for f in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "fp8_gemm_nt",
+              "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
+              "fg_get_device_status", "fg_selftest_wait_timeout"):
+        getattr(lib, f).restype = I
+    _lib = lib
+    return lib
+
+
+def _status_name(s: int) -> str:
+    return {0: "FG_OK", 1: "FG_ERR_INVALID_ARG", 2: "FG_ERR_UNSUPPORTED", 3: "FG_ERR_CUDA",
+            4: "FG_ERR_DEVICE"}.get(s, "FG_ERR_%d" % s)
+
+
+def _check(status: int) -> None:
+    if status != FG_OK:
+        msg = load_library().fg_last_error()
+        raise FP8GemmError(status, msg.decode() if msg else "")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ---------------------------------------------------------------- layouts
+
+def sfa_stride(M: int) -> int:
+    """Row stride (floats) of the MN-major activation-scale layout."""
+    return (M + 3) // 4 * 4
+
+
+def empty_sfa(G: int, M: int, K: int, device) -> torch.Tensor:
+    """Activation scales [G][K/128][stride(M)] (padding entries unused)."""
+    return torch.empty((G, K // 128, sfa_stride(M)), dtype=torch.float32, device=device)
+
+
+def empty_sfb(G: int, N: int, K: int, device) -> torch.Tensor:
+    """Weight scales [G][ceil(N/128)][K/128]."""
+    return torch.empty((G, -(-N // 128), K // 128), dtype=torch.float32, device=device)
+
+
+# ---------------------------------------------------------------- entry points
+
+def per_token_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfa: torch.Tensor,
+                          stream=None) -> None:
+    """x: bf16 [M][K] or [G][M][K] -> q (uint8, same shape), sfa [G][K/128][stride(M)]."""
+    G, M, K = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
+    if x.dtype != torch.bfloat16 or q.dtype != torch.uint8 or sfa.dtype != torch.float32:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "dtypes: x bf16, q uint8, sfa float32")
+    if q.numel() != x.numel() or sfa.numel() < G * (K // 128) * sfa_stride(M):
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "output sizes do not match x")
+    _check(load_library().per_token_cast_to_fp8(_ptr(x), _ptr(q), _ptr(sfa), G, M, K,
+                                                _stream(stream)))
+
+
+def per_block_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfb: torch.Tensor,
+                          stream=None) -> None:
+    """x: bf16 [N][K] or [G][N][K] -> q (uint8, same shape), sfb [G][ceil(N/128)][K/128]."""
+    G, N, K = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
+    if x.dtype != torch.bfloat16 or q.dtype != torch.uint8 or sfb.dtype != torch.float32:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "dtypes: x bf16, q uint8, sfb float32")
+    if q.numel() != x.numel() or sfb.numel() < G * (-(-N // 128)) * (K // 128):
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "output sizes do not match x")
+    _check(load_library().per_block_cast_to_fp8(_ptr(x), _ptr(q), _ptr(sfb), G, N, K,
+                                                _stream(stream)))
+
+
+def fp8_gemm_nt(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor, sfb: torch.Tensor,
+                D: torch.Tensor, stream=None) -> None:
+    """D[M][N] (bf16) = (A * sa)(B * sb)^T; A uint8 [M][K], B uint8 [N][K]."""
+    M, K = A.shape
+    N = B.shape[0]
+    if D.dtype != torch.bfloat16 or tuple(D.shape) != (M, N):
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "D must be bf16 [M][N]")
+    _check(load_library().fp8_gemm_nt(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), M, N, K,
+                                      _stream(stream)))
+
+
+def fp8_grouped_gemm_contiguous(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor,
+                                sfb: torch.Tensor, D: torch.Tensor, m_indices: torch.Tensor,
+                                stream=None) -> None:
+    """A uint8 [M_total][K], B uint8 [G][N][K], m_indices int32 [M_total], D bf16 [M_total][N]."""
+    M_total, K = A.shape
+    G, N, _ = B.shape
+    if m_indices.dtype != torch.int32 or m_indices.numel() != M_total:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "m_indices must be int32 [M_total]")
+    _check(load_library().fp8_grouped_gemm_contiguous(
+        _ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(m_indices), M_total, N, K, G,
+        _stream(stream)))
+
+
+def fp8_grouped_gemm_masked(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor,
+                            sfb: torch.Tensor, D: torch.Tensor, masked_m: torch.Tensor,
+                            expected_m: int, stream=None) -> None:
+    """A uint8 [G][M_max][K], B uint8 [G][N][K], masked_m int32 [G], D bf16 [G][M_max][N]."""
+    G, M_max, K = A.shape
+    N = B.shape[1]
+    if masked_m.dtype != torch.int32 or masked_m.numel() != G:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "masked_m must be int32 [G]")
+    _check(load_library().fp8_grouped_gemm_masked(
+        _ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(masked_m), G, M_max, N, K,
+        int(expected_m), _stream(stream)))
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream and read+clear the device status word (0 = clear)."""
+    code = ctypes.c_int(0)
+    st = load_library().fg_get_device_status(_stream(stream), ctypes.byref(code))
+    if st not in (FG_OK, FG_ERR_DEVICE):
+        _check(st)
+    return int(code.value)
+
+
+def selftest_wait_timeout(timeout_us: int, stream=None) -> None:
+    _check(load_library().fg_selftest_wait_timeout(int(timeout_us), _stream(stream)))

@@ -1,0 +1,522 @@
+// C ABI of the FP8 block-scaled GEMM library (see include/fp8gemm.h):
+// argument validation, TMA descriptor encoding, tile-shape and split-K
+// selection, and kernel launches. One translation unit holds every kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fp8gemm.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace fg {
+namespace {
+
+__device__ int g_status_word;  // device status (FG_DEVICE_*), read by fg_get_device_status
+
+thread_local std::string g_last_error;
+
+fg_status fail(fg_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+fg_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+fg_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FG_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+      return fail(FG_ERR_UNSUPPORTED, "built for sm_100a, device %d is sm_%d%d", dev, major,
+                  minor);
+    e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    d.status = static_cast<int*>(p);
+    d.ready = true;
+  }
+  *out = &d;
+  return FG_OK;
+}
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* s = std::getenv("FG_WAIT_TIMEOUT_MS");
+    const long ms = s ? std::atol(s) : 2000;
+    return static_cast<uint64_t>(ms > 0 ? ms : 2000) * 1000000ull;
+  }();
+  return v;
+}
+
+// ---------------------------------------------------------------- TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+fg_status encode_fn(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!fn) return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *out = fn;
+  return FG_OK;
+}
+
+// 2-D row-major tensor: `inner` elements per row (contiguous), `outer` rows,
+// `row_bytes` between rows; box of box_inner x box_outer elements.
+fg_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swz, const char* what) {
+  EncodeTiledFn fn;
+  fg_status st = encode_fn(&fn);
+  if (st != FG_OK) return st;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FG_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled(%s) failed with %d", what,
+                static_cast<int>(r));
+  return FG_OK;
+}
+
+// ---------------------------------------------------------------- validation
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fg_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(FG_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(FG_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return FG_OK;
+}
+
+#define FG_TRY(expr)                 \
+  do {                               \
+    const fg_status _s = (expr);     \
+    if (_s != FG_OK) return _s;      \
+  } while (0)
+
+int sfa_stride(int M) { return (M + 3) / 4 * 4; }
+
+// ---------------------------------------------------------------- GEMM configs
+
+//                      BT   BW   swap  stages PW split
+using CfgNormal = GemmCfg<128, 128, false, 6, 8, 1>;
+using CfgSwap16 = GemmCfg<16, 128, true, 8, 4, 1>;
+using CfgSwap32 = GemmCfg<32, 128, true, 8, 4, 1>;
+using CfgSwap64 = GemmCfg<64, 128, true, 8, 4, 1>;
+using CfgSwap16S2 = GemmCfg<16, 128, true, 8, 4, 2>;
+using CfgSwap32S2 = GemmCfg<32, 128, true, 8, 4, 2>;
+using CfgSwap64S2 = GemmCfg<64, 128, true, 7, 4, 2>;
+using CfgSwap16S4 = GemmCfg<16, 128, true, 8, 4, 4>;
+using CfgSwap32S4 = GemmCfg<32, 128, true, 8, 4, 4>;
+using CfgSwap64S4 = GemmCfg<64, 128, true, 7, 4, 4>;
+
+struct KernelInfo {
+  bool attr_set = false;
+  int max_clusters = 0;  // max co-resident clusters (split-K configs)
+};
+
+template <class C, int FORM>
+fg_status kernel_info(int dev, KernelInfo** out) {
+  static KernelInfo info[kMaxDevices];
+  KernelInfo& k = info[dev];
+  if (!k.attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<C, FORM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if (C::SPLIT > 1) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = C::SPLIT;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(C::SPLIT * 64);
+      cfg.blockDim = dim3(C::NUM_THREADS);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<C, FORM>, &cfg);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+      if (n < 1) return fail(FG_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", C::SPLIT);
+      k.max_clusters = n;
+    }
+    k.attr_set = true;
+  }
+  *out = &k;
+  return FG_OK;
+}
+
+struct Problem {
+  int form;
+  const uint8_t* A;
+  const float* sfa;
+  const uint8_t* B;
+  const float* sfb;
+  uint16_t* D;
+  const int32_t* m_indices;
+  const int32_t* masked_m;
+  int M;  // rows of one token slab
+  int N, K, G;
+  int slabs;  // token slabs in A (G for masked, else 1)
+};
+
+struct Plan {
+  int bt;      // token rows per tile (128 = normal form, else swapped)
+  int splits;  // CTAs per cluster sharing one tile's K blocks
+  int num_mt, num_nt;
+};
+
+// Tile shape and split-K factor. The swapped product (tokens on the MMA's N
+// side) is used for dense M <= 64 and for masked layouts whose expected rows
+// per expert are <= 64; when it leaves most SMs idle, K is split across a
+// cluster of 2 or 4 CTAs.
+Plan plan_for(const Problem& pr, int sm_count, int expected_m) {
+  Plan pl{};
+  const int KB = pr.K / 128;
+  int small_m = 1 << 30;
+  if (pr.form == kFormDense) small_m = pr.M;
+  if (pr.form == kFormMasked) small_m = expected_m;
+  if (small_m <= 16) pl.bt = 16;
+  else if (small_m <= 32) pl.bt = 32;
+  else if (small_m <= 64) pl.bt = 64;
+  else pl.bt = 128;
+  if (pr.form == kFormMasked && pl.bt < 64) pl.bt = 64;  // one swapped shape for masked
+  pl.num_mt = (pr.M + pl.bt - 1) / pl.bt;
+  pl.num_nt = (pr.N + 127) / 128;
+  pl.splits = 1;
+  if (pr.form == kFormDense && pl.bt < 128) {
+    const int tiles = pl.num_mt * pl.num_nt;
+    for (int s : {4, 2}) {
+      if (tiles * s <= sm_count && KB >= 2 * s) {
+        pl.splits = s;
+        break;
+      }
+    }
+  }
+  return pl;
+}
+
+template <class C, int FORM>
+fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, int dev_id,
+                      cudaStream_t stream) {
+  KernelInfo* ki = nullptr;
+  FG_TRY((kernel_info<C, FORM>(dev_id, &ki)));
+  const int KB = pr.K / 128;
+  CUtensorMap tmA, tmB, tmSA;
+  FG_TRY(make_map(&tmA, pr.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
+                  static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "A"));
+  FG_TRY(make_map(&tmB, pr.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
+                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::BW,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "B"));
+  FG_TRY(make_map(&tmSA, pr.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.M,
+                  static_cast<uint64_t>(pr.slabs) * KB,
+                  static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
+  GemmParams p{};
+  p.M = pr.M;
+  p.N = pr.N;
+  p.K = pr.K;
+  p.G = pr.G;
+  p.KB = KB;
+  p.NB = (pr.N + 127) / 128;
+  p.num_mt = pl.num_mt;
+  p.num_nt = pl.num_nt;
+  p.sfb = pr.sfb;
+  p.D = pr.D;
+  p.m_indices = pr.m_indices;
+  p.masked_m = pr.masked_m;
+  p.status = dev.status;
+  p.timeout_ns = wait_limit_ns();
+  int64_t tiles = static_cast<int64_t>(pl.num_mt) * pl.num_nt;
+  if (FORM == kFormMasked) tiles *= pr.G;  // upper bound: masked_m lives on the device
+  int64_t grid;
+  if (C::SPLIT > 1) {
+    grid = C::SPLIT * std::max<int64_t>(1, std::min<int64_t>(tiles, ki->max_clusters));
+  } else {
+    grid = std::max<int64_t>(1, std::min<int64_t>(tiles, dev.sm_count));
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::NUM_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the
+  attr[0].val.programmaticStreamSerializationAllowed = 1;           // previous kernel
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (C::SPLIT > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C::SPLIT;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<C, FORM>, tmA, tmB, tmSA, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_kernel launch");
+  return FG_OK;
+}
+
+template <int FORM>
+fg_status dispatch(const Problem& pr, const Plan& pl, const DeviceInfo& dev, int dev_id,
+                   cudaStream_t stream) {
+  if (pl.bt == 128) return launch_gemm<CfgNormal, FORM>(pr, pl, dev, dev_id, stream);
+  if constexpr (FORM == kFormMasked) {
+    if (pl.bt == 64) return launch_gemm<CfgSwap64, FORM>(pr, pl, dev, dev_id, stream);
+  }
+  if constexpr (FORM == kFormDense) {
+    switch (pl.bt * 10 + pl.splits) {
+      case 161: return launch_gemm<CfgSwap16, FORM>(pr, pl, dev, dev_id, stream);
+      case 162: return launch_gemm<CfgSwap16S2, FORM>(pr, pl, dev, dev_id, stream);
+      case 164: return launch_gemm<CfgSwap16S4, FORM>(pr, pl, dev, dev_id, stream);
+      case 321: return launch_gemm<CfgSwap32, FORM>(pr, pl, dev, dev_id, stream);
+      case 322: return launch_gemm<CfgSwap32S2, FORM>(pr, pl, dev, dev_id, stream);
+      case 324: return launch_gemm<CfgSwap32S4, FORM>(pr, pl, dev, dev_id, stream);
+      case 641: return launch_gemm<CfgSwap64, FORM>(pr, pl, dev, dev_id, stream);
+      case 642: return launch_gemm<CfgSwap64S2, FORM>(pr, pl, dev, dev_id, stream);
+      case 644: return launch_gemm<CfgSwap64S4, FORM>(pr, pl, dev, dev_id, stream);
+      default: break;
+    }
+  }
+  return fail(FG_ERR_UNSUPPORTED, "no kernel for token tile %d, split %d", pl.bt, pl.splits);
+}
+
+fg_status run_gemm(const Problem& pr, int expected_m, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const Plan pl = plan_for(pr, dev->sm_count, expected_m);
+  if (pr.form == kFormContig && pl.num_mt > kTableMax)
+    return fail(FG_ERR_UNSUPPORTED, "M_total %d exceeds %d rows", pr.M, kTableMax * pl.bt);
+  if (pr.form == kFormMasked && pr.G + 1 > kTableMax)
+    return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d experts", pr.G, kTableMax - 1);
+  switch (pr.form) {
+    case kFormDense: return dispatch<kFormDense>(pr, pl, *dev, dev_id, stream);
+    case kFormContig: return dispatch<kFormContig>(pr, pl, *dev, dev_id, stream);
+    default: return dispatch<kFormMasked>(pr, pl, *dev, dev_id, stream);
+  }
+}
+
+fg_status check_gemm_common(const uint8_t* A, const float* sfa, const uint8_t* B,
+                            const float* sfb, uint16_t* D, int N, int K) {
+  if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
+  if (N <= 0 || N % 16 != 0) return fail(FG_ERR_INVALID_ARG, "N=%d must be a positive multiple of 16", N);
+  FG_TRY(check_ptr(A, "A"));
+  FG_TRY(check_ptr(sfa, "sfa"));
+  FG_TRY(check_ptr(B, "B"));
+  FG_TRY(check_ptr(sfb, "sfb"));
+  FG_TRY(check_ptr(D, "D"));
+  return FG_OK;
+}
+
+// Launch with programmatic stream serialization (the kernel waits on the
+// previous grid with griddepcontrol.wait before touching memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+__global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl ctl{&abort_flag, status, limit_ns};
+    // Nobody arrives on `bar`: the wait must give up after limit_ns.
+    (void)mbar_wait(&bar, 0, ctl);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace fg
+
+using namespace fg;
+
+extern "C" {
+
+int fg_sfa_stride(int M) { return sfa_stride(M); }
+
+fg_status per_token_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfa, int num_groups, int M,
+                                int K, cudaStream_t stream) {
+  if (num_groups < 1) return fail(FG_ERR_INVALID_ARG, "num_groups=%d must be >= 1", num_groups);
+  if (M < 0) return fail(FG_ERR_INVALID_ARG, "M=%d must be >= 0", M);
+  if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
+  if (M == 0) return FG_OK;
+  FG_TRY(check_ptr(x, "x"));
+  FG_TRY(check_ptr(q, "q"));
+  FG_TRY(check_ptr(sfa, "sfa"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  const int64_t slices = static_cast<int64_t>(num_groups) * M * (K / 128);
+  const int64_t blocks_needed = (slices * 16 + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, int64_t(dev->sm_count) * 16));
+  const cudaError_t e = launch_pdl(per_token_cast_kernel, dim3(grid), dim3(256), stream, x, q, sfa,
+                                   num_groups, M, K, sfa_stride(M));
+  if (e != cudaSuccess) return cuda_fail(e, "per_token_cast_kernel launch");
+  return FG_OK;
+}
+
+fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int num_groups, int N,
+                                int K, cudaStream_t stream) {
+  if (num_groups < 1) return fail(FG_ERR_INVALID_ARG, "num_groups=%d must be >= 1", num_groups);
+  if (N <= 0) return fail(FG_ERR_INVALID_ARG, "N=%d must be >= 1", N);
+  if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
+  FG_TRY(check_ptr(x, "x"));
+  FG_TRY(check_ptr(q, "q"));
+  FG_TRY(check_ptr(sfb, "sfb"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  const int64_t blocks = static_cast<int64_t>(num_groups) * ((N + 127) / 128) * (K / 128);
+  if (blocks > 0x7FFFFFFF) return fail(FG_ERR_UNSUPPORTED, "too many blocks");
+  const cudaError_t e = launch_pdl(per_block_cast_kernel, dim3(static_cast<unsigned>(blocks)),
+                                   dim3(256), stream, x, q, sfb, num_groups, N, K);
+  if (e != cudaSuccess) return cuda_fail(e, "per_block_cast_kernel launch");
+  return FG_OK;
+}
+
+fg_status fp8_gemm_nt(const uint8_t* A, const float* sfa, const uint8_t* B, const float* sfb,
+                      uint16_t* D, int M, int N, int K, cudaStream_t stream) {
+  if (M < 0) return fail(FG_ERR_INVALID_ARG, "M=%d must be >= 0", M);
+  if (M == 0) return FG_OK;
+  FG_TRY(check_gemm_common(A, sfa, B, sfb, D, N, K));
+  Problem pr{kFormDense, A, sfa, B, sfb, D, nullptr, nullptr, M, N, K, 1, 1};
+  return run_gemm(pr, M, stream);
+}
+
+fg_status fp8_grouped_gemm_contiguous(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                      const float* sfb, uint16_t* D, const int32_t* m_indices,
+                                      int M_total, int N, int K, int G, cudaStream_t stream) {
+  if (M_total < 0 || M_total % 128 != 0)
+    return fail(FG_ERR_INVALID_ARG, "M_total=%d must be a non-negative multiple of 128", M_total);
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (M_total == 0) return FG_OK;
+  FG_TRY(check_gemm_common(A, sfa, B, sfb, D, N, K));
+  FG_TRY(check_ptr(m_indices, "m_indices"));
+  Problem pr{kFormContig, A, sfa, B, sfb, D, m_indices, nullptr, M_total, N, K, G, 1};
+  return run_gemm(pr, M_total, stream);
+}
+
+fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                  const float* sfb, uint16_t* D, const int32_t* masked_m, int G,
+                                  int M_max, int N, int K, int expected_m, cudaStream_t stream) {
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (M_max < 1) return fail(FG_ERR_INVALID_ARG, "M_max=%d must be >= 1", M_max);
+  FG_TRY(check_gemm_common(A, sfa, B, sfb, D, N, K));
+  FG_TRY(check_ptr(masked_m, "masked_m"));
+  if (expected_m <= 0) expected_m = M_max;
+  Problem pr{kFormMasked, A, sfa, B, sfb, D, nullptr, masked_m, M_max, N, K, G, G};
+  return run_gemm(pr, expected_m, stream);
+}
+
+fg_status fg_get_device_status(cudaStream_t stream, int* code) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(status)");
+  if (code) *code = v;
+  if (v == 0) return FG_OK;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(status)");
+  const char* what = v == FG_DEVICE_WAIT_TIMEOUT   ? "a pipeline wait timed out"
+                     : v == FG_DEVICE_BAD_MASKED_M ? "masked_m outside [0, M_max]"
+                     : v == FG_DEVICE_BAD_M_INDEX  ? "m_indices entry >= G"
+                                                   : "unknown device status";
+  return fail(FG_ERR_DEVICE, "device status %d: %s", v, what);
+}
+
+fg_status fg_selftest_wait_timeout(int timeout_us, cudaStream_t stream) {
+  if (timeout_us <= 0 || timeout_us > 10000000)
+    return fail(FG_ERR_INVALID_ARG, "timeout_us=%d must be in (0, 1e7]", timeout_us);
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(dev->status, static_cast<uint64_t>(timeout_us) * 1000ull);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest_wait_kernel launch");
+  return FG_OK;
+}
+
+const char* fg_status_string(fg_status s) {
+  switch (s) {
+    case FG_OK: return "FG_OK";
+    case FG_ERR_INVALID_ARG: return "FG_ERR_INVALID_ARG";
+    case FG_ERR_UNSUPPORTED: return "FG_ERR_UNSUPPORTED";
+    case FG_ERR_CUDA: return "FG_ERR_CUDA";
+    case FG_ERR_DEVICE: return "FG_ERR_DEVICE";
+  }
+  return "FG_ERR_UNKNOWN";
+}
+
+const char* fg_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

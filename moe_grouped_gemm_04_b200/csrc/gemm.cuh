@@ -1,0 +1,635 @@
+// FP8 e4m3 block-scaled GEMM for sm_100a: tcgen05 MMAs into tensor memory,
+// per-128-K promotion into fp32 registers, persistent tile scheduling over the
+// dense, contiguous-grouped and masked-grouped layouts.
+//
+// The operation (two-level accumulation) follows "一文看懂 DeepSeek 開源項目第三彈"
+// (animattoys.com), section "為現代 AI 計算而造" and the deployment guide's
+// note on promotion, and the "DeepGEMM" overview (zixun.chuxinyishu.com/
+// article/345.html), section "FP8与细粒度缩放":
+//   D[m][n] = sum_kb sa[m][kb] * sb[n/128][kb] * P_kb[m][n],
+//   P_kb[m][n] = sum_{k in block kb} a[m][k] * b[n][k]   (FP8 products, fp32)
+// The grouped layouts follow the same page's paragraph on contiguous and
+// masked MoE grouping, and the swapped product (D^T = B A^T for thin M) its
+// section "swapAB与Mega MoE".
+//
+// CTA roles (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: per K block loads the token tile, the weight
+//               tile and the token scales, all completing on the stage's
+//               "full" barrier.
+//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one
+//               of two TMEM partial buffers, then commits to the stage's
+//               "empty" barrier and the buffer's "tmem full" barrier.
+//   warps 2..   promotion + epilogue: per K block read the partial from TMEM
+//               (tcgen05.ld), add partial * (sa * sb) into fp32 registers
+//               (sb, one value per 128 weight rows and K block, is read from
+//               global memory two K blocks ahead), release the TMEM buffer and
+//               the stage; after the last K block round to bf16 and store D.
+// Two TMEM buffers let the MMA of block kb+1 run while block kb is promoted.
+//
+// Normal form: MMA M = 128 token rows, MMA N = BW weight rows (TMEM lane =
+// token, column = weight). Swapped form: MMA M = 128 weight rows, MMA N = BT
+// tokens (TMEM lane = weight, column = token), used when M is small.
+//
+// Split-K (SPLIT > 1): the K blocks of one output tile are dealt round robin
+// to the SPLIT CTAs of a thread-block cluster (CTA r takes kb = r, r + SPLIT,
+// ...), so that at any moment the cluster reads adjacent 128-byte pieces of
+// the same weight rows. The fp32 partial tiles are then reduce-scattered
+// through distributed shared memory: CTA j owns token rows
+// [j * SLICE_M, (j + 1) * SLICE_M); every CTA pushes its partial values of
+// those rows into CTA j's receive slot for that sender with st.async, whose
+// bytes count down CTA j's "red_ready" mbarrier (no round trips). CTA j then
+// sums its slots in split order and stores its slice of D, so the result
+// does not depend on which CTA finishes first.
+//
+// Programmatic dependent launch: the prologue (barrier init, TMEM
+// allocation, descriptor prefetch) may overlap the previous kernel of the
+// stream; every global-memory access comes after griddepcontrol.wait.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace fg {
+
+enum : int { kFormDense = 0, kFormContig = 1, kFormMasked = 2 };
+
+constexpr int kTableMax = 2048;  // contiguous: token tiles; masked: experts + 1
+constexpr uint64_t kDrainLimitNs = 20000000ull;  // 20 ms for in-flight copies at teardown
+
+struct GemmParams {
+  int M;       // rows of one token slab: dense M, contiguous M_total, masked M_max
+  int N, K, G;
+  int KB;      // K / 128
+  int NB;      // ceil(N / 128)
+  int num_mt;  // token tiles per slab
+  int num_nt;  // weight tiles
+  const float* sfb;
+  uint16_t* D;
+  const int32_t* m_indices;
+  const int32_t* masked_m;
+  int* status;
+  uint64_t timeout_ns;
+};
+
+template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_>
+struct GemmCfg {
+  static constexpr int BT = BT_;          // token rows per tile
+  static constexpr int BW = BW_;          // weight rows per tile
+  static constexpr bool SWAP = SWAP_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr int PW = PW_;          // promotion warps
+  static constexpr int SPLIT = SPLIT_;    // CTAs per cluster sharing one tile's K blocks
+  static constexpr int MMA_N = SWAP ? BT : BW;
+  static_assert(SWAP ? (BW == 128) : (BT == 128), "the lane operand has 128 rows");
+  static_assert(MMA_N % 16 == 0 && MMA_N >= 16 && MMA_N <= 256, "tcgen05 N for M = 128");
+  static_assert(PW % 4 == 0, "promotion warps cover the 4 TMEM lane quadrants");
+  static constexpr int WPQ = PW / 4;      // promotion warps per lane quadrant
+  static constexpr int COLS = MMA_N / WPQ;
+  static_assert(COLS % 8 == 0, "columns per promotion thread");
+  static_assert(SWAP || (COLS <= 128 && (128 % COLS == 0)), "one weight scale per thread");
+  static constexpr int A_BYTES = BT * 128;
+  static constexpr int B_BYTES = BW * 128;
+  static constexpr int SA_BYTES = BT * 4;                       // one TMA box of token scales
+  static constexpr int SA_STAGE = (SA_BYTES + 127) / 128 * 128;  // TMA smem destinations: 128-B aligned
+  static constexpr uint32_t TX_BYTES = A_BYTES + B_BYTES + SA_BYTES;
+  static constexpr int TMEM_USED = 2 * MMA_N;
+  static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
+                                   : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "TMEM has 512 columns");
+  static constexpr int NUM_THREADS = (2 + PW) * 32;
+  // split-K receive slots: SPLIT slots (one per sender) of SLICE_M token rows
+  // x TN weights in fp32, stored as groups of 4 consecutive values along the
+  // dimension a promotion thread holds, with the lane dimension next, so that
+  // the 16-byte pushes of a warp land contiguously:
+  //   swapped form (lane = weight): slot[token / 4][weight][token % 4]
+  //   normal form  (lane = token):  slot[weight / 4][token][weight % 4]
+  static_assert(SPLIT == 1 || (PW == 4 && (SPLIT == 2 || SPLIT == 4 || SPLIT == 8)),
+                "split-K uses 128 promotion threads and 2, 4 or 8 CTAs");
+  static constexpr int TN = SWAP ? 128 : BW;  // weight columns of a tile
+  static constexpr int SLICE_M = BT / SPLIT;
+  static constexpr int SLOT_FLOATS = SLICE_M * TN;
+  static constexpr int RED_BYTES = SPLIT > 1 ? SPLIT * SLOT_FLOATS * 4 : 0;
+  static constexpr uint32_t SLICE_TX = SPLIT * SLICE_M * TN * 4;  // bytes a CTA receives per tile
+  // normal-form reduction: VPT consecutive weights of one token per thread
+  static constexpr int VPT = SPLIT > 1 && !SWAP ? SLICE_M * TN / 128 : 8;
+  static_assert(SPLIT == 1 || (BT % SPLIT == 0 && SLICE_M % 4 == 0 && COLS % 4 == 0),
+                "16-byte pushes of 4 consecutive tokens (swapped) or weights (normal)");
+  static_assert(SPLIT == 1 || SWAP || SLICE_M % 32 == 0, "a warp's tokens share one owner");
+  static_assert(SPLIT == 1 || SWAP || (VPT % 8 == 0 && TN % VPT == 0), "16-byte D stores");
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SA = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_RED = OFF_SA + STAGES * SA_STAGE;
+  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;  // + alignment slack
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
+  static_assert(SA_BYTES % 16 == 0, "TMA box inner extent");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+};
+
+struct Tile {
+  int valid;
+  int e;      // expert (0 for dense)
+  int mt;     // token tile within the slab
+  int nt;     // weight tile
+};
+
+template <int FORM>
+__device__ __forceinline__ int total_tiles(const GemmParams& p, const int* table) {
+  if (FORM == kFormMasked) return table[p.G];
+  return p.num_mt * p.num_nt;
+}
+
+template <int FORM>
+__device__ __forceinline__ Tile resolve_tile(const GemmParams& p, const int* table, int t) {
+  Tile w;
+  if (FORM == kFormMasked) {
+    int lo = 0, hi = p.G;  // table[lo] <= t < table[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (table[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int local = t - table[lo];
+    w.e = lo;
+    w.mt = local / p.num_nt;
+    w.nt = local % p.num_nt;
+    w.valid = 1;
+  } else {
+    w.mt = t / p.num_nt;
+    w.nt = t % p.num_nt;
+    if (FORM == kFormContig) {
+      w.e = table[w.mt];
+      w.valid = w.e >= 0;
+    } else {
+      w.e = 0;
+      w.valid = 1;
+    }
+  }
+  return w;
+}
+
+// Runs on warp 0 before the main loops. Contiguous: expert of every token tile
+// (read from the tile's first row), -1 for padding tiles. Masked: exclusive
+// prefix over experts of the number of (token tile, weight tile) pairs.
+template <class C, int FORM>
+__device__ void build_table(const GemmParams& p, int* table, int lane) {
+  if (FORM == kFormContig) {
+    for (int mt = lane; mt < p.num_mt; mt += 32) {
+      int v = __ldg(p.m_indices + static_cast<int64_t>(mt) * C::BT);
+      if (v >= p.G) {
+        raise_status(p.status, 3 /* FG_DEVICE_BAD_M_INDEX */);
+        v = -1;
+      }
+      table[mt] = v < 0 ? -1 : v;
+    }
+  } else if (FORM == kFormMasked) {
+    const int per = (p.G + 31) / 32;
+    const int e0 = lane * per;
+    const int e1 = min(p.G, e0 + per);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) {
+      int mm = __ldg(p.masked_m + e);
+      if (mm < 0 || mm > p.M) {
+        raise_status(p.status, 2 /* FG_DEVICE_BAD_MASKED_M */);
+        mm = mm < 0 ? 0 : p.M;
+      }
+      const int cnt = (mm + C::BT - 1) / C::BT * p.num_nt;
+      table[e + 1] = cnt;
+      local += cnt;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      run += table[e + 1];
+      table[e + 1] = run;
+    }
+    if (lane == 0) table[0] = 0;
+  }
+}
+
+// Bounded wait used while tearing down: ignores the abort flag, only the
+// time limit, so that copies and MMAs already in flight land before the CTA
+// releases its shared and tensor memory.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+// Stores `NCOL` consecutive accumulator columns of one tile row (TMEM lane)
+// to D. Normal form: the row is a token, the columns weights (16-byte
+// vectors). Swapped form: the row is a weight, the columns tokens (2-byte
+// stores; the 32 lanes of a warp write 32 consecutive weights of one token).
+template <class C, int FORM, int NCOL>
+__device__ __forceinline__ void store_tile_part(const GemmParams& p, const Tile& w, int row,
+                                                int col0, const float* v, int m_valid,
+                                                int row_mi) {
+  const int64_t slab = FORM == kFormMasked ? static_cast<int64_t>(w.e) * p.M : 0;
+  if (!C::SWAP) {
+    const int m = w.mt * C::BT + row;
+    bool ok = m < m_valid;
+    if (FORM == kFormContig) ok = ok && row_mi >= 0;
+    if (!ok) return;
+    uint16_t* dst = p.D + (slab + m) * p.N;
+#pragma unroll
+    for (int j = 0; j < NCOL; j += 8) {
+      const int n = w.nt * C::BW + col0 + j;
+      if (n < p.N) {
+        uint4 q;
+        q.x = pack_bf16x2(v[j + 0], v[j + 1]);
+        q.y = pack_bf16x2(v[j + 2], v[j + 3]);
+        q.z = pack_bf16x2(v[j + 4], v[j + 5]);
+        q.w = pack_bf16x2(v[j + 6], v[j + 7]);
+        *reinterpret_cast<uint4*>(dst + n) = q;
+      }
+    }
+  } else {
+    const int n = w.nt * 128 + row;
+    if (n >= p.N) return;
+#pragma unroll
+    for (int j = 0; j < NCOL; ++j) {
+      const int m = w.mt * C::BT + col0 + j;
+      bool ok = m < m_valid;
+      if (FORM == kFormContig) ok = ok && __ldg(p.m_indices + (m < p.M ? m : 0)) >= 0;
+      if (ok) p.D[(slab + m) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(v[j], 0.0f) & 0xFFFFu);
+    }
+  }
+}
+
+template <class C, int FORM>
+__device__ __forceinline__ void issue_stage(const GemmParams& p, const Tile& w, int kb, uint32_t it,
+                                            uint8_t* sA, uint8_t* sB, uint8_t* sSA, uint64_t* full,
+                                            const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                            const CUtensorMap* tmSA) {
+  const int s = it % C::STAGES;
+  const int a_row = (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
+  const int b_row = w.e * p.N + w.nt * C::BW;
+  const int sa_y = (FORM == kFormMasked ? w.e * p.KB : 0) + kb;
+  mbar_arrive_expect_tx(&full[s], C::TX_BYTES);
+  tma_load_2d(sB + s * C::B_BYTES, tmB, &full[s], kb * 128, b_row);
+  tma_load_2d(sA + s * C::A_BYTES, tmA, &full[s], kb * 128, a_row);
+  tma_load_2d(sSA + s * C::SA_STAGE, tmSA, &full[s], w.mt * C::BT, sa_y);
+}
+
+template <class C, int FORM>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmSA, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sB = smem + C::OFF_B;
+  uint8_t* sSA = smem + C::OFF_SA;
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* red_ready = tempty + 2;    // all partials of the current tile are in place
+  uint64_t* red_free = red_ready + 1;  // every CTA has finished reading them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int* table = reinterpret_cast<int*>(smem + C::OFF_TABLE);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // tiles are dealt to CTAs (or, with split-K, to clusters) round robin;
+  // the K blocks of a tile to the CTAs of its cluster
+  const int t_first = C::SPLIT > 1 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int t_step = C::SPLIT > 1 ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
+  const int kb_first = C::SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  constexpr int kb_step = C::SPLIT;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);               // producer's expect_tx (+ TMA bytes)
+      mbar_init(&empty[s], 1 + C::PW);      // MMA commit + one arrival per promotion warp
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::PW);
+    }
+    mbar_init(red_ready, 1);                 // own expect_tx; peers' bytes complete_tx
+    mbar_init(red_free, C::SPLIT * C::PW);   // one arrival per promotion warp of each CTA
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmSA);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  // Everything above may overlap the previous kernel; memory comes after this.
+  grid_dependency_wait();
+  uint32_t pre_issued = 0;  // first-tile stages the producer issued before the CTA-wide sync
+  if (warp == 0) {
+    build_table<C, FORM>(p, table, lane);
+    __syncwarp();
+    if (lane == 0 && t_first < total_tiles<FORM>(p, table)) {
+      const Tile w = resolve_tile<FORM>(p, table, t_first);
+      if (w.valid) {
+        for (int kb = kb_first; kb < p.KB && pre_issued < C::STAGES; kb += kb_step, ++pre_issued)
+          issue_stage<C, FORM>(p, w, kb, pre_issued, sA, sB, sSA, full, &tmA, &tmB, &tmSA);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  if constexpr (C::SPLIT > 1) cluster_sync_all();  // peers' barriers are initialised
+  tc_fence_after();
+
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+  const int total = total_tiles<FORM>(p, table);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = t_first; t < total; t += t_step) {
+        const Tile w = resolve_tile<FORM>(p, table, t);
+        if (!w.valid) continue;
+        for (int kb = kb_first; kb < p.KB; kb += kb_step, ++it) {
+          if (it < pre_issued) continue;
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) goto producer_done;
+          issue_stage<C, FORM>(p, w, kb, it, sA, sB, sSA, full, &tmA, &tmB, &tmSA);
+        }
+      }
+    producer_done:
+      // Before the CTA exits, the last fill of every stage must have landed
+      // and been released (its TMA bytes and the MMA commit's arrival).
+      it = it > pre_issued ? it : pre_issued;
+      for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
+        const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
+        drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+        drain_wait(&empty[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = mma_idesc_e4m3(128, C::MMA_N);
+      uint32_t it = 0;
+      for (int t = t_first; t < total; t += t_step) {
+        const Tile w = resolve_tile<FORM>(p, table, t);
+        if (!w.valid) continue;
+        for (int kb = kb_first; kb < p.KB; kb += kb_step, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          const int b = it & 1;
+          const uint32_t tph = (it >> 1) & 1u;
+          if (!mbar_wait(&tempty[b], tph ^ 1u, ctl)) goto mma_done;
+          tc_fence_after();
+          if (!mbar_wait(&full[s], ph, ctl)) goto mma_done;
+          tc_fence_after();
+          const uint8_t* lane_tile = C::SWAP ? sB + s * C::B_BYTES : sA + s * C::A_BYTES;
+          const uint8_t* col_tile = C::SWAP ? sA + s * C::A_BYTES : sB + s * C::B_BYTES;
+          const uint64_t adesc = smem_desc_sw128(smem_u32(lane_tile));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(col_tile));
+          const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::MMA_N);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            // advance 32 bytes (= 32 e4m3 along K) inside the 128-byte swizzled row
+            mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[b]);
+        }
+      }
+    mma_done:
+      if (it > 0) drain_wait(&tfull[(it - 1) & 1], ((it - 1) >> 1) & 1u, kDrainLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ promotion + epilogue
+    const int pw = warp - 2;
+    const int quad = warp & 3;          // TMEM lanes this warp may access
+    const int part = pw >> 2;           // column slice of the accumulator
+    const int row = quad * 32 + lane;   // TMEM lane = row of the lane operand
+    const int c0 = part * C::COLS;
+    const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
+    uint32_t it = 0;
+    uint32_t tiles_done = 0;
+    for (int t = t_first; t < total; t += t_step) {
+      const Tile w = resolve_tile<FORM>(p, table, t);
+      if (!w.valid) continue;
+      // row bounds of this tile's token slab (read early, used in the epilogue)
+      int m_valid = p.M;
+      if (FORM == kFormMasked) {
+        m_valid = __ldg(p.masked_m + w.e);
+        m_valid = m_valid < 0 ? 0 : (m_valid > p.M ? p.M : m_valid);
+      }
+      // weight scale of this thread's 128 weight rows, two K blocks ahead
+      const int nb = w.nt * (C::BW / 128) + (C::SWAP ? 0 : c0 / 128);
+      const float* sb_row = p.sfb + (static_cast<int64_t>(w.e) * p.NB + min(nb, p.NB - 1)) * p.KB;
+      float sb_next0 = kb_first < p.KB ? __ldg(sb_row + kb_first) : 0.0f;
+      float sb_next1 = kb_first + kb_step < p.KB ? __ldg(sb_row + kb_first + kb_step) : 0.0f;
+      float acc[C::COLS];
+#pragma unroll
+      for (int j = 0; j < C::COLS; ++j) acc[j] = 0.0f;
+
+      for (int kb = kb_first; kb < p.KB; kb += kb_step, ++it) {
+        const float sbv = sb_next0;
+        sb_next0 = sb_next1;
+        sb_next1 = kb + 2 * kb_step < p.KB ? __ldg(sb_row + kb + 2 * kb_step) : 0.0f;
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1u;
+        const int b = it & 1;
+        const uint32_t tph = (it >> 1) & 1u;
+        if (!mbar_wait(&full[s], ph, ctl)) goto promo_done;
+        if (!mbar_wait(&tfull[b], tph, ctl)) goto promo_done;
+        tc_fence_after();
+        const float* sa_s = reinterpret_cast<const float*>(sSA + s * C::SA_STAGE);
+        const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * C::MMA_N + c0);
+        if (!C::SWAP) {
+          const float scale = sa_s[row] * sbv;
+#pragma unroll
+          for (int ch = 0; ch < C::COLS; ch += 32) {
+            if (C::COLS - ch >= 32) {
+              float v[32];
+              tmem_ld32(taddr + ch, v);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+            } else if (C::COLS - ch >= 16) {
+              float v[16];
+              tmem_ld16(taddr + ch, v);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < C::COLS; ch += 32) {
+            if (C::COLS - ch >= 32) {
+              float v[32];
+              tmem_ld32(taddr + ch, v);
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                acc[ch + j] = fmaf(v[j], sbv * sa_s[c0 + ch + j], acc[ch + j]);
+            } else if (C::COLS - ch >= 16) {
+              float v[16];
+              tmem_ld16(taddr + ch, v);
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                acc[ch + j] = fmaf(v[j], sbv * sa_s[c0 + ch + j], acc[ch + j]);
+            } else {
+              float v[8];
+              tmem_ld8(taddr + ch, v);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                acc[ch + j] = fmaf(v[j], sbv * sa_s[c0 + ch + j], acc[ch + j]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tempty[b]);
+          mbar_arrive(&empty[s]);
+        }
+      }
+
+      // -------------------------------------------------------- epilogue
+      if constexpr (C::SPLIT == 1) {
+        int row_mi = 0;
+        if (FORM == kFormContig && !C::SWAP) {
+          const int m = w.mt * C::BT + row;
+          row_mi = m < p.M ? __ldg(p.m_indices + m) : -1;
+        }
+        store_tile_part<C, FORM, C::COLS>(p, w, row, c0, acc, m_valid, row_mi);
+      } else {
+        const uint32_t red_addr = smem_u32(red);
+        const uint32_t ready_addr = smem_u32(red_ready);
+        const int rank = kb_first;
+        // (1) the receivers must have read the previous tile's slots
+        if (tiles_done > 0 &&
+            !mbar_wait_cluster(red_free, (tiles_done - 1) & 1u, abort_flag, p.status, p.timeout_ns))
+          goto promo_done;
+        // (2) expect this tile's bytes from every sender (including itself)
+        if (threadIdx.x == 64) mbar_arrive_expect_tx(red_ready, C::SLICE_TX);
+        // (3) push this CTA's partial values into their owners' slot `rank`
+        if (C::SWAP) {
+          // lane = weight `row`, columns = tokens c0 .. c0 + COLS
+#pragma unroll
+          for (int j = 0; j < C::COLS; j += 4) {
+            const int m = c0 + j;
+            const uint32_t dst_cta = static_cast<uint32_t>(m / C::SLICE_M);
+            const uint32_t off = static_cast<uint32_t>(
+                (rank * C::SLOT_FLOATS + ((m % C::SLICE_M) / 4 * C::TN + row) * 4) * 4);
+            st_async_f4(mapa_shared(red_addr + off, dst_cta),
+                        make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]),
+                        mapa_shared(ready_addr, dst_cta));
+          }
+        } else {
+          // lane = token `row`, columns = weights c0 .. c0 + COLS
+          const uint32_t dst_cta = static_cast<uint32_t>(row / C::SLICE_M);
+          const uint32_t bar = mapa_shared(ready_addr, dst_cta);
+#pragma unroll
+          for (int j = 0; j < C::COLS; j += 4) {
+            const uint32_t off = static_cast<uint32_t>(
+                (rank * C::SLOT_FLOATS + ((c0 + j) / 4 * C::SLICE_M + row % C::SLICE_M) * 4) * 4);
+            st_async_f4(mapa_shared(red_addr + off, dst_cta),
+                        make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]), bar);
+          }
+        }
+        // (4) wait until every sender's bytes for this CTA's rows have landed
+        if (!mbar_wait_cluster(red_ready, tiles_done & 1u, abort_flag, p.status, p.timeout_ns))
+          goto promo_done;
+        const int tix = threadIdx.x - 64;
+        const bool more = t + t_step < total;  // will peers push into these slots again?
+        if (C::SWAP) {
+          // (5) thread = weight tix: sum its SLICE_M tokens over the slots in
+          //     split order, then store D[token][weight] (32 lanes write 32
+          //     consecutive weights of a token row)
+          float sum[C::SLICE_M];
+#pragma unroll
+          for (int j = 0; j < C::SLICE_M; ++j) sum[j] = 0.0f;
+#pragma unroll
+          for (int r = 0; r < C::SPLIT; ++r) {
+            const float* src = red + r * C::SLOT_FLOATS + tix * 4;
+#pragma unroll
+            for (int j = 0; j < C::SLICE_M; j += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(src + j * C::TN);
+              sum[j] += v.x;
+              sum[j + 1] += v.y;
+              sum[j + 2] += v.z;
+              sum[j + 3] += v.w;
+            }
+          }
+          if (more) {
+            __syncwarp();
+            if (lane == 0)
+              for (int r = 0; r < C::SPLIT; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(red_free), r));
+          }
+          store_tile_part<C, FORM, C::SLICE_M>(p, w, tix, rank * C::SLICE_M, sum, m_valid, 0);
+        } else {
+          // (5) thread: one token row, VPT consecutive weights
+          const int ml = tix / (C::TN / C::VPT);
+          const int n0 = (tix % (C::TN / C::VPT)) * C::VPT;
+          float sum[C::VPT];
+#pragma unroll
+          for (int j = 0; j < C::VPT; ++j) sum[j] = 0.0f;
+#pragma unroll
+          for (int r = 0; r < C::SPLIT; ++r) {
+            const float* src = red + r * C::SLOT_FLOATS + (n0 / 4 * C::SLICE_M + ml) * 4;
+#pragma unroll
+            for (int j = 0; j < C::VPT; j += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(src + j * C::SLICE_M);
+              sum[j] += v.x;
+              sum[j + 1] += v.y;
+              sum[j + 2] += v.z;
+              sum[j + 3] += v.w;
+            }
+          }
+          if (more) {
+            __syncwarp();
+            if (lane == 0)
+              for (int r = 0; r < C::SPLIT; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(red_free), r));
+          }
+          const int srow = rank * C::SLICE_M + ml;
+          int row_mi = 0;
+          if (FORM == kFormContig) {
+            const int m = w.mt * C::BT + srow;
+            row_mi = m < p.M ? __ldg(p.m_indices + m) : -1;
+          }
+          store_tile_part<C, FORM, C::VPT>(p, w, srow, n0, sum, m_valid, row_mi);
+        }
+        ++tiles_done;
+      }
+    }
+  promo_done:;
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // Lane 0 of warps 0 and 1 ran their role alone: reconverge every warp
+  // before the CTA-wide barrier (a barrier reached by part of a warp does not
+  // wait for the rest of the CTA).
+  __syncwarp();
+  tc_fence_before();
+  // No CTA may leave while a peer can still write its shared memory; the
+  // cluster barrier covers every thread of the CTA as well.
+  if constexpr (C::SPLIT > 1) cluster_sync_all(); else __syncthreads();
+  grid_launch_dependents();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fg

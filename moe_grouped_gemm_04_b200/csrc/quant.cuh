@@ -1,0 +1,136 @@
+// FP8 quantizers: per-token (1x128) activation scaling and per-block (128x128)
+// weight scaling. Both are HBM-bound streams: 2 bytes read and 1 byte written
+// per element plus one fp32 scale per group. Loads and stores are 16-byte
+// and 8-byte vectors; the amax reduction is a warp shuffle (per token) or a
+// warp shuffle plus a shared-memory step (per block).
+//
+// Arithmetic (must match the oracle bit for bit):
+//   amax_c = max(amax, 1e-4f); scale = amax_c / 448 (IEEE division);
+//   code = cvt.rn.satfinite.e4m3(x * (448 / amax_c)) with one fp32 multiply.
+// Sources: "DeepGEMM" overview (zixun.chuxinyishu.com/article/345.html),
+// section "FP8与细粒度缩放" (per-slice activation and per-block weight
+// scales); DeepSeek-V3 review (developer.cloud.tencent.cn/article/2686109),
+// "创新之处" item 4 (one scale per 128 elements, 128x128 blocks) and
+// "风险与不足" item 6 (the 448.0 bound).
+#pragma once
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace fg {
+
+constexpr float kFp8Max = 448.0f;
+constexpr float kAmaxFloor = 1e-4f;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 8 bf16 values (one 16-byte word) -> 8 e4m3 codes (one 8-byte word).
+__device__ __forceinline__ uint2 quantize8(uint4 w, float inv) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint16_t p0 = cvt_e4m3x2(__fmul_rn(bf16_lo(in[2 * i]), inv),
+                                   __fmul_rn(bf16_hi(in[2 * i]), inv));
+    const uint16_t p1 = cvt_e4m3x2(__fmul_rn(bf16_lo(in[2 * i + 1]), inv),
+                                   __fmul_rn(bf16_hi(in[2 * i + 1]), inv));
+    out[i] = static_cast<uint32_t>(p0) | (static_cast<uint32_t>(p1) << 16);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+__device__ __forceinline__ float amax8(uint4 w) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, fabsf(bf16_lo(in[i])));
+    m = fmaxf(m, fabsf(bf16_hi(in[i])));
+  }
+  return m;
+}
+
+// One 128-element slice per 16 consecutive threads (8 elements each).
+// Slices are enumerated with the token index fastest so that consecutive
+// slices write consecutive scale entries of the MN-major layout.
+__global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __restrict__ x,
+                                                             uint8_t* __restrict__ q,
+                                                             float* __restrict__ sfa, int G,
+                                                             int M, int K, int stride) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int KB = K / 128;
+  const int64_t slices = static_cast<int64_t>(G) * KB * M;
+  const int sub = threadIdx.x & 15;
+  const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
+  for (int64_t s = first; s < slices; s += step) {
+    const int m = static_cast<int>(s % M);
+    const int64_t gk = s / M;  // g * KB + kb
+    const int kb = static_cast<int>(gk % KB);
+    const int64_t g = gk / KB;
+    const int64_t off = ((g * M + m) * K) + static_cast<int64_t>(kb) * 128 + sub * 8;
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + off));
+    float a = amax8(w);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const float amx = fmaxf(a, kAmaxFloor);
+    const float inv = __fdiv_rn(kFp8Max, amx);
+    *reinterpret_cast<uint2*>(q + off) = quantize8(w, inv);
+    if (sub == 0) sfa[gk * stride + m] = __fdiv_rn(amx, kFp8Max);
+  }
+}
+
+// One CTA (256 threads) per 128x128 block. Thread t covers rows t/16 + 16*i
+// (i = 0..7) and the 8 columns starting at (t%16)*8 of the block.
+__global__ void __launch_bounds__(256) per_block_cast_kernel(const uint16_t* __restrict__ x,
+                                                             uint8_t* __restrict__ q,
+                                                             float* __restrict__ sfb, int G,
+                                                             int N, int K) {
+  __shared__ float warp_max[8];
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int KB = K / 128;
+  const int NB = (N + 127) / 128;
+  const int64_t blk = blockIdx.x;
+  const int kb = static_cast<int>(blk % KB);
+  const int nb = static_cast<int>((blk / KB) % NB);
+  const int64_t g = blk / (static_cast<int64_t>(KB) * NB);
+  const int col = (threadIdx.x & 15) * 8;
+  const int r0 = threadIdx.x >> 4;
+  uint4 w[8];
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = nb * 128 + r0 + 16 * i;
+    if (n < N) {
+      const int64_t off = (g * N + n) * K + static_cast<int64_t>(kb) * 128 + col;
+      w[i] = __ldg(reinterpret_cast<const uint4*>(x + off));
+      a = fmaxf(a, amax8(w[i]));
+    } else {
+      w[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = warp_max[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) a = fmaxf(a, warp_max[i]);
+  const float amx = fmaxf(a, kAmaxFloor);
+  const float inv = __fdiv_rn(kFp8Max, amx);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = nb * 128 + r0 + 16 * i;
+    if (n < N) {
+      const int64_t off = (g * N + n) * K + static_cast<int64_t>(kb) * 128 + col;
+      *reinterpret_cast<uint2*>(q + off) = quantize8(w[i], inv);
+    }
+  }
+  if (threadIdx.x == 0) sfb[blk] = __fdiv_rn(amx, kFp8Max);
+}
+
+}  // namespace fg

@@ -1,0 +1,124 @@
+"""GPU quantizers against the CPU oracle: e4m3 bytes and fp32 scale bits must
+be identical (bit-exact), on seeded inputs with ragged shapes, zero slices,
+tiny values, outliers and N tails, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from helpers import bf16_tensor, sa_from_mn_major
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def fg():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import moe_grouped_gemm_04_b200 as m
+    m.load_library()
+    return m
+
+
+def _special_rows(x: np.ndarray) -> np.ndarray:
+    """Plant the edge cases the quantizer must get right."""
+    x = x.copy()
+    if x.shape[-2] > 4 and x.shape[-1] >= 256:
+        x[..., 1, 128:256] = 0.0            # all-zero slice -> amax floor
+        x[..., 2, :128] *= 1e-7             # amax far below the floor
+        x[..., 3, :] *= 30.0                # outlier row
+        x[..., 4, 5] = 1e-30                # deep underflow element
+    return x
+
+
+def gpu_per_token(fg, bits: np.ndarray):
+    G, M, K = (1, *bits.shape) if bits.ndim == 2 else bits.shape
+    x = bf16_tensor(bits.reshape(G, M, K))
+    q = torch.empty((G, M, K), dtype=torch.uint8, device="cuda")
+    s = torch.full((G, K // 128, fg.sfa_stride(M)), -1.0, dtype=torch.float32, device="cuda")
+    fg.per_token_cast_to_fp8(x, q, s)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+def gpu_per_block(fg, bits: np.ndarray):
+    G, N, K = (1, *bits.shape) if bits.ndim == 2 else bits.shape
+    x = bf16_tensor(bits.reshape(G, N, K))
+    q = torch.empty((G, N, K), dtype=torch.uint8, device="cuda")
+    s = fg.empty_sfb(G, N, K, "cuda")
+    fg.per_block_cast_to_fp8(x, q, s)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+@pytest.mark.parametrize("G,M,K", [(1, 1, 128), (1, 63, 512), (1, 130, 384), (3, 80, 256),
+                                   (1, 64, 7168), (2, 257, 1024)])
+def test_per_token_bit_exact(fg, G, M, K):
+    rng = np.random.default_rng(M * 1000 + K + G)
+    x = _special_rows(rng.standard_normal((G, M, K), dtype=np.float32))
+    bits = workloads.bf16_bits(x)
+    q, s = gpu_per_token(fg, bits)
+    qr, sr = oracle.per_token_cast(bits)
+    assert np.array_equal(q, qr)
+    assert np.array_equal(sa_from_mn_major(s, M).view(np.uint32), sr.view(np.uint32))
+
+
+@pytest.mark.parametrize("G,N,K", [(1, 256, 512), (1, 2112, 768), (2, 130, 256), (1, 64, 128),
+                                   (3, 384, 384)])
+def test_per_block_bit_exact(fg, G, N, K):
+    rng = np.random.default_rng(N * 1000 + K + G)
+    x = _special_rows(rng.standard_normal((G, N, K), dtype=np.float32) * 0.02)
+    bits = workloads.bf16_bits(x)
+    q, s = gpu_per_block(fg, bits)
+    qr, sr = oracle.per_block_cast(bits)
+    assert np.array_equal(q, qr)
+    assert np.array_equal(s.view(np.uint32), sr.view(np.uint32))
+
+
+def test_quantizers_full_size_decode(fg):
+    """decode_64x4096x7168: both operands at full size."""
+    inp = workloads.make("decode_64x4096x7168")
+    q, s = gpu_per_token(fg, inp.a)
+    qr, sr = oracle.per_token_cast(inp.a)
+    assert np.array_equal(q[0], qr)
+    assert np.array_equal(sa_from_mn_major(s, inp.M)[0].view(np.uint32), sr.view(np.uint32))
+    q, s = gpu_per_block(fg, inp.b)
+    qr, sr = oracle.per_block_cast(inp.b)
+    assert np.array_equal(q[0], qr)
+    assert np.array_equal(s[0].view(np.uint32), sr.view(np.uint32))
+
+
+def test_quantizers_full_size_prefill_tail(fg):
+    """prefill_4096x2112x7168: N tail block of 64 rows, K = 7168."""
+    inp = workloads.make("prefill_4096x2112x7168")
+    q, s = gpu_per_block(fg, inp.b)
+    qr, sr = oracle.per_block_cast(inp.b)
+    assert np.array_equal(q[0], qr)
+    assert np.array_equal(s[0].view(np.uint32), sr.view(np.uint32))
+    q, s = gpu_per_token(fg, inp.a)
+    qr, sr = oracle.per_token_cast(inp.a)
+    assert np.array_equal(q[0], qr)
+    assert np.array_equal(sa_from_mn_major(s, inp.M)[0].view(np.uint32), sr.view(np.uint32))
+
+
+def test_per_token_zero_padding_rows(fg):
+    """Contiguous-layout padding rows are zero: codes 0, scale 1e-4/448."""
+    inp = workloads.contiguous(256, 512, counts=np.array([100, 3]), seed=2)
+    q, s = gpu_per_token(fg, inp.a)
+    pad = inp.m_indices < 0
+    assert np.all(q[0][pad] == 0)
+    sa = sa_from_mn_major(s, inp.M_total)[0]
+    assert np.all(sa[pad] == np.float32(1e-4) / np.float32(448.0))
+    qr, sr = oracle.per_token_cast(inp.a)
+    assert np.array_equal(q[0], qr) and np.array_equal(sa.view(np.uint32), sr.view(np.uint32))
+
+
+def test_quantizer_argument_errors(fg):
+    x = torch.zeros((4, 100), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((4, 100), dtype=torch.uint8, device="cuda")
+    s = torch.zeros(64, dtype=torch.float32, device="cuda")
+    with pytest.raises(fg.FP8GemmError) as ei:
+        fg.per_token_cast_to_fp8(x, q, s)
+    assert ei.value.status == fg.FG_ERR_INVALID_ARG

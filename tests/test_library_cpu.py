@@ -1,0 +1,86 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/fp8gemm.h declares, and rejects bad arguments synchronously (before
+any CUDA call), so these run on a CPU-only machine."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8gemm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from moe_grouped_gemm_04_b200 import build as b
+    b.build()
+    import moe_grouped_gemm_04_b200 as m
+    return m.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "fp8_gemm_nt",
+              "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
+              "fg_get_device_status", "fg_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_binding_names_match_header():
+    import moe_grouped_gemm_04_b200 as m
+    assert set(m.EXPORTED) == set(declared_functions())
+
+
+def test_sfa_stride_and_status_strings(lib):
+    assert [lib.fg_sfa_stride(m) for m in (1, 4, 5, 64, 65, 14208)] == [4, 4, 8, 64, 68, 14208]
+    assert lib.fg_status_string(1) == b"FG_ERR_INVALID_ARG"
+    assert lib.fg_status_string(0) == b"FG_OK"
+
+
+FAKE = 0x10000   # never dereferenced: validation fails before any CUDA call
+MISALIGNED = 0x10008
+
+
+def test_validation_rejects_without_touching_the_device(lib):
+    P = ctypes.c_void_p
+    ok = P(FAKE)
+    # K not a multiple of 128
+    assert lib.fp8_gemm_nt(ok, ok, ok, ok, ok, 64, 256, 100, None) == 1
+    # N not a multiple of 16
+    assert lib.fp8_gemm_nt(ok, ok, ok, ok, ok, 64, 250, 256, None) == 1
+    # null and misaligned pointers
+    assert lib.fp8_gemm_nt(None, ok, ok, ok, ok, 64, 256, 256, None) == 1
+    assert lib.fp8_gemm_nt(ok, ok, P(MISALIGNED), ok, ok, 64, 256, 256, None) == 1
+    assert b"aligned" in lib.fg_last_error()
+    # contiguous: M_total must be a multiple of 128
+    assert lib.fp8_grouped_gemm_contiguous(ok, ok, ok, ok, ok, ok, 100, 256, 256, 2, None) == 1
+    assert lib.fp8_grouped_gemm_contiguous(ok, ok, ok, ok, ok, ok, 128, 256, 256, 0, None) == 1
+    # masked: G and M_max positive
+    assert lib.fp8_grouped_gemm_masked(ok, ok, ok, ok, ok, ok, 0, 64, 256, 256, 64, None) == 1
+    assert lib.fp8_grouped_gemm_masked(ok, ok, ok, ok, ok, ok, 2, 0, 256, 256, 64, None) == 1
+    assert lib.fp8_grouped_gemm_masked(ok, ok, ok, ok, ok, None, 2, 64, 256, 256, 64, None) == 1
+    # quantizers
+    assert lib.per_token_cast_to_fp8(ok, ok, ok, 1, 64, 100, None) == 1
+    assert lib.per_token_cast_to_fp8(ok, ok, ok, 0, 64, 128, None) == 1
+    assert lib.per_block_cast_to_fp8(ok, ok, ok, 1, 0, 128, None) == 1
+    assert lib.per_block_cast_to_fp8(ok, P(MISALIGNED), ok, 1, 64, 128, None) == 1
+    assert lib.fg_selftest_wait_timeout(0, None) == 1
+    # empty problems are a no-op success
+    assert lib.fp8_gemm_nt(ok, ok, ok, ok, ok, 0, 256, 256, None) == 0
+    assert lib.per_token_cast_to_fp8(ok, ok, ok, 1, 0, 128, None) == 0
+    assert lib.fp8_grouped_gemm_contiguous(ok, ok, ok, ok, ok, ok, 0, 256, 256, 2, None) == 0

@@ -53,11 +53,24 @@ def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
 
 
 def normal_bf16(rng: np.random.Generator, shape, std: float = 1.0) -> np.ndarray:
-    """bf16 bits of N(0, std^2) samples drawn in float32."""
-    x = rng.standard_normal(size=shape, dtype=np.float32)
-    if std != 1.0:
-        x *= np.float32(std)
-    return bf16_bits(x)
+    """bf16 bits of N(0, std^2) samples drawn in float32.
+
+    Large tensors are drawn in slices along the first axis; the generator's
+    stream is the same as one draw of the whole shape.
+    """
+    shape = tuple(shape)
+    out = np.empty(shape, dtype=np.uint16)
+    rows = shape[0] if shape else 1
+    per_row = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+    chunk = max(1, (1 << 26) // max(per_row, 1))
+    flat = out.reshape(rows, per_row)
+    for r0 in range(0, rows, chunk):
+        r1 = min(rows, r0 + chunk)
+        x = rng.standard_normal(size=(r1 - r0, per_row), dtype=np.float32)
+        if std != 1.0:
+            x *= np.float32(std)
+        flat[r0:r1] = bf16_bits(x)
+    return out
 
 
 def zipf_top8_counts(seed: int, tokens: int = 4096, experts: int = 256,
