@@ -146,17 +146,17 @@ int sfa_stride(int M) { return (M + 3) / 4 * 4; }
 
 // ---------------------------------------------------------------- GEMM configs
 
-//                      BT   BW   swap  stages PW split
-using CfgNormal = GemmCfg<128, 128, false, 6, 8, 1>;
-using CfgSwap16 = GemmCfg<16, 128, true, 8, 4, 1>;
-using CfgSwap32 = GemmCfg<32, 128, true, 8, 4, 1>;
-using CfgSwap64 = GemmCfg<64, 128, true, 8, 4, 1>;
-using CfgSwap16S2 = GemmCfg<16, 128, true, 8, 4, 2>;
-using CfgSwap32S2 = GemmCfg<32, 128, true, 8, 4, 2>;
-using CfgSwap64S2 = GemmCfg<64, 128, true, 7, 4, 2>;
-using CfgSwap16S4 = GemmCfg<16, 128, true, 8, 4, 4>;
-using CfgSwap32S4 = GemmCfg<32, 128, true, 8, 4, 4>;
-using CfgSwap64S4 = GemmCfg<64, 128, true, 7, 4, 4>;
+//                      BT   BW   swap  stages PW split (2 K blocks per stage)
+using CfgNormal = GemmCfg<128, 128, false, 3, 8, 1>;
+using CfgSwap16 = GemmCfg<16, 128, true, 5, 4, 1>;
+using CfgSwap32 = GemmCfg<32, 128, true, 5, 4, 1>;
+using CfgSwap64 = GemmCfg<64, 128, true, 4, 4, 1>;
+using CfgSwap16S2 = GemmCfg<16, 128, true, 5, 4, 2>;
+using CfgSwap32S2 = GemmCfg<32, 128, true, 4, 4, 2>;
+using CfgSwap64S2 = GemmCfg<64, 128, true, 3, 4, 2>;
+using CfgSwap16S4 = GemmCfg<16, 128, true, 5, 4, 4>;
+using CfgSwap32S4 = GemmCfg<32, 128, true, 4, 4, 4>;
+using CfgSwap64S4 = GemmCfg<64, 128, true, 3, 4, 4>;
 
 struct KernelInfo {
   bool attr_set = false;
@@ -232,7 +232,7 @@ Plan plan_for(const Problem& pr, int sm_count, int expected_m) {
   else pl.bt = 128;
   if (pr.form == kFormMasked && pl.bt < 64) pl.bt = 64;  // one swapped shape for masked
   pl.num_mt = (pr.M + pl.bt - 1) / pl.bt;
-  pl.num_nt = (pr.N + 127) / 128;
+  pl.num_nt = (pr.N + CfgNormal::BW - 1) / (pl.bt == 128 ? CfgNormal::BW : 128);
   pl.splits = 1;
   if (pr.form == kFormDense && pl.bt < 128) {
     const int tiles = pl.num_mt * pl.num_nt;

@@ -13,9 +13,11 @@
 // section "swapAB与Mega MoE".
 //
 // CTA roles (one CTA per SM, persistent over output tiles):
-//   warp 0      TMA producer: per K block loads the token tile, the weight
-//               tile and the token scales, all completing on the stage's
-//               "full" barrier.
+//   warp 0      TMA producer: per K block, lane 0 loads the weight tile, lane 1
+//               the token tile and lane 2 the token scales, each onto the
+//               stage's "full" barrier. (A thread's tensor copies complete one
+//               after another at a roughly fixed time per copy, so one thread
+//               per stream keeps three copies in flight per stage.)
 //   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one
 //               of two TMEM partial buffers, then commits to the stage's
 //               "empty" barrier and the buffer's "tmem full" barrier.
@@ -73,7 +75,7 @@ struct GemmParams {
   uint64_t timeout_ns;
 };
 
-template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_>
+template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_, int KPS_ = 2>
 struct GemmCfg {
   static constexpr int BT = BT_;          // token rows per tile
   static constexpr int BW = BW_;          // weight rows per tile
@@ -81,6 +83,7 @@ struct GemmCfg {
   static constexpr int STAGES = STAGES_;
   static constexpr int PW = PW_;          // promotion warps
   static constexpr int SPLIT = SPLIT_;    // CTAs per cluster sharing one tile's K blocks
+  static constexpr int KPS = KPS_;        // K blocks per pipeline stage
   static constexpr int MMA_N = SWAP ? BT : BW;
   static_assert(SWAP ? (BW == 128) : (BT == 128), "the lane operand has 128 rows");
   static_assert(MMA_N % 16 == 0 && MMA_N >= 16 && MMA_N <= 256, "tcgen05 N for M = 128");
@@ -93,12 +96,16 @@ struct GemmCfg {
   static constexpr int B_BYTES = BW * 128;
   static constexpr int SA_BYTES = BT * 4;                       // one TMA box of token scales
   static constexpr int SA_STAGE = (SA_BYTES + 127) / 128 * 128;  // TMA smem destinations: 128-B aligned
-  static constexpr uint32_t TX_BYTES = A_BYTES + B_BYTES + SA_BYTES;
-  static constexpr int TMEM_USED = 2 * MMA_N;
+  static constexpr int STAGE_A = KPS * A_BYTES;
+  static constexpr int STAGE_B = KPS * B_BYTES;
+  static constexpr int STAGE_SA = KPS * SA_STAGE;
+  static constexpr int TMEM_USED = 2 * KPS * MMA_N;  // two stages of KPS partial tiles
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
                                    : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "TMEM has 512 columns");
   static constexpr int NUM_THREADS = (2 + PW) * 32;
+  // the whole register file for the one CTA of an SM (allocation in steps of 8)
+  static constexpr int MAX_REGS = (65536 / NUM_THREADS) / 8 * 8 > 255 ? 255 : (65536 / NUM_THREADS) / 8 * 8;
   // split-K receive slots: SPLIT slots (one per sender) of SLICE_M token rows
   // x TN weights in fp32, stored as groups of 4 consecutive values along the
   // dimension a promotion thread holds, with the lane dimension next, so that
@@ -119,9 +126,9 @@ struct GemmCfg {
   static_assert(SPLIT == 1 || SWAP || SLICE_M % 32 == 0, "a warp's tokens share one owner");
   static_assert(SPLIT == 1 || SWAP || (VPT % 8 == 0 && TN % VPT == 0), "16-byte D stores");
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_SA = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_RED = OFF_SA + STAGES * SA_STAGE;
+  static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
+  static constexpr int OFF_SA = OFF_B + STAGES * STAGE_B;
+  static constexpr int OFF_RED = OFF_SA + STAGES * STAGE_SA;
   static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 4 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -268,23 +275,38 @@ __device__ __forceinline__ void store_tile_part(const GemmParams& p, const Tile&
   }
 }
 
+// One producer lane's share of a stage: stream 0 = weight tiles, 1 = token
+// tiles, 2 = token scales, for the stage's K blocks kq + j * kb_step
+// (j < KPS, those below KB).
 template <class C, int FORM>
-__device__ __forceinline__ void issue_stage(const GemmParams& p, const Tile& w, int kb, uint32_t it,
-                                            uint8_t* sA, uint8_t* sB, uint8_t* sSA, uint64_t* full,
-                                            const CUtensorMap* tmA, const CUtensorMap* tmB,
-                                            const CUtensorMap* tmSA) {
+__device__ __forceinline__ void issue_stage(int stream, const GemmParams& p, const Tile& w, int kq,
+                                            int kb_step, uint32_t it, uint8_t* sA, uint8_t* sB,
+                                            uint8_t* sSA, uint64_t* full, const CUtensorMap* tmA,
+                                            const CUtensorMap* tmB, const CUtensorMap* tmSA) {
   const int s = it % C::STAGES;
-  const int a_row = (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
-  const int b_row = w.e * p.N + w.nt * C::BW;
-  const int sa_y = (FORM == kFormMasked ? w.e * p.KB : 0) + kb;
-  mbar_arrive_expect_tx(&full[s], C::TX_BYTES);
-  tma_load_2d(sB + s * C::B_BYTES, tmB, &full[s], kb * 128, b_row);
-  tma_load_2d(sA + s * C::A_BYTES, tmA, &full[s], kb * 128, a_row);
-  tma_load_2d(sSA + s * C::SA_STAGE, tmSA, &full[s], w.mt * C::BT, sa_y);
+  int nvalid = 0;
+#pragma unroll
+  for (int j = 0; j < C::KPS; ++j) nvalid += kq + j * kb_step < p.KB ? 1 : 0;
+  if (stream == 0) {
+    mbar_arrive_expect_tx(&full[s], nvalid * C::B_BYTES);
+    for (int j = 0; j < nvalid; ++j)
+      tma_load_2d(sB + s * C::STAGE_B + j * C::B_BYTES, tmB, &full[s], (kq + j * kb_step) * 128,
+                  w.e * p.N + w.nt * C::BW);
+  } else if (stream == 1) {
+    mbar_arrive_expect_tx(&full[s], nvalid * C::A_BYTES);
+    for (int j = 0; j < nvalid; ++j)
+      tma_load_2d(sA + s * C::STAGE_A + j * C::A_BYTES, tmA, &full[s], (kq + j * kb_step) * 128,
+                  (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT);
+  } else {
+    mbar_arrive_expect_tx(&full[s], nvalid * C::SA_BYTES);
+    for (int j = 0; j < nvalid; ++j)
+      tma_load_2d(sSA + s * C::STAGE_SA + j * C::SA_STAGE, tmSA, &full[s], w.mt * C::BT,
+                  (FORM == kFormMasked ? w.e * p.KB : 0) + kq + j * kb_step);
+  }
 }
 
 template <class C, int FORM>
-__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+__global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -314,7 +336,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);               // producer's expect_tx (+ TMA bytes)
+      mbar_init(&full[s], 3);               // one expect_tx per producer lane (+ TMA bytes)
       mbar_init(&empty[s], 1 + C::PW);      // MMA commit + one arrival per promotion warp
     }
     for (int b = 0; b < 2; ++b) {
@@ -339,11 +361,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   if (warp == 0) {
     build_table<C, FORM>(p, table, lane);
     __syncwarp();
-    if (lane == 0 && t_first < total_tiles<FORM>(p, table)) {
+    if (lane < 3 && t_first < total_tiles<FORM>(p, table)) {
       const Tile w = resolve_tile<FORM>(p, table, t_first);
       if (w.valid) {
-        for (int kb = kb_first; kb < p.KB && pre_issued < C::STAGES; kb += kb_step, ++pre_issued)
-          issue_stage<C, FORM>(p, w, kb, pre_issued, sA, sB, sSA, full, &tmA, &tmB, &tmSA);
+        for (int kq = kb_first; kq < p.KB && pre_issued < C::STAGES;
+             kq += C::KPS * kb_step, ++pre_issued)
+          issue_stage<C, FORM>(lane, p, w, kq, kb_step, pre_issued, sA, sB, sSA, full, &tmA, &tmB,
+                               &tmSA);
       }
     }
   }
@@ -359,17 +383,17 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane < 3) {
       uint32_t it = 0;
       for (int t = t_first; t < total; t += t_step) {
         const Tile w = resolve_tile<FORM>(p, table, t);
         if (!w.valid) continue;
-        for (int kb = kb_first; kb < p.KB; kb += kb_step, ++it) {
+        for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
           if (it < pre_issued) continue;
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) goto producer_done;
-          issue_stage<C, FORM>(p, w, kb, it, sA, sB, sSA, full, &tmA, &tmB, &tmSA);
+          issue_stage<C, FORM>(lane, p, w, kq, kb_step, it, sA, sB, sSA, full, &tmA, &tmB, &tmSA);
         }
       }
     producer_done:
@@ -390,7 +414,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       for (int t = t_first; t < total; t += t_step) {
         const Tile w = resolve_tile<FORM>(p, table, t);
         if (!w.valid) continue;
-        for (int kb = kb_first; kb < p.KB; kb += kb_step, ++it) {
+        for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
           const int b = it & 1;
@@ -399,15 +423,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           tc_fence_after();
           if (!mbar_wait(&full[s], ph, ctl)) goto mma_done;
           tc_fence_after();
-          const uint8_t* lane_tile = C::SWAP ? sB + s * C::B_BYTES : sA + s * C::A_BYTES;
-          const uint8_t* col_tile = C::SWAP ? sA + s * C::A_BYTES : sB + s * C::B_BYTES;
-          const uint64_t adesc = smem_desc_sw128(smem_u32(lane_tile));
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(col_tile));
-          const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::MMA_N);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            // advance 32 bytes (= 32 e4m3 along K) inside the 128-byte swizzled row
-            mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+          for (int j = 0; j < C::KPS; ++j) {
+            if (kq + j * kb_step >= p.KB) break;
+            const uint8_t* a_tile = sA + s * C::STAGE_A + j * C::A_BYTES;
+            const uint8_t* b_tile = sB + s * C::STAGE_B + j * C::B_BYTES;
+            const uint64_t adesc = smem_desc_sw128(smem_u32(C::SWAP ? b_tile : a_tile));
+            const uint64_t bdesc = smem_desc_sw128(smem_u32(C::SWAP ? a_tile : b_tile));
+            // one fresh partial per K block: slot (b, j) of tensor memory
+            const uint32_t d = tmem_base + static_cast<uint32_t>((b * C::KPS + j) * C::MMA_N);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              // advance 32 bytes (= 32 e4m3 along K) inside the 128-byte swizzled row
+              mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            }
           }
           mma_commit(&empty[s]);
           mma_commit(&tfull[b]);
@@ -435,19 +464,28 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         m_valid = __ldg(p.masked_m + w.e);
         m_valid = m_valid < 0 ? 0 : (m_valid > p.M ? p.M : m_valid);
       }
-      // weight scale of this thread's 128 weight rows, two K blocks ahead
+      // weight scale of this thread's 128 weight rows: one per K block, read
+      // from global memory one stage ahead
       const int nb = w.nt * (C::BW / 128) + (C::SWAP ? 0 : c0 / 128);
       const float* sb_row = p.sfb + (static_cast<int64_t>(w.e) * p.NB + min(nb, p.NB - 1)) * p.KB;
-      float sb_next0 = kb_first < p.KB ? __ldg(sb_row + kb_first) : 0.0f;
-      float sb_next1 = kb_first + kb_step < p.KB ? __ldg(sb_row + kb_first + kb_step) : 0.0f;
+      float sb_next[C::KPS];
+#pragma unroll
+      for (int j = 0; j < C::KPS; ++j) {
+        const int kb = kb_first + j * kb_step;
+        sb_next[j] = kb < p.KB ? __ldg(sb_row + kb) : 0.0f;
+      }
       float acc[C::COLS];
 #pragma unroll
       for (int j = 0; j < C::COLS; ++j) acc[j] = 0.0f;
 
-      for (int kb = kb_first; kb < p.KB; kb += kb_step, ++it) {
-        const float sbv = sb_next0;
-        sb_next0 = sb_next1;
-        sb_next1 = kb + 2 * kb_step < p.KB ? __ldg(sb_row + kb + 2 * kb_step) : 0.0f;
+      for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
+        float sbv[C::KPS];
+#pragma unroll
+        for (int j = 0; j < C::KPS; ++j) {
+          sbv[j] = sb_next[j];
+          const int kb = kq + (C::KPS + j) * kb_step;
+          sb_next[j] = kb < p.KB ? __ldg(sb_row + kb) : 0.0f;
+        }
         const int s = it % C::STAGES;
         const uint32_t ph = (it / C::STAGES) & 1u;
         const int b = it & 1;
@@ -455,45 +493,62 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (!mbar_wait(&full[s], ph, ctl)) goto promo_done;
         if (!mbar_wait(&tfull[b], tph, ctl)) goto promo_done;
         tc_fence_after();
-        const float* sa_s = reinterpret_cast<const float*>(sSA + s * C::SA_STAGE);
-        const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * C::MMA_N + c0);
-        if (!C::SWAP) {
-          const float scale = sa_s[row] * sbv;
 #pragma unroll
-          for (int ch = 0; ch < C::COLS; ch += 32) {
-            if (C::COLS - ch >= 32) {
-              float v[32];
-              tmem_ld32(taddr + ch, v);
+        for (int jk = 0; jk < C::KPS; ++jk) {
+          if (kq + jk * kb_step >= p.KB) break;
+          const float* sa_s = reinterpret_cast<const float*>(sSA + s * C::STAGE_SA + jk * C::SA_STAGE);
+          const uint32_t taddr = tmem_base + t_lane +
+                                 static_cast<uint32_t>((b * C::KPS + jk) * C::MMA_N + c0);
+          if (!C::SWAP) {
+            const float scale = sa_s[row] * sbv[jk];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
-            } else if (C::COLS - ch >= 16) {
-              float v[16];
-              tmem_ld16(taddr + ch, v);
+            for (int ch = 0; ch < C::COLS; ch += (C::COLS - ch >= 64 ? 64 : 32)) {
+              if (C::COLS - ch >= 64) {
+                float v[64];
+                tmem_ld64(taddr + ch, v);
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+                for (int j = 0; j < 64; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+              } else if (C::COLS - ch >= 32) {
+                float v[32];
+                tmem_ld32(taddr + ch, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+              } else if (C::COLS - ch >= 16) {
+                float v[16];
+                tmem_ld16(taddr + ch, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+              }
             }
-          }
-        } else {
+          } else {
+            const float sbs = sbv[jk];
 #pragma unroll
-          for (int ch = 0; ch < C::COLS; ch += 32) {
-            if (C::COLS - ch >= 32) {
-              float v[32];
-              tmem_ld32(taddr + ch, v);
+            for (int ch = 0; ch < C::COLS; ch += (C::COLS - ch >= 64 ? 64 : 32)) {
+              if (C::COLS - ch >= 64) {
+                float v[64];
+                tmem_ld64(taddr + ch, v);
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                acc[ch + j] = fmaf(v[j], sbv * sa_s[c0 + ch + j], acc[ch + j]);
-            } else if (C::COLS - ch >= 16) {
-              float v[16];
-              tmem_ld16(taddr + ch, v);
+                for (int j = 0; j < 64; ++j)
+                  acc[ch + j] = fmaf(v[j], sbs * sa_s[c0 + ch + j], acc[ch + j]);
+              } else if (C::COLS - ch >= 32) {
+                float v[32];
+                tmem_ld32(taddr + ch, v);
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                acc[ch + j] = fmaf(v[j], sbv * sa_s[c0 + ch + j], acc[ch + j]);
-            } else {
-              float v[8];
-              tmem_ld8(taddr + ch, v);
+                for (int j = 0; j < 32; ++j)
+                  acc[ch + j] = fmaf(v[j], sbs * sa_s[c0 + ch + j], acc[ch + j]);
+              } else if (C::COLS - ch >= 16) {
+                float v[16];
+                tmem_ld16(taddr + ch, v);
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                acc[ch + j] = fmaf(v[j], sbv * sa_s[c0 + ch + j], acc[ch + j]);
+                for (int j = 0; j < 16; ++j)
+                  acc[ch + j] = fmaf(v[j], sbs * sa_s[c0 + ch + j], acc[ch + j]);
+              } else {
+                float v[8];
+                tmem_ld8(taddr + ch, v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  acc[ch + j] = fmaf(v[j], sbs * sa_s[c0 + ch + j], acc[ch + j]);
+              }
             }
           }
         }
