@@ -147,7 +147,7 @@ int sfa_stride(int M) { return (M + 3) / 4 * 4; }
 // ---------------------------------------------------------------- GEMM configs
 
 //                      BT   BW   swap  stages PW split (2 K blocks per stage)
-using CfgNormal = GemmCfg<128, 128, false, 3, 8, 1>;
+using CfgNormal = GemmCfg<128, 256, false, 4, 8, 1, 1>;
 using CfgSwap16 = GemmCfg<16, 128, true, 5, 4, 1>;
 using CfgSwap32 = GemmCfg<32, 128, true, 5, 4, 1>;
 using CfgSwap64 = GemmCfg<64, 128, true, 4, 4, 1>;
@@ -172,6 +172,16 @@ fg_status kernel_info(int dev, KernelInfo** out) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if (C::REG_SPLIT) {
+      // the warpgroup register split draws on the launch allocation: it must
+      // be exactly what the split was sized for, or the increase would wait
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, fp8_gemm_kernel<C, FORM>);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      if (fa.numRegs != C::MAX_REGS)
+        return fail(FG_ERR_UNSUPPORTED, "kernel built with %d registers per thread, register split needs %d",
+                    fa.numRegs, C::MAX_REGS);
+    }
     if (C::SPLIT > 1) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];

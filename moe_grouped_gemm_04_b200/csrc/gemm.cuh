@@ -21,7 +21,9 @@
 //   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one
 //               of two TMEM partial buffers, then commits to the stage's
 //               "empty" barrier and the buffer's "tmem full" barrier.
-//   warps 2..   promotion + epilogue: per K block read the partial from TMEM
+//   promotion warps (2..5, or 4..11 in the 8-warp form whose warps 2-3 idle
+//   so that warpgroup 0 holds the single-lane roles and can give registers
+//   to the promotion warpgroups): per K block read the partial from TMEM
 //               (tcgen05.ld), add partial * (sa * sb) into fp32 registers
 //               (sb, one value per 128 weight rows and K block, is read from
 //               global memory two K blocks ahead), release the TMEM buffer and
@@ -103,9 +105,19 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
                                    : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "TMEM has 512 columns");
-  static constexpr int NUM_THREADS = (2 + PW) * 32;
+  static constexpr int PW_BASE = PW == 8 ? 4 : 2;  // first promotion warp
+  static constexpr int NUM_THREADS = (PW_BASE + PW) * 32;
   // the whole register file for the one CTA of an SM (allocation in steps of 8)
   static constexpr int MAX_REGS = (65536 / NUM_THREADS) / 8 * 8 > 255 ? 255 : (65536 / NUM_THREADS) / 8 * 8;
+  // 8 promotion warps: warpgroup 0 (producer, MMA, two idle warps) drops to
+  // REG_LOW registers and the two promotion warpgroups rise to REG_HIGH; the
+  // shares add up to the launch allocation of MAX_REGS per thread.
+  static constexpr bool REG_SPLIT = PW == 8;
+  static constexpr int REG_LOW = 40;
+  static constexpr int REG_HIGH = 232;
+  static_assert(!REG_SPLIT || 128 * REG_LOW + PW * 32 * REG_HIGH <= NUM_THREADS * MAX_REGS,
+                "register split exceeds the launch allocation");
+  static constexpr int SAS = 2 * STAGES;  // token-scale ring (read by the promotion warps)
   // split-K receive slots: SPLIT slots (one per sender) of SLICE_M token rows
   // x TN weights in fp32, stored as groups of 4 consecutive values along the
   // dimension a promotion thread holds, with the lane dimension next, so that
@@ -128,9 +140,9 @@ struct GemmCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
   static constexpr int OFF_SA = OFF_B + STAGES * STAGE_B;
-  static constexpr int OFF_RED = OFF_SA + STAGES * STAGE_SA;
+  static constexpr int OFF_RED = OFF_SA + SAS * STAGE_SA;
   static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * SAS + 4 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;  // + alignment slack
@@ -281,9 +293,11 @@ __device__ __forceinline__ void store_tile_part(const GemmParams& p, const Tile&
 template <class C, int FORM>
 __device__ __forceinline__ void issue_stage(int stream, const GemmParams& p, const Tile& w, int kq,
                                             int kb_step, uint32_t it, uint8_t* sA, uint8_t* sB,
-                                            uint8_t* sSA, uint64_t* full, const CUtensorMap* tmA,
-                                            const CUtensorMap* tmB, const CUtensorMap* tmSA) {
+                                            uint8_t* sSA, uint64_t* full, uint64_t* sa_full,
+                                            const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                            const CUtensorMap* tmSA) {
   const int s = it % C::STAGES;
+  const int q = it % C::SAS;
   int nvalid = 0;
 #pragma unroll
   for (int j = 0; j < C::KPS; ++j) nvalid += kq + j * kb_step < p.KB ? 1 : 0;
@@ -298,15 +312,15 @@ __device__ __forceinline__ void issue_stage(int stream, const GemmParams& p, con
       tma_load_2d(sA + s * C::STAGE_A + j * C::A_BYTES, tmA, &full[s], (kq + j * kb_step) * 128,
                   (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT);
   } else {
-    mbar_arrive_expect_tx(&full[s], nvalid * C::SA_BYTES);
+    mbar_arrive_expect_tx(&sa_full[q], nvalid * C::SA_BYTES);
     for (int j = 0; j < nvalid; ++j)
-      tma_load_2d(sSA + s * C::STAGE_SA + j * C::SA_STAGE, tmSA, &full[s], w.mt * C::BT,
+      tma_load_2d(sSA + q * C::STAGE_SA + j * C::SA_STAGE, tmSA, &sa_full[q], w.mt * C::BT,
                   (FORM == kFormMasked ? w.e * p.KB : 0) + kq + j * kb_step);
   }
 }
 
 template <class C, int FORM>
-__global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -317,7 +331,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* sa_full = empty + C::STAGES;   // token scales of a stage have landed
+  uint64_t* sa_empty = sa_full + C::SAS;   // ... and have been read by the promotion warps
+  uint64_t* tfull = sa_empty + C::SAS;
   uint64_t* tempty = tfull + 2;
   uint64_t* red_ready = tempty + 2;    // all partials of the current tile are in place
   uint64_t* red_free = red_ready + 1;  // every CTA has finished reading them
@@ -336,8 +352,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 3);               // one expect_tx per producer lane (+ TMA bytes)
-      mbar_init(&empty[s], 1 + C::PW);      // MMA commit + one arrival per promotion warp
+      mbar_init(&full[s], 2);               // weight- and token-tile lanes' expect_tx
+      mbar_init(&empty[s], 1);              // the MMA commit
+    }
+    for (int q = 0; q < C::SAS; ++q) {
+      mbar_init(&sa_full[q], 1);            // the scale lane's expect_tx
+      mbar_init(&sa_empty[q], C::PW);       // one arrival per promotion warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -366,8 +386,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
       if (w.valid) {
         for (int kq = kb_first; kq < p.KB && pre_issued < C::STAGES;
              kq += C::KPS * kb_step, ++pre_issued)
-          issue_stage<C, FORM>(lane, p, w, kq, kb_step, pre_issued, sA, sB, sSA, full, &tmA, &tmB,
-                               &tmSA);
+          issue_stage<C, FORM>(lane, p, w, kq, kb_step, pre_issued, sA, sB, sSA, full, sa_full,
+                               &tmA, &tmB, &tmSA);
       }
     }
   }
@@ -381,6 +401,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   const int total = total_tiles<FORM>(p, table);
 
+  if (warp < C::PW_BASE) {
+  if constexpr (C::REG_SPLIT) warpgroup_reg_dealloc<C::REG_LOW>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane < 3) {
@@ -390,20 +412,33 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
         if (!w.valid) continue;
         for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
           if (it < pre_issued) continue;
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) goto producer_done;
-          issue_stage<C, FORM>(lane, p, w, kq, kb_step, it, sA, sB, sSA, full, &tmA, &tmB, &tmSA);
+          if (lane < 2) {
+            const int s = it % C::STAGES;
+            if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1u) ^ 1u, ctl)) goto producer_done;
+          } else {
+            const int q = it % C::SAS;
+            if (!mbar_wait(&sa_empty[q], ((it / C::SAS) & 1u) ^ 1u, ctl)) goto producer_done;
+          }
+          issue_stage<C, FORM>(lane, p, w, kq, kb_step, it, sA, sB, sSA, full, sa_full, &tmA, &tmB,
+                               &tmSA);
         }
       }
     producer_done:
       // Before the CTA exits, the last fill of every stage must have landed
       // and been released (its TMA bytes and the MMA commit's arrival).
       it = it > pre_issued ? it : pre_issued;
-      for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
-        const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
-        drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
-        drain_wait(&empty[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+      if (lane == 0) {
+        for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
+          const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
+          drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+          drain_wait(&empty[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+        }
+      } else if (lane == 2) {
+        for (uint32_t q = 0; q < C::SAS && q < it; ++q) {
+          const uint32_t last = (it - 1 - q) / C::SAS * C::SAS + q;
+          drain_wait(&sa_full[q], (last / C::SAS) & 1u, kDrainLimitNs);
+          drain_wait(&sa_empty[q], (last / C::SAS) & 1u, kDrainLimitNs);
+        }
       }
     }
   } else if (warp == 1) {
@@ -445,9 +480,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
     mma_done:
       if (it > 0) drain_wait(&tfull[(it - 1) & 1], ((it - 1) >> 1) & 1u, kDrainLimitNs);
     }
+  }  // warps 2 .. PW_BASE - 1 (8-warp form) idle
   } else {
     // ------------------------------------------------------------ promotion + epilogue
-    const int pw = warp - 2;
+    if constexpr (C::REG_SPLIT) warpgroup_reg_alloc<C::REG_HIGH>();
+    const int pw = warp - C::PW_BASE;
     const int quad = warp & 3;          // TMEM lanes this warp may access
     const int part = pw >> 2;           // column slice of the accumulator
     const int row = quad * 32 + lane;   // TMEM lane = row of the lane operand
@@ -486,24 +523,23 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
           const int kb = kq + (C::KPS + j) * kb_step;
           sb_next[j] = kb < p.KB ? __ldg(sb_row + kb) : 0.0f;
         }
-        const int s = it % C::STAGES;
-        const uint32_t ph = (it / C::STAGES) & 1u;
+        const int q = it % C::SAS;
         const int b = it & 1;
         const uint32_t tph = (it >> 1) & 1u;
-        if (!mbar_wait(&full[s], ph, ctl)) goto promo_done;
+        if (!mbar_wait(&sa_full[q], (it / C::SAS) & 1u, ctl)) goto promo_done;
         if (!mbar_wait(&tfull[b], tph, ctl)) goto promo_done;
         tc_fence_after();
 #pragma unroll
         for (int jk = 0; jk < C::KPS; ++jk) {
           if (kq + jk * kb_step >= p.KB) break;
-          const float* sa_s = reinterpret_cast<const float*>(sSA + s * C::STAGE_SA + jk * C::SA_STAGE);
+          const float* sa_s = reinterpret_cast<const float*>(sSA + q * C::STAGE_SA + jk * C::SA_STAGE);
           const uint32_t taddr = tmem_base + t_lane +
                                  static_cast<uint32_t>((b * C::KPS + jk) * C::MMA_N + c0);
           if (!C::SWAP) {
             const float scale = sa_s[row] * sbv[jk];
 #pragma unroll
-            for (int ch = 0; ch < C::COLS; ch += (C::COLS - ch >= 64 ? 64 : 32)) {
-              if (C::COLS - ch >= 64) {
+            for (int ch = 0; ch < C::COLS; ch += (C::COLS - ch >= 64 && C::COLS <= 64 ? 64 : 32)) {
+              if (C::COLS - ch >= 64 && C::COLS <= 64) {
                 float v[64];
                 tmem_ld64(taddr + ch, v);
 #pragma unroll
@@ -513,6 +549,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
                 tmem_ld32(taddr + ch, v);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc[ch + j] = fmaf(v[j], scale, acc[ch + j]);
+                if (C::COLS > 64) pin_regs<32>(acc + ch);
               } else if (C::COLS - ch >= 16) {
                 float v[16];
                 tmem_ld16(taddr + ch, v);
@@ -523,8 +560,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
           } else {
             const float sbs = sbv[jk];
 #pragma unroll
-            for (int ch = 0; ch < C::COLS; ch += (C::COLS - ch >= 64 ? 64 : 32)) {
-              if (C::COLS - ch >= 64) {
+            for (int ch = 0; ch < C::COLS; ch += (C::COLS - ch >= 64 && C::COLS <= 64 ? 64 : 32)) {
+              if (C::COLS - ch >= 64 && C::COLS <= 64) {
                 float v[64];
                 tmem_ld64(taddr + ch, v);
 #pragma unroll
@@ -556,7 +593,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&tempty[b]);
-          mbar_arrive(&empty[s]);
+          mbar_arrive(&sa_empty[q]);
         }
       }
 
@@ -577,7 +614,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
             !mbar_wait_cluster(red_free, (tiles_done - 1) & 1u, abort_flag, p.status, p.timeout_ns))
           goto promo_done;
         // (2) expect this tile's bytes from every sender (including itself)
-        if (threadIdx.x == 64) mbar_arrive_expect_tx(red_ready, C::SLICE_TX);
+        if (threadIdx.x == C::PW_BASE * 32) mbar_arrive_expect_tx(red_ready, C::SLICE_TX);
         // (3) push this CTA's partial values into their owners' slot `rank`
         if (C::SWAP) {
           // lane = weight `row`, columns = tokens c0 .. c0 + COLS
@@ -606,7 +643,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) __maxnreg__(C::MAX_REGS)
         // (4) wait until every sender's bytes for this CTA's rows have landed
         if (!mbar_wait_cluster(red_ready, tiles_done & 1u, abort_flag, p.status, p.timeout_ns))
           goto promo_done;
-        const int tix = threadIdx.x - 64;
+        const int tix = threadIdx.x - C::PW_BASE * 32;
         const bool more = t + t_step < total;  // will peers push into these slots again?
         if (C::SWAP) {
           // (5) thread = weight tix: sum its SLICE_M tokens over the slots in

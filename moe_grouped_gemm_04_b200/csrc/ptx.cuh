@@ -65,7 +65,7 @@ __device__ __forceinline__ void raise_status(int* status, int code) {
 // Slow path of mbar_wait: polls until the phase completes, another role of
 // the CTA aborts, or `limit_ns` nanoseconds pass. On the time limit it records
 // FG_DEVICE_WAIT_TIMEOUT and sets the CTA's abort flag so every role stops.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
                                             volatile int* abort_flag, int* status,
                                             uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
@@ -314,7 +314,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 // Bounded wait with cluster-scope acquire (arrivals come from other CTAs).
-__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                int* status, uint64_t limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -364,6 +364,30 @@ __device__ __forceinline__ void grid_dependency_wait() {
 // before it touches memory.
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- register split
+
+// Per-warpgroup register reallocation (all four warps of an aligned
+// warpgroup execute the same one). The registers come from the block's
+// launch allocation, so the shares must add up to at most that.
+template <int N>
+__device__ __forceinline__ void warpgroup_reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void warpgroup_reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Pins `n` values as computed at this point of the program: ordered with the
+// surrounding volatile asm (e.g. the next tensor-memory load), so the compiler
+// cannot defer their computation past it and hold two chunks of loads live.
+template <int N>
+__device__ __forceinline__ void pin_regs(float* v) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
 
 // ---------------------------------------------------------------- misc
