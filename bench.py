@@ -9,12 +9,16 @@ are quantized once before timing, as inference stores them (pass
 --with-weight-quant to quantize them inside every step as well).
 
 The default workload is decode_64x4096x7168 (the swapped-product decode
-shape). Inputs are resident in HBM when the timed region starts; L2 is flushed
-before every timed step (a 256 MiB write, then a 256 MiB read so that no dirty
-flush lines are written back during the step) and the flush is outside the
-step's CUDA events. `value` is FLOPs (2*M_valid*N*K) per step time (no event
-inside the step, so the GEMM's prologue may overlap the quantizer through
-programmatic dependent launch); `roofline` covers the GEMM kernel, timed alone
+shape). Inputs are resident in HBM when the timed region starts. By default
+the step's operands (activations, quantized weights, scales, output) exist in
+several copies whose total is three times the 126 MB L2, used in turn, so that
+no step finds its inputs in L2; the K timed steps run back to back between one
+pair of CUDA events (launch overheads overlap as they do in a serving loop, and
+programmatic dependent launch lets each kernel's prologue overlap its
+predecessor). `--l2 flush` instead flushes L2 before every step (a 256 MiB
+write, then a 256 MiB read so that no dirty flush lines are written back during
+the step) and times each step alone between its own events. `value` is FLOPs
+(2*M_valid*N*K) per step time; `roofline` covers the GEMM kernel, timed alone
 the same way, against the measured HBM bandwidth or FP8 tensor peak; `e2e`
 repeats the step through the public API from pinned host buffers with the
 host<->device copies inside the timed region; `cpu_baseline` times the CPU
@@ -47,6 +51,8 @@ import workloads  # noqa: E402
 
 METRIC = "FP8 block-scaled GEMM TFLOPS (device-timed) and % of B200 FP8/HBM roofline"
 L2_FLUSH_BYTES = 256 << 20
+SENTINEL_BF16 = 0x7FC1  # a bf16 NaN pattern the kernels never produce
+ROTATE_MIN_BYTES = 3 * (126 << 20)  # operand sets in turn: three times the 126 MB L2
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -59,6 +65,11 @@ def parse_args():
     ap.add_argument("--workload", default="decode_64x4096x7168", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--with-weight-quant", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps from Python instead of replaying a CUDA graph")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
+                    help="keep timed steps out of L2 by rotating operand sets larger than L2 "
+                         "(steps back to back) or by flushing L2 before every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -224,10 +235,42 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
 
 # ---------------------------------------------------------------------- GPU leg
 
-class Step:
-    """Device buffers and the launches of one step."""
+class OperandSet:
+    """Device buffers of one copy of a step's operands."""
 
-    def __init__(self, fg, torch, kind, inp, with_weight_quant: bool):
+    def __init__(self, torch, kind, inp, fg, x, w, B, SB, with_weight_quant: bool):
+        dev = "cuda"
+        K, N = inp.K, inp.N
+        self.x = x.clone()
+        self.w = w.clone() if with_weight_quant else None
+        self.B = B.clone()
+        self.SB = SB.clone()
+        if kind == "dense":
+            G, M = 1, inp.M
+            self.A = torch.empty((inp.M, K), dtype=torch.uint8, device=dev)
+            self.D = torch.empty((inp.M, N), dtype=torch.bfloat16, device=dev)
+        elif kind == "contiguous":
+            G, M = 1, inp.M_total
+            self.A = torch.empty((inp.M_total, K), dtype=torch.uint8, device=dev)
+            self.D = torch.empty((inp.M_total, N), dtype=torch.bfloat16, device=dev)
+        else:
+            G, M = inp.G, inp.M_max
+            self.A = torch.empty((inp.G, inp.M_max, K), dtype=torch.uint8, device=dev)
+            self.D = torch.empty((inp.G, inp.M_max, N), dtype=torch.bfloat16, device=dev)
+        self.SA = fg.empty_sfa(G, M, K, dev)
+
+    def nbytes(self):
+        ts = [self.x, self.B, self.SB, self.A, self.D, self.SA] + ([self.w] if self.w is not None else [])
+        return sum(t.numel() * t.element_size() for t in ts)
+
+
+class Step:
+    """The launches of one step over one of several operand sets.
+
+    With `sets` > 1 the copies are used in turn, so that a step's weights and
+    activations are not in L2 when it starts (their total exceeds L2)."""
+
+    def __init__(self, fg, torch, kind, inp, with_weight_quant: bool, min_total_bytes: int):
         self.fg, self.torch, self.kind, self.inp = fg, torch, kind, inp
         self.with_wq = with_weight_quant
         dev = "cuda"
@@ -236,57 +279,48 @@ class Step:
         def bf16(bits):
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
-        self.x = bf16(inp.a)
-        self.w = bf16(inp.b)
-        if kind == "dense":
-            self.G, self.M = 1, inp.M
-            self.A = torch.empty((inp.M, K), dtype=torch.uint8, device=dev)
-            self.B = torch.empty((N, K), dtype=torch.uint8, device=dev)
-            self.D = torch.empty((inp.M, N), dtype=torch.bfloat16, device=dev)
-            Gw = 1
-        elif kind == "contiguous":
-            self.G, self.M = 1, inp.M_total
-            self.A = torch.empty((inp.M_total, K), dtype=torch.uint8, device=dev)
-            self.B = torch.empty((inp.G, N, K), dtype=torch.uint8, device=dev)
-            self.D = torch.empty((inp.M_total, N), dtype=torch.bfloat16, device=dev)
+        x, w = bf16(inp.a), bf16(inp.b)
+        Gw = 1 if kind == "dense" else inp.G
+        B = torch.empty((N, K) if kind == "dense" else (inp.G, N, K), dtype=torch.uint8, device=dev)
+        SB = fg.empty_sfb(Gw, N, K, dev)
+        fg.per_block_cast_to_fp8(w, B, SB)
+        if kind == "contiguous":
             self.mi = torch.from_numpy(inp.m_indices).to(dev)
-            Gw = inp.G
-        else:
-            self.G, self.M = inp.G, inp.M_max
-            self.A = torch.empty((inp.G, inp.M_max, K), dtype=torch.uint8, device=dev)
-            self.B = torch.empty((inp.G, N, K), dtype=torch.uint8, device=dev)
-            self.D = torch.empty((inp.G, inp.M_max, N), dtype=torch.bfloat16, device=dev)
+        if kind == "masked":
             self.mm = torch.from_numpy(inp.masked_m).to(dev)
             self.expected_m = max(1, int(round(float(np.mean(inp.masked_m)))))
-            Gw = inp.G
-        self.SA = fg.empty_sfa(self.G, self.M, K, dev)
-        self.SB = fg.empty_sfb(Gw, N, K, dev)
-        self.quant_weights()
+        first = OperandSet(torch, kind, inp, fg, x, w, B, SB, with_weight_quant)
+        per = first.nbytes()
+        n = max(2, -(-min_total_bytes // per)) if min_total_bytes > 0 else 1
+        self.sets = [first] + [OperandSet(torch, kind, inp, fg, x, w, B, SB, with_weight_quant)
+                               for _ in range(n - 1)]
+        del x, w, B, SB
+        self.set_bytes = per
 
-    def quant_weights(self):
-        self.fg.per_block_cast_to_fp8(self.w, self.B, self.SB)
+    def quant_weights(self, o):
+        self.fg.per_block_cast_to_fp8(o.w, o.B, o.SB)
 
-    def quant_acts(self):
-        self.fg.per_token_cast_to_fp8(self.x, self.A, self.SA)
+    def quant_acts(self, o):
+        self.fg.per_token_cast_to_fp8(o.x, o.A, o.SA)
 
-    def gemm(self):
+    def gemm(self, o):
         fg = self.fg
         if self.kind == "dense":
-            fg.fp8_gemm_nt(self.A, self.SA, self.B, self.SB, self.D)
+            fg.fp8_gemm_nt(o.A, o.SA, o.B, o.SB, o.D)
         elif self.kind == "contiguous":
-            fg.fp8_grouped_gemm_contiguous(self.A, self.SA, self.B, self.SB, self.D, self.mi)
+            fg.fp8_grouped_gemm_contiguous(o.A, o.SA, o.B, o.SB, o.D, self.mi)
         else:
-            fg.fp8_grouped_gemm_masked(self.A, self.SA, self.B, self.SB, self.D, self.mm,
-                                       self.expected_m)
+            fg.fp8_grouped_gemm_masked(o.A, o.SA, o.B, o.SB, o.D, self.mm, self.expected_m)
 
     def launches_per_step(self):
         return 2 + (1 if self.with_wq else 0)
 
-    def run(self):
+    def run(self, i):
+        o = self.sets[i % len(self.sets)]
         if self.with_wq:
-            self.quant_weights()
-        self.quant_acts()
-        self.gemm()
+            self.quant_weights(o)
+        self.quant_acts(o)
+        self.gemm(o)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -299,10 +333,14 @@ def run_ours(args, rank, world, local_rank):
     kind = workloads.WORKLOADS[args.workload][0]
     inp = workloads.make(args.workload, seed=0)
     flops, alg_bytes = workloads.flops_and_bytes(kind, inp)
-    step = Step(fg, torch, kind, inp, args.with_weight_quant)
-    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush_r = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device="cuda")
+    rotate = args.l2 == "rotate"
+    step = Step(fg, torch, kind, inp, args.with_weight_quant,
+                ROTATE_MIN_BYTES if rotate else 0)
+    R = len(step.sets)
     stream = torch.cuda.current_stream()
+    if not rotate:
+        flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        flush_r = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device="cuda")
 
     def flush():
         flush_w.zero_()
@@ -317,69 +355,99 @@ def run_ours(args, rank, world, local_rank):
         if dist is not None:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        flush()
-        step.run()
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def timed(body, K, graph=False):
+        """Mean ms per iteration of body(i) over K iterations. rotate: one
+        event pair around K back-to-back iterations (operand sets in turn),
+        replayed from one CUDA graph when `graph`; flush: L2 flushed before
+        every iteration, outside its event pair."""
+        barrier()
+        torch.cuda.synchronize()
+        if rotate and graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                for i in range(K):
+                    body(i)
+            g.replay()  # untimed: the first replay uploads the graph
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            s = torch.cuda.current_stream()
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+            torch.cuda.synchronize()
+            del g
+            return e0.elapsed_time(e1) / K
+        if rotate:
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            for i in range(K):
+                body(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / K
+        pairs = [(ev(), ev()) for _ in range(K)]
+        for i in range(K):
+            flush()
+            pairs[i][0].record(stream)
+            body(i)
+            pairs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return float(np.mean([x.elapsed_time(y) for x, y in pairs]))
+
+    for i in range(max(args.warmup, R)):
+        if not rotate:
+            flush()
+        step.run(i)
     torch.cuda.synchronize()
     assert fg.get_device_status() == 0
 
     K = args.steps
-    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    ev_gemm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     sampler = ClockSampler(local_rank)
-    barrier()
-    torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)  # let the sampler see the timed region from its start
-    for i in range(K):
-        flush()
-        ev_step[i][0].record(stream)
-        step.run()
-        ev_step[i][1].record(stream)
-    torch.cuda.synchronize()
+    use_graph = rotate and not args.no_graph
+    ms = timed(step.run, K, use_graph)
     barrier()
-    # the GEMM kernel alone (roofline), same flush discipline
-    for i in range(K):
-        flush()
-        if step.with_wq:
-            step.quant_weights()
-        step.quant_acts()
-        flush()
-        ev_gemm[i][0].record(stream)
-        step.gemm()
-        ev_gemm[i][1].record(stream)
-    torch.cuda.synchronize()
+    # the GEMM kernel alone (roofline); every set's activations are quantized.
+    # Outputs start as a NaN sentinel so that the check below sees what the
+    # timed launches wrote.
+    for o in step.sets:
+        o.D.view(torch.int16).fill_(SENTINEL_BF16)
+    gms = timed(lambda i: step.gemm(step.sets[i % R]), K, use_graph)
     barrier()
     clocks = sampler.stop()
     assert fg.get_device_status() == 0
-    step_ms = [a.elapsed_time(b) for a, b in ev_step]
-    gemm_ms = [a.elapsed_time(b) for a, b in ev_gemm]
-    ms = float(np.mean(step_ms))
-    gms = float(np.mean(gemm_ms))
+    # the timed launches did the work: the last output the timed GEMM loop
+    # wrote equals a fresh eager call, bit for bit (the kernels are deterministic)
+    last = step.sets[(K - 1) % R]
+    timed_d = last.D.clone()
+    last.D.view(torch.int16).fill_(SENTINEL_BF16)
+    step.gemm(last)
+    torch.cuda.synchronize()
+    assert torch.equal(timed_d.view(torch.int16), last.D.view(torch.int16)), "timed output differs"
 
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        xh = step.x.cpu().pin_memory()
-        dh = torch.empty(step.D.shape, dtype=step.D.dtype).pin_memory()
-        for _ in range(max(1, args.warmup)):
-            step.x.copy_(xh, non_blocking=True)
-            step.run()
-            dh.copy_(step.D, non_blocking=True)
+        xh = step.sets[0].x.cpu().pin_memory()
+        dh = torch.empty(step.sets[0].D.shape, dtype=step.sets[0].D.dtype).pin_memory()
+
+        def e2e_step(i):
+            o = step.sets[i % R]
+            o.x.copy_(xh, non_blocking=True)
+            step.run(i)
+            dh.copy_(o.D, non_blocking=True)
+
+        for i in range(max(1, args.warmup)):
+            e2e_step(i)
         torch.cuda.synchronize()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        e2e_ms = timed(e2e_step, K)
         barrier()
-        torch.cuda.synchronize()
-        for i in range(K):
-            flush()
-            ev[i][0].record(stream)
-            step.x.copy_(xh, non_blocking=True)
-            step.run()
-            dh.copy_(step.D, non_blocking=True)
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
         e2e = {"ms": e2e_ms, "h2d": xh.numel() * xh.element_size(), "d2h": dh.numel() * dh.element_size()}
 
     # max over ranks
@@ -423,7 +491,11 @@ def run_ours(args, rank, world, local_rank):
 
     value = world * flops / (ms * 1e-3) / 1e12
     cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K,
-           "l2": "flushed before every timed step (256 MiB write + 256 MiB read, outside the step events)",
+           "l2": ("inputs larger than L2: %d operand sets of %.1f MB used in turn, steps back to back"
+                  % (R, step.set_bytes / 1e6)) if rotate else
+                 "flushed before every timed step (256 MiB write + 256 MiB read, outside the step events)",
+           "launch": ("the K timed steps captured in one CUDA graph, replayed once untimed, "
+                      "then once between the events") if use_graph else "eager launches from Python",
            "weights": "quantized inside every step" if args.with_weight_quant else "quantized once before timing",
            "parallelism": "replicas" if world > 1 else "single GPU"}
     if kind == "dense":

@@ -242,7 +242,8 @@ Plan plan_for(const Problem& pr, int sm_count, int expected_m) {
   else pl.bt = 128;
   if (pr.form == kFormMasked && pl.bt < 64) pl.bt = 64;  // one swapped shape for masked
   pl.num_mt = (pr.M + pl.bt - 1) / pl.bt;
-  pl.num_nt = (pr.N + CfgNormal::BW - 1) / (pl.bt == 128 ? CfgNormal::BW : 128);
+  const int tile_w = pl.bt == 128 ? CfgNormal::BW : 128;  // weight rows per tile
+  pl.num_nt = (pr.N + tile_w - 1) / tile_w;
   pl.splits = 1;
   if (pr.form == kFormDense && pl.bt < 128) {
     const int tiles = pl.num_mt * pl.num_nt;
