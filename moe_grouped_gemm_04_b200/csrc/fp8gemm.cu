@@ -263,7 +263,7 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
   KernelInfo* ki = nullptr;
   FG_TRY((kernel_info<C, FORM>(dev_id, &ki)));
   const int KB = pr.K / 128;
-  CUtensorMap tmA, tmB, tmSA;
+  CUtensorMap tmA, tmB, tmSA, tmD;
   FG_TRY(make_map(&tmA, pr.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
                   static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
                   CU_TENSOR_MAP_SWIZZLE_128B, "A"));
@@ -274,6 +274,13 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
                   static_cast<uint64_t>(pr.slabs) * KB,
                   static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 1,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
+  // D as rows x N bf16, box of 32 rows x EPI_COLS columns (normal-form
+  // epilogue; unused, and left zero, by the other forms)
+  std::memset(&tmD, 0, sizeof(tmD));
+  if (C::EPI_TMA)
+    FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
+                    static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2,
+                    C::EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_NONE, "D"));
   GemmParams p{};
   p.M = pr.M;
   p.N = pr.N;
@@ -314,7 +321,7 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<C, FORM>, tmA, tmB, tmSA, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<C, FORM>, tmA, tmB, tmSA, tmD, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_kernel launch");
   return FG_OK;
 }

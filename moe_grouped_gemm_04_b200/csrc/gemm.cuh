@@ -28,6 +28,10 @@
 //               (sb, one value per 128 weight rows and K block, is read from
 //               global memory two K blocks ahead), release the TMEM buffer and
 //               the stage; after the last K block round to bf16 and store D.
+//               Normal form: a warp whose 32 token rows are all stored writes
+//               its slice through shared memory with tensor stores (16
+//               columns per round, two buffers per warp), so that the stores
+//               drain while the warp promotes the next tile.
 // Two TMEM buffers let the MMA of block kb+1 run while block kb is promoted.
 //
 // Normal form: MMA M = 128 token rows, MMA N = BW weight rows (TMEM lane =
@@ -140,7 +144,16 @@ struct GemmCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
   static constexpr int OFF_SA = OFF_B + STAGES * STAGE_B;
-  static constexpr int OFF_RED = OFF_SA + SAS * STAGE_SA;
+  // normal-form epilogue staging: per promotion warp two buffers of 32 rows x
+  // EPI_COLS bf16 (one tensor-store box each)
+  static constexpr bool EPI_TMA = !SWAP && SPLIT == 1;
+  static constexpr int EPI_COLS = 16;
+  static constexpr int EPI_BUF = 32 * EPI_COLS * 2;
+  static constexpr int EPI_BYTES = EPI_TMA ? PW * 2 * EPI_BUF : 0;
+  static_assert(!EPI_TMA || COLS % EPI_COLS == 0, "epilogue rounds");
+  static constexpr int OFF_EPI = EPI_TMA ? (OFF_SA + SAS * STAGE_SA + 1023) / 1024 * 1024
+                                        : OFF_SA + SAS * STAGE_SA;
+  static constexpr int OFF_RED = OFF_EPI + EPI_BYTES;
   static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * SAS + 4 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -148,6 +161,7 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;  // + alignment slack
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(SA_BYTES % 16 == 0, "TMA box inner extent");
+  static_assert(!EPI_TMA || (OFF_EPI % 1024 == 0 && EPI_BUF % 128 == 0), "tensor-store sources");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -322,7 +336,8 @@ __device__ __forceinline__ void issue_stage(int stream, const GemmParams& p, con
 template <class C, int FORM>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmSA, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmD,
+                    const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem + C::OFF_A;
@@ -370,6 +385,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSA);
+    if (C::EPI_TMA) tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -492,6 +508,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     uint32_t it = 0;
     uint32_t tiles_done = 0;
+    uint32_t epi_groups = 0;  // tensor-store groups this warp has issued
     for (int t = t_first; t < total; t += t_step) {
       const Tile w = resolve_tile<FORM>(p, table, t);
       if (!w.valid) continue;
@@ -604,7 +621,44 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           const int m = w.mt * C::BT + row;
           row_mi = m < p.M ? __ldg(p.m_indices + m) : -1;
         }
-        store_tile_part<C, FORM, C::COLS>(p, w, row, c0, acc, m_valid, row_mi);
+        bool staged = false;
+        if constexpr (C::EPI_TMA) {
+          const int m = w.mt * C::BT + row;
+          const bool ok = m < m_valid && (FORM != kFormContig || row_mi >= 0);
+          if (__all_sync(0xffffffffu, ok)) {
+            staged = true;
+            // D rows of this warp: the slab row of its first token
+            const int y = (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT + quad * 32;
+            uint8_t* bufs = smem + C::OFF_EPI + pw * 2 * C::EPI_BUF;
+#pragma unroll
+            for (int ch = 0; ch < C::COLS / C::EPI_COLS; ++ch) {
+              const int x = w.nt * C::BW + c0 + ch * C::EPI_COLS;
+              if (x >= p.N) break;  // columns past N (uniform across the warp)
+              // buffers alternate with the warp's store groups: the group
+              // issued two groups ago used this one and has read it once at
+              // most one group is pending
+              uint8_t* buf = bufs + (epi_groups & 1u) * C::EPI_BUF;
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              uint32_t wv[C::EPI_COLS / 2];
+#pragma unroll
+              for (int j = 0; j < C::EPI_COLS / 2; ++j)
+                wv[j] = pack_bf16x2(acc[ch * C::EPI_COLS + 2 * j], acc[ch * C::EPI_COLS + 2 * j + 1]);
+              uint4* dst = reinterpret_cast<uint4*>(buf + lane * (C::EPI_COLS * 2));
+#pragma unroll
+              for (int j = 0; j < C::EPI_COLS / 8; ++j)
+                dst[j] = make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
+              fence_proxy_async_shared();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmD, buf, x, y);
+                bulk_commit_group();
+              }
+              ++epi_groups;
+            }
+          }
+        }
+        if (!staged) store_tile_part<C, FORM, C::COLS>(p, w, row, c0, acc, m_valid, row_mi);
       } else {
         const uint32_t red_addr = smem_u32(red);
         const uint32_t ready_addr = smem_u32(red_ready);
@@ -705,7 +759,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         ++tiles_done;
       }
     }
-  promo_done:;
+  promo_done:
+    // tensor stores of the epilogue have completed (global writes done,
+    // shared memory no longer read)
+    if (C::EPI_TMA && lane == 0) bulk_wait_group<0>();
   }
 
   // ---------------------------------------------------------------- teardown
