@@ -546,6 +546,38 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (!mbar_wait(&sa_full[q], (it / C::SAS) & 1u, ctl)) goto promo_done;
         if (!mbar_wait(&tfull[b], tph, ctl)) goto promo_done;
         tc_fence_after();
+        if constexpr (!C::SWAP && C::KPS == 1 && C::COLS % 64 == 0) {
+          // normal form: 32-column TMEM loads in two alternating register
+          // sets, the next load in flight while the previous one is folded
+          // in; the TMEM buffer and the scale slot are released once the
+          // last load has completed
+          const float* sa_s = reinterpret_cast<const float*>(sSA + q * C::STAGE_SA);
+          const float scale = sa_s[row] * sbv[0];
+          const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * C::MMA_N + c0);
+          uint32_t r0[32], r1[32];
+          tmem_ld32_issue(taddr, r0);
+          tmem_wait_ld32(r0);
+#pragma unroll
+          for (int ch = 1; ch <= C::COLS / 32; ++ch) {
+            uint32_t(&cur)[32] = (ch & 1) ? r0 : r1;   // loaded by the previous step
+            uint32_t(&nxt)[32] = (ch & 1) ? r1 : r0;
+            if (ch < C::COLS / 32) tmem_ld32_issue(taddr + 32 * ch, nxt);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              acc[(ch - 1) * 32 + j] = fmaf(__uint_as_float(cur[j]), scale, acc[(ch - 1) * 32 + j]);
+            if (ch < C::COLS / 32) {
+              tmem_wait_ld32(nxt);
+              if (ch == C::COLS / 32 - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                  mbar_arrive(&tempty[b]);
+                  mbar_arrive(&sa_empty[q]);
+                }
+              }
+            }
+          }
+        } else {
 #pragma unroll
         for (int jk = 0; jk < C::KPS; ++jk) {
           if (kq + jk * kb_step >= p.KB) break;
@@ -611,6 +643,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (lane == 0) {
           mbar_arrive(&tempty[b]);
           mbar_arrive(&sa_empty[q]);
+        }
         }
       }
 
