@@ -146,17 +146,17 @@ int sfa_stride(int M) { return (M + 3) / 4 * 4; }
 
 // ---------------------------------------------------------------- GEMM configs
 
-//                      BT   BW   swap  stages PW split (2 K blocks per stage)
+//                        BT   BW   swap  stages PW split K blocks/stage
 using CfgNormal = GemmCfg<128, 256, false, 4, 8, 1, 1>;
-using CfgSwap16 = GemmCfg<16, 128, true, 5, 4, 1>;
-using CfgSwap32 = GemmCfg<32, 128, true, 5, 4, 1>;
-using CfgSwap64 = GemmCfg<64, 128, true, 4, 4, 1>;
-using CfgSwap16S2 = GemmCfg<16, 128, true, 5, 4, 2>;
-using CfgSwap32S2 = GemmCfg<32, 128, true, 4, 4, 2>;
-using CfgSwap64S2 = GemmCfg<64, 128, true, 3, 4, 2>;
-using CfgSwap16S4 = GemmCfg<16, 128, true, 5, 4, 4>;
-using CfgSwap32S4 = GemmCfg<32, 128, true, 4, 4, 4>;
-using CfgSwap64S4 = GemmCfg<64, 128, true, 3, 4, 4>;
+using CfgSwap16 = GemmCfg<16, 128, true, 5, 4, 1, 2>;
+using CfgSwap32 = GemmCfg<32, 128, true, 5, 4, 1, 2>;
+using CfgSwap64 = GemmCfg<64, 128, true, 4, 4, 1, 2>;
+using CfgSwap16S2 = GemmCfg<16, 128, true, 5, 4, 2, 2>;
+using CfgSwap32S2 = GemmCfg<32, 128, true, 4, 4, 2, 2>;
+using CfgSwap64S2 = GemmCfg<64, 128, true, 3, 4, 2, 2>;
+using CfgSwap16S4 = GemmCfg<16, 128, true, 5, 4, 4, 2>;
+using CfgSwap32S4 = GemmCfg<32, 128, true, 4, 4, 4, 2>;
+using CfgSwap64S4 = GemmCfg<64, 128, true, 3, 4, 4, 2>;
 
 struct KernelInfo {
   bool attr_set = false;
@@ -170,7 +170,7 @@ fg_status kernel_info(int dev, KernelInfo** out) {
   if (!k.attr_set) {
     cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<C, FORM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
+                                         C::smem_bytes(FORM));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     if (C::REG_SPLIT) {
       // the warpgroup register split draws on the launch allocation: it must
@@ -191,7 +191,7 @@ fg_status kernel_info(int dev, KernelInfo** out) {
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(C::SPLIT * 64);
       cfg.blockDim = dim3(C::NUM_THREADS);
-      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cfg.dynamicSmemBytes = C::smem_bytes(FORM);
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
@@ -274,13 +274,18 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
                   static_cast<uint64_t>(pr.slabs) * KB,
                   static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 1,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
-  // D as rows x N bf16, box of 32 rows x EPI_COLS columns (normal-form
-  // epilogue; unused, and left zero, by the other forms)
+  // D as rows x N bf16: boxes of 32 rows x EPI_COLS columns (normal-form
+  // epilogue) or SLICE_M rows x 128 columns (split-K slices of the swapped
+  // form); unused, and left zero, otherwise
   std::memset(&tmD, 0, sizeof(tmD));
   if (C::EPI_TMA)
     FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
                     static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2,
                     C::EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_NONE, "D"));
+  else if (C::RED_TMA && FORM == kFormDense)
+    FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
+                    static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2,
+                    128, C::SLICE_M, CU_TENSOR_MAP_SWIZZLE_NONE, "D"));
   GemmParams p{};
   p.M = pr.M;
   p.N = pr.N;
@@ -308,7 +313,7 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
   cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(C::NUM_THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.dynamicSmemBytes = C::smem_bytes(FORM);
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the
   attr[0].val.programmaticStreamSerializationAllowed = 1;           // previous kernel

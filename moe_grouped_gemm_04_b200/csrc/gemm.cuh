@@ -122,25 +122,32 @@ struct GemmCfg {
   static_assert(!REG_SPLIT || 128 * REG_LOW + PW * 32 * REG_HIGH <= NUM_THREADS * MAX_REGS,
                 "register split exceeds the launch allocation");
   static constexpr int SAS = 2 * STAGES;  // token-scale ring (read by the promotion warps)
-  // split-K receive slots: SPLIT slots (one per sender) of SLICE_M token rows
-  // x TN weights in fp32, stored as groups of 4 consecutive values along the
-  // dimension a promotion thread holds, with the lane dimension next, so that
-  // the 16-byte pushes of a warp land contiguously:
-  //   swapped form (lane = weight): slot[token / 4][weight][token % 4]
-  //   normal form  (lane = token):  slot[weight / 4][token][weight % 4]
-  static_assert(SPLIT == 1 || (PW == 4 && (SPLIT == 2 || SPLIT == 4 || SPLIT == 8)),
-                "split-K uses 128 promotion threads and 2, 4 or 8 CTAs");
+  // split-K receive slots: SPLIT - 1 slots (one per peer; a CTA keeps its own
+  // values in registers) of SLICE_M token rows x 128 weights in fp32, stored
+  // as groups of 4 consecutive tokens with the weight (TMEM lane) next, so
+  // that the 16-byte pushes of a warp land contiguously:
+  //   slot[token / 4][weight][token % 4]
+  static_assert(SPLIT == 1 || (SWAP && PW == 4 && (SPLIT == 2 || SPLIT == 4 || SPLIT == 8)),
+                "split-K: swapped form, 128 promotion threads, 2, 4 or 8 CTAs");
   static constexpr int TN = SWAP ? 128 : BW;  // weight columns of a tile
   static constexpr int SLICE_M = BT / SPLIT;
   static constexpr int SLOT_FLOATS = SLICE_M * TN;
-  static constexpr int RED_BYTES = SPLIT > 1 ? SPLIT * SLOT_FLOATS * 4 : 0;
-  static constexpr uint32_t SLICE_TX = SPLIT * SLICE_M * TN * 4;  // bytes a CTA receives per tile
-  // normal-form reduction: VPT consecutive weights of one token per thread
-  static constexpr int VPT = SPLIT > 1 && !SWAP ? SLICE_M * TN / 128 : 8;
+  static constexpr int RED_BYTES = SPLIT > 1 ? (SPLIT - 1) * SLOT_FLOATS * 4 : 0;
+  // bytes a CTA receives from its peers per tile
+  static constexpr uint32_t SLICE_TX = (SPLIT - 1) * SLICE_M * TN * 4;
+  // swapped split-K: the reduced slice (SLICE_M tokens x 128 weights, bf16)
+  // leaves through shared memory with one tensor store
+  static constexpr bool RED_TMA = SWAP && SPLIT > 1;
+  static constexpr int RSTG_BYTES = RED_TMA ? SLICE_M * 128 * 2 : 0;
+  // Thin (swapped) shapes are short launches: once the producer has issued
+  // its last load, the next kernel of the stream may launch, so that its
+  // prologue overlaps this kernel's reduction and epilogue.
+  static constexpr bool EARLY_TRIGGER = SWAP;
   static_assert(SPLIT == 1 || (BT % SPLIT == 0 && SLICE_M % 4 == 0 && COLS % 4 == 0),
-                "16-byte pushes of 4 consecutive tokens (swapped) or weights (normal)");
-  static_assert(SPLIT == 1 || SWAP || SLICE_M % 32 == 0, "a warp's tokens share one owner");
-  static_assert(SPLIT == 1 || SWAP || (VPT % 8 == 0 && TN % VPT == 0), "16-byte D stores");
+                "16-byte pushes of 4 consecutive tokens");
+  static_assert(SPLIT == 1 || WPQ == 1, "split-K: a thread holds all tokens of its weight row");
+  // on a CTA's last tile the outgoing partials are staged in the idle ring
+  static_assert(RED_BYTES <= STAGES * (STAGE_A + STAGE_B), "send staging fits in the ring");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
   static constexpr int OFF_SA = OFF_B + STAGES * STAGE_B;
@@ -154,14 +161,20 @@ struct GemmCfg {
   static constexpr int OFF_EPI = EPI_TMA ? (OFF_SA + SAS * STAGE_SA + 1023) / 1024 * 1024
                                         : OFF_SA + SAS * STAGE_SA;
   static constexpr int OFF_RED = OFF_EPI + EPI_BYTES;
-  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * SAS + 4 + 2;
+  static constexpr int OFF_RSTG = OFF_RED + RED_BYTES;  // 128-byte aligned (RED_BYTES is)
+  static constexpr int OFF_BAR = OFF_RSTG + RSTG_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * SAS + 4 + 3;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;  // + alignment slack
+  // the tile table exists for the grouped forms only; + alignment slack
+  static constexpr int smem_bytes(int form) {
+    return OFF_TABLE + (form == kFormDense ? 0 : kTableMax * 4) + 1024;
+  }
+  static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(SA_BYTES % 16 == 0, "TMA box inner extent");
   static_assert(!EPI_TMA || (OFF_EPI % 1024 == 0 && EPI_BUF % 128 == 0), "tensor-store sources");
+  static_assert(!RED_TMA || (OFF_RSTG % 128 == 0 && RSTG_BYTES % 16 == 0), "tensor-store source");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -255,9 +268,9 @@ __device__ void build_table(const GemmParams& p, int* table, int lane) {
 // releases its shared and tensor memory.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = wait_clock();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) return;
+    if (wait_clock() - t0 > wait_cycles(limit_ns)) return;
   }
 }
 
@@ -352,6 +365,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* red_ready = tempty + 2;    // all partials of the current tile are in place
   uint64_t* red_free = red_ready + 1;  // every CTA has finished reading them
+  uint64_t* grp = red_free + 1;        // all promotion warps of this CTA (bounded group sync)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* table = reinterpret_cast<int*>(smem + C::OFF_TABLE);
@@ -380,37 +394,29 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
     mbar_init(red_ready, 1);                 // own expect_tx; peers' bytes complete_tx
     mbar_init(red_free, C::SPLIT * C::PW);   // one arrival per promotion warp of each CTA
+    mbar_init(grp, C::PW);                   // one arrival per promotion warp
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSA);
-    if (C::EPI_TMA) tma_prefetch_desc(&tmD);
+    if (C::EPI_TMA || C::RED_TMA) tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // Peers address this CTA's barriers only after the cluster barrier
+  // completes (its wait comes after the CTA-wide barrier below).
+  __syncwarp();
+  if constexpr (C::SPLIT > 1) cluster_arrive_relaxed();
   // Everything above may overlap the previous kernel; memory comes after this.
   grid_dependency_wait();
-  uint32_t pre_issued = 0;  // first-tile stages the producer issued before the CTA-wide sync
-  if (warp == 0) {
-    build_table<C, FORM>(p, table, lane);
-    __syncwarp();
-    if (lane < 3 && t_first < total_tiles<FORM>(p, table)) {
-      const Tile w = resolve_tile<FORM>(p, table, t_first);
-      if (w.valid) {
-        for (int kq = kb_first; kq < p.KB && pre_issued < C::STAGES;
-             kq += C::KPS * kb_step, ++pre_issued)
-          issue_stage<C, FORM>(lane, p, w, kq, kb_step, pre_issued, sA, sB, sSA, full, sa_full,
-                               &tmA, &tmB, &tmSA);
-      }
-    }
-  }
+  if (warp == 0) build_table<C, FORM>(p, table, lane);
   tc_fence_before();
   __syncwarp();
   __syncthreads();
-  if constexpr (C::SPLIT > 1) cluster_sync_all();  // peers' barriers are initialised
+  if constexpr (C::SPLIT > 1) cluster_wait();  // peers' barriers are initialised
   tc_fence_after();
 
   const uint32_t tmem_base = *tmem_slot;
@@ -427,7 +433,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         const Tile w = resolve_tile<FORM>(p, table, t);
         if (!w.valid) continue;
         for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
-          if (it < pre_issued) continue;
           if (lane < 2) {
             const int s = it % C::STAGES;
             if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1u) ^ 1u, ctl)) goto producer_done;
@@ -439,10 +444,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
                                &tmSA);
         }
       }
+      // every load of this CTA is issued: the next kernel of the stream may
+      // launch (it waits for this grid's completion before touching memory)
+      if (C::EARLY_TRIGGER) grid_launch_dependents();
     producer_done:
       // Before the CTA exits, the last fill of every stage must have landed
       // and been released (its TMA bytes and the MMA commit's arrival).
-      it = it > pre_issued ? it : pre_issued;
       if (lane == 0) {
         for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
           const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
@@ -509,6 +516,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     uint32_t it = 0;
     uint32_t tiles_done = 0;
     uint32_t epi_groups = 0;  // tensor-store groups this warp has issued
+    uint32_t grp_phase = 0;   // uses of the promotion group barrier
     for (int t = t_first; t < total; t += t_step) {
       const Tile w = resolve_tile<FORM>(p, table, t);
       if (!w.valid) continue;
@@ -700,55 +708,80 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (tiles_done > 0 &&
             !mbar_wait_cluster(red_free, (tiles_done - 1) & 1u, abort_flag, p.status, p.timeout_ns))
           goto promo_done;
-        // (2) expect this tile's bytes from every sender (including itself)
+        // (2) expect this tile's bytes from every peer
         if (threadIdx.x == C::PW_BASE * 32) mbar_arrive_expect_tx(red_ready, C::SLICE_TX);
-        // (3) push this CTA's partial values into their owners' slot `rank`
-        if (C::SWAP) {
-          // lane = weight `row`, columns = tokens c0 .. c0 + COLS
+        // (3) push the partial values of the tokens other CTAs own (token m
+        //     belongs to CTA m / SLICE_M) into their slot for this CTA; this
+        //     thread's lane is weight `row`, its columns tokens c0 .. c0 + COLS
+        if (t + t_step >= total) {
+          // last tile of this CTA: the ring is idle (the tile's last MMA has
+          // completed and no load follows), so each peer's slot image is
+          // assembled there and sent with one bulk copy
+          float* images = reinterpret_cast<float*>(smem + C::OFF_A);
 #pragma unroll
           for (int j = 0; j < C::COLS; j += 4) {
             const int m = c0 + j;
-            const uint32_t dst_cta = static_cast<uint32_t>(m / C::SLICE_M);
-            const uint32_t off = static_cast<uint32_t>(
-                (rank * C::SLOT_FLOATS + ((m % C::SLICE_M) / 4 * C::TN + row) * 4) * 4);
-            st_async_f4(mapa_shared(red_addr + off, dst_cta),
-                        make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]),
-                        mapa_shared(ready_addr, dst_cta));
+            const int dst = m / C::SLICE_M;
+            if (dst != rank) {
+              float* img = images + (dst < rank ? dst : dst - 1) * C::SLOT_FLOATS;
+              *reinterpret_cast<float4*>(img + ((m % C::SLICE_M) / 4 * C::TN + row) * 4) =
+                  make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+            }
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(grp);
+          if (!mbar_wait(grp, grp_phase++ & 1u, ctl)) goto promo_done;
+          if (threadIdx.x == C::PW_BASE * 32) {
+            for (int dst = 0; dst < C::SPLIT; ++dst) {
+              if (dst == rank) continue;
+              const uint32_t off = static_cast<uint32_t>((rank < dst ? rank : rank - 1) * C::SLOT_FLOATS * 4);
+              bulk_copy_to_cluster(mapa_shared(red_addr + off, static_cast<uint32_t>(dst)),
+                                   images + (dst < rank ? dst : dst - 1) * C::SLOT_FLOATS,
+                                   C::SLOT_FLOATS * 4, mapa_shared(ready_addr, static_cast<uint32_t>(dst)));
+            }
           }
         } else {
-          // lane = token `row`, columns = weights c0 .. c0 + COLS
-          const uint32_t dst_cta = static_cast<uint32_t>(row / C::SLICE_M);
-          const uint32_t bar = mapa_shared(ready_addr, dst_cta);
 #pragma unroll
           for (int j = 0; j < C::COLS; j += 4) {
-            const uint32_t off = static_cast<uint32_t>(
-                (rank * C::SLOT_FLOATS + ((c0 + j) / 4 * C::SLICE_M + row % C::SLICE_M) * 4) * 4);
-            st_async_f4(mapa_shared(red_addr + off, dst_cta),
-                        make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]), bar);
+            const int m = c0 + j;
+            const int dst = m / C::SLICE_M;
+            if (dst != rank) {
+              const int slot = rank < dst ? rank : rank - 1;
+              const uint32_t off = static_cast<uint32_t>(
+                  (slot * C::SLOT_FLOATS + ((m % C::SLICE_M) / 4 * C::TN + row) * 4) * 4);
+              st_async_f4(mapa_shared(red_addr + off, static_cast<uint32_t>(dst)),
+                          make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]),
+                          mapa_shared(ready_addr, static_cast<uint32_t>(dst)));
+            }
           }
         }
-        // (4) wait until every sender's bytes for this CTA's rows have landed
+        // (4) wait until every peer's bytes for this CTA's tokens have landed
         if (!mbar_wait_cluster(red_ready, tiles_done & 1u, abort_flag, p.status, p.timeout_ns))
           goto promo_done;
-        const int tix = threadIdx.x - C::PW_BASE * 32;
-        const bool more = t + t_step < total;  // will peers push into these slots again?
-        if (C::SWAP) {
-          // (5) thread = weight tix: sum its SLICE_M tokens over the slots in
-          //     split order, then store D[token][weight] (32 lanes write 32
-          //     consecutive weights of a token row)
+        {
+          const bool more = t + t_step < total;  // will peers push into these slots again?
+          // (5) weight `row`: sum its SLICE_M owned tokens over the CTAs in
+          //     split order (its own values from registers), so the result does
+          //     not depend on which CTA finished first
           float sum[C::SLICE_M];
 #pragma unroll
           for (int j = 0; j < C::SLICE_M; ++j) sum[j] = 0.0f;
 #pragma unroll
           for (int r = 0; r < C::SPLIT; ++r) {
-            const float* src = red + r * C::SLOT_FLOATS + tix * 4;
+            if (r == rank) {
 #pragma unroll
-            for (int j = 0; j < C::SLICE_M; j += 4) {
-              const float4 v = *reinterpret_cast<const float4*>(src + j * C::TN);
-              sum[j] += v.x;
-              sum[j + 1] += v.y;
-              sum[j + 2] += v.z;
-              sum[j + 3] += v.w;
+              for (int j = 0; j < C::SLICE_M; ++j) sum[j] += acc[r * C::SLICE_M + j];
+            } else {
+              const float* src = red + (r < rank ? r : r - 1) * C::SLOT_FLOATS + row * 4;
+#pragma unroll
+              for (int j = 0; j < C::SLICE_M; j += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(src + j * C::TN);
+                sum[j] += v.x;
+                sum[j + 1] += v.y;
+                sum[j + 2] += v.z;
+                sum[j + 3] += v.w;
+              }
             }
           }
           if (more) {
@@ -756,38 +789,33 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             if (lane == 0)
               for (int r = 0; r < C::SPLIT; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(red_free), r));
           }
-          store_tile_part<C, FORM, C::SLICE_M>(p, w, tix, rank * C::SLICE_M, sum, m_valid, 0);
-        } else {
-          // (5) thread: one token row, VPT consecutive weights
-          const int ml = tix / (C::TN / C::VPT);
-          const int n0 = (tix % (C::TN / C::VPT)) * C::VPT;
-          float sum[C::VPT];
-#pragma unroll
-          for (int j = 0; j < C::VPT; ++j) sum[j] = 0.0f;
-#pragma unroll
-          for (int r = 0; r < C::SPLIT; ++r) {
-            const float* src = red + r * C::SLOT_FLOATS + (n0 / 4 * C::SLICE_M + ml) * 4;
-#pragma unroll
-            for (int j = 0; j < C::VPT; j += 4) {
-              const float4 v = *reinterpret_cast<const float4*>(src + j * C::SLICE_M);
-              sum[j] += v.x;
-              sum[j + 1] += v.y;
-              sum[j + 2] += v.z;
-              sum[j + 3] += v.w;
+          if constexpr (C::RED_TMA && FORM == kFormDense) {
+            // bf16 slice [SLICE_M tokens][128 weights] in shared memory, then
+            // one tensor store (rows past M and columns past N are clipped)
+            const int y = w.mt * C::BT + rank * C::SLICE_M;
+            uint16_t* stg = reinterpret_cast<uint16_t*>(smem + C::OFF_RSTG);
+            // the previous tile's store has finished reading the buffer: its
+            // issuing thread waits for that before this group barrier
+            if (tiles_done > 0) {
+              if (threadIdx.x == C::PW_BASE * 32) bulk_wait_group_read<0>();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(grp);
+              if (!mbar_wait(grp, grp_phase++ & 1u, ctl)) goto promo_done;
             }
-          }
-          if (more) {
+#pragma unroll
+            for (int j = 0; j < C::SLICE_M; ++j)
+              stg[j * 128 + row] = static_cast<uint16_t>(pack_bf16x2(sum[j], 0.0f) & 0xFFFFu);
+            fence_proxy_async_shared();
             __syncwarp();
-            if (lane == 0)
-              for (int r = 0; r < C::SPLIT; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(red_free), r));
+            if (lane == 0) mbar_arrive(grp);
+            if (!mbar_wait(grp, grp_phase++ & 1u, ctl)) goto promo_done;
+            if (threadIdx.x == C::PW_BASE * 32 && y < m_valid) {
+              tma_store_2d(&tmD, stg, w.nt * 128, y);
+              bulk_commit_group();
+            }
+          } else {
+            store_tile_part<C, FORM, C::SLICE_M>(p, w, row, rank * C::SLICE_M, sum, m_valid, 0);
           }
-          const int srow = rank * C::SLICE_M + ml;
-          int row_mi = 0;
-          if (FORM == kFormContig) {
-            const int m = w.mt * C::BT + srow;
-            row_mi = m < p.M ? __ldg(p.m_indices + m) : -1;
-          }
-          store_tile_part<C, FORM, C::VPT>(p, w, srow, n0, sum, m_valid, row_mi);
         }
         ++tiles_done;
       }
@@ -795,7 +823,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   promo_done:
     // tensor stores of the epilogue have completed (global writes done,
     // shared memory no longer read)
-    if (C::EPI_TMA && lane == 0) bulk_wait_group<0>();
+    // this warp's tensor stores have finished reading shared memory
+    if ((C::EPI_TMA || C::RED_TMA) && lane == 0) bulk_wait_group_read<0>();
   }
 
   // ---------------------------------------------------------------- teardown
@@ -806,7 +835,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   tc_fence_before();
   // No CTA may leave while a peer can still write its shared memory; the
   // cluster barrier covers every thread of the CTA as well.
-  if constexpr (C::SPLIT > 1) cluster_sync_all(); else __syncthreads();
+  if constexpr (C::SPLIT > 1) {
+    // every CTA arrives only after all bytes sent to it have landed, so when
+    // the barrier completes no transfer reads or writes any CTA's memory
+    cluster_arrive_relaxed();
+    cluster_wait();
+  } else {
+    __syncthreads();
+  }
   grid_launch_dependents();
   if (warp == 1) {
     tc_fence_after();

@@ -11,11 +11,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+// Time base of the bounded waits: the SM cycle counter, which is cheap to
+// read (the global nanosecond timer is not). A limit of L nanoseconds is
+// counted as 2 L cycles, which lasts at least L ns at SM clocks up to 2 GHz.
+__device__ __forceinline__ uint64_t wait_clock() { return static_cast<uint64_t>(clock64()); }
+__device__ __forceinline__ uint64_t wait_cycles(uint64_t limit_ns) { return 2 * limit_ns; }
 
 // ---------------------------------------------------------------- mbarrier
 
@@ -68,12 +68,12 @@ __device__ __forceinline__ void raise_status(int* status, int code) {
 __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
                                             volatile int* abort_flag, int* status,
                                             uint64_t limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = wait_clock();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
+      if (wait_clock() - t0 > wait_cycles(limit_ns)) {
         raise_status(status, 1 /* FG_DEVICE_WAIT_TIMEOUT */);
         *abort_flag = 1;
         return false;
@@ -339,10 +339,22 @@ __device__ __forceinline__ uint32_t num_clusters_x() {
 }
 
 // Every thread of every CTA of the cluster (hardware barrier). Only used at
-// kernel start and at teardown, which every thread reaches on every path.
+// teardown, which every thread reaches on every path.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
+}
+
+// The two halves of a cluster barrier, for the kernel start: every thread
+// arrives without release semantics (the barrier initialisations are ordered
+// by fence.mbarrier_init) and waits later, so that work placed in between
+// (the first tensor loads) does not hold the barrier up.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_acq_rel_cluster() {
@@ -378,12 +390,12 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                int* status, uint64_t limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = wait_clock();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
+      if (wait_clock() - t0 > wait_cycles(limit_ns)) {
         raise_status(status, 1 /* FG_DEVICE_WAIT_TIMEOUT */);
         *abort_flag = 1;
         return false;
@@ -400,6 +412,17 @@ __device__ __forceinline__ void st_async_f4(uint32_t dst_cluster_addr, float4 v,
   asm volatile(
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
       ::"r"(dst_cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(mbar_cluster_addr)
+      : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
+// shared memory of a CTA of the cluster; the bytes complete_tx on the
+// mbarrier at `mbar_cluster_addr`, which lives in the destination CTA.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster_addr, const void* src,
+                                                     uint32_t bytes, uint32_t mbar_cluster_addr) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst_cluster_addr), "r"(smem_u32(src)), "r"(bytes), "r"(mbar_cluster_addr)
       : "memory");
 }
 

@@ -59,8 +59,10 @@ __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __r
                                                              uint8_t* __restrict__ q,
                                                              float* __restrict__ sfa, int G,
                                                              int M, int K, int stride) {
-  grid_dependency_wait();
+  // the next kernel may start its prologue now; it waits for this grid
+  // before touching memory
   grid_launch_dependents();
+  grid_dependency_wait();
   const int KB = K / 128;
   const int64_t slices = static_cast<int64_t>(G) * KB * M;
   const int sub = threadIdx.x & 15;
