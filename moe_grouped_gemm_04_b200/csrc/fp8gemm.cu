@@ -147,7 +147,8 @@ int sfa_stride(int M) { return (M + 3) / 4 * 4; }
 // ---------------------------------------------------------------- GEMM configs
 
 //                        BT   BW   swap  stages PW split K blocks/stage
-using CfgNormal = GemmCfg<128, 256, false, 4, 8, 1, 1>;
+using CfgNormal = GemmCfg<128, 256, false, 3, 8, 1, 1>;
+using CfgPair = GemmCfg<128, 256, false, 4, 8, 1, 1, true>;  // dense: CTA pairs, 256 x 256 tiles
 using CfgSwap16 = GemmCfg<16, 128, true, 5, 4, 1, 2>;
 using CfgSwap32 = GemmCfg<32, 128, true, 5, 4, 1, 2>;
 using CfgSwap64 = GemmCfg<64, 128, true, 4, 4, 1, 2>;
@@ -160,7 +161,7 @@ using CfgSwap64S4 = GemmCfg<64, 128, true, 3, 4, 4, 2>;
 
 struct KernelInfo {
   bool attr_set = false;
-  int max_clusters = 0;  // max co-resident clusters (split-K configs)
+  int max_clusters = 0;  // max co-resident clusters (split-K and pair configs)
 };
 
 template <class C, int FORM>
@@ -182,14 +183,14 @@ fg_status kernel_info(int dev, KernelInfo** out) {
         return fail(FG_ERR_UNSUPPORTED, "kernel built with %d registers per thread, register split needs %d",
                     fa.numRegs, C::MAX_REGS);
     }
-    if (C::SPLIT > 1) {
+    if (C::CLUSTER > 1) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = C::SPLIT;
+      attr[0].val.clusterDim.x = C::CLUSTER;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(C::SPLIT * 64);
+      cfg.gridDim = dim3(C::CLUSTER * 64);
       cfg.blockDim = dim3(C::NUM_THREADS);
       cfg.dynamicSmemBytes = C::smem_bytes(FORM);
       cfg.attrs = attr;
@@ -197,7 +198,7 @@ fg_status kernel_info(int dev, KernelInfo** out) {
       int n = 0;
       e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<C, FORM>, &cfg);
       if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-      if (n < 1) return fail(FG_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", C::SPLIT);
+      if (n < 1) return fail(FG_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", C::CLUSTER);
       k.max_clusters = n;
     }
     k.attr_set = true;
@@ -268,20 +269,20 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
                   static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
                   CU_TENSOR_MAP_SWIZZLE_128B, "A"));
   FG_TRY(make_map(&tmB, pr.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
-                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::BW,
+                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::B_ROWS,
                   CU_TENSOR_MAP_SWIZZLE_128B, "B"));
   FG_TRY(make_map(&tmSA, pr.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.M,
                   static_cast<uint64_t>(pr.slabs) * KB,
                   static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 1,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
-  // D as rows x N bf16: boxes of 32 rows x EPI_COLS columns (normal-form
-  // epilogue) or SLICE_M rows x 128 columns (split-K slices of the swapped
-  // form); unused, and left zero, otherwise
+  // D as rows x N bf16: boxes of 32 rows x 64 columns with 128-byte
+  // swizzling (normal-form epilogue) or SLICE_M rows x 128 columns (split-K
+  // slices of the swapped form); unused, and left zero, otherwise
   std::memset(&tmD, 0, sizeof(tmD));
   if (C::EPI_TMA)
     FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
                     static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2,
-                    C::EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_NONE, "D"));
+                    64, 32, CU_TENSOR_MAP_SWIZZLE_128B, "D"));
   else if (C::RED_TMA && FORM == kFormDense)
     FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
                     static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2,
@@ -301,11 +302,11 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
   p.masked_m = pr.masked_m;
   p.status = dev.status;
   p.timeout_ns = wait_limit_ns();
-  int64_t tiles = static_cast<int64_t>(pl.num_mt) * pl.num_nt;
+  int64_t tiles = static_cast<int64_t>(C::PAIR ? (pl.num_mt + 1) / 2 : pl.num_mt) * pl.num_nt;
   if (FORM == kFormMasked) tiles *= pr.G;  // upper bound: masked_m lives on the device
   int64_t grid;
-  if (C::SPLIT > 1) {
-    grid = C::SPLIT * std::max<int64_t>(1, std::min<int64_t>(tiles, ki->max_clusters));
+  if (C::CLUSTER > 1) {
+    grid = C::CLUSTER * std::max<int64_t>(1, std::min<int64_t>(tiles, ki->max_clusters));
   } else {
     grid = std::max<int64_t>(1, std::min<int64_t>(tiles, dev.sm_count));
   }
@@ -319,9 +320,9 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;           // previous kernel
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (C::SPLIT > 1) {
+  if (C::CLUSTER > 1) {
     attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = C::SPLIT;
+    attr[1].val.clusterDim.x = C::CLUSTER;
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
@@ -334,7 +335,10 @@ fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, 
 template <int FORM>
 fg_status dispatch(const Problem& pr, const Plan& pl, const DeviceInfo& dev, int dev_id,
                    cudaStream_t stream) {
-  if (pl.bt == 128) return launch_gemm<CfgNormal, FORM>(pr, pl, dev, dev_id, stream);
+  if (pl.bt == 128) {
+    if constexpr (FORM == kFormDense) return launch_gemm<CfgPair, FORM>(pr, pl, dev, dev_id, stream);
+    return launch_gemm<CfgNormal, FORM>(pr, pl, dev, dev_id, stream);
+  }
   if constexpr (FORM == kFormMasked) {
     if (pl.bt == 64) return launch_gemm<CfgSwap64, FORM>(pr, pl, dev, dev_id, stream);
   }

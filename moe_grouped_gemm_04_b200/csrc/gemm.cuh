@@ -81,7 +81,8 @@ struct GemmParams {
   uint64_t timeout_ns;
 };
 
-template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_, int KPS_ = 2>
+template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_, int KPS_ = 2,
+          bool PAIR_ = false>
 struct GemmCfg {
   static constexpr int BT = BT_;          // token rows per tile
   static constexpr int BW = BW_;          // weight rows per tile
@@ -90,6 +91,15 @@ struct GemmCfg {
   static constexpr int PW = PW_;          // promotion warps
   static constexpr int SPLIT = SPLIT_;    // CTAs per cluster sharing one tile's K blocks
   static constexpr int KPS = KPS_;        // K blocks per pipeline stage
+  // Pair MMA (tcgen05 cta_group::2): the two CTAs of a cluster compute one
+  // tile of 2 * BT tokens x BW weights; each loads its BT token rows and half
+  // of the BW weight rows, the leader issues the MMAs, and each CTA's tensor
+  // memory receives its own BT x BW slice, which it promotes and stores.
+  static constexpr bool PAIR = PAIR_;
+  static_assert(!PAIR || (!SWAP && SPLIT == 1 && KPS == 1), "pair MMA: normal form, no split-K");
+  static constexpr int CLUSTER = PAIR ? 2 : SPLIT;  // CTAs per cluster
+  static constexpr int B_ROWS = PAIR ? BW / 2 : BW;  // weight rows this CTA loads per tile
+  static constexpr int MMA_M = PAIR ? 256 : 128;
   static constexpr int MMA_N = SWAP ? BT : BW;
   static_assert(SWAP ? (BW == 128) : (BT == 128), "the lane operand has 128 rows");
   static_assert(MMA_N % 16 == 0 && MMA_N >= 16 && MMA_N <= 256, "tcgen05 N for M = 128");
@@ -99,7 +109,7 @@ struct GemmCfg {
   static_assert(COLS % 8 == 0, "columns per promotion thread");
   static_assert(SWAP || (COLS <= 128 && (128 % COLS == 0)), "one weight scale per thread");
   static constexpr int A_BYTES = BT * 128;
-  static constexpr int B_BYTES = BW * 128;
+  static constexpr int B_BYTES = B_ROWS * 128;
   static constexpr int SA_BYTES = BT * 4;                       // one TMA box of token scales
   static constexpr int SA_STAGE = (SA_BYTES + 127) / 128 * 128;  // TMA smem destinations: 128-B aligned
   static constexpr int STAGE_A = KPS * A_BYTES;
@@ -151,13 +161,15 @@ struct GemmCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
   static constexpr int OFF_SA = OFF_B + STAGES * STAGE_B;
-  // normal-form epilogue staging: per promotion warp two buffers of 32 rows x
-  // EPI_COLS bf16 (one tensor-store box each)
+  // normal-form epilogue staging: each promotion warp owns a bf16 image of
+  // its 32 rows x COLS columns, as COLS / 64 tensor-store boxes of 32 rows x
+  // 64 columns (128 bytes) in the 128-byte swizzled layout, so the whole
+  // slice is written in one pass and leaves with COLS / 64 stores
   static constexpr bool EPI_TMA = !SWAP && SPLIT == 1;
-  static constexpr int EPI_COLS = 16;
-  static constexpr int EPI_BUF = 32 * EPI_COLS * 2;
-  static constexpr int EPI_BYTES = EPI_TMA ? PW * 2 * EPI_BUF : 0;
-  static_assert(!EPI_TMA || COLS % EPI_COLS == 0, "epilogue rounds");
+  static constexpr int EPI_BOX = 32 * 128;  // bytes of one box
+  static constexpr int EPI_WARP = (COLS / 64) * EPI_BOX;
+  static constexpr int EPI_BYTES = EPI_TMA ? PW * EPI_WARP : 0;
+  static_assert(!EPI_TMA || COLS % 64 == 0, "epilogue boxes of 64 columns");
   static constexpr int OFF_EPI = EPI_TMA ? (OFF_SA + SAS * STAGE_SA + 1023) / 1024 * 1024
                                         : OFF_SA + SAS * STAGE_SA;
   static constexpr int OFF_RED = OFF_EPI + EPI_BYTES;
@@ -173,7 +185,7 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(SA_BYTES % 16 == 0, "TMA box inner extent");
-  static_assert(!EPI_TMA || (OFF_EPI % 1024 == 0 && EPI_BUF % 128 == 0), "tensor-store sources");
+  static_assert(!EPI_TMA || OFF_EPI % 1024 == 0, "swizzled tensor-store sources");
   static_assert(!RED_TMA || (OFF_RSTG % 128 == 0 && RSTG_BYTES % 16 == 0), "tensor-store source");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
@@ -185,16 +197,26 @@ struct Tile {
   int nt;     // weight tile
 };
 
-template <int FORM>
+template <class C, int FORM>
 __device__ __forceinline__ int total_tiles(const GemmParams& p, const int* table) {
   if (FORM == kFormMasked) return table[p.G];
+  if (C::PAIR) return (p.num_mt + 1) / 2 * p.num_nt;  // tiles of two token tiles
   return p.num_mt * p.num_nt;
 }
 
-template <int FORM>
-__device__ __forceinline__ Tile resolve_tile(const GemmParams& p, const int* table, int t) {
+// Tile t of this CTA. With pair MMA the two CTAs of a cluster walk the same
+// pair tiles; CTA `pair_rank` owns token tile 2 * (t / num_nt) + pair_rank
+// (which may lie past M: it still takes part in the MMAs and stores nothing).
+template <class C, int FORM>
+__device__ __forceinline__ Tile resolve_tile(const GemmParams& p, const int* table, int t,
+                                             int pair_rank) {
   Tile w;
-  if (FORM == kFormMasked) {
+  if (C::PAIR) {
+    w.mt = 2 * (t / p.num_nt) + pair_rank;
+    w.nt = t % p.num_nt;
+    w.e = 0;
+    w.valid = 1;
+  } else if (FORM == kFormMasked) {
     int lo = 0, hi = p.G;  // table[lo] <= t < table[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -322,12 +344,28 @@ __device__ __forceinline__ void issue_stage(int stream, const GemmParams& p, con
                                             int kb_step, uint32_t it, uint8_t* sA, uint8_t* sB,
                                             uint8_t* sSA, uint64_t* full, uint64_t* sa_full,
                                             const CUtensorMap* tmA, const CUtensorMap* tmB,
-                                            const CUtensorMap* tmSA) {
+                                            const CUtensorMap* tmSA, int pair_rank) {
   const int s = it % C::STAGES;
   const int q = it % C::SAS;
   int nvalid = 0;
 #pragma unroll
   for (int j = 0; j < C::KPS; ++j) nvalid += kq + j * kb_step < p.KB ? 1 : 0;
+  if constexpr (C::PAIR) {
+    // operand stages of both CTAs complete on the leader's barrier, which
+    // expects the bytes of both
+    if (stream < 2) {
+      const uint32_t leader_full = mapa_shared(smem_u32(&full[s]), 0);
+      if (stream == 0) {
+        if (pair_rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::B_BYTES);
+        tma_load_2d_pair(sB + s * C::STAGE_B, tmB, leader_full, kq * 128,
+                         w.e * p.N + w.nt * C::BW + pair_rank * C::B_ROWS);
+      } else {
+        if (pair_rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::A_BYTES);
+        tma_load_2d_pair(sA + s * C::STAGE_A, tmA, leader_full, kq * 128, w.mt * C::BT);
+      }
+      return;
+    }
+  }
   if (stream == 0) {
     mbar_arrive_expect_tx(&full[s], nvalid * C::B_BYTES);
     for (int j = 0; j < nvalid; ++j)
@@ -374,9 +412,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   // tiles are dealt to CTAs (or, with split-K, to clusters) round robin;
   // the K blocks of a tile to the CTAs of its cluster
-  const int t_first = C::SPLIT > 1 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
-  const int t_step = C::SPLIT > 1 ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
+  static_assert(!C::PAIR || FORM == kFormDense, "pair MMA covers the dense form");
+  const int t_first = C::CLUSTER > 1 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int t_step = C::CLUSTER > 1 ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
   const int kb_first = C::SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int pair_rank = C::PAIR ? static_cast<int>(cluster_ctarank()) : 0;
   constexpr int kb_step = C::SPLIT;
 
   if (threadIdx.x == 0) {
@@ -390,7 +430,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::PW);
+      mbar_init(&tempty[b], C::PAIR ? 2 * C::PW : C::PW);  // pair: the leader's counts both CTAs
     }
     mbar_init(red_ready, 1);                 // own expect_tx; peers' bytes complete_tx
     mbar_init(red_free, C::SPLIT * C::PW);   // one arrival per promotion warp of each CTA
@@ -402,26 +442,37 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&tmSA);
     if (C::EPI_TMA || C::RED_TMA) tma_prefetch_desc(&tmD);
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+  if constexpr (!C::PAIR) {
+    if (warp == 1) {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   // Peers address this CTA's barriers only after the cluster barrier
   // completes (its wait comes after the CTA-wide barrier below).
   __syncwarp();
-  if constexpr (C::SPLIT > 1) cluster_arrive_relaxed();
+  if constexpr (C::CLUSTER > 1) cluster_arrive_relaxed();
   // Everything above may overlap the previous kernel; memory comes after this.
   grid_dependency_wait();
   if (warp == 0) build_table<C, FORM>(p, table, lane);
   tc_fence_before();
   __syncwarp();
   __syncthreads();
-  if constexpr (C::SPLIT > 1) cluster_wait();  // peers' barriers are initialised
+  if constexpr (C::CLUSTER > 1) cluster_wait();  // peers' barriers are initialised
+  if constexpr (C::PAIR) {
+    // the pair's tensor memory, allocated jointly once both CTAs run
+    if (warp == 1) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   tc_fence_after();
 
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-  const int total = total_tiles<FORM>(p, table);
+  const int total = total_tiles<C, FORM>(p, table);
 
   if (warp < C::PW_BASE) {
   if constexpr (C::REG_SPLIT) warpgroup_reg_dealloc<C::REG_LOW>();
@@ -430,7 +481,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     if (lane < 3) {
       uint32_t it = 0;
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = resolve_tile<FORM>(p, table, t);
+        const Tile w = resolve_tile<C, FORM>(p, table, t, pair_rank);
         if (!w.valid) continue;
         for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
           if (lane < 2) {
@@ -441,7 +492,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             if (!mbar_wait(&sa_empty[q], ((it / C::SAS) & 1u) ^ 1u, ctl)) goto producer_done;
           }
           issue_stage<C, FORM>(lane, p, w, kq, kb_step, it, sA, sB, sSA, full, sa_full, &tmA, &tmB,
-                               &tmSA);
+                               &tmSA, pair_rank);
         }
       }
       // every load of this CTA is issued: the next kernel of the stream may
@@ -453,7 +504,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       if (lane == 0) {
         for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
           const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
-          drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+          // (a pair's operand bytes complete on the leader's barrier)
+          if (!C::PAIR || pair_rank == 0) drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
           drain_wait(&empty[s], (last / C::STAGES) & 1u, kDrainLimitNs);
         }
       } else if (lane == 2) {
@@ -466,11 +518,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = mma_idesc_e4m3(128, C::MMA_N);
+    if (lane == 0 && pair_rank == 0) {  // a pair's MMAs are issued by its leader
+      constexpr uint32_t idesc = mma_idesc_e4m3(C::MMA_M, C::MMA_N);
       uint32_t it = 0;
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = resolve_tile<FORM>(p, table, t);
+        const Tile w = resolve_tile<C, FORM>(p, table, t, pair_rank);
         if (!w.valid) continue;
         for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
           const int s = it % C::STAGES;
@@ -493,11 +545,19 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               // advance 32 bytes (= 32 e4m3 along K) inside the 128-byte swizzled row
-              mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+              if constexpr (C::PAIR)
+                mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+              else
+                mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
             }
           }
-          mma_commit(&empty[s]);
-          mma_commit(&tfull[b]);
+          if constexpr (C::PAIR) {
+            mma_commit_pair(&empty[s]);  // both CTAs' stage s and TMEM buffer b
+            mma_commit_pair(&tfull[b]);
+          } else {
+            mma_commit(&empty[s]);
+            mma_commit(&tfull[b]);
+          }
         }
       }
     mma_done:
@@ -515,10 +575,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     uint32_t it = 0;
     uint32_t tiles_done = 0;
-    uint32_t epi_groups = 0;  // tensor-store groups this warp has issued
     uint32_t grp_phase = 0;   // uses of the promotion group barrier
     for (int t = t_first; t < total; t += t_step) {
-      const Tile w = resolve_tile<FORM>(p, table, t);
+      const Tile w = resolve_tile<C, FORM>(p, table, t, pair_rank);
       if (!w.valid) continue;
       // row bounds of this tile's token slab (read early, used in the epilogue)
       int m_valid = p.M;
@@ -555,34 +614,35 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (!mbar_wait(&tfull[b], tph, ctl)) goto promo_done;
         tc_fence_after();
         if constexpr (!C::SWAP && C::KPS == 1 && C::COLS % 64 == 0) {
-          // normal form: 32-column TMEM loads in two alternating register
-          // sets, the next load in flight while the previous one is folded
-          // in; the TMEM buffer and the scale slot are released once the
-          // last load has completed
+          // normal form: the thread's columns in batches of 64 (two 32-column
+          // TMEM loads, one wait); the TMEM buffer and the scale slot are
+          // released as soon as the last batch is in registers, before it is
+          // folded in with packed fused multiply-adds
           const float* sa_s = reinterpret_cast<const float*>(sSA + q * C::STAGE_SA);
           const float scale = sa_s[row] * sbv[0];
           const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * C::MMA_N + c0);
-          uint32_t r0[32], r1[32];
-          tmem_ld32_issue(taddr, r0);
-          tmem_wait_ld32(r0);
 #pragma unroll
-          for (int ch = 1; ch <= C::COLS / 32; ++ch) {
-            uint32_t(&cur)[32] = (ch & 1) ? r0 : r1;   // loaded by the previous step
-            uint32_t(&nxt)[32] = (ch & 1) ? r1 : r0;
-            if (ch < C::COLS / 32) tmem_ld32_issue(taddr + 32 * ch, nxt);
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              acc[(ch - 1) * 32 + j] = fmaf(__uint_as_float(cur[j]), scale, acc[(ch - 1) * 32 + j]);
-            if (ch < C::COLS / 32) {
-              tmem_wait_ld32(nxt);
-              if (ch == C::COLS / 32 - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
+          for (int h = 0; h < C::COLS / 64; ++h) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32_issue(taddr + 64 * h, r0);
+            tmem_ld32_issue(taddr + 64 * h + 32, r1);
+            tmem_wait_ld64(r0, r1);
+            if (h == C::COLS / 64 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if constexpr (C::PAIR)  // the leader's MMA waits for both CTAs
+                  mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+                else
                   mbar_arrive(&tempty[b]);
-                  mbar_arrive(&sa_empty[q]);
-                }
+                mbar_arrive(&sa_empty[q]);
               }
+            }
+            float* a = acc + 64 * h;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              fma2(a[j], a[j + 1], __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]), scale);
+              fma2(a[32 + j], a[33 + j], __uint_as_float(r1[j]), __uint_as_float(r1[j + 1]), scale);
             }
           }
         } else {
@@ -649,7 +709,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&tempty[b]);
+          if constexpr (C::PAIR)
+            mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+          else
+            mbar_arrive(&tempty[b]);
           mbar_arrive(&sa_empty[q]);
         }
         }
@@ -670,32 +733,31 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             staged = true;
             // D rows of this warp: the slab row of its first token
             const int y = (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT + quad * 32;
-            uint8_t* bufs = smem + C::OFF_EPI + pw * 2 * C::EPI_BUF;
+            uint8_t* img = smem + C::OFF_EPI + pw * C::EPI_WARP;
+            // the stores of this warp's previous tile have read the image
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            // row `lane` of box h: 16-byte chunk c (columns h*64 + 8c ..) at
+            // chunk position c ^ (lane % 8), the tensor map's 128-byte swizzle
 #pragma unroll
-            for (int ch = 0; ch < C::COLS / C::EPI_COLS; ++ch) {
-              const int x = w.nt * C::BW + c0 + ch * C::EPI_COLS;
-              if (x >= p.N) break;  // columns past N (uniform across the warp)
-              // buffers alternate with the warp's store groups: the group
-              // issued two groups ago used this one and has read it once at
-              // most one group is pending
-              uint8_t* buf = bufs + (epi_groups & 1u) * C::EPI_BUF;
-              if (lane == 0) bulk_wait_group_read<1>();
-              __syncwarp();
-              uint32_t wv[C::EPI_COLS / 2];
+            for (int h = 0; h < C::COLS / 64; ++h) {
 #pragma unroll
-              for (int j = 0; j < C::EPI_COLS / 2; ++j)
-                wv[j] = pack_bf16x2(acc[ch * C::EPI_COLS + 2 * j], acc[ch * C::EPI_COLS + 2 * j + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(buf + lane * (C::EPI_COLS * 2));
-#pragma unroll
-              for (int j = 0; j < C::EPI_COLS / 8; ++j)
-                dst[j] = make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
-              fence_proxy_async_shared();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&tmD, buf, x, y);
-                bulk_commit_group();
+              for (int c = 0; c < 8; ++c) {
+                const float* v = acc + h * 64 + c * 8;
+                *reinterpret_cast<uint4*>(img + h * C::EPI_BOX + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
               }
-              ++epi_groups;
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll
+              for (int h = 0; h < C::COLS / 64; ++h) {
+                const int x = w.nt * C::BW + c0 + h * 64;
+                if (x < p.N) tma_store_2d(&tmD, img + h * C::EPI_BOX, x, y);  // columns past N clipped
+              }
+              bulk_commit_group();
             }
           }
         }
@@ -835,8 +897,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   tc_fence_before();
   // No CTA may leave while a peer can still write its shared memory; the
   // cluster barrier covers every thread of the CTA as well.
-  if constexpr (C::SPLIT > 1) {
-    // every CTA arrives only after all bytes sent to it have landed, so when
+  if constexpr (C::CLUSTER > 1) {
+    // every CTA arrives only after all bytes sent to it have landed (split-K)
+    // or all MMAs writing its tensor memory have completed (pair), so when
     // the barrier completes no transfer reads or writes any CTA's memory
     cluster_arrive_relaxed();
     cluster_wait();
@@ -846,7 +909,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   grid_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (C::PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
