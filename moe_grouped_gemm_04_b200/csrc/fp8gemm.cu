@@ -261,6 +261,7 @@ Plan plan_for(const Problem& pr, int sm_count, int expected_m) {
 template <class C, int FORM>
 fg_status launch_gemm(const Problem& pr, const Plan& pl, const DeviceInfo& dev, int dev_id,
                       cudaStream_t stream) {
+  static_assert(C::smem_bytes(FORM) <= 232448, "shared memory per CTA");
   KernelInfo* ki = nullptr;
   FG_TRY((kernel_info<C, FORM>(dev_id, &ki)));
   const int KB = pr.K / 128;
@@ -336,6 +337,8 @@ template <int FORM>
 fg_status dispatch(const Problem& pr, const Plan& pl, const DeviceInfo& dev, int dev_id,
                    cudaStream_t stream) {
   if (pl.bt == 128) {
+    // dense: CTA pairs; grouped forms: single-CTA tiles, which are as fast
+    // once promotion is the limit and keep groups 128-row aligned
     if constexpr (FORM == kFormDense) return launch_gemm<CfgPair, FORM>(pr, pl, dev, dev_id, stream);
     return launch_gemm<CfgNormal, FORM>(pr, pl, dev, dev_id, stream);
   }
@@ -444,8 +447,11 @@ fg_status per_token_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfa, int n
   DeviceInfo* dev = nullptr;
   FG_TRY(device_info(&dev));
   const int64_t slices = static_cast<int64_t>(num_groups) * M * (K / 128);
+  if (slices >= (int64_t(1) << 31)) return fail(FG_ERR_UNSUPPORTED, "too many 128-element slices");
+  // one pass for small inputs (latency); up to QUNROLL slice pairs per warp
+  // and pass for large ones (several loads in flight per thread)
   const int64_t blocks_needed = (slices * 16 + 255) / 256;
-  const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, int64_t(dev->sm_count) * 16));
+  const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, int64_t(dev->sm_count) * 8));
   const cudaError_t e = launch_pdl(per_token_cast_kernel, dim3(grid), dim3(256), stream, x, q, sfa,
                                    num_groups, M, K, sfa_stride(M));
   if (e != cudaSuccess) return cuda_fail(e, "per_token_cast_kernel launch");

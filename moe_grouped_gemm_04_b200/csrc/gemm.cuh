@@ -179,15 +179,14 @@ struct GemmCfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
   // the tile table exists for the grouped forms only; + alignment slack
-  static constexpr int smem_bytes(int form) {
-    return OFF_TABLE + (form == kFormDense ? 0 : kTableMax * 4) + 1024;
-  }
-  static constexpr int SMEM_BYTES = OFF_TABLE + kTableMax * 4 + 1024;
+  static constexpr int table_bytes(int form) { return form == kFormDense ? 0 : kTableMax * 4; }
+  static constexpr int smem_bytes(int form) { return OFF_TABLE + table_bytes(form) + 1024; }
+
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(SA_BYTES % 16 == 0, "TMA box inner extent");
   static_assert(!EPI_TMA || OFF_EPI % 1024 == 0, "swizzled tensor-store sources");
   static_assert(!RED_TMA || (OFF_RSTG % 128 == 0 && RSTG_BYTES % 16 == 0), "tensor-store source");
-  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(smem_bytes(kFormDense) <= 232448, "shared memory per CTA");
 };
 
 struct Tile {

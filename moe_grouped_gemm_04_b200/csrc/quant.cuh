@@ -54,7 +54,13 @@ __device__ __forceinline__ float amax8(uint4 w) {
 
 // One 128-element slice per 16 consecutive threads (8 elements each).
 // Slices are enumerated with the token index fastest so that consecutive
-// slices write consecutive scale entries of the MN-major layout.
+// slices write consecutive scale entries of the MN-major layout. A warp
+// covers two adjacent slices and takes QUNROLL such pairs a grid stride apart,
+// issuing all their loads before using any, so that several 16-byte loads per
+// thread are in flight. The host keeps the slice count below 2^31 (32-bit
+// index arithmetic).
+constexpr int QUNROLL = 4;
+
 __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __restrict__ x,
                                                              uint8_t* __restrict__ q,
                                                              float* __restrict__ sfa, int G,
@@ -63,25 +69,41 @@ __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __r
   // before touching memory
   grid_launch_dependents();
   grid_dependency_wait();
-  const int KB = K / 128;
-  const int64_t slices = static_cast<int64_t>(G) * KB * M;
+  const uint32_t KB = static_cast<uint32_t>(K / 128);
+  const uint32_t slices = static_cast<uint32_t>(G) * KB * static_cast<uint32_t>(M);
   const int sub = threadIdx.x & 15;
-  const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-  const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-  for (int64_t s = first; s < slices; s += step) {
-    const int m = static_cast<int>(s % M);
-    const int64_t gk = s / M;  // g * KB + kb
-    const int kb = static_cast<int>(gk % KB);
-    const int64_t g = gk / KB;
-    const int64_t off = ((g * M + m) * K) + static_cast<int64_t>(kb) * 128 + sub * 8;
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + off));
-    float a = amax8(w);
+  const uint32_t half = (threadIdx.x >> 4) & 1;  // which slice of the warp's pair
+  // the loop bound is uniform across a warp (the shuffles below need every
+  // lane); each warp takes the slice pairs base, base + step, ...
+  const uint32_t base0 = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 2;
+  const uint32_t step = ((gridDim.x * blockDim.x) >> 5) * 2;
+  for (uint32_t b0 = base0; b0 < slices; b0 += QUNROLL * step) {
+    uint4 w[QUNROLL];
+    int64_t off[QUNROLL];
+    uint32_t m[QUNROLL], gk[QUNROLL];
+    bool ok[QUNROLL];
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float amx = fmaxf(a, kAmaxFloor);
-    const float inv = __fdiv_rn(kFp8Max, amx);
-    *reinterpret_cast<uint2*>(q + off) = quantize8(w, inv);
-    if (sub == 0) sfa[gk * stride + m] = __fdiv_rn(amx, kFp8Max);
+    for (int u = 0; u < QUNROLL; ++u) {
+      const uint32_t s = b0 + u * step + half;
+      ok[u] = s < slices;
+      m[u] = s % static_cast<uint32_t>(M);
+      gk[u] = s / static_cast<uint32_t>(M);  // g * KB + kb
+      const uint32_t g = gk[u] / KB, kb = gk[u] % KB;
+      off[u] = (static_cast<int64_t>(g) * M + m[u]) * K + kb * 128 + sub * 8;
+      w[u] = ok[u] ? __ldg(reinterpret_cast<const uint4*>(x + off[u])) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < QUNROLL; ++u) {
+      float a = amax8(w[u]);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if (ok[u]) {
+        const float amx = fmaxf(a, kAmaxFloor);
+        const float inv = __fdiv_rn(kFp8Max, amx);
+        *reinterpret_cast<uint2*>(q + off[u]) = quantize8(w[u], inv);
+        if (sub == 0) sfa[static_cast<int64_t>(gk[u]) * stride + m[u]] = __fdiv_rn(amx, kFp8Max);
+      }
+    }
   }
 }
 
