@@ -94,13 +94,20 @@ def _ptr(t: Optional[torch.Tensor]):
         raise FP8GemmError(FG_ERR_INVALID_ARG, "tensor must live on a CUDA device")
     if not t.is_contiguous():
         raise FP8GemmError(FG_ERR_INVALID_ARG, "tensor must be contiguous")
-    return ctypes.c_void_p(t.data_ptr())
+    return t.data_ptr()  # c_void_p argtypes take the integer address
 
 
-def _stream(stream) -> ctypes.c_void_p:
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+# The raw handle of torch's current stream, read without building a Stream
+# object (which costs several microseconds per call).
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 # ---------------------------------------------------------------- layouts
