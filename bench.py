@@ -234,6 +234,17 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
     return flops / dt, desc, dt
 
 
+# ---------------------------------------------------------------------- ranks
+
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of `values` (floats) over all ranks of the
+    process group: the job's time is its slowest rank's."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # ---------------------------------------------------------------------- GPU leg
 
 class OperandSet:
@@ -485,11 +496,9 @@ def run_ours(args, rank, world, local_rank):
 
     # max over ranks
     if dist is not None:
-        t = torch.tensor([ms, gms, e2e["ms"] if e2e else 0.0], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, gms = float(t[0]), float(t[1])
+        ms, gms, e2e_max = max_over_ranks(dist, [ms, gms, e2e["ms"] if e2e else 0.0], "cuda")
         if e2e:
-            e2e["ms"] = float(t[2])
+            e2e["ms"] = e2e_max
 
     if rank != 0:
         return None
