@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
     lib.oracle_e4m3_encode_array.restype = None
     lib.oracle_per_token_cast.argtypes = [P, P, P, I, I, I, I]
     lib.oracle_per_block_cast.argtypes = [P, P, P, I, I, I, I]
+    lib.oracle_per_block_dequant.argtypes = [P, P, P, I, I, I, I]
     lib.oracle_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, I]
     lib.oracle_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
     lib.oracle_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
@@ -124,6 +125,23 @@ def per_block_cast(x_bf16: np.ndarray, threads: int = 0):
     _check(_load().oracle_per_block_cast(_ptr(x), _ptr(q), _ptr(s), G, N, K, threads),
            "per_block_cast")
     return (q[0], s[0]) if squeeze else (q, s)
+
+
+def per_block_dequant(q: np.ndarray, s: np.ndarray, threads: int = 0) -> np.ndarray:
+    """codes [N][K] or [G][N][K] with scales [..., ceil(N/128), K/128] -> bf16 bits like q:
+    bf16(fp32(e4m3(q) * s)), both roundings to nearest even."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    squeeze = q.ndim == 2
+    if squeeze:
+        q, s = q[None], s[None]
+    G, N, K = q.shape
+    if s.shape != (G, -(-N // BLOCK), K // BLOCK):
+        raise ValueError("scale shape %s does not match codes %s" % (s.shape, q.shape))
+    x = np.empty(q.shape, dtype=np.uint16)
+    _check(_load().oracle_per_block_dequant(_ptr(q), _ptr(s), _ptr(x), G, N, K, threads),
+           "per_block_dequant")
+    return x[0] if squeeze else x
 
 
 def gemm_nt(qa, sa, qb, sb, threads: int = 0) -> np.ndarray:

@@ -342,3 +342,81 @@ def test_points_equal_full_gemm():
 def test_oracle_rejects_bad_sizes():
     with pytest.raises(ValueError):
         oracle.per_token_cast(np.zeros((4, 100), np.uint16))
+
+
+# ---------------------------------------------------------------- weight dequantization
+
+def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _block_scales(s: np.ndarray, N: int) -> np.ndarray:
+    """[G][NB][KB] block scales expanded to [G][N][K]."""
+    return np.repeat(np.repeat(s, 128, axis=1)[:, :N], 128, axis=2)
+
+
+def _finite_codes(rng, shape):
+    q = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x00
+    return q
+
+
+def test_dequant_power_of_two_scales_exact():
+    """Power-of-two scales: product and bf16 rounding are exact, so every
+    output is the code's value (torch's independent decoder) times the scale
+    of its 128x128 block. N = 200 has a ragged last block; two groups."""
+    rng = np.random.default_rng(3)
+    G, N, K = 2, 200, 256
+    q = _finite_codes(rng, (G, N, K))
+    s = np.ldexp(1.0, rng.integers(-8, 8, size=(G, 2, 2))).astype(np.float32)
+    got = _bf16_to_f64(oracle.per_block_dequant(q, s))
+    assert np.array_equal(got, torch_decode(q) * _block_scales(s, N))
+
+
+def test_dequant_matches_torch_casts():
+    """General fp32 scales: torch's float8 decode, one float32 multiply and
+    torch's round-to-nearest-even bfloat16 cast give the same bits."""
+    rng = np.random.default_rng(4)
+    G, N, K = 1, 300, 384
+    q = _finite_codes(rng, (G, N, K))
+    s = (rng.random((G, 3, 3)) * 0.01 + 1e-4).astype(np.float32)
+    dec = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float32)
+    want = (dec * torch.from_numpy(_block_scales(s, N).astype(np.float32))).to(torch.bfloat16)
+    got = oracle.per_block_dequant(q, s)
+    assert np.array_equal(got, want.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_dequant_block_indexing():
+    """Every code 1.0 and a distinct power-of-two scale per block: each output
+    equals its own block's scale (a swapped or shifted block index fails)."""
+    G, N, K = 2, 300, 384
+    q = np.full((G, N, K), 0x38, np.uint8)
+    s = np.ldexp(1.0, np.arange(G * 3 * 3).reshape(G, 3, 3) - 9).astype(np.float32)
+    got = _bf16_to_f64(oracle.per_block_dequant(q, s))
+    for g in range(G):
+        for nb in range(3):
+            for kb in range(3):
+                blk = got[g, nb * 128:min(N, nb * 128 + 128), kb * 128:kb * 128 + 128]
+                assert np.all(blk == float(s[g, nb, kb]))
+
+
+def test_dequant_inverts_quantizer():
+    """dequant(per_block_cast(x)) is within half an e4m3 unit of x (relative
+    2^-4, or 2^-10 * s in the subnormal range) plus the bf16 rounding."""
+    rng = np.random.default_rng(5)
+    x = workloads.bf16_bits(rng.standard_normal((300, 512), dtype=np.float32) * 0.02)
+    q, s = oracle.per_block_cast(x)
+    y = _bf16_to_f64(oracle.per_block_dequant(q, s))
+    xv = _bf16_to_f64(x)
+    sf = _block_scales(s[None], 300)[0].astype(np.float64)
+    bound = 2.0 ** -4 * np.abs(xv) + 2.0 ** -10 * sf + 2.0 ** -8 * np.abs(y)
+    assert np.all(np.abs(xv - y) <= bound)
+
+
+def test_dequant_nan_code_gives_nan():
+    q = np.zeros((128, 128), np.uint8)
+    q[3, 5], q[7, 9] = 0x7F, 0xFF
+    y = _bf16_to_f64(oracle.per_block_dequant(q, np.ones((1, 1), np.float32)))
+    assert np.isnan(y[3, 5]) and np.isnan(y[7, 9])
+    assert np.count_nonzero(np.isnan(y)) == 2
