@@ -561,6 +561,111 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+DEQUANT_METRIC = "FP8 weight dequantization (e4m3 + 128x128 scales -> bf16) GB/s (device-timed)"
+
+
+def run_dequant(args, rank, world, local_rank):
+    """The weight dequantizer alone: codes and block scales (quantized once on
+    the GPU) -> bf16, on operand sets whose total exceeds L2, used in turn,
+    K launches replayed from one CUDA graph between one pair of events."""
+    import torch
+
+    import moe_grouped_gemm_04_b200 as fg
+
+    torch.cuda.set_device(local_rank)
+    fg.load_library()
+    inp = workloads.make(args.workload, seed=0)
+    N, K = inp.N, inp.K
+    _, alg_bytes = workloads.flops_and_bytes("dequant", inp)
+    w = torch.from_numpy(np.ascontiguousarray(inp.b).view(np.int16)).cuda().view(torch.bfloat16)
+    q0 = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    s0 = fg.empty_sfb(1, N, K, "cuda")
+    fg.per_block_cast_to_fp8(w, q0, s0)
+    per = int(alg_bytes)
+    R = max(2, -(-ROTATE_MIN_BYTES // per))
+    sets = [(q0.clone(), s0.clone(), torch.empty((N, K), dtype=torch.bfloat16, device="cuda"))
+            for _ in range(R)]
+
+    def launch(i):
+        q, sc, x = sets[i % R]
+        fg.per_block_dequant_to_bf16(q, sc, x)
+
+    for i in range(max(args.warmup, R)):
+        launch(i)
+    torch.cuda.synchronize()
+    steps = args.steps
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for i in range(steps):
+            launch(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    clocks = sampler.stop()
+    # the timed launches did the work: the last output equals a fresh call
+    last = sets[(steps - 1) % R]
+    timed_x = last[2].clone()
+    last[2].view(torch.int16).fill_(SENTINEL_BF16)
+    launch(steps - 1)
+    torch.cuda.synchronize()
+    assert torch.equal(timed_x.view(torch.int16), last[2].view(torch.int16)), "timed output differs"
+    if world > 1:
+        import torch.distributed as dist
+        ms = max_over_ranks(dist, [ms], "cuda")[0]
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = dequant_cpu_sample(inp, args.cpu_seconds)
+    return {
+        "metric": DEQUANT_METRIC, "value": world * gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3->bf16",
+        "data": "synthetic (seeded numpy, random weights)",
+        "config": {"workload": args.workload, "kind": "dequant", "N": N, "K": K,
+                   "l2": "inputs larger than L2: %d operand sets of %.1f MB used in turn" % (R, per / 1e6),
+                   "launch": "K launches captured in one CUDA graph, replayed once untimed, then timed"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "per_block_dequant_kernel", "kernel_ms": ms,
+                     "algorithmic_per_launch": {"bytes": alg_bytes},
+                     "peak_source": "%s HBM copy bandwidth" % peak_src},
+        "cpu_baseline": cpu, "gpu_launches": steps, "clocks": clocks, "e2e": None,
+    }
+
+
+def dequant_cpu_sample(inp, target_s: float):
+    """The oracle's dequantizer on a bounded sample of rows of the same weight."""
+    import oracle
+    threads = oracle.hardware_threads()
+    q, s = oracle.per_block_cast(inp.b, threads=threads)
+    rows = 128
+    while True:
+        t0 = time.perf_counter()
+        oracle.per_block_dequant(q[:rows], s[:-(-rows // 128)], threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= 0.3 * target_s or rows >= inp.N:
+            break
+        rows = min(inp.N, rows * 2)
+    byts = rows * inp.K * 3 + 4 * (-(-rows // 128)) * (inp.K // 128)
+    return {"value": byts / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d rows x K=%d" % (rows, inp.N, inp.K), "seconds": dt}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm, on rank 0 only."""
     if rank != 0:
@@ -598,7 +703,18 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
+    if args.impl == "reference" and workloads.WORKLOADS[args.workload][0] == "dequant":
+        out = None
+        if rank == 0:
+            cpu = dequant_cpu_sample(workloads.make(args.workload, seed=0), min(args.cpu_seconds, 5.0))
+            out = {"impl": "reference", "metric": DEQUANT_METRIC, "value": cpu["value"], "unit": "GB/s",
+                   "n_gpus": world, "steps": 1, "warmup": 0, "higher_is_better": True,
+                   "scaling": "weak", "vs_baseline": None, "dtype": "f32->bf16",
+                   "data": "synthetic (seeded numpy)", "config": {"workload": args.workload},
+                   "cpu_baseline": cpu,
+                   "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}}
+    elif args.impl == "reference":
         out = run_reference(args, rank, world)
     else:
         if world > 1:
@@ -610,7 +726,10 @@ def main():
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                     device_id=torch.device("cuda", local_rank))
         try:
-            out = run_ours(args, rank, world, local_rank)
+            if workloads.WORKLOADS[args.workload][0] == "dequant":
+                out = run_dequant(args, rank, world, local_rank)
+            else:
+                out = run_ours(args, rank, world, local_rank)
         finally:
             if world > 1:
                 import torch.distributed as dist

@@ -107,6 +107,19 @@ fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int n
                                 int N, int K, cudaStream_t stream);
 
 /*
+ * Weight dequantization, the third kernel of the FP8 quantize / dequantize /
+ * GEMM trio (DeepSeek-V3 review "28.5 倍压缩 + 1/10 成本", "创新之处" item 4
+ * and "可复用的模式与技巧" item 3). For every group g, row n and column k:
+ *   x[g][n][k] = bf16( fp32( e4m3(q[g][n][k]) * sfb[g][n/128][k/128] ) )
+ * the fp32 product and the bf16 conversion both round to nearest even; NaN
+ * codes give NaN. q: e4m3 [num_groups][N][K]; sfb: fp32
+ * [num_groups][ceil(N/128)][K/128] (the layout per_block_cast_to_fp8 writes);
+ * x: bf16 [num_groups][N][K]. K % 128 == 0, N >= 1, num_groups >= 1.
+ */
+fg_status per_block_dequant_to_bf16(const uint8_t* q, const float* sfb, uint16_t* x,
+                                    int num_groups, int N, int K, cudaStream_t stream);
+
+/*
  * Dense FP8 GEMM, "NT": D[m][n] = sum_kb sa[m][kb] * sb[n/128][kb] *
  *   sum_{k in kb} e4m3(A[m][k]) * e4m3(B[n][k]), rounded once to bf16.
  * A: e4m3 [M][K] (row-major, K contiguous); sfa: MN-major [K/128][stride(M)];

@@ -8,8 +8,8 @@ fallback: if the library is missing or the device is not sm_100a, every call
 raises.
 
 The functions carry the C names:
-  per_token_cast_to_fp8, per_block_cast_to_fp8, fp8_gemm_nt,
-  fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked
+  per_token_cast_to_fp8, per_block_cast_to_fp8, per_block_dequant_to_bf16,
+  fp8_gemm_nt, fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked
 plus allocation helpers that return tensors in the layouts the kernels use.
 """
 from __future__ import annotations
@@ -31,7 +31,8 @@ FG_ERR_DEVICE = 4
 
 EXPORTED = (
     "fg_sfa_stride", "per_token_cast_to_fp8", "per_block_cast_to_fp8", "fp8_gemm_nt",
-    "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
+    "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
+    "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
 
 
@@ -59,6 +60,7 @@ def load_library() -> ctypes.CDLL:
     lib.fg_sfa_stride.restype = I
     lib.per_token_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
     lib.per_block_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
+    lib.per_block_dequant_to_bf16.argtypes = [P, P, P, I, I, I, P]
     lib.fp8_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, P]
     lib.fp8_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fp8_grouped_gemm_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
@@ -68,7 +70,8 @@ def load_library() -> ctypes.CDLL:
     lib.fg_status_string.restype = ctypes.c_char_p
     lib.fg_last_error.argtypes = []
     lib.fg_last_error.restype = ctypes.c_char_p
-    for f in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "fp8_gemm_nt",
+    for f in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "per_block_dequant_to_bf16",
+              "fp8_gemm_nt",
               "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
@@ -151,6 +154,18 @@ def per_block_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfb: torch.Tensor,
         raise FP8GemmError(FG_ERR_INVALID_ARG, "output sizes do not match x")
     _check(load_library().per_block_cast_to_fp8(_ptr(x), _ptr(q), _ptr(sfb), G, N, K,
                                                 _stream(stream)))
+
+
+def per_block_dequant_to_bf16(q: torch.Tensor, sfb: torch.Tensor, x: torch.Tensor,
+                              stream=None) -> None:
+    """q uint8 [N][K] or [G][N][K], sfb [G][ceil(N/128)][K/128] -> x bf16 (shape of q)."""
+    G, N, K = (1, *q.shape) if q.dim() == 2 else tuple(q.shape)
+    if q.dtype != torch.uint8 or x.dtype != torch.bfloat16 or sfb.dtype != torch.float32:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "dtypes: q uint8, sfb float32, x bf16")
+    if x.numel() != q.numel() or sfb.numel() < G * (-(-N // 128)) * (K // 128):
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "sizes of sfb or x do not match q")
+    _check(load_library().per_block_dequant_to_bf16(_ptr(q), _ptr(sfb), _ptr(x), G, N, K,
+                                                    _stream(stream)))
 
 
 def fp8_gemm_nt(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor, sfb: torch.Tensor,

@@ -519,6 +519,24 @@ fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int n
   return FG_OK;
 }
 
+fg_status per_block_dequant_to_bf16(const uint8_t* q, const float* sfb, uint16_t* x,
+                                    int num_groups, int N, int K, cudaStream_t stream) {
+  if (num_groups < 1) return fail(FG_ERR_INVALID_ARG, "num_groups=%d must be >= 1", num_groups);
+  if (N <= 0) return fail(FG_ERR_INVALID_ARG, "N=%d must be >= 1", N);
+  if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
+  FG_TRY(check_ptr(q, "q"));
+  FG_TRY(check_ptr(sfb, "sfb"));
+  FG_TRY(check_ptr(x, "x"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  const int64_t chunks = static_cast<int64_t>(num_groups) * N * (K / 16);
+  const int grid = static_cast<int>(std::min<int64_t>((chunks + 255) / 256, int64_t(dev->sm_count) * 8));
+  const cudaError_t e = launch_pdl(per_block_dequant_kernel, dim3(grid), dim3(256), stream, q, sfb, x,
+                                   num_groups, N, K);
+  if (e != cudaSuccess) return cuda_fail(e, "per_block_dequant_kernel launch");
+  return FG_OK;
+}
+
 fg_status fp8_gemm_nt(const uint8_t* A, const float* sfa, const uint8_t* B, const float* sfb,
                       uint16_t* D, int M, int N, int K, cudaStream_t stream) {
   if (M < 0) return fail(FG_ERR_INVALID_ARG, "M=%d must be >= 0", M);

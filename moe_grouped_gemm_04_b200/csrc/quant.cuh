@@ -14,6 +14,9 @@
 // "风险与不足" item 6 (the 448.0 bound).
 #pragma once
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -155,6 +158,50 @@ __global__ void __launch_bounds__(256) per_block_cast_kernel(const uint16_t* __r
     }
   }
   if (threadIdx.x == 0) sfb[blk] = __fdiv_rn(amx, kFp8Max);
+}
+
+// Weight dequantization, the third kernel of the FP8 trio (quantize,
+// dequantize, GEMM) the DeepSeek-V3 review describes ("创新之处" item 4):
+//   x = bf16(fp32(e4m3(q) * s)), s the fp32 scale of q's 128x128 block,
+// both roundings to nearest even (e4m3 -> half -> float is exact). HBM-bound:
+// 1 byte read and 2 written per element. A thread converts 16 consecutive
+// codes of one row (K % 128 == 0 keeps them inside one block): one 16-byte
+// load, two 16-byte stores (one chunk per thread and pass measured faster
+// than several loads in flight with fewer threads).
+__global__ void __launch_bounds__(256) per_block_dequant_kernel(const uint8_t* __restrict__ q,
+                                                                const float* __restrict__ sfb,
+                                                                uint16_t* __restrict__ x, int G,
+                                                                int N, int K) {
+  grid_launch_dependents();
+  grid_dependency_wait();
+  const int KB = K / 128;
+  const int NB = (N + 127) / 128;
+  const int64_t chunks = static_cast<int64_t>(G) * N * (K / 16);
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < chunks;
+       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t off = c * 16;
+    const int64_t row = off / K;  // g * N + n
+    const int k = static_cast<int>(off - row * K);
+    const int64_t g = row / N;
+    const int n = static_cast<int>(row - g * N);
+    const float sc = __ldg(sfb + (g * NB + n / 128) * KB + k / 128);
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(q + off));
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t out[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // codes 2i (low byte) and 2i + 1
+      const __nv_fp8x2_storage_t pair =
+          static_cast<__nv_fp8x2_storage_t>((in[i / 2] >> (16 * (i % 2))) & 0xFFFFu);
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float lo = __half2float(__ushort_as_half(h.x));
+      const float hi = __half2float(__ushort_as_half(h.y));
+      out[i] = pack_bf16x2(__fmul_rn(lo, sc), __fmul_rn(hi, sc));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(x + off);
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
 }
 
 }  // namespace fg

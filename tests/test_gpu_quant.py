@@ -122,3 +122,37 @@ def test_quantizer_argument_errors(fg):
     with pytest.raises(fg.FP8GemmError) as ei:
         fg.per_token_cast_to_fp8(x, q, s)
     assert ei.value.status == fg.FG_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- weight dequantization
+
+def gpu_dequant(fg, q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    qt = torch.from_numpy(np.ascontiguousarray(q)).cuda()
+    st = torch.from_numpy(np.ascontiguousarray(s, np.float32)).cuda()
+    x = torch.full(q.shape, -1.0, dtype=torch.bfloat16, device="cuda")
+    fg.per_block_dequant_to_bf16(qt, st, x)
+    torch.cuda.synchronize()
+    return x.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("G,N,K", [(1, 256, 512), (2, 300, 384), (1, 2112, 768), (3, 64, 128)])
+def test_per_block_dequant_bit_exact(fg, G, N, K):
+    """Every finite code and scale bit pattern of the oracle's result."""
+    rng = np.random.default_rng(N + K + G)
+    q = rng.integers(0, 256, size=(G, N, K), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x41
+    s = (rng.random((G, -(-N // 128), K // 128)) * 0.02 + 1e-5).astype(np.float32)
+    assert np.array_equal(gpu_dequant(fg, q, s), oracle.per_block_dequant(q, s))
+
+
+def test_per_block_dequant_round_trip_on_device(fg):
+    """Weights quantized and dequantized on the GPU equal the oracle's chain;
+    NaN codes come back as NaN."""
+    rng = np.random.default_rng(21)
+    bits = workloads.bf16_bits(rng.standard_normal((2, 2112, 512), dtype=np.float32) * 0.02)
+    q, s = gpu_per_block(fg, bits)
+    got = gpu_dequant(fg, q, s)
+    assert np.array_equal(got, oracle.per_block_dequant(*oracle.per_block_cast(bits)))
+    q[0, 7, 3] = 0x7F
+    nan = gpu_dequant(fg, q, s)
+    assert (nan[0, 7, 3] & 0x7F80) == 0x7F80 and (nan[0, 7, 3] & 0x007F) != 0

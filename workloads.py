@@ -163,6 +163,17 @@ def contiguous(N: int, K: int, counts: Optional[np.ndarray] = None, G: int = 8,
                             M_total=M_total, N=N, K=K, G=G)
 
 
+@dataclasses.dataclass
+class DequantInputs:
+    b: np.ndarray  # bf16 bits [N][K] (quantized once, then dequantized)
+    N: int
+    K: int
+
+
+def dequant(N: int, K: int, seed: int = 0, b_std: float = 0.02) -> DequantInputs:
+    return DequantInputs(b=normal_bf16(np.random.default_rng(seed + 1), (N, K), b_std), N=N, K=K)
+
+
 def masked(G: int, M_max: int, N: int, K: int, seed: int = 0,
            masked_m: Optional[np.ndarray] = None, a_std: float = 1.0,
            b_std: float = 0.02) -> MaskedInputs:
@@ -182,6 +193,8 @@ WORKLOADS = {
     "prefill_4096x2112x7168": ("dense", dict(M=4096, N=2112, K=7168)),
     "contiguous_8x4096x7168": ("contiguous", dict(N=4096, K=7168, G=8)),
     "masked_32x256x4096x7168": ("masked", dict(G=32, M_max=256, N=4096, K=7168)),
+    # weight dequantization (e4m3 + 128x128 scales -> bf16) of a prefill weight
+    "dequant_7168x2048": ("dequant", dict(N=7168, K=2048)),
 }
 
 
@@ -191,11 +204,14 @@ def make(name: str, seed: int = 0):
         return dense(seed=seed, **kw)
     if kind == "contiguous":
         return contiguous(seed=seed, **kw)
+    if kind == "dequant":
+        return dequant(seed=seed, **kw)
     return masked(seed=seed, **kw)
 
 
 def flops_and_bytes(kind: str, inp) -> tuple:
-    """Algorithmic FLOPs and HBM bytes of one GEMM call (valid rows only).
+    """Algorithmic FLOPs and HBM bytes of one GEMM call (valid rows only), or of
+    one weight dequantization (bytes only).
 
     FLOPs = 2 * M_valid * N * K. Bytes = A (1 B/elt) + its fp32 scales (one per
     128 elements) + B (1 B/elt) and its fp32 scales (one per 128x128 block) for
@@ -204,6 +220,8 @@ def flops_and_bytes(kind: str, inp) -> tuple:
     N, K = inp.N, inp.K
     nb = -(-N // 128)
     kb = K // 128
+    if kind == "dequant":  # no FLOPs; codes and scales read, bf16 written
+        return 0.0, float(N * K + 4 * nb * kb + 2 * N * K)
     if kind == "dense":
         mv, experts = inp.M, 1
     elif kind == "contiguous":
