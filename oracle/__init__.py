@@ -53,8 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_e4m3_encode_array.argtypes = [P, P, I64]
     lib.oracle_e4m3_encode_array.restype = None
-    lib.oracle_per_token_cast.argtypes = [P, P, P, I, I, I, I]
-    lib.oracle_per_block_cast.argtypes = [P, P, P, I, I, I, I]
+    lib.oracle_per_token_cast.argtypes = [P, P, P, I, I, I, I, I]
+    lib.oracle_per_block_cast.argtypes = [P, P, P, I, I, I, I, I]
     lib.oracle_per_block_dequant.argtypes = [P, P, P, I, I, I, I]
     lib.oracle_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, I]
     lib.oracle_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
@@ -98,8 +98,9 @@ def e4m3_encode(values) -> np.ndarray:
     return out
 
 
-def per_token_cast(x_bf16: np.ndarray, threads: int = 0):
-    """x: bf16 bits [M][K] or [G][M][K] -> (codes like x, scales [..., M, K/128])."""
+def per_token_cast(x_bf16: np.ndarray, threads: int = 0, ue8m0: bool = False):
+    """x: bf16 bits [M][K] or [G][M][K] -> (codes like x, scales [..., M, K/128]).
+    ue8m0: scales rounded up to powers of two (codes of x / s)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     squeeze = x.ndim == 2
     if squeeze:
@@ -107,13 +108,14 @@ def per_token_cast(x_bf16: np.ndarray, threads: int = 0):
     G, M, K = x.shape
     q = np.empty(x.shape, dtype=np.uint8)
     s = np.empty((G, M, K // BLOCK), dtype=np.float32)
-    _check(_load().oracle_per_token_cast(_ptr(x), _ptr(q), _ptr(s), G, M, K, threads),
-           "per_token_cast")
+    _check(_load().oracle_per_token_cast(_ptr(x), _ptr(q), _ptr(s), G, M, K, threads,
+                                         int(ue8m0)), "per_token_cast")
     return (q[0], s[0]) if squeeze else (q, s)
 
 
-def per_block_cast(x_bf16: np.ndarray, threads: int = 0):
-    """x: bf16 bits [N][K] or [G][N][K] -> (codes like x, scales [..., ceil(N/128), K/128])."""
+def per_block_cast(x_bf16: np.ndarray, threads: int = 0, ue8m0: bool = False):
+    """x: bf16 bits [N][K] or [G][N][K] -> (codes like x, scales [..., ceil(N/128), K/128]).
+    ue8m0: scales rounded up to powers of two (codes of x / s)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     squeeze = x.ndim == 2
     if squeeze:
@@ -122,8 +124,8 @@ def per_block_cast(x_bf16: np.ndarray, threads: int = 0):
     NB = -(-N // BLOCK)
     q = np.empty(x.shape, dtype=np.uint8)
     s = np.empty((G, NB, K // BLOCK), dtype=np.float32)
-    _check(_load().oracle_per_block_cast(_ptr(x), _ptr(q), _ptr(s), G, N, K, threads),
-           "per_block_cast")
+    _check(_load().oracle_per_block_cast(_ptr(x), _ptr(q), _ptr(s), G, N, K, threads,
+                                         int(ue8m0)), "per_block_cast")
     return (q[0], s[0]) if squeeze else (q, s)
 
 

@@ -109,15 +109,38 @@ float bf16_to_float(uint16_t b) {
   return f;
 }
 
+// Smallest power of two >= r, for a positive normal float r: 2^E if r is
+// exactly 2^E (zero mantissa field), else 2^(E+1).
+float pow2_ceil(float r) {
+  uint32_t u;
+  std::memcpy(&u, &r, sizeof u);
+  uint32_t e = (u >> 23) & 0xFFu;
+  if ((u & 0x007FFFFFu) != 0) e += 1;
+  const uint32_t v = e << 23;
+  float out;
+  std::memcpy(&out, &v, sizeof out);
+  return out;
+}
+
 // One scaling group: amax -> scale -> codes. `vals` holds the group's
 // elements (already widened from bf16, which is exact).
-float quantize_group(const std::vector<float>& vals, std::vector<uint8_t>& codes) {
+// ue8m0 = 0: s = amax_c / 448, codes of x * (448 / amax_c) (one fp32 rounding).
+// ue8m0 = 1 (the power-of-two scales of the DeepSeek-V3 review, "创新之处"
+// item 4: UE8M0 scales are powers of two): s = the smallest power of two at
+// or above amax_c / 448, codes of x / s (exact: s is a power of two), so no
+// element exceeds 448 before rounding.
+float quantize_group(const std::vector<float>& vals, std::vector<uint8_t>& codes, int ue8m0) {
   float amax = 0.0f;
   for (float x : vals) amax = std::max(amax, std::fabs(x));
   const float amax_c = std::max(amax, 1e-4f);
+  codes.resize(vals.size());
+  if (ue8m0) {
+    const float scale = pow2_ceil(amax_c / 448.0f);
+    for (size_t i = 0; i < vals.size(); ++i) codes[i] = encode(vals[i] / scale);
+    return scale;
+  }
   const float scale = amax_c / 448.0f;
   const float inv = 448.0f / amax_c;
-  codes.resize(vals.size());
   for (size_t i = 0; i < vals.size(); ++i) {
     const float y = vals[i] * inv;  // one fp32 rounding (no contraction)
     codes[i] = encode(y);
@@ -173,7 +196,7 @@ void oracle_e4m3_encode_array(const float* v, uint8_t* out, int64_t n) {
 // x: bf16 bits [G][M][K]; q: e4m3 codes [G][M][K]; s: fp32 [G][M][K/128]
 // (logical order: token, then K block). Returns 0, or -1 on bad sizes.
 int oracle_per_token_cast(const uint16_t* x, uint8_t* q, float* s, int G, int M, int K,
-                          int threads) {
+                          int threads, int ue8m0) {
   if (G < 0 || M < 0 || K <= 0 || K % kBlock != 0) return -1;
   const int KB = K / kBlock;
   parallel_for(static_cast<int64_t>(G) * M, threads, [&](int64_t row) {
@@ -182,7 +205,7 @@ int oracle_per_token_cast(const uint16_t* x, uint8_t* q, float* s, int G, int M,
     for (int kb = 0; kb < KB; ++kb) {
       const int64_t base = row * K + static_cast<int64_t>(kb) * kBlock;
       for (int i = 0; i < kBlock; ++i) vals[i] = bf16_to_float(x[base + i]);
-      s[row * KB + kb] = quantize_group(vals, codes);
+      s[row * KB + kb] = quantize_group(vals, codes, ue8m0);
       std::memcpy(q + base, codes.data(), kBlock);
     }
   });
@@ -193,7 +216,7 @@ int oracle_per_token_cast(const uint16_t* x, uint8_t* q, float* s, int G, int M,
 // x: bf16 bits [G][N][K]; q: [G][N][K]; s: fp32 [G][ceil(N/128)][K/128].
 // A last block that covers fewer than 128 rows uses only its valid rows.
 int oracle_per_block_cast(const uint16_t* x, uint8_t* q, float* s, int G, int N, int K,
-                          int threads) {
+                          int threads, int ue8m0) {
   if (G < 0 || N < 0 || K <= 0 || K % kBlock != 0) return -1;
   const int KB = K / kBlock;
   const int NB = (N + kBlock - 1) / kBlock;
@@ -210,7 +233,7 @@ int oracle_per_block_cast(const uint16_t* x, uint8_t* q, float* s, int G, int N,
       for (int i = 0; i < kBlock; ++i) vals.push_back(bf16_to_float(x[base + i]));
     }
     std::vector<uint8_t> codes;
-    s[blk] = quantize_group(vals, codes);
+    s[blk] = quantize_group(vals, codes, ue8m0);
     size_t j = 0;
     for (int n = n0; n < n1; ++n) {
       const int64_t base = (g * N + n) * K + static_cast<int64_t>(kb) * kBlock;

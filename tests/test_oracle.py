@@ -420,3 +420,67 @@ def test_dequant_nan_code_gives_nan():
     y = _bf16_to_f64(oracle.per_block_dequant(q, np.ones((1, 1), np.float32)))
     assert np.isnan(y[3, 5]) and np.isnan(y[7, 9])
     assert np.count_nonzero(np.isnan(y)) == 2
+
+
+# ---------------------------------------------------------------- power-of-two (UE8M0) scales
+
+def _ue8m0_input(rng, shape):
+    x = rng.standard_normal(shape, dtype=np.float32)
+    x[..., 0, :128] = 0.0                 # all-zero slice: amax floor
+    x[..., 1, :] *= 1e-6                  # tiny row
+    x[..., 2, :] *= 300.0                 # large row
+    x[..., 3, 7] = 448.0 * 2.0 ** -5      # amax exactly 448 * 2^-5: scale exactly 2^-5
+    x[..., 3, 8:128] = 0.0
+    return workloads.bf16_bits(x)
+
+
+def _smallest_pow2_at_least(r: np.ndarray) -> np.ndarray:
+    m, e = np.frexp(r.astype(np.float64))          # r = m * 2^e, m in [0.5, 1)
+    return np.where(m == 0.5, r.astype(np.float64), np.ldexp(1.0, e))
+
+
+def test_ue8m0_token_scales_are_smallest_sufficient_powers_of_two():
+    rng = np.random.default_rng(41)
+    x = _ue8m0_input(rng, (2, 6, 512))
+    q, s = oracle.per_token_cast(x, ue8m0=True)
+    xv = _bf16_to_f64(x).astype(np.float32).reshape(2, 6, 4, 128)
+    amax = np.maximum(np.abs(xv).max(axis=-1), np.float32(1e-4)).astype(np.float32)
+    r = (amax / np.float32(448.0)).astype(np.float32)
+    assert np.array_equal(s.astype(np.float64), _smallest_pow2_at_least(r))
+    assert s[0, 3, 0] == 2.0 ** -5
+
+
+def test_ue8m0_token_codes_are_x_over_s_rounded():
+    """x / s is exact (s a power of two) and at most 448 in magnitude; the codes
+    are torch's independent encoding of it."""
+    rng = np.random.default_rng(42)
+    x = _ue8m0_input(rng, (6, 384))
+    q, s = oracle.per_token_cast(x, ue8m0=True)
+    y = (_bf16_to_f64(x) / np.repeat(s, 128, axis=1)).astype(np.float32)
+    assert np.all(np.abs(y) <= 448.0)
+    assert np.array_equal(q, torch_encode(y))
+
+
+def test_ue8m0_block_scales_and_codes():
+    rng = np.random.default_rng(43)
+    x = workloads.bf16_bits(rng.standard_normal((300, 256), dtype=np.float32) * 0.02)
+    q, s = oracle.per_block_cast(x, ue8m0=True)
+    xv = _bf16_to_f64(x)
+    for nb in range(3):
+        for kb in range(2):
+            blk = xv[nb * 128:min(300, nb * 128 + 128), kb * 128:kb * 128 + 128].astype(np.float32)
+            amax = np.float32(max(float(np.abs(blk).max()), 1e-4))
+            want = _smallest_pow2_at_least(np.array([amax / np.float32(448.0)], np.float32))[0]
+            assert s[nb, kb] == want
+    y = (xv / _block_scales(s[None], 300)[0]).astype(np.float32)
+    assert np.array_equal(q, torch_encode(y))
+
+
+def test_ue8m0_round_trip_within_half_unit():
+    rng = np.random.default_rng(44)
+    x = workloads.bf16_bits(rng.standard_normal((256, 512), dtype=np.float32))
+    q, s = oracle.per_block_cast(x, ue8m0=True)
+    y = _bf16_to_f64(oracle.per_block_dequant(q, s))
+    xv = _bf16_to_f64(x)
+    sf = _block_scales(s[None], 256)[0].astype(np.float64)
+    assert np.all(np.abs(xv - y) <= 2.0 ** -4 * np.abs(xv) + 2.0 ** -10 * sf + 2.0 ** -8 * np.abs(y))
