@@ -107,6 +107,21 @@ fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int n
                                 int N, int K, cudaStream_t stream);
 
 /*
+ * The same two quantizers with power-of-two scales (the UE8M0 scale format of
+ * DeepSeek-V3.1; DeepSeek-V3 review "28.5 倍压缩 + 1/10 成本", "创新之处"
+ * item 4: scales quantized to powers of two, so a shift replaces a multiply):
+ *   scale = the smallest power of two at or above max(amax, 1e-4f) / 448
+ *           (from the fp32 bits of the quotient)
+ *   q     = e4m3_rne_satfinite(x / scale)   (exact: no element exceeds 448)
+ * Layouts, sizes and errors as for the fp32-scale forms above; the scales are
+ * written as fp32 values, so every GEMM entry point accepts them.
+ */
+fg_status per_token_cast_to_fp8_ue8m0(const uint16_t* x, uint8_t* q, float* sfa, int num_groups,
+                                      int M, int K, cudaStream_t stream);
+fg_status per_block_cast_to_fp8_ue8m0(const uint16_t* x, uint8_t* q, float* sfb, int num_groups,
+                                      int N, int K, cudaStream_t stream);
+
+/*
  * Weight dequantization, the third kernel of the FP8 quantize / dequantize /
  * GEMM trio (DeepSeek-V3 review "28.5 倍压缩 + 1/10 成本", "创新之处" item 4
  * and "可复用的模式与技巧" item 3). For every group g, row n and column k:

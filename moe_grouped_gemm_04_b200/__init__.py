@@ -30,7 +30,8 @@ FG_ERR_CUDA = 3
 FG_ERR_DEVICE = 4
 
 EXPORTED = (
-    "fg_sfa_stride", "per_token_cast_to_fp8", "per_block_cast_to_fp8", "fp8_gemm_nt",
+    "fg_sfa_stride", "per_token_cast_to_fp8", "per_block_cast_to_fp8",
+    "per_token_cast_to_fp8_ue8m0", "per_block_cast_to_fp8_ue8m0", "fp8_gemm_nt",
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
@@ -60,6 +61,8 @@ def load_library() -> ctypes.CDLL:
     lib.fg_sfa_stride.restype = I
     lib.per_token_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
     lib.per_block_cast_to_fp8.argtypes = [P, P, P, I, I, I, P]
+    lib.per_token_cast_to_fp8_ue8m0.argtypes = [P, P, P, I, I, I, P]
+    lib.per_block_cast_to_fp8_ue8m0.argtypes = [P, P, P, I, I, I, P]
     lib.per_block_dequant_to_bf16.argtypes = [P, P, P, I, I, I, P]
     lib.fp8_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, P]
     lib.fp8_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
@@ -70,7 +73,8 @@ def load_library() -> ctypes.CDLL:
     lib.fg_status_string.restype = ctypes.c_char_p
     lib.fg_last_error.argtypes = []
     lib.fg_last_error.restype = ctypes.c_char_p
-    for f in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "per_block_dequant_to_bf16",
+    for f in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "per_token_cast_to_fp8_ue8m0",
+              "per_block_cast_to_fp8_ue8m0", "per_block_dequant_to_bf16",
               "fp8_gemm_nt",
               "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
@@ -132,28 +136,46 @@ def empty_sfb(G: int, N: int, K: int, device) -> torch.Tensor:
 
 # ---------------------------------------------------------------- entry points
 
-def per_token_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfa: torch.Tensor,
-                          stream=None) -> None:
-    """x: bf16 [M][K] or [G][M][K] -> q (uint8, same shape), sfa [G][K/128][stride(M)]."""
+def _token_cast(fn, x, q, sfa, stream):
     G, M, K = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
     if x.dtype != torch.bfloat16 or q.dtype != torch.uint8 or sfa.dtype != torch.float32:
         raise FP8GemmError(FG_ERR_INVALID_ARG, "dtypes: x bf16, q uint8, sfa float32")
     if q.numel() != x.numel() or sfa.numel() < G * (K // 128) * sfa_stride(M):
         raise FP8GemmError(FG_ERR_INVALID_ARG, "output sizes do not match x")
-    _check(load_library().per_token_cast_to_fp8(_ptr(x), _ptr(q), _ptr(sfa), G, M, K,
-                                                _stream(stream)))
+    _check(fn(_ptr(x), _ptr(q), _ptr(sfa), G, M, K, _stream(stream)))
 
 
-def per_block_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfb: torch.Tensor,
-                          stream=None) -> None:
-    """x: bf16 [N][K] or [G][N][K] -> q (uint8, same shape), sfb [G][ceil(N/128)][K/128]."""
+def _block_cast(fn, x, q, sfb, stream):
     G, N, K = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
     if x.dtype != torch.bfloat16 or q.dtype != torch.uint8 or sfb.dtype != torch.float32:
         raise FP8GemmError(FG_ERR_INVALID_ARG, "dtypes: x bf16, q uint8, sfb float32")
     if q.numel() != x.numel() or sfb.numel() < G * (-(-N // 128)) * (K // 128):
         raise FP8GemmError(FG_ERR_INVALID_ARG, "output sizes do not match x")
-    _check(load_library().per_block_cast_to_fp8(_ptr(x), _ptr(q), _ptr(sfb), G, N, K,
-                                                _stream(stream)))
+    _check(fn(_ptr(x), _ptr(q), _ptr(sfb), G, N, K, _stream(stream)))
+
+
+def per_token_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfa: torch.Tensor,
+                          stream=None) -> None:
+    """x: bf16 [M][K] or [G][M][K] -> q (uint8, same shape), sfa [G][K/128][stride(M)]."""
+    _token_cast(load_library().per_token_cast_to_fp8, x, q, sfa, stream)
+
+
+def per_token_cast_to_fp8_ue8m0(x: torch.Tensor, q: torch.Tensor, sfa: torch.Tensor,
+                                stream=None) -> None:
+    """As per_token_cast_to_fp8 with power-of-two scales."""
+    _token_cast(load_library().per_token_cast_to_fp8_ue8m0, x, q, sfa, stream)
+
+
+def per_block_cast_to_fp8(x: torch.Tensor, q: torch.Tensor, sfb: torch.Tensor,
+                          stream=None) -> None:
+    """x: bf16 [N][K] or [G][N][K] -> q (uint8, same shape), sfb [G][ceil(N/128)][K/128]."""
+    _block_cast(load_library().per_block_cast_to_fp8, x, q, sfb, stream)
+
+
+def per_block_cast_to_fp8_ue8m0(x: torch.Tensor, q: torch.Tensor, sfb: torch.Tensor,
+                                stream=None) -> None:
+    """As per_block_cast_to_fp8 with power-of-two scales."""
+    _block_cast(load_library().per_block_cast_to_fp8_ue8m0, x, q, sfb, stream)
 
 
 def per_block_dequant_to_bf16(q: torch.Tensor, sfb: torch.Tensor, x: torch.Tensor,

@@ -469,17 +469,8 @@ __global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
   __syncthreads();
 }
 
-}  // namespace
-}  // namespace fg
-
-using namespace fg;
-
-extern "C" {
-
-int fg_sfa_stride(int M) { return sfa_stride(M); }
-
-fg_status per_token_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfa, int num_groups, int M,
-                                int K, cudaStream_t stream) {
+fg_status run_per_token(const uint16_t* x, uint8_t* q, float* sfa, int num_groups, int M, int K,
+                        bool ue8m0, cudaStream_t stream) {
   if (num_groups < 1) return fail(FG_ERR_INVALID_ARG, "num_groups=%d must be >= 1", num_groups);
   if (M < 0) return fail(FG_ERR_INVALID_ARG, "M=%d must be >= 0", M);
   if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
@@ -495,14 +486,14 @@ fg_status per_token_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfa, int n
   // and pass for large ones (several loads in flight per thread)
   const int64_t blocks_needed = (slices * 16 + 255) / 256;
   const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, int64_t(dev->sm_count) * 8));
-  const cudaError_t e = launch_pdl(per_token_cast_kernel, dim3(grid), dim3(256), stream, x, q, sfa,
+  const cudaError_t e = launch_pdl(ue8m0 ? per_token_cast_kernel<true> : per_token_cast_kernel<false>, dim3(grid), dim3(256), stream, x, q, sfa,
                                    num_groups, M, K, sfa_stride(M));
   if (e != cudaSuccess) return cuda_fail(e, "per_token_cast_kernel launch");
   return FG_OK;
 }
 
-fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int num_groups, int N,
-                                int K, cudaStream_t stream) {
+fg_status run_per_block(const uint16_t* x, uint8_t* q, float* sfb, int num_groups, int N, int K,
+                        bool ue8m0, cudaStream_t stream) {
   if (num_groups < 1) return fail(FG_ERR_INVALID_ARG, "num_groups=%d must be >= 1", num_groups);
   if (N <= 0) return fail(FG_ERR_INVALID_ARG, "N=%d must be >= 1", N);
   if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
@@ -513,10 +504,40 @@ fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int n
   FG_TRY(device_info(&dev));
   const int64_t blocks = static_cast<int64_t>(num_groups) * ((N + 127) / 128) * (K / 128);
   if (blocks > 0x7FFFFFFF) return fail(FG_ERR_UNSUPPORTED, "too many blocks");
-  const cudaError_t e = launch_pdl(per_block_cast_kernel, dim3(static_cast<unsigned>(blocks)),
+  const cudaError_t e = launch_pdl(ue8m0 ? per_block_cast_kernel<true> : per_block_cast_kernel<false>,
+                                   dim3(static_cast<unsigned>(blocks)),
                                    dim3(256), stream, x, q, sfb, num_groups, N, K);
   if (e != cudaSuccess) return cuda_fail(e, "per_block_cast_kernel launch");
   return FG_OK;
+}
+
+}  // namespace
+}  // namespace fg
+
+using namespace fg;
+
+extern "C" {
+
+int fg_sfa_stride(int M) { return sfa_stride(M); }
+
+fg_status per_token_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfa, int num_groups, int M,
+                                int K, cudaStream_t stream) {
+  return run_per_token(x, q, sfa, num_groups, M, K, false, stream);
+}
+
+fg_status per_token_cast_to_fp8_ue8m0(const uint16_t* x, uint8_t* q, float* sfa, int num_groups,
+                                      int M, int K, cudaStream_t stream) {
+  return run_per_token(x, q, sfa, num_groups, M, K, true, stream);
+}
+
+fg_status per_block_cast_to_fp8(const uint16_t* x, uint8_t* q, float* sfb, int num_groups, int N,
+                                int K, cudaStream_t stream) {
+  return run_per_block(x, q, sfb, num_groups, N, K, false, stream);
+}
+
+fg_status per_block_cast_to_fp8_ue8m0(const uint16_t* x, uint8_t* q, float* sfb, int num_groups,
+                                      int N, int K, cudaStream_t stream) {
+  return run_per_block(x, q, sfb, num_groups, N, K, true, stream);
 }
 
 fg_status per_block_dequant_to_bf16(const uint8_t* q, const float* sfb, uint16_t* x,

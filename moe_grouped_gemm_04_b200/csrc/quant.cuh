@@ -6,7 +6,9 @@
 //
 // Arithmetic (must match the oracle bit for bit):
 //   amax_c = max(amax, 1e-4f); scale = amax_c / 448 (IEEE division);
-//   code = cvt.rn.satfinite.e4m3(x * (448 / amax_c)) with one fp32 multiply.
+//   code = cvt.rn.satfinite.e4m3(x * (448 / amax_c)) with one fp32 multiply;
+// or, with power-of-two (UE8M0) scales, scale = the smallest power of two at
+// or above amax_c / 448 and code = cvt.rn.satfinite.e4m3(x / scale), exact.
 // Sources: "DeepGEMM" overview (zixun.chuxinyishu.com/article/345.html),
 // section "FP8与细粒度缩放" (per-slice activation and per-block weight
 // scales); DeepSeek-V3 review (developer.cloud.tencent.cn/article/2686109),
@@ -44,6 +46,25 @@ __device__ __forceinline__ uint2 quantize8(uint4 w, float inv) {
   return make_uint2(out[0], out[1]);
 }
 
+// Scale and its reciprocal for a group with amax_c = max(amax, 1e-4).
+// UE8M0 = false: s = amax_c / 448, inv = 448 / amax_c (IEEE divisions).
+// UE8M0 = true: s = the smallest power of two at or above amax_c / 448 (from
+// the fp32 bits of the quotient: 2^E if its mantissa field is zero, else
+// 2^(E+1)), inv = 1 / s exactly (biased exponent 254 - e), so that x * inv
+// equals x / s.
+template <bool UE8M0>
+__device__ __forceinline__ void group_scale(float amx, float& scale, float& inv) {
+  if constexpr (UE8M0) {
+    const uint32_t u = __float_as_uint(__fdiv_rn(amx, kFp8Max));
+    const uint32_t e = ((u >> 23) & 0xFFu) + ((u & 0x007FFFFFu) != 0 ? 1u : 0u);
+    scale = __uint_as_float(e << 23);
+    inv = __uint_as_float((254u - e) << 23);
+  } else {
+    scale = __fdiv_rn(amx, kFp8Max);
+    inv = __fdiv_rn(kFp8Max, amx);
+  }
+}
+
 __device__ __forceinline__ float amax8(uint4 w) {
   const uint32_t in[4] = {w.x, w.y, w.z, w.w};
   float m = 0.0f;
@@ -64,6 +85,7 @@ __device__ __forceinline__ float amax8(uint4 w) {
 // index arithmetic).
 constexpr int QUNROLL = 4;
 
+template <bool UE8M0>
 __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __restrict__ x,
                                                              uint8_t* __restrict__ q,
                                                              float* __restrict__ sfa, int G,
@@ -101,10 +123,10 @@ __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __r
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
       if (ok[u]) {
-        const float amx = fmaxf(a, kAmaxFloor);
-        const float inv = __fdiv_rn(kFp8Max, amx);
+        float scale, inv;
+        group_scale<UE8M0>(fmaxf(a, kAmaxFloor), scale, inv);
         *reinterpret_cast<uint2*>(q + off[u]) = quantize8(w[u], inv);
-        if (sub == 0) sfa[static_cast<int64_t>(gk[u]) * stride + m[u]] = __fdiv_rn(amx, kFp8Max);
+        if (sub == 0) sfa[static_cast<int64_t>(gk[u]) * stride + m[u]] = scale;
       }
     }
   }
@@ -112,6 +134,7 @@ __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __r
 
 // One CTA (256 threads) per 128x128 block. Thread t covers rows t/16 + 16*i
 // (i = 0..7) and the 8 columns starting at (t%16)*8 of the block.
+template <bool UE8M0>
 __global__ void __launch_bounds__(256) per_block_cast_kernel(const uint16_t* __restrict__ x,
                                                              uint8_t* __restrict__ q,
                                                              float* __restrict__ sfb, int G,
@@ -147,8 +170,8 @@ __global__ void __launch_bounds__(256) per_block_cast_kernel(const uint16_t* __r
   a = warp_max[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) a = fmaxf(a, warp_max[i]);
-  const float amx = fmaxf(a, kAmaxFloor);
-  const float inv = __fdiv_rn(kFp8Max, amx);
+  float scale, inv;
+  group_scale<UE8M0>(fmaxf(a, kAmaxFloor), scale, inv);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int n = nb * 128 + r0 + 16 * i;
@@ -157,7 +180,7 @@ __global__ void __launch_bounds__(256) per_block_cast_kernel(const uint16_t* __r
       *reinterpret_cast<uint2*>(q + off) = quantize8(w[i], inv);
     }
   }
-  if (threadIdx.x == 0) sfb[blk] = __fdiv_rn(amx, kFp8Max);
+  if (threadIdx.x == 0) sfb[blk] = scale;
 }
 
 // Weight dequantization, the third kernel of the FP8 trio (quantize,

@@ -156,3 +156,33 @@ def test_per_block_dequant_round_trip_on_device(fg):
     q[0, 7, 3] = 0x7F
     nan = gpu_dequant(fg, q, s)
     assert (nan[0, 7, 3] & 0x7F80) == 0x7F80 and (nan[0, 7, 3] & 0x007F) != 0
+
+
+# ---------------------------------------------------------------- power-of-two (UE8M0) scales
+
+@pytest.mark.parametrize("G,M,K", [(1, 1, 128), (1, 130, 384), (3, 80, 256), (1, 64, 7168)])
+def test_per_token_ue8m0_bit_exact(fg, G, M, K):
+    rng = np.random.default_rng(M * 3 + K + G)
+    bits = workloads.bf16_bits(_special_rows(rng.standard_normal((G, M, K), dtype=np.float32)))
+    x = bf16_tensor(bits)
+    q = torch.empty((G, M, K), dtype=torch.uint8, device="cuda")
+    s = torch.full((G, K // 128, fg.sfa_stride(M)), -1.0, dtype=torch.float32, device="cuda")
+    fg.per_token_cast_to_fp8_ue8m0(x, q, s)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.per_token_cast(bits, ue8m0=True)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sa_from_mn_major(s.cpu().numpy(), M).view(np.uint32), s_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("G,N,K", [(1, 256, 512), (2, 300, 384), (1, 2112, 768)])
+def test_per_block_ue8m0_bit_exact(fg, G, N, K):
+    rng = np.random.default_rng(N * 3 + K + G)
+    bits = workloads.bf16_bits(rng.standard_normal((G, N, K), dtype=np.float32) * 0.02)
+    x = bf16_tensor(bits)
+    q = torch.empty((G, N, K), dtype=torch.uint8, device="cuda")
+    s = fg.empty_sfb(G, N, K, "cuda")
+    fg.per_block_cast_to_fp8_ue8m0(x, q, s)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.per_block_cast(bits, ue8m0=True)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
