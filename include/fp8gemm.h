@@ -182,6 +182,45 @@ fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint
                                   int M_max, int N, int K, int expected_m, cudaStream_t stream);
 
 /*
+ * The three GEMMs above for power-of-two scales (the UE8M0 scale format;
+ * DeepSeek-V3 review "28.5 倍压缩 + 1/10 成本", "创新之处" item 4: scales
+ * quantized to powers of two so that applying one is a shift). Same operation,
+ * arguments, layouts, contracts and errors as fp8_gemm_nt,
+ * fp8_grouped_gemm_contiguous and fp8_grouped_gemm_masked; additionally every
+ * sfa and sfb entry that is read must be a power of two in the fp32 normal
+ * range (what per_token_cast_to_fp8_ue8m0 / per_block_cast_to_fp8_ue8m0
+ * write). The kernel keeps only each scale's exponent field: a scale that is
+ * not a power of two acts as the power of two at or below it, zero as 2^-127.
+ *
+ * For token tiles of 128 rows the scales are applied inside the tensor core
+ * (tcgen05.mma kind::mxf8f6f4.block_scale, one UE8M0 scale per row per 32 K
+ * elements), and the whole K range accumulates in tensor memory in fp32 with
+ * no promotion pass; the products a * b * sa * sb are exact, only the order of
+ * the fp32 additions differs from the promoted form. Thin shapes (dense
+ * M <= 64, masked expected_m <= 64) run the promoted swapped kernel, which is
+ * exact per K block for power-of-two scales as well.
+ */
+fg_status fp8_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                            const float* sfb, uint16_t* D, int M, int N, int K,
+                            cudaStream_t stream);
+fg_status fp8_grouped_gemm_contiguous_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                            const float* sfb, uint16_t* D,
+                                            const int32_t* m_indices, int M_total, int N, int K,
+                                            int G, cudaStream_t stream);
+fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                        const float* sfb, uint16_t* D, const int32_t* masked_m,
+                                        int G, int M_max, int N, int K, int expected_m,
+                                        cudaStream_t stream);
+
+/*
+ * Tuning knob of the three _ue8m0 GEMMs (process-wide): 0 = choose the weight
+ * tile width per shape (default); 128, 224 or 256 = always use that width and
+ * the block-scaled kernel, thin shapes included. Other values:
+ * FG_ERR_INVALID_ARG.
+ */
+fg_status fg_set_ue8m0_tile_width(int width);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns FG_OK when it was clear, FG_ERR_DEVICE otherwise
  * (the detail is in fg_last_error and *code, which may be NULL).

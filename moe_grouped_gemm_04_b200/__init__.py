@@ -9,7 +9,10 @@ raises.
 
 The functions carry the C names:
   per_token_cast_to_fp8, per_block_cast_to_fp8, per_block_dequant_to_bf16,
-  fp8_gemm_nt, fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked
+  fp8_gemm_nt, fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked,
+  per_token_cast_to_fp8_ue8m0, per_block_cast_to_fp8_ue8m0, and the GEMMs for
+  power-of-two scales fp8_gemm_nt_ue8m0, fp8_grouped_gemm_contiguous_ue8m0,
+  fp8_grouped_gemm_masked_ue8m0 (set_ue8m0_tile_width tunes them)
 plus allocation helpers that return tensors in the layouts the kernels use.
 """
 from __future__ import annotations
@@ -33,7 +36,8 @@ EXPORTED = (
     "fg_sfa_stride", "per_token_cast_to_fp8", "per_block_cast_to_fp8",
     "per_token_cast_to_fp8_ue8m0", "per_block_cast_to_fp8_ue8m0", "fp8_gemm_nt",
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
-    "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
+    "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
+    "fg_set_ue8m0_tile_width", "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
 
 
@@ -67,6 +71,10 @@ def load_library() -> ctypes.CDLL:
     lib.fp8_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, P]
     lib.fp8_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fp8_grouped_gemm_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+    lib.fp8_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, I, I, I, P]
+    lib.fp8_grouped_gemm_contiguous_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+    lib.fp8_grouped_gemm_masked_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+    lib.fg_set_ue8m0_tile_width.argtypes = [I]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
     lib.fg_status_string.argtypes = [I]
@@ -77,6 +85,8 @@ def load_library() -> ctypes.CDLL:
               "per_block_cast_to_fp8_ue8m0", "per_block_dequant_to_bf16",
               "fp8_gemm_nt",
               "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
+              "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0",
+              "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile_width",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
     _lib = lib
@@ -190,41 +200,79 @@ def per_block_dequant_to_bf16(q: torch.Tensor, sfb: torch.Tensor, x: torch.Tenso
                                                     _stream(stream)))
 
 
-def fp8_gemm_nt(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor, sfb: torch.Tensor,
-                D: torch.Tensor, stream=None) -> None:
-    """D[M][N] (bf16) = (A * sa)(B * sb)^T; A uint8 [M][K], B uint8 [N][K]."""
+def _gemm_nt(fn, A, sfa, B, sfb, D, stream):
     M, K = A.shape
     N = B.shape[0]
     if D.dtype != torch.bfloat16 or tuple(D.shape) != (M, N):
         raise FP8GemmError(FG_ERR_INVALID_ARG, "D must be bf16 [M][N]")
-    _check(load_library().fp8_gemm_nt(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), M, N, K,
-                                      _stream(stream)))
+    _check(fn(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), M, N, K, _stream(stream)))
+
+
+def _gemm_contiguous(fn, A, sfa, B, sfb, D, m_indices, stream):
+    M_total, K = A.shape
+    G, N, _ = B.shape
+    if m_indices.dtype != torch.int32 or m_indices.numel() != M_total:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "m_indices must be int32 [M_total]")
+    _check(fn(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(m_indices), M_total, N, K, G,
+              _stream(stream)))
+
+
+def _gemm_masked(fn, A, sfa, B, sfb, D, masked_m, expected_m, stream):
+    G, M_max, K = A.shape
+    N = B.shape[1]
+    if masked_m.dtype != torch.int32 or masked_m.numel() != G:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "masked_m must be int32 [G]")
+    _check(fn(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(masked_m), G, M_max, N, K,
+              int(expected_m), _stream(stream)))
+
+
+def fp8_gemm_nt(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor, sfb: torch.Tensor,
+                D: torch.Tensor, stream=None) -> None:
+    """D[M][N] (bf16) = (A * sa)(B * sb)^T; A uint8 [M][K], B uint8 [N][K]."""
+    _gemm_nt(load_library().fp8_gemm_nt, A, sfa, B, sfb, D, stream)
 
 
 def fp8_grouped_gemm_contiguous(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor,
                                 sfb: torch.Tensor, D: torch.Tensor, m_indices: torch.Tensor,
                                 stream=None) -> None:
     """A uint8 [M_total][K], B uint8 [G][N][K], m_indices int32 [M_total], D bf16 [M_total][N]."""
-    M_total, K = A.shape
-    G, N, _ = B.shape
-    if m_indices.dtype != torch.int32 or m_indices.numel() != M_total:
-        raise FP8GemmError(FG_ERR_INVALID_ARG, "m_indices must be int32 [M_total]")
-    _check(load_library().fp8_grouped_gemm_contiguous(
-        _ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(m_indices), M_total, N, K, G,
-        _stream(stream)))
+    _gemm_contiguous(load_library().fp8_grouped_gemm_contiguous, A, sfa, B, sfb, D, m_indices,
+                     stream)
 
 
 def fp8_grouped_gemm_masked(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor,
                             sfb: torch.Tensor, D: torch.Tensor, masked_m: torch.Tensor,
                             expected_m: int, stream=None) -> None:
     """A uint8 [G][M_max][K], B uint8 [G][N][K], masked_m int32 [G], D bf16 [G][M_max][N]."""
-    G, M_max, K = A.shape
-    N = B.shape[1]
-    if masked_m.dtype != torch.int32 or masked_m.numel() != G:
-        raise FP8GemmError(FG_ERR_INVALID_ARG, "masked_m must be int32 [G]")
-    _check(load_library().fp8_grouped_gemm_masked(
-        _ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(masked_m), G, M_max, N, K,
-        int(expected_m), _stream(stream)))
+    _gemm_masked(load_library().fp8_grouped_gemm_masked, A, sfa, B, sfb, D, masked_m, expected_m,
+                 stream)
+
+
+def fp8_gemm_nt_ue8m0(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor, sfb: torch.Tensor,
+                      D: torch.Tensor, stream=None) -> None:
+    """fp8_gemm_nt with power-of-two scales (block-scaled tensor-core MMAs)."""
+    _gemm_nt(load_library().fp8_gemm_nt_ue8m0, A, sfa, B, sfb, D, stream)
+
+
+def fp8_grouped_gemm_contiguous_ue8m0(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor,
+                                      sfb: torch.Tensor, D: torch.Tensor,
+                                      m_indices: torch.Tensor, stream=None) -> None:
+    """fp8_grouped_gemm_contiguous with power-of-two scales."""
+    _gemm_contiguous(load_library().fp8_grouped_gemm_contiguous_ue8m0, A, sfa, B, sfb, D,
+                     m_indices, stream)
+
+
+def fp8_grouped_gemm_masked_ue8m0(A: torch.Tensor, sfa: torch.Tensor, B: torch.Tensor,
+                                  sfb: torch.Tensor, D: torch.Tensor, masked_m: torch.Tensor,
+                                  expected_m: int, stream=None) -> None:
+    """fp8_grouped_gemm_masked with power-of-two scales."""
+    _gemm_masked(load_library().fp8_grouped_gemm_masked_ue8m0, A, sfa, B, sfb, D, masked_m,
+                 expected_m, stream)
+
+
+def set_ue8m0_tile_width(width: int) -> None:
+    """0 = automatic (default); 128, 224 or 256 = force that weight-tile width."""
+    _check(load_library().fg_set_ue8m0_tile_width(int(width)))
 
 
 def get_device_status(stream=None) -> int:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -14,6 +15,7 @@
 
 #include "fp8gemm.h"
 #include "gemm.cuh"
+#include "gemm_mx.cuh"
 #include "quant.cuh"
 
 namespace fg {
@@ -422,6 +424,137 @@ fg_status run_gemm(const Problem& pr, int expected_m, cudaStream_t stream) {
   }
 }
 
+// ---------------------------------------------------------------- UE8M0 GEMM
+
+//                  BW  stages accumulators epilogue warps per quadrant
+using MxN128 = MxCfg<128, 5, 2, 1>;
+using MxN224 = MxCfg<224, 4, 2, 1>;
+using MxN256 = MxCfg<256, 3, 1, 2>;
+
+template <class C, int FORM>
+fg_status mx_kernel_attr(int dev) {
+  static bool done[kMaxDevices] = {};
+  if (!done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(fp8_gemm_mx_kernel<C, FORM>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               C::smem_bytes(FORM));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    done[dev] = true;
+  }
+  return FG_OK;
+}
+
+template <class C, int FORM>
+fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
+  static_assert(C::smem_bytes(FORM) <= 232448, "shared memory per CTA");
+  FG_TRY((mx_kernel_attr<C, FORM>(dev_id)));
+  const int KB = pr.K / 128;
+  CUtensorMap tmA, tmB, tmSA, tmD;
+  FG_TRY(make_map(&tmA, pr.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
+                  static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "A"));
+  FG_TRY(make_map(&tmB, pr.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
+                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::BW,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "B"));
+  FG_TRY(make_map(&tmSA, pr.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.M,
+                  static_cast<uint64_t>(pr.slabs) * KB,
+                  static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
+  // D as rows x N bf16 in boxes of 32 rows x 32 columns, 64-byte swizzled
+  FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
+                  static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2, 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_64B, "D"));
+  GemmParams p{};
+  p.M = pr.M;
+  p.N = pr.N;
+  p.K = pr.K;
+  p.G = pr.G;
+  p.KB = KB;
+  p.NB = (pr.N + 127) / 128;
+  p.num_mt = (pr.M + C::BT - 1) / C::BT;
+  p.num_nt = (pr.N + C::BW - 1) / C::BW;
+  p.sfb = pr.sfb;
+  p.D = pr.D;
+  p.m_indices = pr.m_indices;
+  p.masked_m = pr.masked_m;
+  p.status = dev.status;
+  p.timeout_ns = wait_limit_ns();
+  int64_t tiles = static_cast<int64_t>(p.num_mt) * p.num_nt;
+  if (FORM == kFormMasked) tiles *= pr.G;  // upper bound: masked_m lives on the device
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(tiles, dev.sm_count));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::NUM_THREADS);
+  cfg.dynamicSmemBytes = C::smem_bytes(FORM);
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_mx_kernel<C, FORM>, tmA, tmB, tmSA,
+                                           tmD, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_mx_kernel launch");
+  return FG_OK;
+}
+
+// Weight-tile width of the block-scaled kernel: the candidate whose tiles
+// fill the SMs in the fewest rounds, counting a round by its MMA work (the
+// tile width) and a small surcharge for the narrow tile (its MMAs read more
+// shared memory per flop) and the single-accumulator one (its MMAs wait for
+// each tile's accumulator to be read).
+int mx_tile_width(const Problem& pr, int sm_count, int expected_m) {
+  int64_t token_tiles = (pr.M + 127) / 128;
+  if (pr.form == kFormMasked) token_tiles = static_cast<int64_t>((expected_m + 127) / 128) * pr.G;
+  const struct { int bw; double weight; } cand[] = {{224, 1.0}, {256, 1.03}, {128, 1.10}};
+  int best = 224;
+  double best_cost = 1e300;
+  for (const auto& c : cand) {
+    const int64_t tiles = token_tiles * ((pr.N + c.bw - 1) / c.bw);
+    const int64_t rounds = (tiles + sm_count - 1) / sm_count;
+    const double cost = static_cast<double>(rounds) * c.bw * c.weight;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = c.bw;
+    }
+  }
+  return best;
+}
+
+template <int FORM>
+fg_status dispatch_mx(const Problem& pr, int bw, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
+  switch (bw) {
+    case 128: return launch_mx<MxN128, FORM>(pr, dev, dev_id, stream);
+    case 256: return launch_mx<MxN256, FORM>(pr, dev, dev_id, stream);
+    default: return launch_mx<MxN224, FORM>(pr, dev, dev_id, stream);
+  }
+}
+
+// Power-of-two scales: the block-scaled kernel for token tiles of 128 rows;
+// thin shapes (dense M <= 64, masked with expected_m <= 64) take the swapped
+// promotion kernel, whose per-block scaling is exact for such scales too.
+std::atomic<int> g_mx_tile_width{0};  // fg_set_ue8m0_tile_width (0 = automatic)
+
+fg_status run_gemm_mx(const Problem& pr, int expected_m, cudaStream_t stream) {
+  const int force_bw = g_mx_tile_width.load(std::memory_order_relaxed);
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const int small_m = pr.form == kFormDense ? pr.M : pr.form == kFormMasked ? expected_m : 1 << 30;
+  if (small_m <= 64 && force_bw == 0) return run_gemm(pr, expected_m, stream);
+  if (pr.form == kFormContig && (pr.M + 127) / 128 > kTableMax)
+    return fail(FG_ERR_UNSUPPORTED, "M_total %d exceeds %d rows", pr.M, kTableMax * 128);
+  if (pr.form == kFormMasked && pr.G + 1 > kTableMax)
+    return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d experts", pr.G, kTableMax - 1);
+  const int bw = force_bw ? force_bw : mx_tile_width(pr, dev->sm_count, expected_m);
+  switch (pr.form) {
+    case kFormDense: return dispatch_mx<kFormDense>(pr, bw, *dev, dev_id, stream);
+    case kFormContig: return dispatch_mx<kFormContig>(pr, bw, *dev, dev_id, stream);
+    default: return dispatch_mx<kFormMasked>(pr, bw, *dev, dev_id, stream);
+  }
+}
+
 fg_status check_gemm_common(const uint8_t* A, const float* sfa, const uint8_t* B,
                             const float* sfb, uint16_t* D, int N, int K) {
   if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
@@ -590,6 +723,49 @@ fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint
   if (expected_m <= 0) expected_m = M_max;
   Problem pr{kFormMasked, A, sfa, B, sfb, D, nullptr, masked_m, M_max, N, K, G, G};
   return run_gemm(pr, expected_m, stream);
+}
+
+fg_status fp8_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B, const float* sfb,
+                            uint16_t* D, int M, int N, int K, cudaStream_t stream) {
+  if (M < 0) return fail(FG_ERR_INVALID_ARG, "M=%d must be >= 0", M);
+  if (M == 0) return FG_OK;
+  FG_TRY(check_gemm_common(A, sfa, B, sfb, D, N, K));
+  Problem pr{kFormDense, A, sfa, B, sfb, D, nullptr, nullptr, M, N, K, 1, 1};
+  return run_gemm_mx(pr, M, stream);
+}
+
+fg_status fp8_grouped_gemm_contiguous_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                            const float* sfb, uint16_t* D,
+                                            const int32_t* m_indices, int M_total, int N, int K,
+                                            int G, cudaStream_t stream) {
+  if (M_total < 0 || M_total % 128 != 0)
+    return fail(FG_ERR_INVALID_ARG, "M_total=%d must be a non-negative multiple of 128", M_total);
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (M_total == 0) return FG_OK;
+  FG_TRY(check_gemm_common(A, sfa, B, sfb, D, N, K));
+  FG_TRY(check_ptr(m_indices, "m_indices"));
+  Problem pr{kFormContig, A, sfa, B, sfb, D, m_indices, nullptr, M_total, N, K, G, 1};
+  return run_gemm_mx(pr, M_total, stream);
+}
+
+fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                        const float* sfb, uint16_t* D, const int32_t* masked_m,
+                                        int G, int M_max, int N, int K, int expected_m,
+                                        cudaStream_t stream) {
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (M_max < 1) return fail(FG_ERR_INVALID_ARG, "M_max=%d must be >= 1", M_max);
+  FG_TRY(check_gemm_common(A, sfa, B, sfb, D, N, K));
+  FG_TRY(check_ptr(masked_m, "masked_m"));
+  if (expected_m <= 0) expected_m = M_max;
+  Problem pr{kFormMasked, A, sfa, B, sfb, D, nullptr, masked_m, M_max, N, K, G, G};
+  return run_gemm_mx(pr, expected_m, stream);
+}
+
+fg_status fg_set_ue8m0_tile_width(int width) {
+  if (width != 0 && width != 128 && width != 224 && width != 256)
+    return fail(FG_ERR_INVALID_ARG, "tile width %d: 0 (automatic), 128, 224 or 256", width);
+  g_mx_tile_width.store(width, std::memory_order_relaxed);
+  return FG_OK;
 }
 
 fg_status fg_get_device_status(cudaStream_t stream, int* code) {

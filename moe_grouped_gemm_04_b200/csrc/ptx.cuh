@@ -91,6 +91,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 
 // ---------------------------------------------------------------- TMA / cp.async
 
+// 4-byte asynchronous copy global -> shared (L1-allocating).
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+
+// Arrive on `bar` once all of this thread's earlier cp.async copies have
+// landed; the arrival is counted in the barrier's expected count (noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -240,6 +253,72 @@ __host__ __device__ constexpr uint32_t mma_idesc_e4m3(int M, int N) {
          | (0u << 15) | (0u << 16)                  // A, B K-major
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale: e4m3 A
+// and B, both K-major, shape M x N, scale factors in UE8M0 (power-of-two)
+// format, scale-factor id 0 for both operands (byte 0 of each scale word).
+__host__ __device__ constexpr uint32_t mma_idesc_e4m3_bs(int M, int N) {
+  return (0u << 4)                                  // B scale-factor id
+         | (0u << 7) | (0u << 10)                   // A, B format: e4m3
+         | (0u << 15) | (0u << 16)                  // A, B K-major
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (1u << 23)                               // scale format: UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
+         | (0u << 29);                              // A scale-factor id
+}
+
+// D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T with one UE8M0 scale per
+// row (column) per 32 K elements, read from tensor memory at sfa_tmem and
+// sfb_tmem; FP8 e4m3 inputs, fp32 accumulator.
+__device__ __forceinline__ void mma_f8_bs(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copies one 512-byte scale-factor group from shared memory into 4 tensor
+// memory columns: 32 rows of 16 bytes, replicated into all four 32-lane
+// quadrants. Shared layout [r0 < 32][r1 < 4][byte < 4]: the scale word of row
+// r0 + 32 * r1 lands in column taddr + r1 of lane r0 of every quadrant.
+__device__ __forceinline__ void tmem_cp_sf_group(uint32_t taddr, uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address / 16
+  d |= static_cast<uint64_t>(128 >> 4) << 16;           // leading-dim offset (one core matrix)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;           // 8-row core matrices 128 bytes apart
+  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version; no swizzle
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
+// Pair forms (issued by the leader CTA of a CTA pair). The block-scaled pair
+// MMA reads, in each CTA's tensor memory, the A scales of that CTA's rows and
+// the B scales of all N columns; the pair copy moves each CTA's shared group
+// into that CTA's own tensor memory.
+__device__ __forceinline__ void mma_f8_bs_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t sfa_tmem,
+                                               uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf_group_pair(uint32_t taddr, uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA

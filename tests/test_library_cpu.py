@@ -89,3 +89,24 @@ def test_validation_rejects_without_touching_the_device(lib):
     assert lib.fp8_gemm_nt(ok, ok, ok, ok, ok, 0, 256, 256, None) == 0
     assert lib.per_token_cast_to_fp8(ok, ok, ok, 1, 0, 128, None) == 0
     assert lib.fp8_grouped_gemm_contiguous(ok, ok, ok, ok, ok, ok, 0, 256, 256, 2, None) == 0
+
+
+def test_ue8m0_gemm_validation_without_the_device(lib):
+    P = ctypes.c_void_p
+    ok = P(FAKE)
+    assert lib.fp8_gemm_nt_ue8m0(ok, ok, ok, ok, ok, 64, 256, 100, None) == 1
+    assert lib.fp8_gemm_nt_ue8m0(ok, ok, ok, ok, ok, 256, 250, 256, None) == 1
+    assert lib.fp8_gemm_nt_ue8m0(ok, ok, ok, ok, None, 256, 256, 256, None) == 1
+    assert lib.fp8_grouped_gemm_contiguous_ue8m0(ok, ok, ok, ok, ok, ok, 100, 256, 256, 2, None) == 1
+    assert lib.fp8_grouped_gemm_contiguous_ue8m0(ok, ok, ok, ok, ok, None, 128, 256, 256, 2, None) == 1
+    assert lib.fp8_grouped_gemm_masked_ue8m0(ok, ok, ok, ok, ok, ok, 0, 64, 256, 256, 64, None) == 1
+    assert lib.fp8_grouped_gemm_masked_ue8m0(ok, ok, P(MISALIGNED), ok, ok, ok, 2, 64, 256, 256, 64,
+                                             None) == 1
+    assert lib.fp8_gemm_nt_ue8m0(ok, ok, ok, ok, ok, 0, 256, 256, None) == 0
+    assert lib.fp8_grouped_gemm_contiguous_ue8m0(ok, ok, ok, ok, ok, ok, 0, 256, 256, 2, None) == 0
+    # the tile-width knob takes 0, 128, 224 and 256 only
+    for w in (0, 128, 224, 256):
+        assert lib.fg_set_ue8m0_tile_width(w) == 0
+    for w in (-1, 64, 192, 512):
+        assert lib.fg_set_ue8m0_tile_width(w) == 1
+    assert lib.fg_set_ue8m0_tile_width(0) == 0
