@@ -192,10 +192,11 @@ fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint
  * write). The kernel keeps only each scale's exponent field: a scale that is
  * not a power of two acts as the power of two at or below it, zero as 2^-127.
  *
- * For token tiles of 128 rows the scales are applied inside the tensor core
- * (tcgen05.mma kind::mxf8f6f4.block_scale, one UE8M0 scale per row per 32 K
- * elements), and the whole K range accumulates in tensor memory in fp32 with
- * no promotion pass; the products a * b * sa * sb are exact, only the order of
+ * For token tiles of 128 rows (dense: pairs of them, computed by the two CTAs
+ * of a cluster) the scales are applied inside the tensor core (tcgen05.mma
+ * kind::mxf8f6f4.block_scale, one UE8M0 scale per row per 32 K elements), and
+ * the whole K range accumulates in tensor memory in fp32 with no promotion
+ * pass; the products a * b * sa * sb are exact, only the order of
  * the fp32 additions differs from the promoted form. Thin shapes (dense
  * M <= 64, masked expected_m <= 64) run the promoted swapped kernel, which is
  * exact per K block for power-of-two scales as well.
@@ -213,12 +214,14 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
                                         cudaStream_t stream);
 
 /*
- * Tuning knob of the three _ue8m0 GEMMs (process-wide): 0 = choose the weight
- * tile width per shape (default); 128, 224 or 256 = always use that width and
- * the block-scaled kernel, thin shapes included. Other values:
- * FG_ERR_INVALID_ARG.
+ * Tuning knob of the three _ue8m0 GEMMs (process-wide). width = 0: choose the
+ * tile per shape (default). Otherwise always use the block-scaled kernel, thin
+ * shapes included, with weight tiles of `width` rows: 128, 224 or 256 with
+ * pair = 0 (one CTA per 128-token tile), or 224 with pair = 1 (two CTAs of a
+ * cluster per 256-token tile, tcgen05 cta_group::2; dense layout only, the
+ * grouped layouts fall back to pair = 0). Other values: FG_ERR_INVALID_ARG.
  */
-fg_status fg_set_ue8m0_tile_width(int width);
+fg_status fg_set_ue8m0_tile(int width, int pair);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

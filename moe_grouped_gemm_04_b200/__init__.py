@@ -12,7 +12,7 @@ The functions carry the C names:
   fp8_gemm_nt, fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked,
   per_token_cast_to_fp8_ue8m0, per_block_cast_to_fp8_ue8m0, and the GEMMs for
   power-of-two scales fp8_gemm_nt_ue8m0, fp8_grouped_gemm_contiguous_ue8m0,
-  fp8_grouped_gemm_masked_ue8m0 (set_ue8m0_tile_width tunes them)
+  fp8_grouped_gemm_masked_ue8m0 (set_ue8m0_tile tunes them)
 plus allocation helpers that return tensors in the layouts the kernels use.
 """
 from __future__ import annotations
@@ -37,7 +37,7 @@ EXPORTED = (
     "per_token_cast_to_fp8_ue8m0", "per_block_cast_to_fp8_ue8m0", "fp8_gemm_nt",
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
     "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
-    "fg_set_ue8m0_tile_width", "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
+    "fg_set_ue8m0_tile", "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
 
 
@@ -74,7 +74,7 @@ def load_library() -> ctypes.CDLL:
     lib.fp8_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, I, I, I, P]
     lib.fp8_grouped_gemm_contiguous_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fp8_grouped_gemm_masked_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
-    lib.fg_set_ue8m0_tile_width.argtypes = [I]
+    lib.fg_set_ue8m0_tile.argtypes = [I, I]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
     lib.fg_status_string.argtypes = [I]
@@ -86,7 +86,7 @@ def load_library() -> ctypes.CDLL:
               "fp8_gemm_nt",
               "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
               "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0",
-              "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile_width",
+              "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
     _lib = lib
@@ -270,9 +270,10 @@ def fp8_grouped_gemm_masked_ue8m0(A: torch.Tensor, sfa: torch.Tensor, B: torch.T
                  expected_m, stream)
 
 
-def set_ue8m0_tile_width(width: int) -> None:
-    """0 = automatic (default); 128, 224 or 256 = force that weight-tile width."""
-    _check(load_library().fg_set_ue8m0_tile_width(int(width)))
+def set_ue8m0_tile(width: int, pair: bool = False) -> None:
+    """0 = automatic (default); else force weight tiles of `width` rows (128,
+    224 or 256 single-CTA, or 224 as a CTA pair)."""
+    _check(load_library().fg_set_ue8m0_tile(int(width), 1 if pair else 0))
 
 
 def get_device_status(stream=None) -> int:

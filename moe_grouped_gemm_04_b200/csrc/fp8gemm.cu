@@ -426,39 +426,64 @@ fg_status run_gemm(const Problem& pr, int expected_m, cudaStream_t stream) {
 
 // ---------------------------------------------------------------- UE8M0 GEMM
 
-//                  BW  stages accumulators epilogue warps per quadrant
-using MxN128 = MxCfg<128, 5, 2, 1>;
-using MxN224 = MxCfg<224, 4, 2, 1>;
-using MxN256 = MxCfg<256, 3, 1, 2>;
+//                  BW  stages accumulators epilogue-warps/quadrant pair K-blocks/stage
+using MxN128 = MxCfg<128, 5, 2, 1, false, 1>;
+using MxN224 = MxCfg<224, 4, 2, 1, false, 1>;
+using MxN256 = MxCfg<256, 3, 1, 2, false, 1>;
+using MxP224 = MxCfg<224, 3, 2, 1, true, 2>;  // dense: CTA pairs, 256 x 224 tiles
 
+// Shared-memory attribute and, for pair configs, the number of co-resident
+// clusters (the persistent grid's size).
 template <class C, int FORM>
-fg_status mx_kernel_attr(int dev) {
+fg_status mx_kernel_attr(int dev, int* max_clusters) {
   static bool done[kMaxDevices] = {};
+  static int clusters[kMaxDevices] = {};
   if (!done[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(fp8_gemm_mx_kernel<C, FORM>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               C::smem_bytes(FORM));
+    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_mx_kernel<C, FORM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::smem_bytes(FORM));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if (C::CLUSTER > 1) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = C::CLUSTER;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(C::CLUSTER * 64);
+      cfg.blockDim = dim3(C::NUM_THREADS);
+      cfg.dynamicSmemBytes = C::smem_bytes(FORM);
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, fp8_gemm_mx_kernel<C, FORM>, &cfg);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+      if (n < 1) return fail(FG_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", C::CLUSTER);
+      clusters[dev] = n;
+    }
     done[dev] = true;
   }
+  *max_clusters = clusters[dev];
   return FG_OK;
 }
 
 template <class C, int FORM>
 fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
   static_assert(C::smem_bytes(FORM) <= 232448, "shared memory per CTA");
-  FG_TRY((mx_kernel_attr<C, FORM>(dev_id)));
+  int max_clusters = 0;
+  FG_TRY((mx_kernel_attr<C, FORM>(dev_id, &max_clusters)));
   const int KB = pr.K / 128;
   CUtensorMap tmA, tmB, tmSA, tmD;
   FG_TRY(make_map(&tmA, pr.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
                   static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
                   CU_TENSOR_MAP_SWIZZLE_128B, "A"));
   FG_TRY(make_map(&tmB, pr.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
-                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::BW,
+                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::B_ROWS,
                   CU_TENSOR_MAP_SWIZZLE_128B, "B"));
+  // token scales: boxes of 128 tokens x 4 K blocks (one quad)
   FG_TRY(make_map(&tmSA, pr.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.M,
                   static_cast<uint64_t>(pr.slabs) * KB,
-                  static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 1,
+                  static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 4,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
   // D as rows x N bf16 in boxes of 32 rows x 32 columns, 64-byte swizzled
   FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
@@ -479,11 +504,12 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
   p.masked_m = pr.masked_m;
   p.status = dev.status;
   p.timeout_ns = wait_limit_ns();
-  int64_t tiles = static_cast<int64_t>(p.num_mt) * p.num_nt;
+  int64_t tiles = static_cast<int64_t>(C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
   if (FORM == kFormMasked) tiles *= pr.G;  // upper bound: masked_m lives on the device
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(tiles, dev.sm_count));
+  const int64_t grid = C::PAIR ? C::CLUSTER * std::max<int64_t>(1, std::min<int64_t>(tiles, max_clusters))
+                               : std::max<int64_t>(1, std::min<int64_t>(tiles, dev.sm_count));
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(C::NUM_THREADS);
   cfg.dynamicSmemBytes = C::smem_bytes(FORM);
@@ -492,66 +518,88 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (C::CLUSTER > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C::CLUSTER;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_mx_kernel<C, FORM>, tmA, tmB, tmSA,
                                            tmD, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_mx_kernel launch");
   return FG_OK;
 }
 
-// Weight-tile width of the block-scaled kernel: the candidate whose tiles
-// fill the SMs in the fewest rounds, counting a round by its MMA work (the
-// tile width) and a small surcharge for the narrow tile (its MMAs read more
-// shared memory per flop) and the single-accumulator one (its MMAs wait for
-// each tile's accumulator to be read).
-int mx_tile_width(const Problem& pr, int sm_count, int expected_m) {
+// Tile of the block-scaled kernel: the candidate whose tiles fill the SMs in
+// the fewest rounds, a round costed by its MMA work (the tile width) times a
+// per-candidate factor for how close the candidate's MMAs run to the tensor
+// peak (the single-CTA tiles stream more operand bytes per MMA than the stage
+// ring keeps in flight; the narrow tile also reads more shared memory per
+// flop; the single-accumulator tile waits for each accumulator to be read).
+struct MxPlan {
+  int bw;
+  bool pair;
+};
+
+MxPlan mx_plan(const Problem& pr, int sm_count, int expected_m) {
   int64_t token_tiles = (pr.M + 127) / 128;
   if (pr.form == kFormMasked) token_tiles = static_cast<int64_t>((expected_m + 127) / 128) * pr.G;
-  const struct { int bw; double weight; } cand[] = {{224, 1.0}, {256, 1.03}, {128, 1.10}};
-  int best = 224;
+  const struct { int bw; bool pair; double weight; } cand[] = {
+      {224, true, 1.0}, {224, false, 1.45}, {256, false, 1.5}, {128, false, 1.6}};
+  MxPlan best{224, false};
   double best_cost = 1e300;
   for (const auto& c : cand) {
-    const int64_t tiles = token_tiles * ((pr.N + c.bw - 1) / c.bw);
-    const int64_t rounds = (tiles + sm_count - 1) / sm_count;
+    if (c.pair && pr.form != kFormDense) continue;  // pair tiles: dense layout
+    const int64_t nt = (pr.N + c.bw - 1) / c.bw;
+    const int64_t tiles = c.pair ? (token_tiles + 1) / 2 * nt : token_tiles * nt;
+    const int64_t units = c.pair ? sm_count / 2 : sm_count;
+    const int64_t rounds = (tiles + units - 1) / units;
     const double cost = static_cast<double>(rounds) * c.bw * c.weight;
     if (cost < best_cost) {
       best_cost = cost;
-      best = c.bw;
+      best = MxPlan{c.bw, c.pair};
     }
   }
   return best;
 }
 
 template <int FORM>
-fg_status dispatch_mx(const Problem& pr, int bw, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
-  switch (bw) {
+fg_status dispatch_mx(const Problem& pr, MxPlan pl, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
+  if constexpr (FORM == kFormDense) {
+    if (pl.pair) return launch_mx<MxP224, FORM>(pr, dev, dev_id, stream);
+  }
+  switch (pl.bw) {
     case 128: return launch_mx<MxN128, FORM>(pr, dev, dev_id, stream);
     case 256: return launch_mx<MxN256, FORM>(pr, dev, dev_id, stream);
     default: return launch_mx<MxN224, FORM>(pr, dev, dev_id, stream);
   }
 }
 
+// fg_set_ue8m0_tile: 0 = automatic, else the forced width (+ pair flag)
+std::atomic<int> g_mx_tile{0};
+
 // Power-of-two scales: the block-scaled kernel for token tiles of 128 rows;
 // thin shapes (dense M <= 64, masked with expected_m <= 64) take the swapped
 // promotion kernel, whose per-block scaling is exact for such scales too.
-std::atomic<int> g_mx_tile_width{0};  // fg_set_ue8m0_tile_width (0 = automatic)
-
 fg_status run_gemm_mx(const Problem& pr, int expected_m, cudaStream_t stream) {
-  const int force_bw = g_mx_tile_width.load(std::memory_order_relaxed);
+  const int forced = g_mx_tile.load(std::memory_order_relaxed);
   DeviceInfo* dev = nullptr;
   FG_TRY(device_info(&dev));
   int dev_id = 0;
   cudaGetDevice(&dev_id);
   const int small_m = pr.form == kFormDense ? pr.M : pr.form == kFormMasked ? expected_m : 1 << 30;
-  if (small_m <= 64 && force_bw == 0) return run_gemm(pr, expected_m, stream);
+  if (small_m <= 64 && forced == 0) return run_gemm(pr, expected_m, stream);
   if (pr.form == kFormContig && (pr.M + 127) / 128 > kTableMax)
     return fail(FG_ERR_UNSUPPORTED, "M_total %d exceeds %d rows", pr.M, kTableMax * 128);
   if (pr.form == kFormMasked && pr.G + 1 > kTableMax)
     return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d experts", pr.G, kTableMax - 1);
-  const int bw = force_bw ? force_bw : mx_tile_width(pr, dev->sm_count, expected_m);
+  MxPlan pl = forced ? MxPlan{forced & 0xFFFF, (forced >> 16) != 0} : mx_plan(pr, dev->sm_count, expected_m);
+  if (pl.pair && pr.form != kFormDense) pl.pair = false;  // pair tiles: dense layout
   switch (pr.form) {
-    case kFormDense: return dispatch_mx<kFormDense>(pr, bw, *dev, dev_id, stream);
-    case kFormContig: return dispatch_mx<kFormContig>(pr, bw, *dev, dev_id, stream);
-    default: return dispatch_mx<kFormMasked>(pr, bw, *dev, dev_id, stream);
+    case kFormDense: return dispatch_mx<kFormDense>(pr, pl, *dev, dev_id, stream);
+    case kFormContig: return dispatch_mx<kFormContig>(pr, pl, *dev, dev_id, stream);
+    default: return dispatch_mx<kFormMasked>(pr, pl, *dev, dev_id, stream);
   }
 }
 
@@ -761,10 +809,12 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
   return run_gemm_mx(pr, expected_m, stream);
 }
 
-fg_status fg_set_ue8m0_tile_width(int width) {
-  if (width != 0 && width != 128 && width != 224 && width != 256)
-    return fail(FG_ERR_INVALID_ARG, "tile width %d: 0 (automatic), 128, 224 or 256", width);
-  g_mx_tile_width.store(width, std::memory_order_relaxed);
+fg_status fg_set_ue8m0_tile(int width, int pair) {
+  const bool ok = width == 0 || (pair ? width == 224 : (width == 128 || width == 224 || width == 256));
+  if (!ok)
+    return fail(FG_ERR_INVALID_ARG, "tile %d%s: 0 (automatic), 128, 224, 256, or 224 as a pair",
+                width, pair ? " (pair)" : "");
+  g_mx_tile.store(width == 0 ? 0 : (width | (pair ? 1 << 16 : 0)), std::memory_order_relaxed);
   return FG_OK;
 }
 

@@ -14,24 +14,36 @@
 // fp32 in global memory (the layouts of gemm.cuh); the kernel takes their
 // exponent bytes.
 //
+// Scale words: the block-scaled MMA reads, per row, a 32-bit word from tensor
+// memory and uses the byte its scale-factor id selects. One word carries the
+// scales of four consecutive 128-wide K blocks (byte k = K block 4q + k), so
+// the scale groups are converted and copied to tensor memory once per four K
+// blocks (a "quad"), through their own ring of SFS slots.
+//
+// The MMA-issuing thread is the critical resource: on sm_100a each tcgen05
+// instruction occupies it for tens of cycles, so everything else it does per
+// K block (barrier waits, scale copies, commits, bookkeeping) directly idles
+// the tensor pipe. Hence quads, KPS K blocks per pipeline stage (one wait and
+// one commit per stage) and a non-blocking peek at the next stage's barrier
+// while the current stage's MMAs are being issued.
+//
 // CTA roles (one CTA per SM, persistent over 128-token x BW-weight tiles):
-//   warp 0      producer: lane 0 loads the weight tile, lane 1 the token
-//               tile of each K block onto the stage's "full" barrier (TMA);
-//               lane 2 the fp32 scales of the stage onto its "sa full"
-//               barrier: the 128 token scales with one TMA copy, the (at most
-//               three) weight-block scales the tile's rows touch with 4-byte
-//               cp.async copies.
-//   warp 1      MMA issuer: per K block copies the stage's scale groups from
-//               shared to tensor memory (tcgen05.cp) and issues 4 block-scaled
-//               MMAs (K = 32 each) into the tile's accumulator; commits the
-//               stage to "empty" and, after the last K block, the accumulator
-//               to "tmem full".
-//   warp 2      scale converter: per K block takes the staged fp32 scales of
-//               the tile's 128 token rows and BW weight rows, keeps their
-//               exponent bytes (UE8M0 has the fp32 exponent's bias) and writes
-//               them in the shared layout tcgen05.cp expects, then arrives on
-//               the stage's "sf full" barrier. (Everything it reads is already
-//               in shared memory, staged as deep as the operand tiles.)
+//   warp 0      producer: lane 0 loads the weight tiles, lane 1 the token
+//               tiles of each stage's K blocks onto its "full" barrier (TMA);
+//               lane 2 the fp32 scales of each quad onto its "sa full"
+//               barrier: the 128 x 4 token scales with one TMA copy, the (at
+//               most three per K block) weight-block scales the tile's rows
+//               touch with 4-byte cp.async copies.
+//   warp 1      MMA issuer (converged warp, one elected lane issues): per
+//               quad, waits for its scale groups and copies
+//               them to tensor memory (tcgen05.cp); per K block 4 block-scaled
+//               MMAs (K = 32 each) into the tile's accumulator; commits each
+//               stage to "empty", each quad to "sf empty" and each finished
+//               accumulator to "tmem full".
+//   warp 2      scale converter: per quad takes the staged fp32 scales,
+//               keeps their exponent bytes (UE8M0 has the fp32 exponent's
+//               bias), packs four K blocks per word in the shared layout
+//               tcgen05.cp expects and arrives on the slot's "sf full".
 //   warp 3      idle (keeps the epilogue warps aligned to TMEM lane quadrants)
 //   warps 4..   epilogue: per tile, 32 accumulator columns at a time from
 //               tensor memory to registers, bf16, a 64-byte-swizzled shared
@@ -40,6 +52,16 @@
 // With two accumulators (BW <= 224) the epilogue of one tile overlaps the
 // MMAs of the next; with BW = 256 the MMAs wait for the accumulator to be
 // read (8 epilogue warps keep that short).
+//
+// Pair form (PAIR, dense layout): the two CTAs of a cluster compute one tile
+// of 256 tokens x BW weights with tcgen05 cta_group::2. Each CTA loads its 128
+// token rows and half of the weight rows. The block-scaled pair MMA reads, in
+// each CTA's tensor memory, the scales of that CTA's token rows and of all BW
+// weight rows, so both CTAs stage and convert the weight scales of the whole
+// tile. The leader (rank 0) issues the copies, MMAs and commits, which arrive
+// on both CTAs' barriers; operand bytes of both CTAs complete on the leader's
+// "full" barrier; the peer's converter and epilogue arrive on the leader's
+// "sf full" and "tmem empty" barriers through the cluster.
 #pragma once
 
 #include <cstdint>
@@ -50,44 +72,56 @@
 
 namespace fg {
 
-template <int BW_, int STAGES_, int ACC_, int EPQ_>
+template <int BW_, int STAGES_, int ACC_, int EPQ_, bool PAIR_, int KPS_>
 struct MxCfg {
-  static constexpr int BT = 128;          // token rows per tile (MMA M)
+  static constexpr int BT = 128;          // token rows per CTA tile
   static constexpr int BW = BW_;          // weight rows per tile (MMA N)
   static constexpr bool SWAP = false;     // tile helpers of gemm.cuh: tokens on the lanes
-  static constexpr bool PAIR = false;
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int CLUSTER = PAIR ? 2 : 1;
+  static constexpr int MMA_M = PAIR ? 256 : 128;
+  static constexpr int B_ROWS = PAIR ? BW / 2 : BW;  // weight rows this CTA loads
   static constexpr int STAGES = STAGES_;
+  static constexpr int KPS = KPS_;        // K blocks per pipeline stage
+  static_assert(KPS == 1 || KPS == 2 || KPS == 4, "stages tile the 4-block quads");
   static constexpr int ACC = ACC_;        // accumulators in tensor memory
   static constexpr int EPQ = EPQ_;        // epilogue warps per TMEM lane quadrant
-  static_assert(BW % 32 == 0 && BW >= 32 && BW <= 256, "tcgen05 N for M = 128, 32-column chunks");
+  static_assert(BW % 32 == 0 && BW >= 32 && BW <= 256, "tcgen05 N, 32-column chunks");
+  static_assert(!PAIR || B_ROWS % 16 == 0, "pair: half tiles of whole 8-row swizzle atoms");
   static constexpr int EW = 4 * EPQ;      // epilogue warps
   static constexpr int ECOLS = BW / EPQ;  // accumulator columns per epilogue warp
   static_assert(ECOLS % 32 == 0, "epilogue chunks of 32 columns");
   static constexpr int EPI_BASE = 4;      // first epilogue warp
   static constexpr int NUM_THREADS = (EPI_BASE + EW) * 32;
-  // scale-factor groups per stage: 128 token rows, ceil(BW / 128) x 128 weight rows
+  // scale groups of one slot: 128 token rows, ceil(BW / 128) x 128 weight rows
   static constexpr int SFB_GROUPS = (BW + 127) / 128;
-  static constexpr int SF_COLS = 4 * (1 + SFB_GROUPS);    // tensor-memory columns per stage
-  static constexpr int SF_BYTES = 512 * (1 + SFB_GROUPS);  // shared bytes per stage
-  // staged fp32 scales per stage: 128 token scales, then the scales of the
-  // (at most NBT) 128-row weight blocks the tile's rows touch
+  static constexpr int SF_COLS = 4 * (1 + SFB_GROUPS);    // tensor-memory columns per slot
+  static constexpr int SF_BYTES = 512 * (1 + SFB_GROUPS);  // shared bytes per slot
+  static constexpr int SFS = 3;           // scale slots (quads in flight)
+  // staged fp32 scales of a quad: 4 x 128 token scales (one TMA box), then
+  // 4 x NBT weight-block scales ([k][j]: K block 4q + k, block nb0 + j)
   static constexpr int NBT = SFB_GROUPS + 1;
-  static constexpr int RAW_BYTES = 512 + 128;
-  static constexpr int TMEM_USED = ACC * BW + STAGES * SF_COLS;
+  static constexpr int RAW_A = 4 * 512;
+  static constexpr int RAW_BYTES = RAW_A + 128;
+  static constexpr int RAWS = 2;          // staged-scale ring
+  static_assert(4 * NBT * 4 <= RAW_BYTES - RAW_A, "staged weight-block scales");
+  static constexpr int TMEM_USED = ACC * BW + SFS * SF_COLS;
   static_assert(TMEM_USED <= 512, "TMEM has 512 columns");
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
                                    : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
-  static constexpr int A_BYTES = BT * 128;
-  static constexpr int B_BYTES = BW * 128;
+  static constexpr int A_BYTES = BT * 128;       // one K block of the token tile
+  static constexpr int B_BYTES = B_ROWS * 128;   // one K block of this CTA's weight rows
+  static constexpr int STAGE_A = KPS * A_BYTES;
+  static constexpr int STAGE_B = KPS * B_BYTES;
   static constexpr int EPI_RING = 2;         // image buffers per epilogue warp
   static constexpr int BOX_BYTES = 32 * 64;  // 32 rows x 32 bf16 columns
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_RAW = OFF_SF + STAGES * SF_BYTES;  // 128-byte aligned
-  static constexpr int OFF_EPI = (OFF_RAW + STAGES * RAW_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
+  static constexpr int OFF_SF = OFF_B + STAGES * STAGE_B;
+  static constexpr int OFF_RAW = OFF_SF + SFS * SF_BYTES;  // 128-byte aligned
+  static constexpr int OFF_EPI = (OFF_RAW + RAWS * RAW_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_EPI + EW * EPI_RING * BOX_BYTES;
-  static constexpr int NUM_BARS = 4 * STAGES + 2 * ACC;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * SFS + 2 * RAWS + 2 * ACC;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int table_bytes(int form) { return form == kFormDense ? 0 : kTableMax * 4; }
@@ -96,8 +130,7 @@ struct MxCfg {
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(OFF_SF % 128 == 0 && OFF_RAW % 128 == 0 && RAW_BYTES % 128 == 0,
                 "scale groups and staged scales: 128-byte aligned");
-  static_assert(NBT * 4 <= RAW_BYTES - 512, "staged weight-block scales");
-  static_assert(smem_bytes(kFormContig) <= 232448, "shared memory per CTA");
+  static_assert(smem_bytes(PAIR ? kFormDense : kFormContig) <= 232448, "shared memory per CTA");
 };
 
 // 16-byte chunk c (columns 8c .. 8c + 7) of row r of a 32-row x 64-byte box
@@ -105,11 +138,8 @@ struct MxCfg {
 // offset are XORed with bits 7-8, i.e. with (r / 2) % 4.
 __device__ __forceinline__ int sw64_offset(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
 
-// UE8M0 byte of an fp32 power of two: its biased exponent, replicated into
-// the four bytes of a scale word (the MMA reads byte 0).
-__device__ __forceinline__ uint32_t ue8m0_word(float s) {
-  return ((__float_as_uint(s) >> 23) & 0xFFu) * 0x01010101u;
-}
+// UE8M0 byte of an fp32 power of two: its biased exponent.
+__device__ __forceinline__ uint32_t ue8m0_byte(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
 // Bounded wait of a whole warp: lane 0 polls, every lane returns its verdict.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
@@ -118,11 +148,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// Position in a ring of N slots, advanced one use at a time: slot index and
+// the parity of the slot's current phase.
+template <int N>
+struct Ring {
+  uint32_t slot = 0, phase = 0;
+  __device__ __forceinline__ void next() {
+    if (++slot == N) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 template <class C, int FORM>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmD,
                        const GemmParams p) {
+  static_assert(!C::PAIR || FORM == kFormDense, "pair tiles cover the dense layout");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem + C::OFF_A;
@@ -131,27 +175,38 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   uint8_t* sRAW = smem + C::OFF_RAW;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* sf_full = empty + C::STAGES;  // the stage's scale groups are written
-  uint64_t* sa_full = sf_full + C::STAGES;  // the stage's fp32 scales have landed
-  uint64_t* tfull = sa_full + C::STAGES;  // an accumulator holds a finished tile
-  uint64_t* tempty = tfull + C::ACC;      // ... and has been read by the epilogue
+  uint64_t* sf_full = empty + C::STAGES;    // a scale slot's groups are written (both CTAs)
+  uint64_t* sf_empty = sf_full + C::SFS;    // ... and the quad's MMAs have completed
+  uint64_t* sa_full = sf_empty + C::SFS;    // a quad's fp32 scales have landed
+  uint64_t* sa_empty = sa_full + C::RAWS;   // ... and the converter has read them
+  uint64_t* tfull = sa_empty + C::RAWS;     // an accumulator holds a finished tile
+  uint64_t* tempty = tfull + C::ACC;        // ... and has been read by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* table = reinterpret_cast<int*>(smem + C::OFF_TABLE);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int rank = C::PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int t_first = C::PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int t_step = C::PAIR ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 2);      // weight- and token-tile lanes' expect_tx
+      mbar_init(&full[s], 2);      // weight- and token-tile lanes' expect_tx (the leader's, for a pair)
       mbar_init(&empty[s], 1);     // the MMA commit
-      mbar_init(&sf_full[s], 1);   // the converter warp
-      mbar_init(&sa_full[s], 2);   // scale lane: expect_tx (TMA) + cp.async arrival
+    }
+    for (int q = 0; q < C::SFS; ++q) {
+      mbar_init(&sf_full[q], C::CLUSTER);  // the converter warp of each CTA
+      mbar_init(&sf_empty[q], 1);          // the MMA commit after the quad
+    }
+    for (int r = 0; r < C::RAWS; ++r) {
+      mbar_init(&sa_full[r], 2);   // scale lane: expect_tx (TMA) + cp.async arrival
+      mbar_init(&sa_empty[r], 1);  // the converter
     }
     for (int b = 0; b < C::ACC; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::EW);  // one arrival per epilogue warp
+      mbar_init(&tempty[b], C::CLUSTER * C::EW);  // one arrival per epilogue warp (of both CTAs)
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -160,53 +215,63 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&tmSA);
     tma_prefetch_desc(&tmD);
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+  if constexpr (!C::PAIR) {
+    if (warp == 1) {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
+  // Peers address this CTA's barriers only after the cluster barrier
+  // completes (its wait comes after the CTA-wide barrier below).
+  __syncwarp();
+  if constexpr (C::PAIR) cluster_arrive_relaxed();
   // Everything above may overlap the previous kernel; memory comes after this.
   grid_dependency_wait();
   if (warp == 0) build_table<C, FORM>(p, table, lane);
   tc_fence_before();
-  __syncwarp();
   __syncthreads();
+  if constexpr (C::PAIR) {
+    cluster_wait();
+    // the pair's tensor memory, allocated jointly once both CTAs run
+    if (warp == 1) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   tc_fence_after();
 
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_sf = tmem_base + static_cast<uint32_t>(C::ACC * C::BW);
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   const int total = total_tiles<C, FORM>(p, table);
+  const int KQ = (p.KB + 3) >> 2;  // quads per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane < 3) {
-      uint32_t it = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
-        const Tile w = resolve_tile<C, FORM>(p, table, t, 0);
+    if (lane < 2) {
+      Ring<C::STAGES> st;
+      uint32_t fills = 0;
+      for (int t = t_first; t < total; t += t_step) {
+        const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
         if (!w.valid) continue;
-        // weight blocks the tile's rows touch (clamped: rows past N are never stored)
-        const int nb0 = (w.nt * C::BW) >> 7;
-        const float* sfb_e = p.sfb + static_cast<int64_t>(w.e) * p.NB * p.KB;
-        for (int kb = 0; kb < p.KB; ++kb, ++it) {
-          const int s = it % C::STAGES;
-          if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1u) ^ 1u, ctl)) goto producer_done;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[s], C::B_BYTES);
-            tma_load_2d(sB + s * C::B_BYTES, &tmB, &full[s], kb * 128, w.e * p.N + w.nt * C::BW);
-          } else if (lane == 1) {
-            mbar_arrive_expect_tx(&full[s], C::A_BYTES);
-            tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * 128,
-                        (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT);
+        const int row = lane == 0 ? w.e * p.N + w.nt * C::BW + rank * C::B_ROWS
+                                  : (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
+        const CUtensorMap* map = lane == 0 ? &tmB : &tmA;
+        const uint32_t bytes = lane == 0 ? C::B_BYTES : C::A_BYTES;
+        for (int kb0 = 0; kb0 < p.KB; kb0 += C::KPS, st.next(), ++fills) {
+          if (!mbar_wait(&empty[st.slot], st.phase ^ 1u, ctl)) goto producer_done;
+          const int nk = min(C::KPS, p.KB - kb0);
+          uint8_t* dst = lane == 0 ? sB + st.slot * C::STAGE_B : sA + st.slot * C::STAGE_A;
+          if constexpr (C::PAIR) {
+            // both CTAs' operand bytes complete on the leader's barrier
+            if (rank == 0) mbar_arrive_expect_tx(&full[st.slot], 2 * nk * bytes);
+            const uint32_t bar = mapa_shared(smem_u32(&full[st.slot]), 0);
+            for (int j = 0; j < nk; ++j) tma_load_2d_pair(dst + j * bytes, map, bar, (kb0 + j) * 128, row);
           } else {
-            uint8_t* raw = sRAW + s * C::RAW_BYTES;
-            mbar_arrive_expect_tx(&sa_full[s], 512);
-            // token scales past M read as zero (their rows are never stored)
-            tma_load_2d(raw, &tmSA, &sa_full[s], w.mt * C::BT,
-                        (FORM == kFormMasked ? w.e * p.KB : 0) + kb);
-#pragma unroll
-            for (int j = 0; j < C::NBT; ++j)
-              cp_async_4(raw + 512 + 4 * j, sfb_e + static_cast<int64_t>(min(nb0 + j, p.NB - 1)) * p.KB + kb);
-            cp_async_mbar_arrive(&sa_full[s]);
+            mbar_arrive_expect_tx(&full[st.slot], nk * bytes);
+            for (int j = 0; j < nk; ++j) tma_load_2d(dst + j * bytes, map, &full[st.slot], (kb0 + j) * 128, row);
           }
         }
       }
@@ -214,62 +279,140 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       // the last fill of every stage has landed and been consumed before the
       // CTA releases its shared memory
       if (lane == 0) {
-        for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
-          const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
-          drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
-          drain_wait(&empty[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+        for (uint32_t s = 0; s < C::STAGES && s < fills; ++s) {
+          const uint32_t last = (fills - 1 - s) / C::STAGES * C::STAGES + s;
+          // (a pair's operand bytes complete on the leader's barrier)
+          if (!C::PAIR || rank == 0) drain_wait(&full[last % C::STAGES], (last / C::STAGES) & 1u, kDrainLimitNs);
+          drain_wait(&empty[last % C::STAGES], (last / C::STAGES) & 1u, kDrainLimitNs);
         }
-      } else if (lane == 2) {
-        for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
-          const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
-          drain_wait(&sa_full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
+      }
+    } else if (lane == 2) {
+      Ring<C::RAWS> rr;
+      uint32_t fills = 0;
+      for (int t = t_first; t < total; t += t_step) {
+        const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
+        if (!w.valid) continue;
+        // weight blocks the tile's rows touch (clamped: rows past N are never stored)
+        const int nb0 = (w.nt * C::BW) >> 7;
+        const float* sfb_e = p.sfb + static_cast<int64_t>(w.e) * p.NB * p.KB;
+        for (int qi = 0; qi < KQ; ++qi, rr.next(), ++fills) {
+          if (!mbar_wait(&sa_empty[rr.slot], rr.phase ^ 1u, ctl)) goto scales_done;
+          uint8_t* raw = sRAW + rr.slot * C::RAW_BYTES;
+          mbar_arrive_expect_tx(&sa_full[rr.slot], C::RAW_A);
+          // 4 K blocks of token scales; rows past M read as zero, K blocks past
+          // the tile's last one are never used
+          tma_load_2d(raw, &tmSA, &sa_full[rr.slot], w.mt * C::BT,
+                      (FORM == kFormMasked ? w.e * p.KB : 0) + 4 * qi);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int kb = min(4 * qi + k, p.KB - 1);
+#pragma unroll
+            for (int j = 0; j < C::NBT; ++j)
+              cp_async_4(raw + C::RAW_A + 4 * (k * C::NBT + j),
+                         sfb_e + static_cast<int64_t>(min(nb0 + j, p.NB - 1)) * p.KB + kb);
+          }
+          cp_async_mbar_arrive(&sa_full[rr.slot]);
         }
+      }
+    scales_done:
+      for (uint32_t r = 0; r < C::RAWS && r < fills; ++r) {
+        const uint32_t last = (fills - 1 - r) / C::RAWS * C::RAWS + r;
+        drain_wait(&sa_full[last % C::RAWS], (last / C::RAWS) & 1u, kDrainLimitNs);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = mma_idesc_e4m3_bs(C::BT, C::BW);
-      uint32_t it = 0, tc = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
-        const Tile w = resolve_tile<C, FORM>(p, table, t, 0);
+    // The whole warp runs the loop (converged, so that descriptors and
+    // addresses stay warp-uniform); one elected lane issues the tcgen05
+    // instructions, the same lane every time (copies and the MMAs that read
+    // them must come from one thread).
+    if (rank == 0) {  // a pair's MMAs are issued by its leader
+      constexpr uint32_t idesc = mma_idesc_e4m3_bs(C::MMA_M, C::BW);
+      Ring<C::STAGES> st;
+      Ring<C::SFS> sq;
+      uint32_t tc = 0;
+      bool ready = false;  // the current stage's "full" phase was seen complete by a peek
+      for (int t = t_first; t < total; t += t_step) {
+        const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
         if (!w.valid) continue;
         const int b = tc % C::ACC;
-        if (!mbar_wait(&tempty[b], ((tc / C::ACC) & 1u) ^ 1u, ctl)) goto mma_done;
+        if (!warp_wait(&tempty[b], ((tc / C::ACC) & 1u) ^ 1u, ctl, lane)) goto mma_done;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::BW);
-        for (int kb = 0; kb < p.KB; ++kb, ++it) {
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(&full[s], ph, ctl)) goto mma_done;
-          if (!mbar_wait(&sf_full[s], ph, ctl)) goto mma_done;
+        for (int kb0 = 0; kb0 < p.KB; kb0 += C::KPS, st.next()) {
+          if (!ready && !warp_wait(&full[st.slot], st.phase, ctl, lane)) goto mma_done;
           tc_fence_after();
-          // the stage's scale groups into its own tensor-memory columns
-          // (a copy is ordered before the MMAs this thread issues after it)
-          const uint32_t sf = tmem_sf + static_cast<uint32_t>(s * C::SF_COLS);
-          const uint32_t sf_smem = smem_u32(sSF + s * C::SF_BYTES);
-          tmem_cp_sf_group(sf, sf_smem);
+          const uint32_t a_base = smem_u32(sA + st.slot * C::STAGE_A);
+          const uint32_t b_base = smem_u32(sB + st.slot * C::STAGE_B);
 #pragma unroll
-          for (int g = 0; g < C::SFB_GROUPS; ++g)
-            tmem_cp_sf_group(sf + 4 + 4 * g, sf_smem + 512 * (1 + g));
-          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * C::A_BYTES));
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * C::B_BYTES));
+          for (int j = 0; j < C::KPS; ++j) {
+            const int kb = kb0 + j;
+            if (kb >= p.KB) break;
+            const uint32_t k4 = static_cast<uint32_t>(kb & 3);
+            const uint32_t sf = tmem_sf + sq.slot * C::SF_COLS;
+            if (k4 == 0) {
+              // a new quad: its scale groups (both CTAs') into tensor memory
+              if (!warp_wait(&sf_full[sq.slot], sq.phase, ctl, lane)) goto mma_done;
+              tc_fence_after();
+              const uint32_t src = smem_u32(sSF + sq.slot * C::SF_BYTES);
+              if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)  // 32 bytes (= 32 e4m3 along K) per MMA
-            mma_f8_bs(d, adesc + 2 * k, bdesc + 2 * k, idesc, sf, sf + 4, (kb | k) != 0 ? 1u : 0u);
-          mma_commit(&empty[s]);
+                for (int g = 0; g <= C::SFB_GROUPS; ++g) {
+                  if constexpr (C::PAIR) tmem_cp_sf_group_pair(sf + 4 * g, src + 512 * g);
+                  else tmem_cp_sf_group(sf + 4 * g, src + 512 * g);
+                }
+              }
+            }
+            // byte k4 of each scale word: this K block's scales
+            const uint32_t sfa = sf | (k4 << 30);
+            const uint32_t sfb = (sf + 4) | (k4 << 30);
+            const uint32_t id = idesc | (k4 << 4) | (k4 << 29);
+            const uint64_t adesc = smem_desc_sw128(a_base + j * C::A_BYTES);
+            const uint64_t bdesc = smem_desc_sw128(b_base + j * C::B_BYTES);
+            const bool last_of_quad = k4 == 3 || kb == p.KB - 1;
+            if (elect_one()) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {  // 32 bytes (= 32 e4m3 along K) per MMA
+                if constexpr (C::PAIR)
+                  mma_f8_bs_pair(d, adesc + 2 * k, bdesc + 2 * k, id, sfa, sfb, (kb | k) != 0 ? 1u : 0u);
+                else
+                  mma_f8_bs(d, adesc + 2 * k, bdesc + 2 * k, id, sfa, sfb, (kb | k) != 0 ? 1u : 0u);
+              }
+              if (last_of_quad) {
+                // the quad's scale slot is free once these MMAs complete
+                if constexpr (C::PAIR) mma_commit_pair(&sf_empty[sq.slot]);
+                else mma_commit(&sf_empty[sq.slot]);
+              }
+            }
+            if (last_of_quad) sq.next();
+          }
+          // peek at the next stage while this stage's MMAs execute
+          {
+            Ring<C::STAGES> nx = st;
+            nx.next();
+            const int r = lane == 0 ? (mbar_test_wait(&full[nx.slot], nx.phase) ? 1 : 0) : 0;
+            ready = __shfl_sync(0xffffffffu, r, 0) != 0;
+          }
+          if (elect_one()) {
+            if constexpr (C::PAIR) mma_commit_pair(&empty[st.slot]);  // both CTAs' stage
+            else mma_commit(&empty[st.slot]);
+          }
         }
-        mma_commit(&tfull[b]);
+        if (elect_one()) {
+          if constexpr (C::PAIR) mma_commit_pair(&tfull[b]);
+          else mma_commit(&tfull[b]);
+        }
         ++tc;
       }
     mma_done:
-      if (tc > 0) drain_wait(&tfull[(tc - 1) % C::ACC], ((tc - 1) / C::ACC) & 1u, kDrainLimitNs);
+      if (tc > 0 && lane == 0) drain_wait(&tfull[(tc - 1) % C::ACC], ((tc - 1) / C::ACC) & 1u, kDrainLimitNs);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale converter
-    uint32_t it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile w = resolve_tile<C, FORM>(p, table, t, 0);
+    Ring<C::RAWS> rr;
+    Ring<C::SFS> sq;
+    for (int t = t_first; t < total; t += t_step) {
+      const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
       if (!w.valid) continue;
       // staged weight-block index of this lane's weight rows lane + 32 r1 + 128 g
       const int n0 = w.nt * C::BW;
@@ -278,23 +421,52 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       for (int g = 0; g < C::SFB_GROUPS; ++g)
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1) jb[g][r1] = ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
-      for (int kb = 0; kb < p.KB; ++kb, ++it) {
-        const int s = it % C::STAGES;
-        // the stage's scales have landed (and, since the producer refilled the
-        // stage, its previous scale groups have been copied out)
-        if (!warp_wait(&sa_full[s], (it / C::STAGES) & 1u, ctl, lane)) goto convert_done;
-        const float* raw = reinterpret_cast<const float*>(sRAW + s * C::RAW_BYTES);
-        uint8_t* grp = sSF + s * C::SF_BYTES + lane * 16;
-        *reinterpret_cast<uint4*>(grp) = make_uint4(ue8m0_word(raw[lane]), ue8m0_word(raw[lane + 32]),
-                                                    ue8m0_word(raw[lane + 64]), ue8m0_word(raw[lane + 96]));
+      for (int qi = 0; qi < KQ; ++qi, rr.next(), sq.next()) {
+        // the quad's scales have landed, and the slot's previous quad has
+        // been copied out and its MMAs have completed
+        if (!warp_wait(&sa_full[rr.slot], rr.phase, ctl, lane)) goto convert_done;
+        if (!warp_wait(&sf_empty[sq.slot], sq.phase ^ 1u, ctl, lane)) goto convert_done;
+        const float* raw = reinterpret_cast<const float*>(sRAW + rr.slot * C::RAW_BYTES);
+        const int nk = min(4, p.KB - 4 * qi);  // K blocks of this quad
+        uint32_t wa[4] = {0, 0, 0, 0};
+        uint32_t wb[C::SFB_GROUPS][4];
 #pragma unroll
         for (int g = 0; g < C::SFB_GROUPS; ++g)
-          *reinterpret_cast<uint4*>(grp + 512 * (1 + g)) =
-              make_uint4(ue8m0_word(raw[128 + jb[g][0]]), ue8m0_word(raw[128 + jb[g][1]]),
-                         ue8m0_word(raw[128 + jb[g][2]]), ue8m0_word(raw[128 + jb[g][3]]));
-        fence_proxy_async_shared();  // visible to tcgen05.cp (async proxy)
+#pragma unroll
+          for (int r1 = 0; r1 < 4; ++r1) wb[g][r1] = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (k < nk) {
+#pragma unroll
+            for (int r1 = 0; r1 < 4; ++r1) wa[r1] |= ue8m0_byte(raw[k * 128 + 32 * r1 + lane]) << (8 * k);
+#pragma unroll
+            for (int g = 0; g < C::SFB_GROUPS; ++g)
+#pragma unroll
+              for (int r1 = 0; r1 < 4; ++r1)
+                wb[g][r1] |= ue8m0_byte(raw[C::RAW_A / 4 + k * C::NBT + jb[g][r1]]) << (8 * k);
+          }
+        }
+        uint8_t* grp = sSF + sq.slot * C::SF_BYTES + lane * 16;
+        *reinterpret_cast<uint4*>(grp) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+#pragma unroll
+        for (int g = 0; g < C::SFB_GROUPS; ++g)
+          *reinterpret_cast<uint4*>(grp + 512 * (1 + g)) = make_uint4(wb[g][0], wb[g][1], wb[g][2], wb[g][3]);
+        // visible to this CTA's async proxy (which executes tcgen05.cp for
+        // this CTA's shared memory, also when the leader issues it) before
+        // the arrival leaves this thread
+        fence_proxy_async_shared();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_full[s]);
+        if (lane == 0) {
+          mbar_arrive(&sa_empty[rr.slot]);
+          // (a remote arrival with cluster-scope release stalls the issuing
+          // thread for about a microsecond; the leader issues the copy only
+          // after observing this arrival, by which time the writes above are
+          // visible to the async proxy)
+          if (C::PAIR && rank != 0)
+            mbar_arrive_remote(mapa_shared(smem_u32(&sf_full[sq.slot]), 0));
+          else
+            mbar_arrive(&sf_full[sq.slot]);
+        }
       }
     }
   convert_done:;
@@ -303,12 +475,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     const int ew = warp - C::EPI_BASE;
     const int quad = warp & 3;          // TMEM lanes this warp may access
     const int c0 = (ew >> 2) * C::ECOLS;
-    const int row = quad * 32 + lane;   // token row of the tile
+    const int row = quad * 32 + lane;   // token row of this CTA's tile
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     uint8_t* ring = smem + C::OFF_EPI + ew * C::EPI_RING * C::BOX_BYTES;
     uint32_t tc = 0, boxes = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile w = resolve_tile<C, FORM>(p, table, t, 0);
+    for (int t = t_first; t < total; t += t_step) {
+      const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
       if (!w.valid) continue;
       int m_valid = p.M;
       if (FORM == kFormMasked) {
@@ -334,7 +506,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           // the accumulator is in registers: the next tile's MMAs may start
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[b]);
+          if (lane == 0) {
+            if (C::PAIR && rank != 0)  // the leader's MMA waits for both CTAs
+              mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+            else
+              mbar_arrive(&tempty[b]);
+          }
         }
         if (staged) {
           uint8_t* img = ring + (boxes % C::EPI_RING) * C::BOX_BYTES;
@@ -373,11 +550,19 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   // ---------------------------------------------------------------- teardown
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (C::PAIR) {
+    // each CTA arrives only after the MMAs writing its tensor memory and
+    // reading its shared memory have completed (drained above)
+    cluster_arrive_relaxed();
+    cluster_wait();
+  } else {
+    __syncthreads();
+  }
   grid_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (C::PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 

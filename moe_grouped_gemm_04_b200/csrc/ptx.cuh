@@ -50,6 +50,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One lane of a converged warp (the lowest active one) gets true. Issuing
+// tcgen05 instructions from converged warp code under this election keeps
+// their descriptors and addresses warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared state every bounded wait consults: a CTA-wide abort flag in shared
 // memory and the device status word in global memory.
 struct WaitCtl {
@@ -257,15 +283,17 @@ __host__ __device__ constexpr uint32_t mma_idesc_e4m3(int M, int N) {
 
 // Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale: e4m3 A
 // and B, both K-major, shape M x N, scale factors in UE8M0 (power-of-two)
-// format, scale-factor id 0 for both operands (byte 0 of each scale word).
-__host__ __device__ constexpr uint32_t mma_idesc_e4m3_bs(int M, int N) {
-  return (0u << 4)                                  // B scale-factor id
+// format; `sf_id` selects the byte of each 32-bit scale word that scales this
+// MMA's 32-wide K slice (the same id goes into bits 30-31 of the scale
+// tensor-memory addresses).
+__host__ __device__ constexpr uint32_t mma_idesc_e4m3_bs(int M, int N, uint32_t sf_id = 0) {
+  return (sf_id << 4)                               // B scale-factor id
          | (0u << 7) | (0u << 10)                   // A, B format: e4m3
          | (0u << 15) | (0u << 16)                  // A, B K-major
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (1u << 23)                               // scale format: UE8M0
          | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
-         | (0u << 29);                              // A scale-factor id
+         | (sf_id << 29);                           // A scale-factor id
 }
 
 // D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T with one UE8M0 scale per

@@ -22,7 +22,8 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 SENTINEL = 0xFFFF
-WIDTHS = [128, 224, 256]
+# forced tiles: (weight rows, CTA pair); (0, False) = the automatic choice
+TILES = [(128, False), (224, False), (256, False), (224, True), (0, False)]
 
 
 @pytest.fixture(scope="module")
@@ -32,14 +33,15 @@ def fg():
     import moe_grouped_gemm_04_b200 as m
     m.load_library()
     yield m
-    m.set_ue8m0_tile_width(0)
+    m.set_ue8m0_tile(0)
 
 
-@pytest.fixture(params=WIDTHS + [0], ids=lambda w: "w%d" % w if w else "auto")
+@pytest.fixture(params=TILES, ids=lambda t: ("p%d" if t[1] else "w%d") % t[0] if t[0] else "auto")
 def width(request, fg):
-    fg.set_ue8m0_tile_width(request.param)
-    yield request.param
-    fg.set_ue8m0_tile_width(0)
+    w, pair = request.param
+    fg.set_ue8m0_tile(w, pair)
+    yield w + (1000 if pair else 0)
+    fg.set_ue8m0_tile(0)
 
 
 def _d_tensor(shape):
