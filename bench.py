@@ -1,6 +1,7 @@
 """Benchmark of the FP8 block-scaled GEMM hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--scales fp32|ue8m0]
 
 One step is one pass of the per-call hot path over one batch of synthetic
 input: the activation quantizer (per token, per 128 channels) followed by the
@@ -24,6 +25,8 @@ repeats the step through the public API from pinned host buffers with the
 host<->device copies inside the timed region (uploads, compute and downloads
 of consecutive steps pipelined on three streams, as a serving loop would);
 `cpu_baseline` times the CPU oracle on a bounded sample of the same workload.
+`--scales ue8m0` quantizes with power-of-two scales and runs the block-scaled
+GEMM entry points (the oracle then uses the same power-of-two quantizers).
 
 Multi-GPU (torchrun, one process per GPU): the path does not shard across
 GPUs within one call, so every rank runs an independent replica (weak
@@ -66,6 +69,9 @@ def parse_args():
     ap.add_argument("--workload", default="decode_64x4096x7168", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--with-weight-quant", action="store_true")
+    ap.add_argument("--scales", default="fp32", choices=["fp32", "ue8m0"],
+                    help="fp32: scale = amax / 448 (the promoted GEMM); ue8m0: power-of-two "
+                         "scales (the _ue8m0 quantizers and the block-scaled GEMM)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps from Python instead of replaying a CUDA graph")
     ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
@@ -172,7 +178,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------- CPU legs
 
-def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
+def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict, ue8m0: bool = False):
     """Oracle on a bounded sample of the workload: quantize the sampled A rows
     and compute their outputs against all N columns (weights are quantized
     outside the timed part, as on the GPU side). Returns
@@ -193,7 +199,7 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
     def weights(e):
         if e not in cache:
             b = inp.b if kind == "dense" else inp.b[e]
-            cache[e] = oracle.per_block_cast(b, threads=threads)
+            cache[e] = oracle.per_block_cast(b, threads=threads, ue8m0=ue8m0)
         return cache[e]
 
     order = np.random.default_rng(0).permutation(len(a_rows))
@@ -203,7 +209,7 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
         for e in np.unique(experts[take]):
             weights(int(e))
         t0 = time.perf_counter()
-        qa, sa = oracle.per_token_cast(a_rows[take], threads=threads)
+        qa, sa = oracle.per_token_cast(a_rows[take], threads=threads, ue8m0=ue8m0)
         for e in np.unique(experts[take]):
             sub = np.nonzero(experts[take] == e)[0]
             qb, sb = weights(int(e))
@@ -220,7 +226,7 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict):
         passes = max(1, int(target_s / max(dt, 1e-3)))
         t0 = time.perf_counter()
         for _ in range(passes):
-            qa, sa = oracle.per_token_cast(a_rows, threads=threads)
+            qa, sa = oracle.per_token_cast(a_rows, threads=threads, ue8m0=ue8m0)
             for e in np.unique(experts):
                 sub = np.nonzero(experts == e)[0]
                 qb, sb = weights(int(e))
@@ -246,6 +252,13 @@ def max_over_ranks(dist, values, device):
 
 
 # ---------------------------------------------------------------------- GPU leg
+
+def gemm_kernel_name(kind: str, inp, ue8m0: bool) -> str:
+    """The GEMM kernel a step launches (the library's choice for the shape)."""
+    thin = (kind == "dense" and inp.M <= 64) or (
+        kind == "masked" and max(1, int(round(float(np.mean(inp.masked_m))))) <= 64)
+    return "fp8_gemm_mx_kernel" if ue8m0 and not thin else "fp8_gemm_kernel"
+
 
 class OperandSet:
     """Device buffers of one copy of a step's operands."""
@@ -282,9 +295,17 @@ class Step:
     With `sets` > 1 the copies are used in turn, so that a step's weights and
     activations are not in L2 when it starts (their total exceeds L2)."""
 
-    def __init__(self, fg, torch, kind, inp, with_weight_quant: bool, min_total_bytes: int):
+    def __init__(self, fg, torch, kind, inp, with_weight_quant: bool, min_total_bytes: int,
+                 ue8m0: bool = False):
         self.fg, self.torch, self.kind, self.inp = fg, torch, kind, inp
         self.with_wq = with_weight_quant
+        self.ue8m0 = ue8m0
+        sfx = "_ue8m0" if ue8m0 else ""
+        self.q_token = getattr(fg, "per_token_cast_to_fp8" + sfx)
+        self.q_block = getattr(fg, "per_block_cast_to_fp8" + sfx)
+        self.g_dense = getattr(fg, "fp8_gemm_nt" + sfx)
+        self.g_contig = getattr(fg, "fp8_grouped_gemm_contiguous" + sfx)
+        self.g_masked = getattr(fg, "fp8_grouped_gemm_masked" + sfx)
         dev = "cuda"
         K, N = inp.K, inp.N
 
@@ -295,7 +316,7 @@ class Step:
         Gw = 1 if kind == "dense" else inp.G
         B = torch.empty((N, K) if kind == "dense" else (inp.G, N, K), dtype=torch.uint8, device=dev)
         SB = fg.empty_sfb(Gw, N, K, dev)
-        fg.per_block_cast_to_fp8(w, B, SB)
+        self.q_block(w, B, SB)
         if kind == "contiguous":
             self.mi = torch.from_numpy(inp.m_indices).to(dev)
         if kind == "masked":
@@ -310,19 +331,18 @@ class Step:
         self.set_bytes = per
 
     def quant_weights(self, o):
-        self.fg.per_block_cast_to_fp8(o.w, o.B, o.SB)
+        self.q_block(o.w, o.B, o.SB)
 
     def quant_acts(self, o):
-        self.fg.per_token_cast_to_fp8(o.x, o.A, o.SA)
+        self.q_token(o.x, o.A, o.SA)
 
     def gemm(self, o):
-        fg = self.fg
         if self.kind == "dense":
-            fg.fp8_gemm_nt(o.A, o.SA, o.B, o.SB, o.D)
+            self.g_dense(o.A, o.SA, o.B, o.SB, o.D)
         elif self.kind == "contiguous":
-            fg.fp8_grouped_gemm_contiguous(o.A, o.SA, o.B, o.SB, o.D, self.mi)
+            self.g_contig(o.A, o.SA, o.B, o.SB, o.D, self.mi)
         else:
-            fg.fp8_grouped_gemm_masked(o.A, o.SA, o.B, o.SB, o.D, self.mm, self.expected_m)
+            self.g_masked(o.A, o.SA, o.B, o.SB, o.D, self.mm, self.expected_m)
 
     def launches_per_step(self):
         return 2 + (1 if self.with_wq else 0)
@@ -346,8 +366,9 @@ def run_ours(args, rank, world, local_rank):
     inp = workloads.make(args.workload, seed=0)
     flops, alg_bytes = workloads.flops_and_bytes(kind, inp)
     rotate = args.l2 == "rotate"
+    ue8m0 = args.scales == "ue8m0"
     step = Step(fg, torch, kind, inp, args.with_weight_quant,
-                ROTATE_MIN_BYTES if rotate else 0)
+                ROTATE_MIN_BYTES if rotate else 0, ue8m0)
     R = len(step.sets)
     stream = torch.cuda.current_stream()
     if not rotate:
@@ -518,7 +539,7 @@ def run_ours(args, rank, world, local_rank):
                 "frac": achieved / peak}
         peak_note = "%s HBM copy bandwidth (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
     roof["traffic"] = traffic_for(args.workload)
-    roof["kernel"] = "fp8_gemm_kernel"
+    roof["kernel"] = gemm_kernel_name(kind, inp, ue8m0)
     roof["algorithmic_per_launch"] = {"flops": flops, "bytes": alg_bytes}
     roof["kernel_ms"] = gms
     roof["peak_source"] = peak_note
@@ -527,7 +548,7 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_cpu_baseline:
         import oracle
         threads = oracle.hardware_threads()
-        fps, desc, secs = cpu_sample(inp, kind, args.cpu_seconds, threads, {})
+        fps, desc, secs = cpu_sample(inp, kind, args.cpu_seconds, threads, {}, ue8m0)
         cpu = {"value": fps / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc, "seconds": secs}
 
@@ -539,6 +560,8 @@ def run_ours(args, rank, world, local_rank):
            "launch": ("the K timed steps captured in one CUDA graph, replayed once untimed, "
                       "then once between the events") if use_graph else "eager launches from Python",
            "weights": "quantized inside every step" if args.with_weight_quant else "quantized once before timing",
+           "scales": ("power-of-two (UE8M0) scales, block-scaled tensor-core GEMM" if ue8m0 else
+                      "fp32 scales amax/448, promoted per 128-wide K block"),
            "parallelism": "replicas" if world > 1 else "single GPU"}
     if kind == "dense":
         cfg["M"] = inp.M
@@ -676,17 +699,19 @@ def run_reference(args, rank, world):
     threads = oracle.hardware_threads()
     per_step = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     cache = {}
+    ue8m0 = args.scales == "ue8m0"
     for _ in range(args.warmup):
-        cpu_sample(inp, kind, per_step, threads, cache)
+        cpu_sample(inp, kind, per_step, threads, cache, ue8m0)
     vals, descs, secs = [], [], []
     for _ in range(args.steps):
-        fps, desc, s = cpu_sample(inp, kind, per_step, threads, cache)
+        fps, desc, s = cpu_sample(inp, kind, per_step, threads, cache, ue8m0)
         vals.append(fps)
         descs.append(desc)
         secs.append(s)
     value = float(np.mean(vals)) / 1e12
     ms = float(np.mean(secs)) * 1e3
-    cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K}
+    cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K,
+           "scales": "power-of-two (UE8M0)" if ue8m0 else "fp32 amax/448"}
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,

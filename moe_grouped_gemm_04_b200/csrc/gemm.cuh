@@ -18,9 +18,10 @@
 //               stage's "full" barrier. (A thread's tensor copies complete one
 //               after another at a roughly fixed time per copy, so one thread
 //               per stream keeps three copies in flight per stage.)
-//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one
-//               of two TMEM partial buffers, then commits to the stage's
-//               "empty" barrier and the buffer's "tmem full" barrier.
+//   warp 1      MMA issuer (converged warp, one elected lane issues): 4 x
+//               tcgen05.mma (K = 32 each) per K block into one of two TMEM
+//               partial buffers, then commits to the stage's "empty" barrier
+//               and the buffer's "tmem full" barrier.
 //   promotion warps (2..5, or 4..11 in the 8-warp form whose warps 2-3 idle
 //   so that warpgroup 0 holds the single-lane roles and can give registers
 //   to the promotion warpgroups): per K block read the partial from TMEM
@@ -517,7 +518,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && pair_rank == 0) {  // a pair's MMAs are issued by its leader
+    // The whole warp runs the loop (converged: descriptors stay
+    // warp-uniform, which keeps each tcgen05 issue short); one elected lane
+    // issues the MMAs and commits.
+    if (pair_rank == 0) {  // a pair's MMAs are issued by its leader
       constexpr uint32_t idesc = mma_idesc_e4m3(C::MMA_M, C::MMA_N);
       uint32_t it = 0;
       for (int t = t_first; t < total; t += t_step) {
@@ -528,39 +532,41 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           const uint32_t ph = (it / C::STAGES) & 1u;
           const int b = it & 1;
           const uint32_t tph = (it >> 1) & 1u;
-          if (!mbar_wait(&tempty[b], tph ^ 1u, ctl)) goto mma_done;
+          if (!warp_wait(&tempty[b], tph ^ 1u, ctl, lane)) goto mma_done;
           tc_fence_after();
-          if (!mbar_wait(&full[s], ph, ctl)) goto mma_done;
+          if (!warp_wait(&full[s], ph, ctl, lane)) goto mma_done;
           tc_fence_after();
+          if (elect_one()) {
 #pragma unroll
-          for (int j = 0; j < C::KPS; ++j) {
-            if (kq + j * kb_step >= p.KB) break;
-            const uint8_t* a_tile = sA + s * C::STAGE_A + j * C::A_BYTES;
-            const uint8_t* b_tile = sB + s * C::STAGE_B + j * C::B_BYTES;
-            const uint64_t adesc = smem_desc_sw128(smem_u32(C::SWAP ? b_tile : a_tile));
-            const uint64_t bdesc = smem_desc_sw128(smem_u32(C::SWAP ? a_tile : b_tile));
-            // one fresh partial per K block: slot (b, j) of tensor memory
-            const uint32_t d = tmem_base + static_cast<uint32_t>((b * C::KPS + j) * C::MMA_N);
+            for (int j = 0; j < C::KPS; ++j) {
+              if (kq + j * kb_step >= p.KB) break;
+              const uint8_t* a_tile = sA + s * C::STAGE_A + j * C::A_BYTES;
+              const uint8_t* b_tile = sB + s * C::STAGE_B + j * C::B_BYTES;
+              const uint64_t adesc = smem_desc_sw128(smem_u32(C::SWAP ? b_tile : a_tile));
+              const uint64_t bdesc = smem_desc_sw128(smem_u32(C::SWAP ? a_tile : b_tile));
+              // one fresh partial per K block: slot (b, j) of tensor memory
+              const uint32_t d = tmem_base + static_cast<uint32_t>((b * C::KPS + j) * C::MMA_N);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              // advance 32 bytes (= 32 e4m3 along K) inside the 128-byte swizzled row
-              if constexpr (C::PAIR)
-                mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-              else
-                mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+              for (int k = 0; k < 4; ++k) {
+                // advance 32 bytes (= 32 e4m3 along K) inside the 128-byte swizzled row
+                if constexpr (C::PAIR)
+                  mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+                else
+                  mma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+              }
             }
-          }
-          if constexpr (C::PAIR) {
-            mma_commit_pair(&empty[s]);  // both CTAs' stage s and TMEM buffer b
-            mma_commit_pair(&tfull[b]);
-          } else {
-            mma_commit(&empty[s]);
-            mma_commit(&tfull[b]);
+            if constexpr (C::PAIR) {
+              mma_commit_pair(&empty[s]);  // both CTAs' stage s and TMEM buffer b
+              mma_commit_pair(&tfull[b]);
+            } else {
+              mma_commit(&empty[s]);
+              mma_commit(&tfull[b]);
+            }
           }
         }
       }
     mma_done:
-      if (it > 0) drain_wait(&tfull[(it - 1) & 1], ((it - 1) >> 1) & 1u, kDrainLimitNs);
+      if (it > 0 && lane == 0) drain_wait(&tfull[(it - 1) & 1], ((it - 1) >> 1) & 1u, kDrainLimitNs);
     }
   }  // warps 2 .. PW_BASE - 1 (8-warp form) idle
   } else {

@@ -141,13 +141,6 @@ __device__ __forceinline__ int sw64_offset(int r, int c) { return r * 64 + ((c ^
 // UE8M0 byte of an fp32 power of two: its biased exponent.
 __device__ __forceinline__ uint32_t ue8m0_byte(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
-// Bounded wait of a whole warp: lane 0 polls, every lane returns its verdict.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
-  int ok = 1;
-  if (lane == 0) ok = mbar_wait(bar, parity, ctl) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 // Position in a ring of N slots, advanced one use at a time: slot index and
 // the parity of the slot's current phase.
 template <int N>

@@ -115,6 +115,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   return mbar_wait_slow(bar, parity, ctl.abort_flag, ctl.status, ctl.limit_ns);
 }
 
+// Bounded wait of a whole warp: lane 0 polls, every lane returns its verdict.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int lane) {
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(bar, parity, ctl) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // ---------------------------------------------------------------- TMA / cp.async
 
 // 4-byte asynchronous copy global -> shared (L1-allocating).
