@@ -192,8 +192,8 @@ fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint
  * write). The kernel keeps only each scale's exponent field: a scale that is
  * not a power of two acts as the power of two at or below it, zero as 2^-127.
  *
- * For token tiles of 128 rows (dense: pairs of them, computed by the two CTAs
- * of a cluster) the scales are applied inside the tensor core (tcgen05.mma
+ * For token tiles of 128 rows (or pairs of them of one expert, computed by
+ * the two CTAs of a cluster) the scales are applied inside the tensor core (tcgen05.mma
  * kind::mxf8f6f4.block_scale, one UE8M0 scale per row per 32 K elements), and
  * the whole K range accumulates in tensor memory in fp32 with no promotion
  * pass; the products a * b * sa * sb are exact, only the order of
@@ -218,8 +218,8 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
  * tile per shape (default). Otherwise always use the block-scaled kernel, thin
  * shapes included, with weight tiles of `width` rows: 128, 224 or 256 with
  * pair = 0 (one CTA per 128-token tile), or 224 with pair = 1 (two CTAs of a
- * cluster per 256-token tile, tcgen05 cta_group::2; dense layout only, the
- * grouped layouts fall back to pair = 0). Other values: FG_ERR_INVALID_ARG.
+ * cluster per pair of token tiles of one expert, tcgen05 cta_group::2).
+ * Other values: FG_ERR_INVALID_ARG.
  */
 fg_status fg_set_ue8m0_tile(int width, int pair);
 

@@ -430,7 +430,7 @@ fg_status run_gemm(const Problem& pr, int expected_m, cudaStream_t stream) {
 using MxN128 = MxCfg<128, 5, 2, 1, false, 1>;
 using MxN224 = MxCfg<224, 4, 2, 1, false, 1>;
 using MxN256 = MxCfg<256, 3, 1, 2, false, 1>;
-using MxP224 = MxCfg<224, 3, 2, 1, true, 2>;  // dense: CTA pairs, 256 x 224 tiles
+using MxP224 = MxCfg<224, 3, 2, 1, true, 2>;  // CTA pairs, 256 x 224 tiles
 
 // Shared-memory attribute and, for pair configs, the number of co-resident
 // clusters (the persistent grid's size).
@@ -543,16 +543,24 @@ struct MxPlan {
 };
 
 MxPlan mx_plan(const Problem& pr, int sm_count, int expected_m) {
+  // token tiles, and token-tile pairs (pairs never span experts: masked
+  // slabs pair within an expert; contiguous runs likewise, counted here as
+  // if the groups' tiles paired perfectly)
   int64_t token_tiles = (pr.M + 127) / 128;
-  if (pr.form == kFormMasked) token_tiles = static_cast<int64_t>((expected_m + 127) / 128) * pr.G;
+  int64_t pairs = (token_tiles + 1) / 2;
+  if (pr.form == kFormMasked) {
+    const int64_t per_expert = (expected_m + 127) / 128;
+    token_tiles = per_expert * pr.G;
+    pairs = (per_expert + 1) / 2 * pr.G;
+  }
+  // relative cost of one tile's MMA work per SM, measured on B200
   const struct { int bw; bool pair; double weight; } cand[] = {
-      {224, true, 1.0}, {224, false, 1.45}, {256, false, 1.5}, {128, false, 1.6}};
+      {224, true, 1.0}, {224, false, 1.15}, {256, false, 1.4}, {128, false, 1.5}};
   MxPlan best{224, false};
   double best_cost = 1e300;
   for (const auto& c : cand) {
-    if (c.pair && pr.form != kFormDense) continue;  // pair tiles: dense layout
     const int64_t nt = (pr.N + c.bw - 1) / c.bw;
-    const int64_t tiles = c.pair ? (token_tiles + 1) / 2 * nt : token_tiles * nt;
+    const int64_t tiles = (c.pair ? pairs : token_tiles) * nt;
     const int64_t units = c.pair ? sm_count / 2 : sm_count;
     const int64_t rounds = (tiles + units - 1) / units;
     const double cost = static_cast<double>(rounds) * c.bw * c.weight;
@@ -566,9 +574,7 @@ MxPlan mx_plan(const Problem& pr, int sm_count, int expected_m) {
 
 template <int FORM>
 fg_status dispatch_mx(const Problem& pr, MxPlan pl, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
-  if constexpr (FORM == kFormDense) {
-    if (pl.pair) return launch_mx<MxP224, FORM>(pr, dev, dev_id, stream);
-  }
+  if (pl.pair) return launch_mx<MxP224, FORM>(pr, dev, dev_id, stream);
   switch (pl.bw) {
     case 128: return launch_mx<MxN128, FORM>(pr, dev, dev_id, stream);
     case 256: return launch_mx<MxN256, FORM>(pr, dev, dev_id, stream);
@@ -595,7 +601,6 @@ fg_status run_gemm_mx(const Problem& pr, int expected_m, cudaStream_t stream) {
   if (pr.form == kFormMasked && pr.G + 1 > kTableMax)
     return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d experts", pr.G, kTableMax - 1);
   MxPlan pl = forced ? MxPlan{forced & 0xFFFF, (forced >> 16) != 0} : mx_plan(pr, dev->sm_count, expected_m);
-  if (pl.pair && pr.form != kFormDense) pl.pair = false;  // pair tiles: dense layout
   switch (pr.form) {
     case kFormDense: return dispatch_mx<kFormDense>(pr, pl, *dev, dev_id, stream);
     case kFormContig: return dispatch_mx<kFormContig>(pr, pl, *dev, dev_id, stream);

@@ -53,8 +53,13 @@
 // MMAs of the next; with BW = 256 the MMAs wait for the accumulator to be
 // read (8 epilogue warps keep that short).
 //
-// Pair form (PAIR, dense layout): the two CTAs of a cluster compute one tile
-// of 256 tokens x BW weights with tcgen05 cta_group::2. Each CTA loads its 128
+// Pair form (PAIR): the two CTAs of a cluster compute one tile of 256 tokens
+// x BW weights with tcgen05 cta_group::2. Dense: token tiles 2j and 2j + 1.
+// Masked: consecutive token tiles of one expert's slab. Contiguous: a "pair
+// unit" table built by warp 0 pairs consecutive token tiles within each run
+// of tiles of one expert; a run of odd length ends with a unit whose second
+// tile belongs to no row of that expert (it still loads its half of the
+// weight tile, which the leader's MMAs need, and stores nothing). Each CTA loads its 128
 // token rows and half of the weight rows. The block-scaled pair MMA reads, in
 // each CTA's tensor memory, the scales of that CTA's token rows and of all BW
 // weight rows, so both CTAs stage and convert the weight scales of the whole
@@ -124,13 +129,16 @@ struct MxCfg {
   static constexpr int NUM_BARS = 2 * STAGES + 2 * SFS + 2 * RAWS + 2 * ACC;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int table_bytes(int form) { return form == kFormDense ? 0 : kTableMax * 4; }
+  // grouped layouts: token-tile table; contiguous pairs: + the pair-unit table
+  static constexpr int table_bytes(int form) {
+    return form == kFormDense ? 0 : (form == kFormContig && PAIR ? 2 : 1) * kTableMax * 4;
+  }
   static constexpr int smem_bytes(int form) { return OFF_TABLE + table_bytes(form) + 1024; }
 
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(OFF_SF % 128 == 0 && OFF_RAW % 128 == 0 && RAW_BYTES % 128 == 0,
                 "scale groups and staged scales: 128-byte aligned");
-  static_assert(smem_bytes(PAIR ? kFormDense : kFormContig) <= 232448, "shared memory per CTA");
+  static_assert(smem_bytes(kFormContig) <= 232448, "shared memory per CTA");
 };
 
 // 16-byte chunk c (columns 8c .. 8c + 7) of row r of a 32-row x 64-byte box
@@ -140,6 +148,123 @@ __device__ __forceinline__ int sw64_offset(int r, int c) { return r * 64 + ((c ^
 
 // UE8M0 byte of an fp32 power of two: its biased exponent.
 __device__ __forceinline__ uint32_t ue8m0_byte(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
+
+// Tables of the grouped layouts, built by warp 0 before the main loops.
+// Contiguous: table[mt] = expert of token tile mt (from its first row; -1 for
+// padding tiles); with pairs also units[u] = first token tile of pair unit u
+// and *num_units. Masked: table[e] = exclusive prefix over experts of the
+// number of (token tile or tile pair, weight tile) work items.
+template <class C, int FORM>
+__device__ void mx_build_table(const GemmParams& p, int* table, int* num_units, int lane) {
+  if constexpr (FORM == kFormContig) {
+    for (int mt = lane; mt < p.num_mt; mt += 32) {
+      int v = __ldg(p.m_indices + static_cast<int64_t>(mt) * C::BT);
+      if (v >= p.G) {
+        raise_status(p.status, 3 /* FG_DEVICE_BAD_M_INDEX */);
+        v = -1;
+      }
+      table[mt] = v < 0 ? -1 : v;
+    }
+    if constexpr (C::PAIR) {
+      __syncwarp();
+      int* units = table + kTableMax;
+      int count = 0;
+      int run_start = 0;  // first tile of the run the previous chunk ended in
+      int prev_e = -2;    // expert of the previous chunk's last tile
+      for (int base = 0; base < p.num_mt; base += 32) {
+        const int mt = base + lane;
+        const int e = mt < p.num_mt ? table[mt] : -3;
+        int e_before = __shfl_up_sync(0xffffffffu, e, 1);
+        if (lane == 0) e_before = prev_e;
+        // start of this tile's run: the last run start at or before it
+        int rs = (mt < p.num_mt && e != e_before) ? mt : -1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, rs, o);
+          if (lane >= o) rs = max(rs, v);
+        }
+        if (rs < 0) rs = run_start;
+        // a unit starts at every other tile of a run of one expert
+        const bool unit = mt < p.num_mt && e >= 0 && ((mt - rs) & 1) == 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, unit);
+        if (unit) units[count + __popc(bal & ((1u << lane) - 1u))] = mt;
+        count += __popc(bal);
+        run_start = __shfl_sync(0xffffffffu, rs, 31);
+        prev_e = __shfl_sync(0xffffffffu, e, 31);
+      }
+      if (lane == 0) *num_units = count;
+    }
+  } else if constexpr (FORM == kFormMasked) {
+    const int per = (p.G + 31) / 32;
+    const int e0 = lane * per;
+    const int e1 = min(p.G, e0 + per);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) {
+      int mm = __ldg(p.masked_m + e);
+      if (mm < 0 || mm > p.M) {
+        raise_status(p.status, 2 /* FG_DEVICE_BAD_MASKED_M */);
+        mm = mm < 0 ? 0 : p.M;
+      }
+      int rows = (mm + C::BT - 1) / C::BT;  // token tiles
+      if (C::PAIR) rows = (rows + 1) / 2;    // ... or tile pairs
+      const int cnt = rows * p.num_nt;
+      table[e + 1] = cnt;
+      local += cnt;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      run += table[e + 1];
+      table[e + 1] = run;
+    }
+    if (lane == 0) table[0] = 0;
+  }
+}
+
+template <class C, int FORM>
+__device__ __forceinline__ int mx_total(const GemmParams& p, const int* table, int num_units) {
+  if (FORM == kFormMasked) return table[p.G];
+  if (FORM == kFormContig && C::PAIR) return num_units * p.num_nt;
+  return (C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
+}
+
+// Work item t of this CTA (rank = its place in the pair; 0 without pairs).
+template <class C, int FORM>
+__device__ __forceinline__ Tile mx_resolve(const GemmParams& p, const int* table, int t, int rank) {
+  Tile w;
+  w.valid = 1;
+  if (FORM == kFormMasked) {
+    int lo = 0, hi = p.G;  // table[lo] <= t < table[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (table[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int local = t - table[lo];
+    w.e = lo;
+    w.mt = C::PAIR ? 2 * (local / p.num_nt) + rank : local / p.num_nt;
+    w.nt = local % p.num_nt;
+  } else if (FORM == kFormContig && C::PAIR) {
+    const int mt0 = table[kTableMax + t / p.num_nt];
+    w.e = table[mt0];
+    w.mt = mt0 + rank;
+    w.nt = t % p.num_nt;
+  } else {
+    w.mt = C::PAIR ? 2 * (t / p.num_nt) + rank : t / p.num_nt;
+    w.nt = t % p.num_nt;
+    if (FORM == kFormContig) {
+      w.e = table[w.mt];
+      w.valid = w.e >= 0;
+    } else {
+      w.e = 0;
+    }
+  }
+  return w;
+}
 
 // Position in a ring of N slots, advanced one use at a time: slot index and
 // the parity of the slot's current phase.
@@ -159,7 +284,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmD,
                        const GemmParams p) {
-  static_assert(!C::PAIR || FORM == kFormDense, "pair tiles cover the dense layout");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem + C::OFF_A;
@@ -177,6 +301,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* table = reinterpret_cast<int*>(smem + C::OFF_TABLE);
+  int* num_units = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -220,7 +345,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   if constexpr (C::PAIR) cluster_arrive_relaxed();
   // Everything above may overlap the previous kernel; memory comes after this.
   grid_dependency_wait();
-  if (warp == 0) build_table<C, FORM>(p, table, lane);
+  if (warp == 0) mx_build_table<C, FORM>(p, table, num_units, lane);
   tc_fence_before();
   __syncthreads();
   if constexpr (C::PAIR) {
@@ -238,7 +363,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_sf = tmem_base + static_cast<uint32_t>(C::ACC * C::BW);
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-  const int total = total_tiles<C, FORM>(p, table);
+  const int total = mx_total<C, FORM>(p, table, *num_units);
   const int KQ = (p.KB + 3) >> 2;  // quads per tile
 
   if (warp == 0) {
@@ -247,7 +372,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       Ring<C::STAGES> st;
       uint32_t fills = 0;
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
+        const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
         if (!w.valid) continue;
         const int row = lane == 0 ? w.e * p.N + w.nt * C::BW + rank * C::B_ROWS
                                   : (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
@@ -283,7 +408,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       Ring<C::RAWS> rr;
       uint32_t fills = 0;
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
+        const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
         if (!w.valid) continue;
         // weight blocks the tile's rows touch (clamped: rows past N are never stored)
         const int nb0 = (w.nt * C::BW) >> 7;
@@ -326,7 +451,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       uint32_t tc = 0;
       bool ready = false;  // the current stage's "full" phase was seen complete by a peek
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
+        const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
         if (!w.valid) continue;
         const int b = tc % C::ACC;
         if (!warp_wait(&tempty[b], ((tc / C::ACC) & 1u) ^ 1u, ctl, lane)) goto mma_done;
@@ -405,7 +530,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     Ring<C::RAWS> rr;
     Ring<C::SFS> sq;
     for (int t = t_first; t < total; t += t_step) {
-      const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
+      const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
       if (!w.valid) continue;
       // staged weight-block index of this lane's weight rows lane + 32 r1 + 128 g
       const int n0 = w.nt * C::BW;
@@ -473,7 +598,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     uint8_t* ring = smem + C::OFF_EPI + ew * C::EPI_RING * C::BOX_BYTES;
     uint32_t tc = 0, boxes = 0;
     for (int t = t_first; t < total; t += t_step) {
-      const Tile w = resolve_tile<C, FORM>(p, table, t, rank);
+      const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
       if (!w.valid) continue;
       int m_valid = p.M;
       if (FORM == kFormMasked) {
@@ -482,7 +607,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       }
       const int m = w.mt * C::BT + row;
       int row_mi = 0;
-      if (FORM == kFormContig) row_mi = m < p.M ? __ldg(p.m_indices + m) : -1;
+      // contiguous: a row is stored if it belongs to the tile's expert (rows of
+      // padding, and rows of a pair unit's partner tile that belong to another
+      // expert, are not)
+      if (FORM == kFormContig) row_mi = (m < p.M && __ldg(p.m_indices + m) == w.e) ? 0 : -1;
       const bool ok = m < m_valid && (FORM != kFormContig || row_mi >= 0);
       // a warp whose 32 rows are all stored writes through tensor stores
       const bool staged = __all_sync(0xffffffffu, ok);

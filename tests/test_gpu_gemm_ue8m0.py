@@ -161,6 +161,32 @@ def test_contiguous_parity_small(fg, width, counts, N, K):
     assert np.all(got[~valid] == SENTINEL), "padding rows must stay unwritten"
 
 
+def test_contiguous_padding_tiles_and_odd_runs(fg, width):
+    """Padding tiles between groups, an expert split into two runs, runs of
+    odd length and groups meeting inside an aligned pair of token tiles: pair
+    units join two tiles of one run only, and a unit's partner tile of
+    another expert or of padding stores nothing."""
+    N, K = 384, 512
+    experts = [0, -1, 0, 1, 1, 1, -1, 2, 3, 3, 3, 0]   # expert of each 128-row tile
+    rows = [128, 0, 77, 128, 128, 5, 0, 128, 128, 128, 64, 100]  # valid rows of each tile
+    M_total = 128 * len(experts)
+    m_indices = np.full(M_total, -1, np.int32)
+    for t, (e, r) in enumerate(zip(experts, rows)):
+        if e >= 0:
+            m_indices[t * 128:t * 128 + r] = e
+    rng = np.random.default_rng(13)
+    a = np.zeros((M_total, K), np.uint16)
+    valid = m_indices >= 0
+    a[valid] = workloads.bf16_bits(rng.standard_normal((int(valid.sum()), K), dtype=np.float32))
+    b = workloads.normal_bf16(np.random.default_rng(14), (4, N, K), 0.02)
+    qa, sa = oracle.per_token_cast(a, ue8m0=True)
+    qb, sb = oracle.per_block_cast(b, ue8m0=True)
+    ref = oracle.grouped_contiguous(qa, sa, qb, sb, m_indices)
+    got = run_contiguous(fg, qa, sa, qb, sb, m_indices)
+    check_gemm(bf16_bits_to_f64(got[valid]), ref[valid], "ue8m0 contiguous padding tiles")
+    assert np.all(got[~valid] == SENTINEL), "padding rows must stay unwritten"
+
+
 def test_contiguous_full_size_sampled(fg):
     inp = workloads.make("contiguous_8x4096x7168")
     qa, sa = oracle.per_token_cast(inp.a, ue8m0=True)
