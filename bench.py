@@ -102,7 +102,7 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_for(workload: str):
+def traffic_for(workload: str, ue8m0: bool = False):
     """DRAM bytes per GEMM launch from a committed ncu summary, if it was taken
     on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -110,7 +110,7 @@ def traffic_for(workload: str):
         return None
     with open(path) as f:
         d = json.load(f)
-    e = d.get(workload)
+    e = d.get(workload + ("@ue8m0" if ue8m0 else ""))
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
     return e.get("dram_bytes_per_launch")
@@ -538,7 +538,7 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak}
         peak_note = "%s HBM copy bandwidth (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
-    roof["traffic"] = traffic_for(args.workload)
+    roof["traffic"] = traffic_for(args.workload, ue8m0)
     roof["kernel"] = gemm_kernel_name(kind, inp, ue8m0)
     roof["algorithmic_per_launch"] = {"flops": flops, "bytes": alg_bytes}
     roof["kernel_ms"] = gms
