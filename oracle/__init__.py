@@ -60,6 +60,14 @@ def _load() -> ctypes.CDLL:
     lib.oracle_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
     lib.oracle_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
     lib.oracle_gemm_points.argtypes = [P, P, P, P, P, P, P, I64, P, I, I, I, I]
+    lib.oracle_exp_f32.argtypes = [ctypes.c_float]
+    lib.oracle_exp_f32.restype = ctypes.c_float
+    lib.oracle_silu_f32.argtypes = [ctypes.c_float]
+    lib.oracle_silu_f32.restype = ctypes.c_float
+    lib.oracle_swiglu.argtypes = [P, P, P, I64]
+    lib.oracle_swiglu.restype = None
+    lib.oracle_f64_to_bf16.argtypes = [P, P, I64]
+    lib.oracle_f64_to_bf16.restype = None
     for f in ("oracle_per_token_cast", "oracle_per_block_cast", "oracle_gemm_nt",
               "oracle_grouped_contiguous", "oracle_grouped_masked", "oracle_gemm_points",
               "oracle_hardware_threads"):
@@ -216,3 +224,66 @@ def gemm_points(qa, sa, qb, sb, a_rows, experts, cols, threads: int = 0) -> np.n
                                       _ptr(n), r.size, _ptr(out), N, K, G, threads),
            "gemm_points")
     return out
+
+
+# ---------------------------------------------------------------- expert FFN
+
+def exp_f32(x) -> np.ndarray:
+    """exp in fp32 by the oracle's fixed operation sequence (elementwise)."""
+    lib = _load()
+    x = np.asarray(x, np.float32)
+    return np.array([lib.oracle_exp_f32(float(v)) for v in x.ravel()], np.float32).reshape(x.shape)
+
+
+def silu_f32(x) -> np.ndarray:
+    """silu(g) = g / (1 + exp(-g)) in fp32 (elementwise)."""
+    lib = _load()
+    x = np.asarray(x, np.float32)
+    return np.array([lib.oracle_silu_f32(float(v)) for v in x.ravel()], np.float32).reshape(x.shape)
+
+
+def swiglu(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
+    """h = bf16(silu(gate) * up) for bf16 bit patterns of equal shape."""
+    g = np.ascontiguousarray(g_bits, np.uint16)
+    u = np.ascontiguousarray(u_bits, np.uint16)
+    assert g.shape == u.shape
+    h = np.empty_like(g)
+    _load().oracle_swiglu(_ptr(g), _ptr(u), _ptr(h), g.size)
+    return h
+
+
+def f64_to_bf16(v: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of fp64 values (nearest even, one rounding)."""
+    v = np.ascontiguousarray(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    _load().oracle_f64_to_bf16(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def moe_ffn_contiguous(xq, sx, w1q, sw1, w2q, sw2, m_indices, threads: int = 0):
+    """Expert FFN on the contiguous layout with power-of-two scales: the first
+    grouped GEMM (W1 rows: I gate rows, then I up rows), its result rounded to
+    bf16, h = swiglu(gate, up), h quantized per token per 128 channels with
+    power-of-two scales, the second grouped GEMM. Returns (gu_bits [M][2I],
+    hq [M][I], sh [M][I/128], y fp64 [M][H]); rows with m_indices < 0 are
+    computed as the grouped GEMM defines them (zero) and ignored by callers."""
+    I = w1q.shape[1] // 2
+    gu = f64_to_bf16(grouped_contiguous(xq, sx, w1q, sw1, m_indices, threads))
+    h = swiglu(gu[:, :I], gu[:, I:])
+    hq, sh = per_token_cast(h, threads=threads, ue8m0=True)
+    y = grouped_contiguous(hq, sh, w2q, sw2, m_indices, threads)
+    return gu, hq, sh, y
+
+
+def moe_ffn_masked(xq, sx, w1q, sw1, w2q, sw2, masked_m, threads: int = 0):
+    """The same chain on the masked layout ([G][M_max][...] slabs)."""
+    G, M_max, _ = xq.shape
+    I = w1q.shape[1] // 2
+    y1 = grouped_masked(xq, sx, w1q, sw1, masked_m, threads)
+    for e in range(G):  # rows past masked_m are not computed: their intermediate is zero
+        y1[e, int(masked_m[e]):] = 0.0
+    gu = f64_to_bf16(y1)
+    h = swiglu(gu[..., :I], gu[..., I:])
+    hq, sh = per_token_cast(h, threads=threads, ue8m0=True)
+    y = grouped_masked(hq, sh, w2q, sw2, masked_m, threads)
+    return gu, hq, sh, y

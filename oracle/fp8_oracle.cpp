@@ -34,6 +34,17 @@
 //    only the two scale multiplies and the outer sum over K blocks round in
 //    fp64. The result is kept in fp64, not rounded to bf16.
 //
+//  * The expert FFN's activation (the "Mega MoE" kernel fuses both expert
+//    GEMMs with the SwiGLU activation: "DeepGEMM" overview, section
+//    "swapAB与Mega MoE"; the pages name SwiGLU without a formula). Reading
+//    taken: h = silu(gate) * up with silu(g) = g / (1 + exp(-g)), gate and up
+//    the bf16 outputs of the first GEMM, evaluated in fp32 and rounded once to
+//    bf16. exp is evaluated by one fixed sequence of IEEE fp32 operations
+//    (Cody and Waite's argument reduction, "Software Manual for the
+//    Elementary Functions", 1980, then the degree-7 Taylor polynomial in
+//    Horner form with fused multiply-adds), so that a second implementation
+//    of the same method can agree with it bit for bit.
+//
 // Build: g++ -O2 -std=c++17 -fPIC -shared -pthread -ffp-contract=off
 // (no fast-math: the quantizer's fp32 divide and multiply must be IEEE).
 
@@ -147,6 +158,36 @@ float quantize_group(const std::vector<float>& vals, std::vector<uint8_t>& codes
   }
   return scale;
 }
+
+// ---- SwiGLU -------------------------------------------------------------------
+
+// exp(x) in fp32: x clamped to [-87, 88] (so that 2^n below stays a normal
+// number), n = nearest integer to x * log2(e), r = x - n * ln2 with ln2 split
+// into C1 = 355/512 (n * C1 is exact) and C2 = ln2 - C1, then
+// exp(r) = sum_{k<=7} r^k / k! by Horner's rule with fused multiply-adds, and
+// the result p * 2^n (one rounding).
+float exp_f32(float x) {
+  x = std::fmin(std::fmax(x, -87.0f), 88.0f);
+  const float n = std::nearbyint(x * 1.44269504088896341f);
+  const float c1 = 0.693359375f;
+  const float c2 = -2.12194440e-4f;
+  float r = std::fma(-n, c1, x);
+  r = std::fma(-n, c2, r);
+  float p = 1.0f / 5040.0f;
+  p = std::fma(p, r, 1.0f / 720.0f);
+  p = std::fma(p, r, 1.0f / 120.0f);
+  p = std::fma(p, r, 1.0f / 24.0f);
+  p = std::fma(p, r, 1.0f / 6.0f);
+  p = std::fma(p, r, 0.5f);
+  p = std::fma(p, r, 1.0f);
+  p = std::fma(p, r, 1.0f);
+  uint32_t bits = static_cast<uint32_t>(static_cast<int>(n) + 127) << 23;  // 2^n, n in [-126, 127]
+  float two_n;
+  std::memcpy(&two_n, &bits, 4);
+  return p * two_n;
+}
+
+float silu_f32(float g) { return g / (1.0f + exp_f32(-g)); }
 
 template <typename F>
 void parallel_for(int64_t n, int threads, F&& body) {
@@ -368,6 +409,46 @@ int oracle_gemm_points(const uint8_t* qa, const float* sa, const uint8_t* qb, co
     out[p] = dot_blocked(qa + a_row[p] * K, sa + a_row[p] * KB, brow, srow, K);
   });
   return 0;
+}
+
+float oracle_exp_f32(float x) { return exp_f32(x); }
+float oracle_silu_f32(float g) { return silu_f32(g); }
+
+// h = bf16(silu(g) * u) elementwise; g, u, h bf16 bit patterns.
+void oracle_swiglu(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n) {
+  for (int64_t i = 0; i < n; ++i)
+    h[i] = float_to_bf16_rne(silu_f32(bf16_to_float(g[i])) * bf16_to_float(u[i]));
+}
+
+// bf16 nearest-even rounding of fp64 values (one rounding from the exact
+// value; magnitudes beyond the largest finite bf16 round to infinity).
+void oracle_f64_to_bf16(const double* v, uint16_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double x = v[i];
+    if (std::isnan(x)) {
+      out[i] = 0x7FC0;
+      continue;
+    }
+    const uint16_t sign = std::signbit(x) ? 0x8000 : 0;
+    const double a = std::fabs(x);
+    if (a == 0.0) {
+      out[i] = sign;
+      continue;
+    }
+    // spacing of bf16 values at a's binade (subnormals share the smallest)
+    int e;
+    std::frexp(a, &e);                 // a = f * 2^e, f in [0.5, 1)
+    int q = std::max(e - 8, -133);     // bf16: 8 significant bits; subnormal spacing 2^-133
+    const double unit = std::ldexp(1.0, q);
+    const double m = a / unit;         // exact (power-of-two scaling)
+    double r = std::nearbyint(m);      // ties to even (default rounding mode)
+    const double y = r * unit;
+    const float f = y > 3.3895313892515355e38 ? std::numeric_limits<float>::infinity()
+                                              : static_cast<float>(y);  // exact: <= 8 significant bits
+    uint32_t b;
+    std::memcpy(&b, &f, 4);
+    out[i] = static_cast<uint16_t>(sign | ((b >> 16) & 0x7FFF));
+  }
 }
 
 int oracle_hardware_threads(void) {

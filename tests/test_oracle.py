@@ -484,3 +484,132 @@ def test_ue8m0_round_trip_within_half_unit():
     xv = _bf16_to_f64(x)
     sf = _block_scales(s[None], 256)[0].astype(np.float64)
     assert np.all(np.abs(xv - y) <= 2.0 ** -4 * np.abs(xv) + 2.0 ** -10 * sf + 2.0 ** -8 * np.abs(y))
+
+
+# ---------------------------------------------------------------- expert FFN pieces
+
+def _ulp32(x):
+    x = np.abs(np.asarray(x, np.float32))
+    return np.spacing(x).astype(np.float64)
+
+
+def test_exp_f32_within_two_ulp_of_exp():
+    """The fixed-sequence fp32 exp against the fp64 exp over its whole
+    unclamped range (a wrong constant, a dropped Taylor term or a wrong
+    exponent reassembly fails this)."""
+    x = np.linspace(-87.0, 88.0, 40001).astype(np.float32)
+    got = oracle.exp_f32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    err = np.abs(got - ref) / _ulp32(ref)
+    assert err.max() <= 2.0, err.max()
+
+
+def test_exp_f32_exact_points_and_clamp():
+    assert oracle.exp_f32(np.float32(0.0)) == 1.0
+    k = np.arange(-120, 121).astype(np.float32)
+    x = (k.astype(np.float64) * np.log(2.0)).astype(np.float32)
+    got = oracle.exp_f32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    assert np.all(np.abs(got - ref) <= 2 * _ulp32(ref))
+    assert oracle.exp_f32(np.float32(200.0)) == oracle.exp_f32(np.float32(88.0))
+    assert oracle.exp_f32(np.float32(-200.0)) == oracle.exp_f32(np.float32(-87.0))
+
+
+def test_silu_identities():
+    """silu(0) = 0; silu(x) - silu(-x) = x; silu(x) = x once exp(-x) is below
+    half an ulp of 1; close to the fp64 formula."""
+    assert oracle.silu_f32(np.float32(0.0)) == 0.0
+    x = np.linspace(0.01, 15.0, 3001).astype(np.float32)
+    d = oracle.silu_f32(x).astype(np.float64) - oracle.silu_f32(-x).astype(np.float64)
+    assert np.all(np.abs(d - x) <= 4 * _ulp32(x))
+    big = np.array([17.0, 20.0, 100.0, 3e4], np.float32)
+    assert np.array_equal(oracle.silu_f32(big), big)
+    xs = np.linspace(-30.0, 30.0, 6001).astype(np.float32)
+    ref = xs.astype(np.float64) / (1.0 + np.exp(-xs.astype(np.float64)))
+    got = oracle.silu_f32(xs).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 4 * _ulp32(ref) + 1e-45)
+
+
+def _bf16_neighbours(v):
+    """The two bf16 values around each fp64 v (from fp32 bit patterns)."""
+    f = np.asarray(v, np.float64).astype(np.float32)
+    b = f.view(np.uint32) & np.uint32(0xFFFF0000)
+    lo = b.view(np.float32).astype(np.float64)
+    hi = (b + np.uint32(0x10000)).view(np.float32).astype(np.float64)
+    return lo, hi
+
+
+def test_f64_to_bf16_single_rounding():
+    """Hand cases (ties to even, subnormal, overflow) and random values against
+    the nearest of the two neighbouring bf16 values (ties to even)."""
+    cases = {1.0: 0x3F80, 1 + 2 ** -8: 0x3F80, 1 + 3 * 2 ** -8: 0x3F82, -2.5: 0xC020,
+             1e-40: 0x0001, 3.39e38: 0x7F7F, 3.4e38: 0x7F80, 0.0: 0x0000}
+    got = oracle.f64_to_bf16(np.array(list(cases)))
+    assert got.tolist() == list(cases.values())
+    rng = np.random.default_rng(21)
+    v = rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))
+    v = v[np.abs(v) > 1e-30]
+    got = oracle.f64_to_bf16(v)
+    gv = (got.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    lo, hi = _bf16_neighbours(np.abs(v))
+    a = np.abs(v)
+    nearest = np.where(a - lo < hi - a, lo, hi)
+    tie = (a - lo) == (hi - a)
+    even = np.where(((lo.astype(np.float32).view(np.uint32) >> 16) & 1) == 0, lo, hi)
+    nearest = np.where(tie, even, nearest) * np.sign(v)
+    assert np.array_equal(gv, nearest)
+
+
+def test_swiglu_against_fp64_formula():
+    """h = bf16(silu(g) * u): equal to the bf16 rounding of the fp64 formula
+    except where the fp32 evaluation sits within a few ulp of a rounding
+    boundary (then the neighbouring bf16 value)."""
+    rng = np.random.default_rng(22)
+    g = workloads.bf16_bits(rng.standard_normal(20000).astype(np.float32) * 3)
+    u = workloads.bf16_bits(rng.standard_normal(20000).astype(np.float32))
+    h = oracle.swiglu(g, u)
+    gf = (g.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    uf = (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    ref = oracle.f64_to_bf16(gf / (1.0 + np.exp(-gf)) * uf)
+    diff = np.abs(h.astype(np.int64) - ref.astype(np.int64))
+    assert np.all(diff <= 1) and np.mean(diff == 0) > 0.999
+
+
+def test_ffn_chain_closed_form():
+    """All-ones operands: gate = 2, up = 1, so h = bf16(silu(2)) = 1.765625;
+    its power-of-two scale is 2^-7 (1.7656/448 is just above 2^-8) and its code
+    e4m3(226) = 224; with all-ones W2 at scale 2^-7 every output is
+    I * 224 * 2^-7 * 2^-7 = 1.75 (I = 128)."""
+    H = I = 128
+    M = 5
+    xq = np.full((M, H), 0x38, np.uint8)
+    sx = np.full((M, 1), 2.0 ** -7, np.float32)
+    w1q = np.full((1, 2 * I, H), 0x38, np.uint8)
+    sw1 = np.array([[[2.0], [1.0]]], np.float32)  # gate block x2, up block x1
+    w2q = np.full((1, H, I), 0x38, np.uint8)
+    sw2 = np.full((1, 1, 1), 2.0 ** -7, np.float32)
+    mi = np.zeros(M, np.int32)
+    gu, hq, sh, y = oracle.moe_ffn_contiguous(xq, sx, w1q, sw1, w2q, sw2, mi)
+    assert np.all(gu[:, :I] == 0x4000) and np.all(gu[:, I:] == 0x3F80)   # 2.0, 1.0
+    assert np.all(sh == 2.0 ** -7)
+    assert np.all(hq == oracle.e4m3_encode(np.float32(224.0)))
+    assert np.all(y == 1.75)
+
+
+def test_ffn_masked_matches_contiguous_per_expert():
+    """The masked chain equals the contiguous chain on each expert's valid rows."""
+    rng = np.random.default_rng(23)
+    G, M_max, H, I = 2, 40, 256, 128
+    mm = np.array([40, 17], np.int32)
+    x = workloads.bf16_bits(rng.standard_normal((G, M_max, H)).astype(np.float32))
+    xq, sx = oracle.per_token_cast(x, ue8m0=True)
+    w1q, sw1 = oracle.per_block_cast(workloads.normal_bf16(rng, (G, 2 * I, H), 0.05), ue8m0=True)
+    w2q, sw2 = oracle.per_block_cast(workloads.normal_bf16(rng, (G, H, I), 0.05), ue8m0=True)
+    gu_m, hq_m, sh_m, y_m = oracle.moe_ffn_masked(xq, sx, w1q, sw1, w2q, sw2, mm)
+    for e in range(G):
+        v = int(mm[e])
+        mi = np.full(v, e, np.int32)
+        gu_c, hq_c, sh_c, y_c = oracle.moe_ffn_contiguous(xq[e, :v], sx[e, :v], w1q, sw1, w2q, sw2, mi)
+        assert np.array_equal(gu_m[e, :v], gu_c)
+        assert np.array_equal(hq_m[e, :v], hq_c)
+        assert np.array_equal(y_m[e, :v], y_c)
