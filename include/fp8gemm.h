@@ -214,6 +214,41 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
                                         cudaStream_t stream);
 
 /*
+ * MoE expert FFN with power-of-two scales: for every expert e,
+ *   GU = bf16(X_e W1_e^T)          (first grouped GEMM; W1_e has 2I rows: I gate
+ *                                   rows, then I up rows)
+ *   h  = bf16(silu(gate) * up)     (silu(g) = g / (1 + exp(-g)) in fp32, exp by a
+ *                                   fixed Cody-Waite + degree-7 Taylor sequence)
+ *   Hq, sfh = per_token_cast_to_fp8_ue8m0(h)
+ *   Y  = bf16(Hq W2_e^T)           (second grouped GEMM; W2_e is H x I)
+ * the single-GPU part of the "Mega MoE" kernel, which fuses both expert GEMMs
+ * with the SwiGLU activation ("DeepGEMM" overview, section "swapAB与Mega MoE").
+ * The SwiGLU and the requantization run in the first GEMM's epilogue (no bf16
+ * intermediate goes to memory); the second GEMM is fp8_grouped_gemm_*_ue8m0.
+ * Scales must be powers of two (as for the _ue8m0 GEMMs).
+ * Contiguous: X e4m3 [M_total][H], sfx MN-major [H/128][stride(M_total)],
+ *   m_indices int32 [M_total] (contract of fp8_grouped_gemm_contiguous);
+ *   Hq e4m3 [M_total][I], sfh [I/128][stride(M_total)], Y bf16 [M_total][H].
+ * Masked: X [G][M_max][H], sfx [G][H/128][stride(M_max)], masked_m int32 [G];
+ *   Hq [G][M_max][I], sfh [G][I/128][stride(M_max)], Y [G][M_max][H].
+ * W1 e4m3 [G][2I][H], sfw1 [G][2I/128][H/128]; W2 e4m3 [G][H][I],
+ * sfw2 [G][H/128][I/128]. GU: optional (NULL = not written) bf16 [rows][2I]
+ * output of the first GEMM (gate columns, then up columns), which the SwiGLU
+ * backward pass needs. Hq, sfh and Y (and GU) are written on valid rows only.
+ * H % 128 == 0, I % 128 == 0, G >= 1; other limits as for the grouped GEMMs.
+ */
+fg_status fp8_moe_ffn_contiguous_ue8m0(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                      const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                      uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                      const int32_t* m_indices, int M_total, int H, int I, int G,
+                                      cudaStream_t stream);
+fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                  const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                  uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                  const int32_t* masked_m, int G, int M_max, int H, int I,
+                                  int expected_m, cudaStream_t stream);
+
+/*
  * Tuning knob of the three _ue8m0 GEMMs (process-wide). width = 0: choose the
  * tile per shape (default). Otherwise always use the block-scaled kernel, thin
  * shapes included, with weight tiles of `width` rows: 128, 224 or 256 with

@@ -12,7 +12,8 @@ The functions carry the C names:
   fp8_gemm_nt, fp8_grouped_gemm_contiguous, fp8_grouped_gemm_masked,
   per_token_cast_to_fp8_ue8m0, per_block_cast_to_fp8_ue8m0, and the GEMMs for
   power-of-two scales fp8_gemm_nt_ue8m0, fp8_grouped_gemm_contiguous_ue8m0,
-  fp8_grouped_gemm_masked_ue8m0 (set_ue8m0_tile tunes them)
+  fp8_grouped_gemm_masked_ue8m0 (set_ue8m0_tile tunes them), and the expert FFN
+  fp8_moe_ffn_contiguous_ue8m0, fp8_moe_ffn_masked_ue8m0
 plus allocation helpers that return tensors in the layouts the kernels use.
 """
 from __future__ import annotations
@@ -37,7 +38,8 @@ EXPORTED = (
     "per_token_cast_to_fp8_ue8m0", "per_block_cast_to_fp8_ue8m0", "fp8_gemm_nt",
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
     "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
-    "fg_set_ue8m0_tile", "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
+    "fg_set_ue8m0_tile", "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
+    "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
 
 
@@ -75,6 +77,8 @@ def load_library() -> ctypes.CDLL:
     lib.fp8_grouped_gemm_contiguous_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fp8_grouped_gemm_masked_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
     lib.fg_set_ue8m0_tile.argtypes = [I, I]
+    lib.fp8_moe_ffn_contiguous_ue8m0.argtypes = [P] * 11 + [I, I, I, I, P]
+    lib.fp8_moe_ffn_masked_ue8m0.argtypes = [P] * 11 + [I, I, I, I, I, P]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
     lib.fg_status_string.argtypes = [I]
@@ -87,6 +91,7 @@ def load_library() -> ctypes.CDLL:
               "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
               "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0",
               "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile",
+              "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
     _lib = lib
@@ -268,6 +273,34 @@ def fp8_grouped_gemm_masked_ue8m0(A: torch.Tensor, sfa: torch.Tensor, B: torch.T
     """fp8_grouped_gemm_masked with power-of-two scales."""
     _gemm_masked(load_library().fp8_grouped_gemm_masked_ue8m0, A, sfa, B, sfb, D, masked_m,
                  expected_m, stream)
+
+
+def fp8_moe_ffn_contiguous_ue8m0(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, m_indices, GU=None,
+                                 stream=None) -> None:
+    """Expert FFN (contiguous layout): X uint8 [M_total][H], W1 uint8 [G][2I][H],
+    W2 uint8 [G][H][I] -> Hq uint8 [M_total][I], sfh [I/128][stride], Y bf16
+    [M_total][H] (and GU bf16 [M_total][2I] if given)."""
+    M_total, H = X.shape
+    G, I2, _ = W1.shape
+    if m_indices.dtype != torch.int32 or m_indices.numel() != M_total:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "m_indices must be int32 [M_total]")
+    _check(load_library().fp8_moe_ffn_contiguous_ue8m0(
+        _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
+        _ptr(GU), _ptr(Y), _ptr(m_indices), M_total, H, I2 // 2, G, _stream(stream)))
+
+
+def fp8_moe_ffn_masked_ue8m0(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, masked_m, expected_m,
+                             GU=None, stream=None) -> None:
+    """Expert FFN (masked layout): X uint8 [G][M_max][H] -> Hq [G][M_max][I],
+    sfh [G][I/128][stride], Y bf16 [G][M_max][H] (and GU [G][M_max][2I])."""
+    G, M_max, H = X.shape
+    I2 = W1.shape[1]
+    if masked_m.dtype != torch.int32 or masked_m.numel() != G:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "masked_m must be int32 [G]")
+    _check(load_library().fp8_moe_ffn_masked_ue8m0(
+        _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
+        _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m),
+        _stream(stream)))
 
 
 def set_ue8m0_tile(width: int, pair: bool = False) -> None:

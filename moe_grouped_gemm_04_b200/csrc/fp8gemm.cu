@@ -431,6 +431,17 @@ using MxN128 = MxCfg<128, 5, 2, 1, false, 1>;
 using MxN224 = MxCfg<224, 4, 2, 1, false, 1>;
 using MxN256 = MxCfg<256, 3, 1, 2, false, 1>;
 using MxP224 = MxCfg<224, 3, 2, 1, true, 2>;  // CTA pairs, 256 x 224 tiles
+// first GEMM of the expert FFN with the fused SwiGLU + requantization epilogue
+using MxFfnP = MxCfg<256, 3, 1, 1, true, 2, 1>;
+using MxFfnS = MxCfg<256, 4, 1, 1, false, 1, 1>;
+
+// Outputs of the fused expert-FFN epilogue.
+struct FfnOut {
+  uint8_t* hq;
+  float* sfh;
+  uint16_t* gu;
+  int I;
+};
 
 // Shared-memory attribute and, for pair configs, the number of co-resident
 // clusters (the persistent grid's size).
@@ -468,7 +479,8 @@ fg_status mx_kernel_attr(int dev, int* max_clusters) {
 }
 
 template <class C, int FORM>
-fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
+fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaStream_t stream,
+                    const FfnOut* ffn = nullptr) {
   static_assert(C::smem_bytes(FORM) <= 232448, "shared memory per CTA");
   int max_clusters = 0;
   FG_TRY((mx_kernel_attr<C, FORM>(dev_id, &max_clusters)));
@@ -478,7 +490,7 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
                   static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
                   CU_TENSOR_MAP_SWIZZLE_128B, "A"));
   FG_TRY(make_map(&tmB, pr.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
-                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::B_ROWS,
+                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::B_BOX,
                   CU_TENSOR_MAP_SWIZZLE_128B, "B"));
   // token scales: boxes of 128 tokens x 4 K blocks (one quad)
   FG_TRY(make_map(&tmSA, pr.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.M,
@@ -486,9 +498,12 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
                   static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 4,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
   // D as rows x N bf16 in boxes of 32 rows x 32 columns, 64-byte swizzled
-  FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
-                  static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2, 32, 32,
-                  CU_TENSOR_MAP_SWIZZLE_64B, "D"));
+  // (the fused FFN epilogue writes no D)
+  std::memset(&tmD, 0, sizeof(tmD));
+  if (C::EPI == 0)
+    FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
+                    static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B, "D"));
   GemmParams p{};
   p.M = pr.M;
   p.N = pr.N;
@@ -504,6 +519,14 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
   p.masked_m = pr.masked_m;
   p.status = dev.status;
   p.timeout_ns = wait_limit_ns();
+  if (C::EPI == 1) {
+    p.hq = ffn->hq;
+    p.sfh = ffn->sfh;
+    p.gu = ffn->gu;
+    p.I = ffn->I;
+    p.sfh_stride = sfa_stride(pr.M);
+    p.num_nt = ffn->I / 128;  // one tile = 128 gate + 128 up rows
+  }
   int64_t tiles = static_cast<int64_t>(C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
   if (FORM == kFormMasked) tiles *= pr.G;  // upper bound: masked_m lives on the device
   const int64_t grid = C::PAIR ? C::CLUSTER * std::max<int64_t>(1, std::min<int64_t>(tiles, max_clusters))
@@ -606,6 +629,59 @@ fg_status run_gemm_mx(const Problem& pr, int expected_m, cudaStream_t stream) {
     case kFormContig: return dispatch_mx<kFormContig>(pr, pl, *dev, dev_id, stream);
     default: return dispatch_mx<kFormMasked>(pr, pl, *dev, dev_id, stream);
   }
+}
+
+// The expert FFN: the first grouped GEMM with the fused SwiGLU + requant
+// epilogue (pairs unless the masked layout's experts hold about one token
+// tile), then the second grouped GEMM on the quantized activations.
+fg_status run_ffn(int form, const uint8_t* X, const float* sfx, const uint8_t* W1, const float* sfw1,
+                  const uint8_t* W2, const float* sfw2, uint8_t* Hq, float* sfh, uint16_t* GU,
+                  uint16_t* Y, const int32_t* m_indices, const int32_t* masked_m, int M, int H,
+                  int I, int G, int expected_m, cudaStream_t stream) {
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (H <= 0 || H % 128 != 0) return fail(FG_ERR_INVALID_ARG, "H=%d must be a positive multiple of 128", H);
+  if (I <= 0 || I % 128 != 0) return fail(FG_ERR_INVALID_ARG, "I=%d must be a positive multiple of 128", I);
+  if (form == kFormContig) {
+    if (M < 0 || M % 128 != 0)
+      return fail(FG_ERR_INVALID_ARG, "M_total=%d must be a non-negative multiple of 128", M);
+    if (M == 0) return FG_OK;
+    FG_TRY(check_ptr(m_indices, "m_indices"));
+    if ((M + 127) / 128 > kTableMax)
+      return fail(FG_ERR_UNSUPPORTED, "M_total %d exceeds %d rows", M, kTableMax * 128);
+  } else {
+    if (M < 1) return fail(FG_ERR_INVALID_ARG, "M_max=%d must be >= 1", M);
+    FG_TRY(check_ptr(masked_m, "masked_m"));
+    if (G + 1 > kTableMax) return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d experts", G, kTableMax - 1);
+    if (expected_m <= 0) expected_m = M;
+  }
+  FG_TRY(check_ptr(X, "X"));
+  FG_TRY(check_ptr(sfx, "sfx"));
+  FG_TRY(check_ptr(W1, "W1"));
+  FG_TRY(check_ptr(sfw1, "sfw1"));
+  FG_TRY(check_ptr(W2, "W2"));
+  FG_TRY(check_ptr(sfw2, "sfw2"));
+  FG_TRY(check_ptr(Hq, "Hq"));
+  FG_TRY(check_ptr(sfh, "sfh"));
+  FG_TRY(check_ptr(Y, "Y"));
+  if (GU) FG_TRY(check_ptr(GU, "GU"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  const int slabs = form == kFormMasked ? G : 1;
+  const FfnOut out{Hq, sfh, GU, I};
+  Problem p1{form, X, sfx, W1, sfw1, nullptr, m_indices, masked_m, M, 2 * I, H, G, slabs};
+  const bool pair = form == kFormContig || expected_m > 128;
+  fg_status st;
+  if (form == kFormContig)
+    st = pair ? launch_mx<MxFfnP, kFormContig>(p1, *dev, dev_id, stream, &out)
+              : launch_mx<MxFfnS, kFormContig>(p1, *dev, dev_id, stream, &out);
+  else
+    st = pair ? launch_mx<MxFfnP, kFormMasked>(p1, *dev, dev_id, stream, &out)
+              : launch_mx<MxFfnS, kFormMasked>(p1, *dev, dev_id, stream, &out);
+  if (st != FG_OK) return st;
+  Problem p2{form, Hq, sfh, W2, sfw2, Y, m_indices, masked_m, M, H, I, G, slabs};
+  return run_gemm_mx(p2, expected_m, stream);
 }
 
 fg_status check_gemm_common(const uint8_t* A, const float* sfa, const uint8_t* B,
@@ -812,6 +888,24 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
   if (expected_m <= 0) expected_m = M_max;
   Problem pr{kFormMasked, A, sfa, B, sfb, D, nullptr, masked_m, M_max, N, K, G, G};
   return run_gemm_mx(pr, expected_m, stream);
+}
+
+fg_status fp8_moe_ffn_contiguous_ue8m0(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                      const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                      uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                      const int32_t* m_indices, int M_total, int H, int I, int G,
+                                      cudaStream_t stream) {
+  return run_ffn(kFormContig, X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, GU, Y, m_indices, nullptr,
+                 M_total, H, I, G, M_total, stream);
+}
+
+fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                  const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                  uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                  const int32_t* masked_m, int G, int M_max, int H, int I,
+                                  int expected_m, cudaStream_t stream) {
+  return run_ffn(kFormMasked, X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, GU, Y, nullptr, masked_m, M_max,
+                 H, I, G, expected_m, stream);
 }
 
 fg_status fg_set_ue8m0_tile(int width, int pair) {

@@ -80,6 +80,14 @@ struct GemmParams {
   const int32_t* masked_m;
   int* status;
   uint64_t timeout_ns;
+  // fused expert-FFN epilogue of the block-scaled kernel (otherwise unused):
+  // quantized activations h [rows][I] with their per-token scales (MN-major,
+  // row stride sfh_stride) and, optionally, the bf16 gate/up values [rows][2I]
+  uint8_t* hq;
+  float* sfh;
+  uint16_t* gu;
+  int I;
+  int sfh_stride;
 };
 
 template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_, int KPS_ = 2,

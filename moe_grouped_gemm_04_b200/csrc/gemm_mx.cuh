@@ -67,18 +67,31 @@
 // on both CTAs' barriers; operand bytes of both CTAs complete on the leader's
 // "full" barrier; the peer's converter and epilogue arrive on the leader's
 // "sf full" and "tmem empty" barriers through the cluster.
+//
+// Fused expert-FFN epilogue (EPI = 1, first GEMM of the expert FFN): W1 holds
+// I gate rows then I up rows per expert; the tile of weight tile nt is the
+// 128 gate rows nt*128.. and the 128 up rows I + nt*128.. (a pair's CTAs load
+// one block each), so each token row of the tile holds 128 gate and the
+// matching 128 up values. The epilogue rounds them to bf16, computes
+// h = bf16(silu(gate) * up) (act.cuh), takes the row's 128-wide amax and its
+// power-of-two scale, and writes the e4m3 codes of h and the scale in the
+// per-token layout the second GEMM reads (optionally also the bf16 gate and
+// up values). The arithmetic is that of per_token_cast_to_fp8_ue8m0.
 #pragma once
 
 #include <cstdint>
 #include <cuda.h>
 
+#include "act.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fg {
 
-template <int BW_, int STAGES_, int ACC_, int EPQ_, bool PAIR_, int KPS_>
+template <int BW_, int STAGES_, int ACC_, int EPQ_, bool PAIR_, int KPS_, int EPI_ = 0>
 struct MxCfg {
+  static constexpr int EPI = EPI_;        // 0: bf16 D; 1: SwiGLU + UE8M0 requantization
   static constexpr int BT = 128;          // token rows per CTA tile
   static constexpr int BW = BW_;          // weight rows per tile (MMA N)
   static constexpr bool SWAP = false;     // tile helpers of gemm.cuh: tokens on the lanes
@@ -93,6 +106,11 @@ struct MxCfg {
   static constexpr int EPQ = EPQ_;        // epilogue warps per TMEM lane quadrant
   static_assert(BW % 32 == 0 && BW >= 32 && BW <= 256, "tcgen05 N, 32-column chunks");
   static_assert(!PAIR || B_ROWS % 16 == 0, "pair: half tiles of whole 8-row swizzle atoms");
+  static_assert(EPI == 0 || (BW == 256 && ACC == 1 && EPQ == 1),
+                "fused FFN epilogue: 128 gate + 128 up columns, one accumulator, one warp per quadrant");
+  // weight rows per tensor load: the fused FFN tile is two 128-row blocks
+  static constexpr int B_BOX = EPI == 1 ? 128 : B_ROWS;
+  static constexpr int B_LOADS = B_ROWS / B_BOX;
   static constexpr int EW = 4 * EPQ;      // epilogue warps
   static constexpr int ECOLS = BW / EPQ;  // accumulator columns per epilogue warp
   static_assert(ECOLS % 32 == 0, "epilogue chunks of 32 columns");
@@ -105,7 +123,7 @@ struct MxCfg {
   static constexpr int SFS = 3;           // scale slots (quads in flight)
   // staged fp32 scales of a quad: 4 x 128 token scales (one TMA box), then
   // 4 x NBT weight-block scales ([k][j]: K block 4q + k, block nb0 + j)
-  static constexpr int NBT = SFB_GROUPS + 1;
+  static constexpr int NBT = EPI == 1 ? 2 : SFB_GROUPS + 1;
   static constexpr int RAW_A = 4 * 512;
   static constexpr int RAW_BYTES = RAW_A + 128;
   static constexpr int RAWS = 2;          // staged-scale ring
@@ -125,7 +143,7 @@ struct MxCfg {
   static constexpr int OFF_SF = OFF_B + STAGES * STAGE_B;
   static constexpr int OFF_RAW = OFF_SF + SFS * SF_BYTES;  // 128-byte aligned
   static constexpr int OFF_EPI = (OFF_RAW + RAWS * RAW_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_BAR = OFF_EPI + EW * EPI_RING * BOX_BYTES;
+  static constexpr int OFF_BAR = OFF_EPI + (EPI == 0 ? EW * EPI_RING * BOX_BYTES : 0);
   static constexpr int NUM_BARS = 2 * STAGES + 2 * SFS + 2 * RAWS + 2 * ACC;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
@@ -374,10 +392,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       for (int t = t_first; t < total; t += t_step) {
         const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
         if (!w.valid) continue;
-        const int row = lane == 0 ? w.e * p.N + w.nt * C::BW + rank * C::B_ROWS
+        // fused FFN: gate block nt*128.. and up block I + nt*128.. of the
+        // expert's 2I rows (a pair's CTAs load one block each)
+        const int row = lane == 0 ? (C::EPI == 1 ? w.e * p.N + (C::PAIR ? rank : 0) * p.I + w.nt * 128
+                                                 : w.e * p.N + w.nt * C::BW + rank * C::B_ROWS)
                                   : (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
         const CUtensorMap* map = lane == 0 ? &tmB : &tmA;
         const uint32_t bytes = lane == 0 ? C::B_BYTES : C::A_BYTES;
+        const int loads = lane == 0 ? C::B_LOADS : 1;  // tensor loads per K block
+        const int load_step = C::EPI == 1 ? p.I : 0;   // rows between them
         for (int kb0 = 0; kb0 < p.KB; kb0 += C::KPS, st.next(), ++fills) {
           if (!mbar_wait(&empty[st.slot], st.phase ^ 1u, ctl)) goto producer_done;
           const int nk = min(C::KPS, p.KB - kb0);
@@ -386,10 +409,16 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             // both CTAs' operand bytes complete on the leader's barrier
             if (rank == 0) mbar_arrive_expect_tx(&full[st.slot], 2 * nk * bytes);
             const uint32_t bar = mapa_shared(smem_u32(&full[st.slot]), 0);
-            for (int j = 0; j < nk; ++j) tma_load_2d_pair(dst + j * bytes, map, bar, (kb0 + j) * 128, row);
+            for (int j = 0; j < nk; ++j)
+              for (int h = 0; h < loads; ++h)
+                tma_load_2d_pair(dst + j * bytes + h * C::B_BOX * 128, map, bar, (kb0 + j) * 128,
+                                 row + h * load_step);
           } else {
             mbar_arrive_expect_tx(&full[st.slot], nk * bytes);
-            for (int j = 0; j < nk; ++j) tma_load_2d(dst + j * bytes, map, &full[st.slot], (kb0 + j) * 128, row);
+            for (int j = 0; j < nk; ++j)
+              for (int h = 0; h < loads; ++h)
+                tma_load_2d(dst + j * bytes + h * C::B_BOX * 128, map, &full[st.slot], (kb0 + j) * 128,
+                            row + h * load_step);
           }
         }
       }
@@ -425,9 +454,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           for (int k = 0; k < 4; ++k) {
             const int kb = min(4 * qi + k, p.KB - 1);
 #pragma unroll
-            for (int j = 0; j < C::NBT; ++j)
-              cp_async_4(raw + C::RAW_A + 4 * (k * C::NBT + j),
-                         sfb_e + static_cast<int64_t>(min(nb0 + j, p.NB - 1)) * p.KB + kb);
+            for (int j = 0; j < C::NBT; ++j) {
+              // fused FFN: the gate block nt and the up block I/128 + nt
+              const int nb = C::EPI == 1 ? (j == 0 ? w.nt : (p.I >> 7) + w.nt) : min(nb0 + j, p.NB - 1);
+              cp_async_4(raw + C::RAW_A + 4 * (k * C::NBT + j), sfb_e + static_cast<int64_t>(nb) * p.KB + kb);
+            }
           }
           cp_async_mbar_arrive(&sa_full[rr.slot]);
         }
@@ -538,7 +569,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
       for (int g = 0; g < C::SFB_GROUPS; ++g)
 #pragma unroll
-        for (int r1 = 0; r1 < 4; ++r1) jb[g][r1] = ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
+        for (int r1 = 0; r1 < 4; ++r1)
+          jb[g][r1] = C::EPI == 1 ? g : ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
       for (int qi = 0; qi < KQ; ++qi, rr.next(), sq.next()) {
         // the quad's scales have landed, and the slot's previous quad has
         // been copied out and its MMAs have completed
@@ -588,6 +620,89 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       }
     }
   convert_done:;
+  } else if (C::EPI == 1 && warp >= C::EPI_BASE) {
+    // ------------------------------------------------------------ fused FFN epilogue
+    const int quad = warp & 3;          // TMEM lanes this warp may access (one warp per quadrant)
+    const int row = quad * 32 + lane;   // token row of this CTA's tile
+    const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
+    const int IB = p.I >> 7;
+    uint32_t tc = 0;
+    for (int t = t_first; t < total; t += t_step) {
+      const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+      if (!w.valid) continue;
+      int m_valid = p.M;
+      if (FORM == kFormMasked) {
+        m_valid = __ldg(p.masked_m + w.e);
+        m_valid = m_valid < 0 ? 0 : (m_valid > p.M ? p.M : m_valid);
+      }
+      const int m = w.mt * C::BT + row;
+      bool ok = m < m_valid;
+      if (FORM == kFormContig) ok = ok && __ldg(p.m_indices + m) == w.e;
+      const int64_t grow = (FORM == kFormMasked ? static_cast<int64_t>(w.e) * p.M : 0) + m;
+      if (!warp_wait(&tfull[0], tc & 1u, ctl, lane)) goto ffn_done;
+      tc_fence_after();
+      float h[128];
+      float amax = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rg[32], ru[32];
+        tmem_ld32_issue(tmem_base + t_lane + static_cast<uint32_t>(32 * c), rg);
+        tmem_ld32_issue(tmem_base + t_lane + static_cast<uint32_t>(128 + 32 * c), ru);
+        tmem_wait_ld64(rg, ru);
+        if (c == 3) {
+          // the accumulator is in registers: the next tile's MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (C::PAIR && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[0]), 0));
+            else mbar_arrive(&tempty[0]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float hv = round_bf16(__fmul_rn(silu_fixed(round_bf16(__uint_as_float(rg[j]))),
+                                                round_bf16(__uint_as_float(ru[j]))));
+          h[32 * c + j] = hv;
+          amax = fmaxf(amax, fabsf(hv));
+        }
+        if (p.gu != nullptr && ok) {
+          // bf16 gate at columns nt*128 + 32c.., up at I + nt*128 + 32c..
+          uint16_t* gdst = p.gu + grow * (2 * p.I) + w.nt * 128 + 32 * c;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            *reinterpret_cast<uint4*>(gdst + j) = make_uint4(
+                pack_bf16x2(__uint_as_float(rg[j]), __uint_as_float(rg[j + 1])),
+                pack_bf16x2(__uint_as_float(rg[j + 2]), __uint_as_float(rg[j + 3])),
+                pack_bf16x2(__uint_as_float(rg[j + 4]), __uint_as_float(rg[j + 5])),
+                pack_bf16x2(__uint_as_float(rg[j + 6]), __uint_as_float(rg[j + 7])));
+            *reinterpret_cast<uint4*>(gdst + p.I + j) = make_uint4(
+                pack_bf16x2(__uint_as_float(ru[j]), __uint_as_float(ru[j + 1])),
+                pack_bf16x2(__uint_as_float(ru[j + 2]), __uint_as_float(ru[j + 3])),
+                pack_bf16x2(__uint_as_float(ru[j + 4]), __uint_as_float(ru[j + 5])),
+                pack_bf16x2(__uint_as_float(ru[j + 6]), __uint_as_float(ru[j + 7])));
+          }
+        }
+      }
+      if (ok) {
+        // the per-token power-of-two quantization of per_token_cast_to_fp8_ue8m0
+        float scale, inv;
+        group_scale<true>(fmaxf(amax, kAmaxFloor), scale, inv);
+        uint8_t* qdst = p.hq + grow * p.I + w.nt * 128;
+#pragma unroll
+        for (int j = 0; j < 128; j += 16) {
+          uint32_t v[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            v[i] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(h[j + 4 * i], inv), __fmul_rn(h[j + 4 * i + 1], inv))) |
+                   (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(h[j + 4 * i + 2], inv),
+                                                     __fmul_rn(h[j + 4 * i + 3], inv))) << 16);
+          *reinterpret_cast<uint4*>(qdst + j) = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+        p.sfh[static_cast<int64_t>((FORM == kFormMasked ? w.e * IB : 0) + w.nt) * p.sfh_stride + m] = scale;
+      }
+      ++tc;
+    }
+  ffn_done:;
   } else if (warp >= C::EPI_BASE) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - C::EPI_BASE;

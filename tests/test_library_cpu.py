@@ -110,3 +110,25 @@ def test_ue8m0_gemm_validation_without_the_device(lib):
     for w, pair in ((-1, 0), (64, 0), (192, 0), (512, 0), (128, 1), (256, 1)):
         assert lib.fg_set_ue8m0_tile(w, pair) == 1
     assert lib.fg_set_ue8m0_tile(0, 0) == 0
+
+
+def test_ffn_validation_without_the_device(lib):
+    P = ctypes.c_void_p
+    ok = P(FAKE)
+    args = [ok] * 11
+    # I and H must be positive multiples of 128; M_total a multiple of 128
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 100, 2, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 200, 128, 2, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 100, 256, 128, 2, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 128, 0, None) == 1
+    bad = list(args)
+    bad[6] = P(MISALIGNED)  # Hq
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*bad, 256, 256, 128, 2, None) == 1
+    margs = list(args)
+    margs[10] = None  # masked_m
+    assert lib.fp8_moe_ffn_masked_ue8m0(*margs, 2, 64, 256, 128, 32, None) == 1
+    assert lib.fp8_moe_ffn_masked_ue8m0(*args, 2, 0, 256, 128, 32, None) == 1
+    # an empty contiguous problem is a no-op success; GU may be NULL
+    nogu = list(args)
+    nogu[8] = None
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*nogu, 0, 256, 128, 2, None) == 0
