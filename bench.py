@@ -185,6 +185,8 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict, ue8m0
     (flops_per_second, description, seconds)."""
     import oracle
 
+    if kind == "ffn":
+        return ffn_cpu_sample(inp, target_s, threads, cache)
     K, N = inp.K, inp.N
     if kind == "dense":
         a_rows, experts = inp.a, np.zeros(inp.M, np.int64)
@@ -240,6 +242,48 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict, ue8m0
     return flops / dt, desc, dt
 
 
+def ffn_cpu_sample(inp, target_s: float, threads: int, cache: dict):
+    """The oracle's expert-FFN chain (UE8M0 quantization of the sampled rows,
+    first GEMM, bf16, SwiGLU, requantization, second GEMM) on a bounded sample
+    of valid rows; expert weights are quantized outside the timed part."""
+    import oracle
+
+    H, I = inp.H, inp.I
+    valid = np.nonzero(inp.m_indices >= 0)[0]
+    experts = inp.m_indices[valid].astype(np.int64)
+
+    def weights(e):
+        if ("w", e) not in cache:
+            cache[("w", e)] = (oracle.per_block_cast(inp.w1[e], threads=threads, ue8m0=True),
+                               oracle.per_block_cast(inp.w2[e], threads=threads, ue8m0=True))
+        return cache[("w", e)]
+
+    order = np.random.default_rng(0).permutation(len(valid))
+    rows = cache.get("rows", 1)
+    while True:
+        take = order[:min(rows, len(order))]
+        for e in np.unique(experts[take]):
+            weights(int(e))
+        t0 = time.perf_counter()
+        qa, sa = oracle.per_token_cast(inp.a[valid[take]], threads=threads, ue8m0=True)
+        for e in np.unique(experts[take]):
+            sub = np.nonzero(experts[take] == e)[0]
+            (w1q, sw1), (w2q, sw2) = weights(int(e))
+            gu = oracle.f64_to_bf16(oracle.gemm_nt(qa[sub], sa[sub], w1q, sw1, threads=threads))
+            h = oracle.swiglu(gu[:, :I], gu[:, I:])
+            hq, sh = oracle.per_token_cast(h, threads=threads, ue8m0=True)
+            oracle.gemm_nt(hq, sh, w2q, sw2, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or len(take) >= len(order):
+            break
+        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9))
+    cache["rows"] = rows
+    flops = 6.0 * len(take) * H * I
+    desc = ("%d of %d valid rows through the whole expert FFN (quantization, first GEMM, "
+            "SwiGLU, requantization, second GEMM), H=%d, I=%d" % (len(take), len(order), H, I))
+    return flops / dt, desc, dt
+
+
 # ---------------------------------------------------------------------- ranks
 
 def max_over_ranks(dist, values, device):
@@ -255,6 +299,8 @@ def max_over_ranks(dist, values, device):
 
 def gemm_kernel_name(kind: str, inp, ue8m0: bool) -> str:
     """The GEMM kernel a step launches (the library's choice for the shape)."""
+    if kind == "ffn":
+        return "fp8_gemm_mx_kernel x2 (first GEMM with fused SwiGLU + requantization, second GEMM)"
     thin = (kind == "dense" and inp.M <= 64) or (
         kind == "masked" and max(1, int(round(float(np.mean(inp.masked_m))))) <= 64)
     return "fp8_gemm_mx_kernel" if ue8m0 and not thin else "fp8_gemm_kernel"
@@ -263,13 +309,25 @@ def gemm_kernel_name(kind: str, inp, ue8m0: bool) -> str:
 class OperandSet:
     """Device buffers of one copy of a step's operands."""
 
-    def __init__(self, torch, kind, inp, fg, x, w, B, SB, with_weight_quant: bool):
+    def __init__(self, torch, kind, inp, fg, x, w, B, SB, with_weight_quant: bool, extra=None):
         dev = "cuda"
         K, N = inp.K, inp.N
         self.x = x.clone()
         self.w = w.clone() if with_weight_quant else None
         self.B = B.clone()
         self.SB = SB.clone()
+        self.extra = []
+        if kind == "ffn":
+            W2, SW2 = extra
+            self.W2, self.SW2 = W2.clone(), SW2.clone()
+            M, H, I = inp.M_total, inp.H, inp.I
+            self.A = torch.empty((M, H), dtype=torch.uint8, device=dev)
+            self.SA = fg.empty_sfa(1, M, H, dev)
+            self.Hq = torch.empty((M, I), dtype=torch.uint8, device=dev)
+            self.SH = fg.empty_sfa(1, M, I, dev)
+            self.D = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+            self.extra = [self.W2, self.SW2, self.Hq, self.SH]
+            return
         if kind == "dense":
             G, M = 1, inp.M
             self.A = torch.empty((inp.M, K), dtype=torch.uint8, device=dev)
@@ -286,6 +344,7 @@ class OperandSet:
 
     def nbytes(self):
         ts = [self.x, self.B, self.SB, self.A, self.D, self.SA] + ([self.w] if self.w is not None else [])
+        ts += self.extra
         return sum(t.numel() * t.element_size() for t in ts)
 
 
@@ -312,20 +371,34 @@ class Step:
         def bf16(bits):
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
-        x, w = bf16(inp.a), bf16(inp.b)
-        Gw = 1 if kind == "dense" else inp.G
-        B = torch.empty((N, K) if kind == "dense" else (inp.G, N, K), dtype=torch.uint8, device=dev)
-        SB = fg.empty_sfb(Gw, N, K, dev)
-        self.q_block(w, B, SB)
-        if kind == "contiguous":
+        extra = None
+        if kind == "ffn":
+            # W1 [G][2I][H] in B/SB, W2 [G][H][I] alongside
+            x, w = bf16(inp.a), bf16(inp.w1)
+            B = torch.empty((inp.G, 2 * inp.I, inp.H), dtype=torch.uint8, device=dev)
+            SB = fg.empty_sfb(inp.G, 2 * inp.I, inp.H, dev)
+            self.q_block(w, B, SB)
+            w2 = bf16(inp.w2)
+            W2 = torch.empty((inp.G, inp.H, inp.I), dtype=torch.uint8, device=dev)
+            SW2 = fg.empty_sfb(inp.G, inp.H, inp.I, dev)
+            self.q_block(w2, W2, SW2)
+            extra = (W2, SW2)
+            del w2
+        else:
+            x, w = bf16(inp.a), bf16(inp.b)
+            Gw = 1 if kind == "dense" else inp.G
+            B = torch.empty((N, K) if kind == "dense" else (inp.G, N, K), dtype=torch.uint8, device=dev)
+            SB = fg.empty_sfb(Gw, N, K, dev)
+            self.q_block(w, B, SB)
+        if kind in ("contiguous", "ffn"):
             self.mi = torch.from_numpy(inp.m_indices).to(dev)
         if kind == "masked":
             self.mm = torch.from_numpy(inp.masked_m).to(dev)
             self.expected_m = max(1, int(round(float(np.mean(inp.masked_m)))))
-        first = OperandSet(torch, kind, inp, fg, x, w, B, SB, with_weight_quant)
+        first = OperandSet(torch, kind, inp, fg, x, w, B, SB, with_weight_quant, extra)
         per = first.nbytes()
         n = max(2, -(-min_total_bytes // per)) if min_total_bytes > 0 else 1
-        self.sets = [first] + [OperandSet(torch, kind, inp, fg, x, w, B, SB, with_weight_quant)
+        self.sets = [first] + [OperandSet(torch, kind, inp, fg, x, w, B, SB, with_weight_quant, extra)
                                for _ in range(n - 1)]
         del x, w, B, SB
         self.set_bytes = per
@@ -337,7 +410,10 @@ class Step:
         self.q_token(o.x, o.A, o.SA)
 
     def gemm(self, o):
-        if self.kind == "dense":
+        if self.kind == "ffn":
+            self.fg.fp8_moe_ffn_contiguous_ue8m0(o.A, o.SA, o.B, o.SB, o.W2, o.SW2, o.Hq, o.SH, o.D,
+                                                 self.mi)
+        elif self.kind == "dense":
             self.g_dense(o.A, o.SA, o.B, o.SB, o.D)
         elif self.kind == "contiguous":
             self.g_contig(o.A, o.SA, o.B, o.SB, o.D, self.mi)
@@ -345,7 +421,7 @@ class Step:
             self.g_masked(o.A, o.SA, o.B, o.SB, o.D, self.mm, self.expected_m)
 
     def launches_per_step(self):
-        return 2 + (1 if self.with_wq else 0)
+        return (3 if self.kind == "ffn" else 2) + (1 if self.with_wq else 0)
 
     def run(self, i):
         o = self.sets[i % len(self.sets)]
@@ -366,7 +442,9 @@ def run_ours(args, rank, world, local_rank):
     inp = workloads.make(args.workload, seed=0)
     flops, alg_bytes = workloads.flops_and_bytes(kind, inp)
     rotate = args.l2 == "rotate"
-    ue8m0 = args.scales == "ue8m0"
+    ue8m0 = args.scales == "ue8m0" or kind == "ffn"  # the expert FFN uses power-of-two scales
+    if kind == "ffn" and args.with_weight_quant:
+        raise SystemExit("--with-weight-quant is not supported for the expert FFN workload")
     step = Step(fg, torch, kind, inp, args.with_weight_quant,
                 ROTATE_MIN_BYTES if rotate else 0, ue8m0)
     R = len(step.sets)
@@ -563,7 +641,9 @@ def run_ours(args, rank, world, local_rank):
            "scales": ("power-of-two (UE8M0) scales, block-scaled tensor-core GEMM" if ue8m0 else
                       "fp32 scales amax/448, promoted per 128-wide K block"),
            "parallelism": "replicas" if world > 1 else "single GPU"}
-    if kind == "dense":
+    if kind == "ffn":
+        cfg.update(H=inp.H, I=inp.I, G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
+    elif kind == "dense":
         cfg["M"] = inp.M
     elif kind == "contiguous":
         cfg.update(G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
@@ -699,7 +779,7 @@ def run_reference(args, rank, world):
     threads = oracle.hardware_threads()
     per_step = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     cache = {}
-    ue8m0 = args.scales == "ue8m0"
+    ue8m0 = args.scales == "ue8m0" or kind == "ffn"
     for _ in range(args.warmup):
         cpu_sample(inp, kind, per_step, threads, cache, ue8m0)
     vals, descs, secs = [], [], []

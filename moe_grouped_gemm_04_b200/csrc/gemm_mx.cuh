@@ -641,47 +641,47 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       const int64_t grow = (FORM == kFormMasked ? static_cast<int64_t>(w.e) * p.M : 0) + m;
       if (!warp_wait(&tfull[0], tc & 1u, ctl, lane)) goto ffn_done;
       tc_fence_after();
-      float h[128];
-      float amax = 0.0f;
+      // gate and up values as packed bf16 pairs (the activation takes them in
+      // bf16): all 256 columns are read first, so that the accumulator goes
+      // back to the MMA before the activation arithmetic
+      uint32_t gp[64], upk[64];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t rg[32], ru[32];
         tmem_ld32_issue(tmem_base + t_lane + static_cast<uint32_t>(32 * c), rg);
         tmem_ld32_issue(tmem_base + t_lane + static_cast<uint32_t>(128 + 32 * c), ru);
         tmem_wait_ld64(rg, ru);
-        if (c == 3) {
-          // the accumulator is in registers: the next tile's MMAs may start
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (C::PAIR && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[0]), 0));
-            else mbar_arrive(&tempty[0]);
-          }
-        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float hv = round_bf16(__fmul_rn(silu_fixed(round_bf16(__uint_as_float(rg[j]))),
-                                                round_bf16(__uint_as_float(ru[j]))));
-          h[32 * c + j] = hv;
-          amax = fmaxf(amax, fabsf(hv));
+        for (int j = 0; j < 16; ++j) {
+          gp[16 * c + j] = pack_bf16x2(__uint_as_float(rg[2 * j]), __uint_as_float(rg[2 * j + 1]));
+          upk[16 * c + j] = pack_bf16x2(__uint_as_float(ru[2 * j]), __uint_as_float(ru[2 * j + 1]));
         }
-        if (p.gu != nullptr && ok) {
-          // bf16 gate at columns nt*128 + 32c.., up at I + nt*128 + 32c..
-          uint16_t* gdst = p.gu + grow * (2 * p.I) + w.nt * 128 + 32 * c;
+      }
+      // the accumulator is in registers: the next tile's MMAs may start
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (C::PAIR && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[0]), 0));
+        else mbar_arrive(&tempty[0]);
+      }
+      if (p.gu != nullptr && ok) {
+        // bf16 gate at columns nt*128.., up at I + nt*128..
+        uint16_t* gdst = p.gu + grow * (2 * p.I) + w.nt * 128;
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            *reinterpret_cast<uint4*>(gdst + j) = make_uint4(
-                pack_bf16x2(__uint_as_float(rg[j]), __uint_as_float(rg[j + 1])),
-                pack_bf16x2(__uint_as_float(rg[j + 2]), __uint_as_float(rg[j + 3])),
-                pack_bf16x2(__uint_as_float(rg[j + 4]), __uint_as_float(rg[j + 5])),
-                pack_bf16x2(__uint_as_float(rg[j + 6]), __uint_as_float(rg[j + 7])));
-            *reinterpret_cast<uint4*>(gdst + p.I + j) = make_uint4(
-                pack_bf16x2(__uint_as_float(ru[j]), __uint_as_float(ru[j + 1])),
-                pack_bf16x2(__uint_as_float(ru[j + 2]), __uint_as_float(ru[j + 3])),
-                pack_bf16x2(__uint_as_float(ru[j + 4]), __uint_as_float(ru[j + 5])),
-                pack_bf16x2(__uint_as_float(ru[j + 6]), __uint_as_float(ru[j + 7])));
-          }
+        for (int j = 0; j < 64; j += 4) {
+          *reinterpret_cast<uint4*>(gdst + 2 * j) = make_uint4(gp[j], gp[j + 1], gp[j + 2], gp[j + 3]);
+          *reinterpret_cast<uint4*>(gdst + p.I + 2 * j) = make_uint4(upk[j], upk[j + 1], upk[j + 2], upk[j + 3]);
         }
+      }
+      // h = bf16(silu(gate) * up), kept as packed bf16 pairs, and its amax
+      uint32_t hp[64];
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const float h0 = round_bf16(__fmul_rn(silu_fixed(bf16_lo(gp[j])), bf16_lo(upk[j])));
+        const float h1 = round_bf16(__fmul_rn(silu_fixed(bf16_hi(gp[j])), bf16_hi(upk[j])));
+        amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
+        hp[j] = pack_bf16x2(h0, h1);
       }
       if (ok) {
         // the per-token power-of-two quantization of per_token_cast_to_fp8_ue8m0
@@ -689,14 +689,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         group_scale<true>(fmaxf(amax, kAmaxFloor), scale, inv);
         uint8_t* qdst = p.hq + grow * p.I + w.nt * 128;
 #pragma unroll
-        for (int j = 0; j < 128; j += 16) {
+        for (int j = 0; j < 64; j += 8) {
           uint32_t v[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            v[i] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(h[j + 4 * i], inv), __fmul_rn(h[j + 4 * i + 1], inv))) |
-                   (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(h[j + 4 * i + 2], inv),
-                                                     __fmul_rn(h[j + 4 * i + 3], inv))) << 16);
-          *reinterpret_cast<uint4*>(qdst + j) = make_uint4(v[0], v[1], v[2], v[3]);
+            v[i] = static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(bf16_lo(hp[j + 2 * i]), inv),
+                                                    __fmul_rn(bf16_hi(hp[j + 2 * i]), inv))) |
+                   (static_cast<uint32_t>(cvt_e4m3x2(__fmul_rn(bf16_lo(hp[j + 2 * i + 1]), inv),
+                                                     __fmul_rn(bf16_hi(hp[j + 2 * i + 1]), inv))) << 16);
+          *reinterpret_cast<uint4*>(qdst + 2 * j) = make_uint4(v[0], v[1], v[2], v[3]);
         }
         p.sfh[static_cast<int64_t>((FORM == kFormMasked ? w.e * IB : 0) + w.nt) * p.sfh_stride + m] = scale;
       }

@@ -20,9 +20,15 @@ inference shapes"):
                            each group padded to a multiple of 128, padding
                            rows zero, m_indices = -1 on padding rows
   masked_32x256x4096x7168  32 experts, capacity 256, masked_m ~ U{0..256}
+  ffn_contiguous_8x7168x2048  expert FFN (DeepSeek-V3 expert shape: hidden
+                           7168, intermediate 2048) on the contiguous
+                           workload's 8 experts and token counts; W1 [8][4096][7168]
+                           (gate rows, then up rows) and W2 [8][7168][2048]
+                           ~ N(0, 0.02)
 
 Seeds: every tensor draws from its own ``numpy.random.default_rng(seed + i)``
-with i = 0 for A, 1 for B, 2 for the routing and 3 for masked_m.
+with i = 0 for A, 1 for B (the FFN's W1), 2 for the routing, 3 for masked_m
+and 5 for the FFN's W2.
 """
 from __future__ import annotations
 
@@ -164,6 +170,35 @@ def contiguous(N: int, K: int, counts: Optional[np.ndarray] = None, G: int = 8,
 
 
 @dataclasses.dataclass
+class FfnInputs:
+    a: np.ndarray          # bf16 bits [M_total][H], padding rows zero
+    w1: np.ndarray         # bf16 bits [G][2I][H]: I gate rows, then I up rows
+    w2: np.ndarray         # bf16 bits [G][H][I]
+    m_indices: np.ndarray  # int32 [M_total]
+    counts: np.ndarray     # int64 [G]
+    M_total: int
+    H: int
+    I: int
+    G: int
+
+    @property
+    def N(self) -> int:  # output columns (of the second GEMM)
+        return self.H
+
+    @property
+    def K(self) -> int:  # contraction of the first GEMM
+        return self.H
+
+
+def ffn_contiguous(H: int, I: int, G: int = 8, seed: int = 0, a_std: float = 1.0,
+                   w_std: float = 0.02) -> FfnInputs:
+    c = contiguous(N=2 * I, K=H, G=G, seed=seed, a_std=a_std, b_std=w_std)
+    w2 = normal_bf16(np.random.default_rng(seed + 5), (c.G, H, I), w_std)
+    return FfnInputs(a=c.a, w1=c.b, w2=w2, m_indices=c.m_indices, counts=c.counts,
+                     M_total=c.M_total, H=H, I=I, G=c.G)
+
+
+@dataclasses.dataclass
 class DequantInputs:
     b: np.ndarray  # bf16 bits [N][K] (quantized once, then dequantized)
     N: int
@@ -195,6 +230,8 @@ WORKLOADS = {
     "masked_32x256x4096x7168": ("masked", dict(G=32, M_max=256, N=4096, K=7168)),
     # weight dequantization (e4m3 + 128x128 scales -> bf16) of a prefill weight
     "dequant_7168x2048": ("dequant", dict(N=7168, K=2048)),
+    # expert FFN (first GEMM + SwiGLU + requantization, second GEMM)
+    "ffn_contiguous_8x7168x2048": ("ffn", dict(H=7168, I=2048, G=8)),
 }
 
 
@@ -206,6 +243,8 @@ def make(name: str, seed: int = 0):
         return contiguous(seed=seed, **kw)
     if kind == "dequant":
         return dequant(seed=seed, **kw)
+    if kind == "ffn":
+        return ffn_contiguous(seed=seed, **kw)
     return masked(seed=seed, **kw)
 
 
@@ -217,6 +256,17 @@ def flops_and_bytes(kind: str, inp) -> tuple:
     128 elements) + B (1 B/elt) and its fp32 scales (one per 128x128 block) for
     every expert with at least one valid row + D (2 B/elt) over valid rows.
     """
+    if kind == "ffn":
+        # both GEMMs; bytes: X and its scales, W1 and W2 with their block
+        # scales for every expert with a token, h written and read back with
+        # its scales, Y
+        H, I = inp.H, inp.I
+        mv = int(inp.counts.sum())
+        experts = int((inp.counts > 0).sum())
+        flops = 2.0 * mv * (2 * I) * H + 2.0 * mv * H * I
+        wbytes = experts * (3 * I * H + 4 * ((2 * I // 128) * (H // 128) + (H // 128) * (I // 128)))
+        byts = mv * H + 4 * mv * (H // 128) + wbytes + 2 * (mv * I + 4 * mv * (I // 128)) + 2 * mv * H
+        return flops, float(byts)
     N, K = inp.N, inp.K
     nb = -(-N // 128)
     kb = K // 128
