@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
     lib.oracle_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
     lib.oracle_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
     lib.oracle_gemm_points.argtypes = [P, P, P, P, P, P, P, I64, P, I, I, I, I]
+    lib.oracle_k_grouped.argtypes = [P, P, P, P, P, P, I, I, I, I, I]
+    lib.oracle_k_grouped.restype = ctypes.c_int
     lib.oracle_exp_f32.argtypes = [ctypes.c_float]
     lib.oracle_exp_f32.restype = ctypes.c_float
     lib.oracle_silu_f32.argtypes = [ctypes.c_float]
@@ -287,3 +289,24 @@ def moe_ffn_masked(xq, sx, w1q, sw1, w2q, sw2, masked_m, threads: int = 0):
     hq, sh = per_token_cast(h, threads=threads, ue8m0=True)
     y = grouped_masked(hq, sh, w2q, sw2, masked_m, threads)
     return gu, hq, sh, y
+
+
+# ---------------------------------------------------------------- K-grouped GEMM
+
+def k_grouped(qa, sa, qb, sb, ks, threads: int = 0) -> np.ndarray:
+    """D[e][m][n] (fp64) of the K-grouped GEMM: qa [M][T], sa [M][T/128],
+    qb [N][T], sb [N][T/128] (one scale per row per 128-token block on both
+    sides), ks [G] token counts (multiples of 128, summing to T)."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    ks = np.ascontiguousarray(ks, dtype=np.int32)
+    M, T = qa.shape
+    N = qb.shape[0]
+    G = ks.size
+    assert qb.shape[1] == T and sa.shape == (M, T // BLOCK) and sb.shape == (N, T // BLOCK)
+    out = np.empty((G, M, N), dtype=np.float64)
+    _check(_load().oracle_k_grouped(_ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), _ptr(ks), _ptr(out),
+                                    G, M, N, T, threads), "k_grouped")
+    return out

@@ -34,6 +34,16 @@
 //    only the two scale multiplies and the outer sum over K blocks round in
 //    fp64. The result is kept in fp64, not rounded to bf16.
 //
+//  * The K-grouped GEMM of FP8 training's expert weight gradients (the
+//    animattoys.com page, section "為現代 AI 計算而造", names FP8 training
+//    among DeepGEMM's uses; the DeepSeek-V3 review's quantize / dequantize /
+//    GEMM trio, "创新之处" item 4, scales every operand per 128 elements of
+//    the contraction). Reading taken: the contraction runs over tokens, the
+//    experts' token ranges are stacked along it (each a multiple of 128), and
+//    both operands carry one scale per row per 128-token block:
+//      D[e][m][n] = sum over expert e's token blocks tb of
+//                   sa[m][tb] * sb[n][tb] * sum_{t in tb} a[m][t] * b[n][t].
+//    Exact block sums, fp64 result (as for the GEMM above).
 //  * The expert FFN's activation (the "Mega MoE" kernel fuses both expert
 //    GEMMs with the SwiGLU activation: "DeepGEMM" overview, section
 //    "swapAB与Mega MoE"; the pages name SwiGLU without a formula). Reading
@@ -408,6 +418,37 @@ int oracle_gemm_points(const uint8_t* qa, const float* sa, const uint8_t* qb, co
     const float* srow = sb + (e[p] * NB + n[p] / kBlock) * KB;
     out[p] = dot_blocked(qa + a_row[p] * K, sa + a_row[p] * KB, brow, srow, K);
   });
+  return 0;
+}
+
+// K-grouped GEMM. qa: e4m3 [M][T]; sa: fp32 [M][T/128]; qb: e4m3 [N][T];
+// sb: fp32 [N][T/128]; ks: int32 [G] token counts (multiples of 128, summing
+// to T); out: fp64 [G][M][N]. Returns 0, or -1 on bad sizes or counts.
+int oracle_k_grouped(const uint8_t* qa, const float* sa, const uint8_t* qb, const float* sb,
+                     const int32_t* ks, double* out, int G, int M, int N, int T, int threads) {
+  if (G < 1 || M < 0 || N < 0 || T < 0 || T % kBlock != 0) return -1;
+  int64_t total = 0;
+  for (int e = 0; e < G; ++e) {
+    if (ks[e] < 0 || ks[e] % kBlock != 0) return -1;
+    total += ks[e];
+  }
+  if (total != T) return -1;
+  const int TB = T / kBlock;
+  int64_t t0 = 0;
+  for (int e = 0; e < G; ++e) {
+    const int64_t tb0 = t0 / kBlock;
+    const int len = ks[e];
+    double* oe = out + static_cast<int64_t>(e) * M * N;
+    parallel_for(M, threads, [&](int64_t m) {
+      for (int n = 0; n < N; ++n) {
+        oe[m * N + n] = len == 0 ? 0.0
+                                 : dot_blocked(qa + m * T + t0, sa + m * TB + tb0,
+                                               qb + static_cast<int64_t>(n) * T + t0,
+                                               sb + static_cast<int64_t>(n) * TB + tb0, len);
+      }
+    });
+    t0 += len;
+  }
   return 0;
 }
 

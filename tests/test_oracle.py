@@ -613,3 +613,89 @@ def test_ffn_masked_matches_contiguous_per_expert():
         assert np.array_equal(gu_m[e, :v], gu_c)
         assert np.array_equal(hq_m[e, :v], hq_c)
         assert np.array_equal(y_m[e, :v], y_c)
+
+
+# ---------------------------------------------------------------- K-grouped GEMM
+
+def _kg_operands(rng, M, N, ks, ue8m0=True):
+    T = int(sum(ks))
+    a = workloads.bf16_bits(rng.standard_normal((M, T)).astype(np.float32))
+    b = workloads.bf16_bits(rng.standard_normal((N, T)).astype(np.float32))
+    qa, sa = oracle.per_token_cast(a, ue8m0=ue8m0)
+    qb, sb = oracle.per_token_cast(b, ue8m0=ue8m0)
+    return qa, sa, qb, sb
+
+
+def test_k_grouped_single_group_is_the_dense_gemm():
+    """One expert and B row scales constant over each 128-row block: the dense
+    block-scaled GEMM (a swapped row/block index or operand fails this)."""
+    rng = np.random.default_rng(41)
+    M, N, T = 130, 256, 384
+    qa, sa, qb, _ = _kg_operands(rng, M, N, [T])
+    sbb = (2.0 ** rng.integers(-6, 3, size=(N // 128, T // 128))).astype(np.float32)
+    sb_rows = np.repeat(sbb, 128, axis=0)
+    d = oracle.k_grouped(qa, sa, qb, sb_rows, np.array([T], np.int32))
+    ref = oracle.gemm_nt(qa, sa, qb, sbb)
+    assert np.array_equal(d[0], ref)
+
+
+def test_k_grouped_sums_to_the_whole_range():
+    """Linearity: the experts' results add up to one GEMM over all tokens."""
+    rng = np.random.default_rng(42)
+    M, N = 64, 96
+    ks = [256, 0, 128, 384]
+    qa, sa, qb, sb = _kg_operands(rng, M, N, ks)
+    d = oracle.k_grouped(qa, sa, qb, sb, np.array(ks, np.int32))
+    whole = oracle.k_grouped(qa, sa, qb, sb, np.array([sum(ks)], np.int32))[0]
+    rms = np.sqrt(np.mean(whole ** 2))
+    assert np.max(np.abs(d.sum(axis=0) - whole)) <= 1e-12 * rms * len(ks)
+    assert np.all(d[1] == 0.0)  # the empty expert
+
+
+def test_k_grouped_brute_force_per_expert():
+    """Each expert's result is the fp64 product of its decoded, scaled token
+    slices (both scales indexed by row and 128-token block)."""
+    rng = np.random.default_rng(43)
+    M, N = 20, 24
+    ks = [128, 256]
+    qa, sa, qb, sb = _kg_operands(rng, M, N, ks)
+    d = oracle.k_grouped(qa, sa, qb, sb, np.array(ks, np.int32))
+    av = oracle.e4m3_decode(qa) * np.repeat(sa, 128, axis=1)
+    bv = oracle.e4m3_decode(qb) * np.repeat(sb, 128, axis=1)
+    t0 = 0
+    for e, k in enumerate(ks):
+        ref = av[:, t0:t0 + k] @ bv[:, t0:t0 + k].T
+        assert np.allclose(d[e], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+        t0 += k
+
+
+def test_k_grouped_integer_exact():
+    """Entries in {-1, 0, 1} with power-of-two scales: exact (integer matmul)."""
+    rng = np.random.default_rng(44)
+    M, N = 33, 40
+    ks = [128, 384]
+    T = sum(ks)
+    ia = rng.integers(-1, 2, size=(M, T))
+    ib = rng.integers(-1, 2, size=(N, T))
+    qa = oracle.e4m3_encode(ia.astype(np.float32))
+    qb = oracle.e4m3_encode(ib.astype(np.float32))
+    sa = (2.0 ** rng.integers(-3, 3, size=(M, T // 128))).astype(np.float32)
+    sb = (2.0 ** rng.integers(-3, 3, size=(N, T // 128))).astype(np.float32)
+    d = oracle.k_grouped(qa, sa, qb, sb, np.array(ks, np.int32))
+    t0 = 0
+    for e, k in enumerate(ks):
+        ref = np.zeros((M, N))
+        for tb in range(t0 // 128, (t0 + k) // 128):
+            blk = slice(tb * 128, (tb + 1) * 128)
+            ref += np.outer(sa[:, tb], sb[:, tb]) * (ia[:, blk] @ ib[:, blk].T)
+        assert np.array_equal(d[e], ref)
+        t0 += k
+
+
+def test_k_grouped_rejects_bad_counts():
+    qa = np.zeros((4, 256), np.uint8)
+    sa = np.ones((4, 2), np.float32)
+    with pytest.raises(ValueError):
+        oracle.k_grouped(qa, sa, qa, sa, np.array([100, 156], np.int32))
+    with pytest.raises(ValueError):
+        oracle.k_grouped(qa, sa, qa, sa, np.array([128], np.int32))
