@@ -76,6 +76,7 @@ typedef enum {
 #define FG_DEVICE_WAIT_TIMEOUT 1   /* a bounded pipeline wait gave up */
 #define FG_DEVICE_BAD_MASKED_M 2   /* masked_m[e] < 0 or > M_max (clamped) */
 #define FG_DEVICE_BAD_M_INDEX 3    /* m_indices entry >= G (tile skipped) */
+#define FG_DEVICE_BAD_K_GROUP 4    /* ks entry < 0, not a multiple of 128, or sum > T (truncated) */
 
 /* Row stride (in floats) of the MN-major activation-scale layout. */
 int fg_sfa_stride(int M);
@@ -247,6 +248,29 @@ fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uin
                                   uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
                                   const int32_t* masked_m, int G, int M_max, int H, int I,
                                   int expected_m, cudaStream_t stream);
+
+/*
+ * K-grouped GEMM with power-of-two scales, for the weight gradients of MoE
+ * experts in FP8 training (dW_e = dY_e^T X_e: the contraction runs over the
+ * tokens routed to each expert). The experts' token ranges are stacked along
+ * K; both operands carry one scale per row per 128-token block:
+ *   D[e][m][n] = sum over expert e's token blocks tb of
+ *                sa[m][tb] * sb[n][tb] * sum_{t in tb} a[m][t] * b[n][t],
+ * accumulated in fp32 (block-scaled tensor-core MMAs, whole range in tensor
+ * memory). Sources: FP8 training among DeepGEMM's uses ("一文看懂 DeepSeek
+ * 開源項目第三彈", section "為現代 AI 計算而造") and per-128-element scaling
+ * of every GEMM operand (DeepSeek-V3 review, "创新之处" item 4).
+ * A: e4m3 [M][T] (K contiguous); sfa: fp32 MN-major [T/128][stride(M)]
+ * (the layout per_token_cast_to_fp8_ue8m0 writes for a [M][T] input);
+ * B: e4m3 [N][T]; sfb: fp32 MN-major [T/128][stride(N)]; D: fp32 [G][M][N];
+ * ks: int32 [G] device array of token counts, each a multiple of 128 and
+ * summing to T (violations set FG_DEVICE_BAD_K_GROUP; the counts are then
+ * truncated). An expert with ks[e] = 0 gets D[e] = 0. Scales must be powers of
+ * two. G >= 1, M >= 1, N % 16 == 0, T % 128 == 0 (T = 0 allowed).
+ */
+fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                     const float* sfb, float* D, const int32_t* ks, int G, int M,
+                                     int N, int T, cudaStream_t stream);
 
 /*
  * Tuning knob of the three _ue8m0 GEMMs (process-wide). width = 0: choose the

@@ -13,7 +13,8 @@ The functions carry the C names:
   per_token_cast_to_fp8_ue8m0, per_block_cast_to_fp8_ue8m0, and the GEMMs for
   power-of-two scales fp8_gemm_nt_ue8m0, fp8_grouped_gemm_contiguous_ue8m0,
   fp8_grouped_gemm_masked_ue8m0 (set_ue8m0_tile tunes them), and the expert FFN
-  fp8_moe_ffn_contiguous_ue8m0, fp8_moe_ffn_masked_ue8m0
+  fp8_moe_ffn_contiguous_ue8m0, fp8_moe_ffn_masked_ue8m0, and the K-grouped
+  (expert weight-gradient) GEMM fp8_k_grouped_gemm_nt_ue8m0
 plus allocation helpers that return tensors in the layouts the kernels use.
 """
 from __future__ import annotations
@@ -39,6 +40,7 @@ EXPORTED = (
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
     "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
     "fg_set_ue8m0_tile", "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
+    "fp8_k_grouped_gemm_nt_ue8m0",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
 
@@ -79,6 +81,7 @@ def load_library() -> ctypes.CDLL:
     lib.fg_set_ue8m0_tile.argtypes = [I, I]
     lib.fp8_moe_ffn_contiguous_ue8m0.argtypes = [P] * 11 + [I, I, I, I, P]
     lib.fp8_moe_ffn_masked_ue8m0.argtypes = [P] * 11 + [I, I, I, I, I, P]
+    lib.fp8_k_grouped_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
     lib.fg_status_string.argtypes = [I]
@@ -92,6 +95,7 @@ def load_library() -> ctypes.CDLL:
               "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0",
               "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile",
               "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
+              "fp8_k_grouped_gemm_nt_ue8m0",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
     _lib = lib
@@ -301,6 +305,21 @@ def fp8_moe_ffn_masked_ue8m0(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, masked_m, e
         _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
         _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m),
         _stream(stream)))
+
+
+def fp8_k_grouped_gemm_nt_ue8m0(A, sfa, B, sfb, D, ks, stream=None) -> None:
+    """K-grouped GEMM (expert weight gradients): A uint8 [M][T], sfa [T/128][stride(M)],
+    B uint8 [N][T], sfb [T/128][stride(N)], ks int32 [G] token counts (device),
+    D float32 [G][M][N]."""
+    M, T = A.shape
+    N = B.shape[0]
+    G = ks.numel()
+    if ks.dtype != torch.int32:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "ks must be int32 [G]")
+    if D.dtype != torch.float32 or tuple(D.shape) != (G, M, N):
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "D must be float32 [G][M][N]")
+    _check(load_library().fp8_k_grouped_gemm_nt_ue8m0(
+        _ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), _ptr(ks), G, M, N, T, _stream(stream)))
 
 
 def set_ue8m0_tile(width: int, pair: bool = False) -> None:

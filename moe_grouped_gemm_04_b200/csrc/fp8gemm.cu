@@ -434,6 +434,9 @@ using MxP224 = MxCfg<224, 3, 2, 1, true, 2>;  // CTA pairs, 256 x 224 tiles
 // first GEMM of the expert FFN with the fused SwiGLU + requantization epilogue
 using MxFfnP = MxCfg<256, 3, 1, 1, true, 2, 1>;
 using MxFfnS = MxCfg<256, 4, 1, 1, false, 1, 1>;
+// K-grouped GEMM (expert weight gradients): fp32 output, per-row B scales
+using MxKgP = MxCfg<224, 3, 2, 1, true, 2, 2>;
+using MxKgS = MxCfg<224, 4, 2, 1, false, 1, 2>;
 
 // Outputs of the fused expert-FFN epilogue.
 struct FfnOut {
@@ -478,28 +481,44 @@ fg_status mx_kernel_attr(int dev, int* max_clusters) {
   return FG_OK;
 }
 
+// The K-grouped problem's fp32 output travels in the Problem's D slot.
+float* ffn_d32(const Problem& pr) { return reinterpret_cast<float*>(pr.D); }
+
 template <class C, int FORM>
 fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaStream_t stream,
-                    const FfnOut* ffn = nullptr) {
+                    const FfnOut* ffn = nullptr, int kb_override = -1) {
   static_assert(C::smem_bytes(FORM) <= 232448, "shared memory per CTA");
   int max_clusters = 0;
   FG_TRY((mx_kernel_attr<C, FORM>(dev_id, &max_clusters)));
   const int KB = pr.K / 128;
-  CUtensorMap tmA, tmB, tmSA, tmD;
+  CUtensorMap tmA, tmB, tmSA, tmSB, tmD;
   FG_TRY(make_map(&tmA, pr.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
                   static_cast<uint64_t>(pr.slabs) * pr.M, pr.K, 128, C::BT,
                   CU_TENSOR_MAP_SWIZZLE_128B, "A"));
+  // (K-grouped: one B of N rows whose K range the experts share)
   FG_TRY(make_map(&tmB, pr.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K,
-                  static_cast<uint64_t>(pr.G) * pr.N, pr.K, 128, C::B_BOX,
+                  static_cast<uint64_t>(FORM == kFormKGrouped ? 1 : pr.G) * pr.N, pr.K, 128, C::B_BOX,
                   CU_TENSOR_MAP_SWIZZLE_128B, "B"));
   // token scales: boxes of 128 tokens x 4 K blocks (one quad)
   FG_TRY(make_map(&tmSA, pr.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.M,
                   static_cast<uint64_t>(pr.slabs) * KB,
                   static_cast<uint64_t>(sfa_stride(pr.M)) * 4, C::BT, 4,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "SFA"));
+  // K-grouped: per-row weight scales, MN-major [K/128][stride(N)], boxes of
+  // BW rows x 4 K blocks
+  std::memset(&tmSB, 0, sizeof(tmSB));
+  if (C::EPI == 2)
+    FG_TRY(make_map(&tmSB, pr.sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.N, KB,
+                    static_cast<uint64_t>(sfa_stride(pr.N)) * 4, C::BW, 4,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, "SFB"));
   // D as rows x N bf16 in boxes of 32 rows x 32 columns, 64-byte swizzled
-  // (the fused FFN epilogue writes no D)
+  // (K-grouped: fp32 in 32 x 32 boxes, 128-byte swizzled; the fused FFN
+  // epilogue writes no D)
   std::memset(&tmD, 0, sizeof(tmD));
+  if (C::EPI == 2)
+    FG_TRY(make_map(&tmD, ffn_d32(pr), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.N,
+                    static_cast<uint64_t>(pr.G) * pr.M, static_cast<uint64_t>(pr.N) * 4, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B, "D"));
   if (C::EPI == 0)
     FG_TRY(make_map(&tmD, pr.D, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.N,
                     static_cast<uint64_t>(pr.slabs) * pr.M, static_cast<uint64_t>(pr.N) * 2, 32, 32,
@@ -509,7 +528,7 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
   p.N = pr.N;
   p.K = pr.K;
   p.G = pr.G;
-  p.KB = KB;
+  p.KB = kb_override >= 0 ? kb_override : KB;  // (K-grouped with T = 0: no K blocks)
   p.NB = (pr.N + 127) / 128;
   p.num_mt = (pr.M + C::BT - 1) / C::BT;
   p.num_nt = (pr.N + C::BW - 1) / C::BW;
@@ -527,8 +546,12 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
     p.sfh_stride = sfa_stride(pr.M);
     p.num_nt = ffn->I / 128;  // one tile = 128 gate + 128 up rows
   }
+  if (C::EPI == 2) {
+    p.ks = pr.m_indices;  // token counts per expert (device)
+    p.d32 = ffn_d32(pr);
+  }
   int64_t tiles = static_cast<int64_t>(C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
-  if (FORM == kFormMasked) tiles *= pr.G;  // upper bound: masked_m lives on the device
+  if (FORM == kFormMasked || FORM == kFormKGrouped) tiles *= pr.G;  // (masked: an upper bound)
   const int64_t grid = C::PAIR ? C::CLUSTER * std::max<int64_t>(1, std::min<int64_t>(tiles, max_clusters))
                                : std::max<int64_t>(1, std::min<int64_t>(tiles, dev.sm_count));
   cudaLaunchConfig_t cfg = {};
@@ -549,7 +572,7 @@ fg_status launch_mx(const Problem& pr, const DeviceInfo& dev, int dev_id, cudaSt
     cfg.numAttrs = 2;
   }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_gemm_mx_kernel<C, FORM>, tmA, tmB, tmSA,
-                                           tmD, p);
+                                           tmSB, tmD, p);
   if (e != cudaSuccess) return cuda_fail(e, "fp8_gemm_mx_kernel launch");
   return FG_OK;
 }
@@ -908,6 +931,34 @@ fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uin
                  H, I, G, expected_m, stream);
 }
 
+fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
+                                     const float* sfb, float* D, const int32_t* ks, int G, int M,
+                                     int N, int T, cudaStream_t stream) {
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (G + 1 > kTableMax) return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d groups", G, kTableMax - 1);
+  if (M < 1) return fail(FG_ERR_INVALID_ARG, "M=%d must be >= 1", M);
+  if (N <= 0 || N % 16 != 0) return fail(FG_ERR_INVALID_ARG, "N=%d must be a positive multiple of 16", N);
+  if (T < 0 || T % 128 != 0) return fail(FG_ERR_INVALID_ARG, "T=%d must be a non-negative multiple of 128", T);
+  FG_TRY(check_ptr(A, "A"));
+  FG_TRY(check_ptr(sfa, "sfa"));
+  FG_TRY(check_ptr(B, "B"));
+  FG_TRY(check_ptr(sfb, "sfb"));
+  FG_TRY(check_ptr(D, "D"));
+  FG_TRY(check_ptr(ks, "ks"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  // (T = 0: every group is empty; the kernel writes zeros. The tensor maps
+  // need a nonzero extent, so the K extent is at least one block.)
+  Problem pr{kFormKGrouped, A, sfa, B, sfb, reinterpret_cast<uint16_t*>(D), ks, nullptr, M, N,
+             std::max(T, 128), G, 1};
+  if (T == 0) pr.K = 128;
+  // pairs unless there is a single token tile
+  if (M > 128) return launch_mx<MxKgP, kFormKGrouped>(pr, *dev, dev_id, stream, nullptr, T / 128);
+  return launch_mx<MxKgS, kFormKGrouped>(pr, *dev, dev_id, stream, nullptr, T / 128);
+}
+
 fg_status fg_set_ue8m0_tile(int width, int pair) {
   const bool ok = width == 0 || (pair ? width == 224 : (width == 128 || width == 224 || width == 256));
   if (!ok)
@@ -931,6 +982,7 @@ fg_status fg_get_device_status(cudaStream_t stream, int* code) {
   const char* what = v == FG_DEVICE_WAIT_TIMEOUT   ? "a pipeline wait timed out"
                      : v == FG_DEVICE_BAD_MASKED_M ? "masked_m outside [0, M_max]"
                      : v == FG_DEVICE_BAD_M_INDEX  ? "m_indices entry >= G"
+                     : v == FG_DEVICE_BAD_K_GROUP  ? "ks entry negative, not a multiple of 128, or past T"
                                                    : "unknown device status";
   return fail(FG_ERR_DEVICE, "device status %d: %s", v, what);
 }

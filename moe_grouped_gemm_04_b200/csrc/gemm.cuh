@@ -62,7 +62,7 @@
 
 namespace fg {
 
-enum : int { kFormDense = 0, kFormContig = 1, kFormMasked = 2 };
+enum : int { kFormDense = 0, kFormContig = 1, kFormMasked = 2, kFormKGrouped = 3 };
 
 constexpr int kTableMax = 2048;  // contiguous: token tiles; masked: experts + 1
 constexpr uint64_t kDrainLimitNs = 20000000ull;  // 20 ms for in-flight copies at teardown
@@ -88,6 +88,10 @@ struct GemmParams {
   uint16_t* gu;
   int I;
   int sfh_stride;
+  // K-grouped GEMM of the block-scaled kernel: token counts per expert
+  // (device) and the fp32 output [G][M][N]
+  const int32_t* ks;
+  float* d32;
 };
 
 template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_, int KPS_ = 2,
@@ -203,6 +207,8 @@ struct Tile {
   int e;      // expert (0 for dense)
   int mt;     // token tile within the slab
   int nt;     // weight tile
+  int kb0;    // first K block (block-scaled kernel; K-grouped: the expert's first token block)
+  int nkb;    // K blocks of the tile
 };
 
 template <class C, int FORM>

@@ -77,6 +77,14 @@
 // power-of-two scale, and writes the e4m3 codes of h and the scale in the
 // per-token layout the second GEMM reads (optionally also the bf16 gate and
 // up values). The arithmetic is that of per_token_cast_to_fp8_ue8m0.
+//
+// K-grouped GEMM (EPI = 2, form kFormKGrouped: the weight gradients of the
+// experts in FP8 training): the contraction runs over tokens whose expert
+// ranges are stacked along K, so a tile (expert e, mt, nt) runs over the K
+// blocks of expert e only; both operands carry one scale per row per
+// 128-token block (the per-row B scales arrive with a second TMA box beside
+// the token scales); the fp32 result goes out through 128-byte-swizzled
+// 32 x 32 boxes. An expert without tokens gets zeros (no MMA runs for it).
 #pragma once
 
 #include <cstdint>
@@ -91,7 +99,7 @@ namespace fg {
 
 template <int BW_, int STAGES_, int ACC_, int EPQ_, bool PAIR_, int KPS_, int EPI_ = 0>
 struct MxCfg {
-  static constexpr int EPI = EPI_;        // 0: bf16 D; 1: SwiGLU + UE8M0 requantization
+  static constexpr int EPI = EPI_;        // 0: bf16 D; 1: SwiGLU + UE8M0 requantization; 2: K-grouped, fp32 D
   static constexpr int BT = 128;          // token rows per CTA tile
   static constexpr int BW = BW_;          // weight rows per tile (MMA N)
   static constexpr bool SWAP = false;     // tile helpers of gemm.cuh: tokens on the lanes
@@ -106,7 +114,7 @@ struct MxCfg {
   static constexpr int EPQ = EPQ_;        // epilogue warps per TMEM lane quadrant
   static_assert(BW % 32 == 0 && BW >= 32 && BW <= 256, "tcgen05 N, 32-column chunks");
   static_assert(!PAIR || B_ROWS % 16 == 0, "pair: half tiles of whole 8-row swizzle atoms");
-  static_assert(EPI == 0 || (BW == 256 && ACC == 1 && EPQ == 1),
+  static_assert(EPI != 1 || (BW == 256 && ACC == 1 && EPQ == 1),
                 "fused FFN epilogue: 128 gate + 128 up columns, one accumulator, one warp per quadrant");
   // weight rows per tensor load: the fused FFN tile is two 128-row blocks
   static constexpr int B_BOX = EPI == 1 ? 128 : B_ROWS;
@@ -125,9 +133,11 @@ struct MxCfg {
   // 4 x NBT weight-block scales ([k][j]: K block 4q + k, block nb0 + j)
   static constexpr int NBT = EPI == 1 ? 2 : SFB_GROUPS + 1;
   static constexpr int RAW_A = 4 * 512;
-  static constexpr int RAW_BYTES = RAW_A + 128;
+  // K-grouped: per-row weight scales, BW rows x 4 K blocks (one TMA box)
+  static constexpr int RAW_B = EPI == 2 ? 4 * BW * 4 : 128;
+  static constexpr int RAW_BYTES = RAW_A + (RAW_B + 127) / 128 * 128;
   static constexpr int RAWS = 2;          // staged-scale ring
-  static_assert(4 * NBT * 4 <= RAW_BYTES - RAW_A, "staged weight-block scales");
+  static_assert(EPI == 2 || 4 * NBT * 4 <= RAW_BYTES - RAW_A, "staged weight-block scales");
   static constexpr int TMEM_USED = ACC * BW + SFS * SF_COLS;
   static_assert(TMEM_USED <= 512, "TMEM has 512 columns");
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
@@ -136,14 +146,16 @@ struct MxCfg {
   static constexpr int B_BYTES = B_ROWS * 128;   // one K block of this CTA's weight rows
   static constexpr int STAGE_A = KPS * A_BYTES;
   static constexpr int STAGE_B = KPS * B_BYTES;
-  static constexpr int EPI_RING = 2;         // image buffers per epilogue warp
-  static constexpr int BOX_BYTES = 32 * 64;  // 32 rows x 32 bf16 columns
+  // epilogue image buffers per warp, each one box of 32 rows x 32 columns
+  // (bf16: 64-byte rows; fp32: 128-byte rows)
+  static constexpr int EPI_RING = EPI == 2 ? 1 : 2;
+  static constexpr int BOX_BYTES = EPI == 2 ? 32 * 128 : 32 * 64;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * STAGE_A;
   static constexpr int OFF_SF = OFF_B + STAGES * STAGE_B;
   static constexpr int OFF_RAW = OFF_SF + SFS * SF_BYTES;  // 128-byte aligned
   static constexpr int OFF_EPI = (OFF_RAW + RAWS * RAW_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_BAR = OFF_EPI + (EPI == 0 ? EW * EPI_RING * BOX_BYTES : 0);
+  static constexpr int OFF_BAR = OFF_EPI + (EPI == 1 ? 0 : EW * EPI_RING * BOX_BYTES);  // (the fused FFN stages no D)
   static constexpr int NUM_BARS = 2 * STAGES + 2 * SFS + 2 * RAWS + 2 * ACC;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
@@ -152,11 +164,12 @@ struct MxCfg {
     return form == kFormDense ? 0 : (form == kFormContig && PAIR ? 2 : 1) * kTableMax * 4;
   }
   static constexpr int smem_bytes(int form) { return OFF_TABLE + table_bytes(form) + 1024; }
+  static_assert(EPI != 2 || smem_bytes(kFormKGrouped) <= 232448, "shared memory per CTA");
 
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(OFF_SF % 128 == 0 && OFF_RAW % 128 == 0 && RAW_BYTES % 128 == 0,
                 "scale groups and staged scales: 128-byte aligned");
-  static_assert(smem_bytes(kFormContig) <= 232448, "shared memory per CTA");
+  static_assert(EPI == 2 || smem_bytes(kFormContig) <= 232448, "shared memory per CTA");
 };
 
 // 16-byte chunk c (columns 8c .. 8c + 7) of row r of a 32-row x 64-byte box
@@ -212,6 +225,34 @@ __device__ void mx_build_table(const GemmParams& p, int* table, int* num_units, 
       }
       if (lane == 0) *num_units = count;
     }
+  } else if constexpr (FORM == kFormKGrouped) {
+    // table[e] = first token block of expert e (exclusive prefix of ks / 128)
+    const int per = (p.G + 31) / 32;
+    const int e0 = lane * per;
+    const int e1 = min(p.G, e0 + per);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) {
+      int k = __ldg(p.ks + e);
+      if (k < 0 || (k & 127) != 0) {
+        raise_status(p.status, 4 /* FG_DEVICE_BAD_K_GROUP */);
+        k = k < 0 ? 0 : k & ~127;
+      }
+      table[e + 1] = k >> 7;
+      local += k >> 7;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      run += table[e + 1];
+      table[e + 1] = min(run, p.KB);  // token blocks past T are dropped (status raised below)
+    }
+    if (lane == 31 && incl > p.KB) raise_status(p.status, 4 /* FG_DEVICE_BAD_K_GROUP */);
+    if (lane == 0) table[0] = 0;
   } else if constexpr (FORM == kFormMasked) {
     const int per = (p.G + 31) / 32;
     const int e0 = lane * per;
@@ -247,6 +288,7 @@ __device__ void mx_build_table(const GemmParams& p, int* table, int* num_units, 
 template <class C, int FORM>
 __device__ __forceinline__ int mx_total(const GemmParams& p, const int* table, int num_units) {
   if (FORM == kFormMasked) return table[p.G];
+  if (FORM == kFormKGrouped) return p.G * (C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
   if (FORM == kFormContig && C::PAIR) return num_units * p.num_nt;
   return (C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
 }
@@ -256,7 +298,17 @@ template <class C, int FORM>
 __device__ __forceinline__ Tile mx_resolve(const GemmParams& p, const int* table, int t, int rank) {
   Tile w;
   w.valid = 1;
-  if (FORM == kFormMasked) {
+  w.kb0 = 0;
+  w.nkb = p.KB;
+  if (FORM == kFormKGrouped) {
+    const int per = (C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
+    w.e = t / per;
+    const int local = t - w.e * per;
+    w.mt = C::PAIR ? 2 * (local / p.num_nt) + rank : local / p.num_nt;
+    w.nt = local % p.num_nt;
+    w.kb0 = table[w.e];
+    w.nkb = table[w.e + 1] - table[w.e];
+  } else if (FORM == kFormMasked) {
     int lo = 0, hi = p.G;  // table[lo] <= t < table[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -300,8 +352,8 @@ struct Ring {
 template <class C, int FORM>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmD,
-                       const GemmParams p) {
+                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                       const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem + C::OFF_A;
@@ -337,7 +389,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       mbar_init(&sf_empty[q], 1);          // the MMA commit after the quad
     }
     for (int r = 0; r < C::RAWS; ++r) {
-      mbar_init(&sa_full[r], 2);   // scale lane: expect_tx (TMA) + cp.async arrival
+      // scale lane: expect_tx (TMA), plus the cp.async arrival (weight-block scales)
+      mbar_init(&sa_full[r], C::EPI == 2 ? 1 : 2);
       mbar_init(&sa_empty[r], 1);  // the converter
     }
     for (int b = 0; b < C::ACC; ++b) {
@@ -349,7 +402,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSA);
-    tma_prefetch_desc(&tmD);
+    if (C::EPI == 2) tma_prefetch_desc(&tmSB);
+    if (C::EPI != 1) tma_prefetch_desc(&tmD);
   }
   if constexpr (!C::PAIR) {
     if (warp == 1) {
@@ -382,7 +436,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   const uint32_t tmem_sf = tmem_base + static_cast<uint32_t>(C::ACC * C::BW);
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   const int total = mx_total<C, FORM>(p, table, *num_units);
-  const int KQ = (p.KB + 3) >> 2;  // quads per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -394,16 +447,19 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (!w.valid) continue;
         // fused FFN: gate block nt*128.. and up block I + nt*128.. of the
         // expert's 2I rows (a pair's CTAs load one block each)
-        const int row = lane == 0 ? (C::EPI == 1 ? w.e * p.N + (C::PAIR ? rank : 0) * p.I + w.nt * 128
-                                                 : w.e * p.N + w.nt * C::BW + rank * C::B_ROWS)
+        // (K-grouped: B is one matrix whose K range the experts share)
+        const int b_base = FORM == kFormKGrouped ? 0 : w.e * p.N;
+        const int row = lane == 0 ? (C::EPI == 1 ? b_base + (C::PAIR ? rank : 0) * p.I + w.nt * 128
+                                                 : b_base + w.nt * C::BW + rank * C::B_ROWS)
                                   : (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
         const CUtensorMap* map = lane == 0 ? &tmB : &tmA;
         const uint32_t bytes = lane == 0 ? C::B_BYTES : C::A_BYTES;
         const int loads = lane == 0 ? C::B_LOADS : 1;  // tensor loads per K block
         const int load_step = C::EPI == 1 ? p.I : 0;   // rows between them
-        for (int kb0 = 0; kb0 < p.KB; kb0 += C::KPS, st.next(), ++fills) {
+        for (int kb0 = 0; kb0 < w.nkb; kb0 += C::KPS, st.next(), ++fills) {
           if (!mbar_wait(&empty[st.slot], st.phase ^ 1u, ctl)) goto producer_done;
-          const int nk = min(C::KPS, p.KB - kb0);
+          const int nk = min(C::KPS, w.nkb - kb0);
+          const int kx = (w.kb0 + kb0) * 128;  // K coordinate of the stage's first block
           uint8_t* dst = lane == 0 ? sB + st.slot * C::STAGE_B : sA + st.slot * C::STAGE_A;
           if constexpr (C::PAIR) {
             // both CTAs' operand bytes complete on the leader's barrier
@@ -411,13 +467,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             const uint32_t bar = mapa_shared(smem_u32(&full[st.slot]), 0);
             for (int j = 0; j < nk; ++j)
               for (int h = 0; h < loads; ++h)
-                tma_load_2d_pair(dst + j * bytes + h * C::B_BOX * 128, map, bar, (kb0 + j) * 128,
+                tma_load_2d_pair(dst + j * bytes + h * C::B_BOX * 128, map, bar, kx + j * 128,
                                  row + h * load_step);
           } else {
             mbar_arrive_expect_tx(&full[st.slot], nk * bytes);
             for (int j = 0; j < nk; ++j)
               for (int h = 0; h < loads; ++h)
-                tma_load_2d(dst + j * bytes + h * C::B_BOX * 128, map, &full[st.slot], (kb0 + j) * 128,
+                tma_load_2d(dst + j * bytes + h * C::B_BOX * 128, map, &full[st.slot], kx + j * 128,
                             row + h * load_step);
           }
         }
@@ -442,17 +498,25 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         // weight blocks the tile's rows touch (clamped: rows past N are never stored)
         const int nb0 = (w.nt * C::BW) >> 7;
         const float* sfb_e = p.sfb + static_cast<int64_t>(w.e) * p.NB * p.KB;
+        const int KQ = (w.nkb + 3) >> 2;  // quads of the tile
         for (int qi = 0; qi < KQ; ++qi, rr.next(), ++fills) {
           if (!mbar_wait(&sa_empty[rr.slot], rr.phase ^ 1u, ctl)) goto scales_done;
           uint8_t* raw = sRAW + rr.slot * C::RAW_BYTES;
-          mbar_arrive_expect_tx(&sa_full[rr.slot], C::RAW_A);
           // 4 K blocks of token scales; rows past M read as zero, K blocks past
           // the tile's last one are never used
-          tma_load_2d(raw, &tmSA, &sa_full[rr.slot], w.mt * C::BT,
-                      (FORM == kFormMasked ? w.e * p.KB : 0) + 4 * qi);
+          const int ky = (FORM == kFormMasked ? w.e * p.KB : 0) + w.kb0 + 4 * qi;
+          if constexpr (C::EPI == 2) {
+            // per-row weight scales: BW rows x 4 K blocks beside them
+            mbar_arrive_expect_tx(&sa_full[rr.slot], C::RAW_A + C::RAW_B);
+            tma_load_2d(raw, &tmSA, &sa_full[rr.slot], w.mt * C::BT, ky);
+            tma_load_2d(raw + C::RAW_A, &tmSB, &sa_full[rr.slot], w.nt * C::BW, ky);
+            continue;
+          }
+          mbar_arrive_expect_tx(&sa_full[rr.slot], C::RAW_A);
+          tma_load_2d(raw, &tmSA, &sa_full[rr.slot], w.mt * C::BT, ky);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int kb = min(4 * qi + k, p.KB - 1);
+            const int kb = w.kb0 + min(4 * qi + k, w.nkb - 1);
 #pragma unroll
             for (int j = 0; j < C::NBT; ++j) {
               // fused FFN: the gate block nt and the up block I/128 + nt
@@ -483,12 +547,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ready = false;  // the current stage's "full" phase was seen complete by a peek
       for (int t = t_first; t < total; t += t_step) {
         const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
-        if (!w.valid) continue;
+        if (!w.valid || w.nkb == 0) continue;  // (an expert without tokens: no MMA)
         const int b = tc % C::ACC;
         if (!warp_wait(&tempty[b], ((tc / C::ACC) & 1u) ^ 1u, ctl, lane)) goto mma_done;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::BW);
-        for (int kb0 = 0; kb0 < p.KB; kb0 += C::KPS, st.next()) {
+        for (int kb0 = 0; kb0 < w.nkb; kb0 += C::KPS, st.next()) {
           if (!ready && !warp_wait(&full[st.slot], st.phase, ctl, lane)) goto mma_done;
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + st.slot * C::STAGE_A);
@@ -496,7 +560,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < C::KPS; ++j) {
             const int kb = kb0 + j;
-            if (kb >= p.KB) break;
+            if (kb >= w.nkb) break;
             const uint32_t k4 = static_cast<uint32_t>(kb & 3);
             const uint32_t sf = tmem_sf + sq.slot * C::SF_COLS;
             if (k4 == 0) {
@@ -518,7 +582,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             const uint32_t id = idesc | (k4 << 4) | (k4 << 29);
             const uint64_t adesc = smem_desc_sw128(a_base + j * C::A_BYTES);
             const uint64_t bdesc = smem_desc_sw128(b_base + j * C::B_BYTES);
-            const bool last_of_quad = k4 == 3 || kb == p.KB - 1;
+            const bool last_of_quad = k4 == 3 || kb == w.nkb - 1;
             if (elect_one()) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {  // 32 bytes (= 32 e4m3 along K) per MMA
@@ -571,13 +635,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1)
           jb[g][r1] = C::EPI == 1 ? g : ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
+      const int KQ = (w.nkb + 3) >> 2;  // quads of the tile
       for (int qi = 0; qi < KQ; ++qi, rr.next(), sq.next()) {
         // the quad's scales have landed, and the slot's previous quad has
         // been copied out and its MMAs have completed
         if (!warp_wait(&sa_full[rr.slot], rr.phase, ctl, lane)) goto convert_done;
         if (!warp_wait(&sf_empty[sq.slot], sq.phase ^ 1u, ctl, lane)) goto convert_done;
         const float* raw = reinterpret_cast<const float*>(sRAW + rr.slot * C::RAW_BYTES);
-        const int nk = min(4, p.KB - 4 * qi);  // K blocks of this quad
+        const int nk = min(4, w.nkb - 4 * qi);  // K blocks of this quad
         uint32_t wa[4] = {0, 0, 0, 0};
         uint32_t wb[C::SFB_GROUPS][4];
 #pragma unroll
@@ -592,8 +657,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
             for (int g = 0; g < C::SFB_GROUPS; ++g)
 #pragma unroll
-              for (int r1 = 0; r1 < 4; ++r1)
-                wb[g][r1] |= ue8m0_byte(raw[C::RAW_A / 4 + k * C::NBT + jb[g][r1]]) << (8 * k);
+              for (int r1 = 0; r1 < 4; ++r1) {
+                if constexpr (C::EPI == 2) {
+                  // per-row weight scale of tile row 128 g + 32 r1 + lane
+                  const int n = 128 * g + 32 * r1 + lane;
+                  wb[g][r1] |= (n < C::BW ? ue8m0_byte(raw[C::RAW_A / 4 + k * C::BW + n]) : 127u) << (8 * k);
+                } else {
+                  wb[g][r1] |= ue8m0_byte(raw[C::RAW_A / 4 + k * C::NBT + jb[g][r1]]) << (8 * k);
+                }
+              }
           }
         }
         uint8_t* grp = sSF + sq.slot * C::SF_BYTES + lane * 16;
@@ -730,46 +802,70 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       const bool ok = m < m_valid && (FORM != kFormContig || row_mi >= 0);
       // a warp whose 32 rows are all stored writes through tensor stores
       const bool staged = __all_sync(0xffffffffu, ok);
-      const int y = (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT + quad * 32;
+      const int y = (FORM == kFormMasked || FORM == kFormKGrouped ? w.e * p.M : 0) + w.mt * C::BT + quad * 32;
+      const bool zero = w.nkb == 0;  // K-grouped expert without tokens: zeros, no accumulator
       const int b = tc % C::ACC;
-      if (!warp_wait(&tfull[b], (tc / C::ACC) & 1u, ctl, lane)) goto epi_done;
-      tc_fence_after();
+      if (!zero) {
+        if (!warp_wait(&tfull[b], (tc / C::ACC) & 1u, ctl, lane)) goto epi_done;
+        tc_fence_after();
+      }
 #pragma unroll 1
       for (int ch = 0; ch < C::ECOLS / 32; ++ch) {
         uint32_t r[32];
-        tmem_ld32_issue(tmem_base + t_lane + static_cast<uint32_t>(b * C::BW + c0 + ch * 32), r);
-        tmem_wait_ld32(r);
-        if (ch == C::ECOLS / 32 - 1) {
-          // the accumulator is in registers: the next tile's MMAs may start
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (C::PAIR && rank != 0)  // the leader's MMA waits for both CTAs
-              mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
-            else
-              mbar_arrive(&tempty[b]);
+        if (zero) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+        } else {
+          tmem_ld32_issue(tmem_base + t_lane + static_cast<uint32_t>(b * C::BW + c0 + ch * 32), r);
+          tmem_wait_ld32(r);
+          if (ch == C::ECOLS / 32 - 1) {
+            // the accumulator is in registers: the next tile's MMAs may start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (C::PAIR && rank != 0)  // the leader's MMA waits for both CTAs
+                mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+              else
+                mbar_arrive(&tempty[b]);
+            }
           }
         }
+        const int x = w.nt * C::BW + c0 + ch * 32;
         if (staged) {
           uint8_t* img = ring + (boxes % C::EPI_RING) * C::BOX_BYTES;
           // the tensor store that last used this buffer has read it
           if (boxes >= C::EPI_RING && lane == 0) bulk_wait_group_read<C::EPI_RING - 1>();
           __syncwarp();
+          if constexpr (C::EPI == 2) {
+            // fp32: row `lane` of the box is 128 bytes; 16-byte chunk c at
+            // position c ^ (lane % 8) (the tensor map's 128-byte swizzle)
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(img + sw64_offset(lane, c)) = make_uint4(
-                pack_bf16x2(__uint_as_float(r[8 * c + 0]), __uint_as_float(r[8 * c + 1])),
-                pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
-                pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
-                pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(img + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(img + sw64_offset(lane, c)) = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[8 * c + 0]), __uint_as_float(r[8 * c + 1])),
+                  pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                  pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                  pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+          }
           fence_proxy_async_shared();
           __syncwarp();
           if (lane == 0) {
-            const int x = w.nt * C::BW + c0 + ch * 32;
             if (x < p.N) tma_store_2d(&tmD, img, x, y);  // columns past N are clipped
             bulk_commit_group();  // (possibly empty: keeps one group per buffer use)
           }
           ++boxes;
+        } else if constexpr (C::EPI == 2) {
+          if (ok) {
+            float* dst = p.d32 + (static_cast<int64_t>(w.e) * p.M + m) * p.N;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              if (x + j < p.N) *reinterpret_cast<uint4*>(dst + x + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+          }
         } else {
           float v[32];
 #pragma unroll
@@ -777,7 +873,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           store_tile_part<C, FORM, 32>(p, w, row, c0 + ch * 32, v, m_valid, row_mi);
         }
       }
-      ++tc;
+      if (!zero) ++tc;
     }
   epi_done:
     // this warp's tensor stores have finished reading shared memory

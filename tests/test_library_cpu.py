@@ -132,3 +132,19 @@ def test_ffn_validation_without_the_device(lib):
     nogu = list(args)
     nogu[8] = None
     assert lib.fp8_moe_ffn_contiguous_ue8m0(*nogu, 0, 256, 128, 2, None) == 0
+
+
+def test_k_grouped_validation_without_the_device(lib):
+    P = ctypes.c_void_p
+    ok = P(FAKE)
+    args = [ok] * 6
+    assert lib.fp8_k_grouped_gemm_nt_ue8m0(*args, 0, 128, 256, 256, None) == 1   # G
+    assert lib.fp8_k_grouped_gemm_nt_ue8m0(*args, 2, 0, 256, 256, None) == 1     # M
+    assert lib.fp8_k_grouped_gemm_nt_ue8m0(*args, 2, 128, 250, 256, None) == 1   # N % 16
+    assert lib.fp8_k_grouped_gemm_nt_ue8m0(*args, 2, 128, 256, 200, None) == 1   # T % 128
+    bad = list(args)
+    bad[5] = None  # ks
+    assert lib.fp8_k_grouped_gemm_nt_ue8m0(*bad, 2, 128, 256, 256, None) == 1
+    bad = list(args)
+    bad[4] = P(MISALIGNED)  # D
+    assert lib.fp8_k_grouped_gemm_nt_ue8m0(*bad, 2, 128, 256, 256, None) == 1
