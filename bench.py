@@ -187,6 +187,8 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict, ue8m0
 
     if kind == "ffn":
         return ffn_cpu_sample(inp, target_s, threads, cache)
+    if kind == "kgrouped":
+        return kgrouped_cpu_sample(inp, target_s, threads, cache)
     K, N = inp.K, inp.N
     if kind == "dense":
         a_rows, experts = inp.a, np.zeros(inp.M, np.int64)
@@ -284,6 +286,33 @@ def ffn_cpu_sample(inp, target_s: float, threads: int, cache: dict):
     return flops / dt, desc, dt
 
 
+def kgrouped_cpu_sample(inp, target_s: float, threads: int, cache: dict):
+    """The oracle's K-grouped GEMM for a bounded sample of A rows (quantized per
+    row per 128 tokens) against all of B (quantized outside the timed part)."""
+    import oracle
+
+    if "qb" not in cache:
+        cache["qb"] = oracle.per_token_cast(inp.b, threads=threads, ue8m0=True)
+    qb, sb = cache["qb"]
+    tv = int(inp.counts.sum())
+    order = np.random.default_rng(0).permutation(inp.M)
+    rows = cache.get("rows", 1)
+    while True:
+        take = np.sort(order[:min(rows, inp.M)])
+        t0 = time.perf_counter()
+        qa, sa = oracle.per_token_cast(inp.a[take], threads=threads, ue8m0=True)
+        oracle.k_grouped(qa, sa, qb, sb, inp.ks, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or len(take) >= inp.M:
+            break
+        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9))
+    cache["rows"] = rows
+    flops = 2.0 * len(take) * inp.N * tv
+    desc = ("%d of %d A rows x all %d B rows over all %d experts' tokens (T=%d, quantization "
+            "of the sampled rows + K-grouped GEMM)" % (len(take), inp.M, inp.N, inp.G, inp.T))
+    return flops / dt, desc, dt
+
+
 # ---------------------------------------------------------------------- ranks
 
 def max_over_ranks(dist, values, device):
@@ -301,6 +330,8 @@ def gemm_kernel_name(kind: str, inp, ue8m0: bool) -> str:
     """The GEMM kernel a step launches (the library's choice for the shape)."""
     if kind == "ffn":
         return "fp8_gemm_mx_kernel x2 (first GEMM with fused SwiGLU + requantization, second GEMM)"
+    if kind == "kgrouped":
+        return "fp8_gemm_mx_kernel (K-grouped, fp32 output)"
     thin = (kind == "dense" and inp.M <= 64) or (
         kind == "masked" and max(1, int(round(float(np.mean(inp.masked_m))))) <= 64)
     return "fp8_gemm_mx_kernel" if ue8m0 and not thin else "fp8_gemm_kernel"
@@ -314,9 +345,21 @@ class OperandSet:
         K, N = inp.K, inp.N
         self.x = x.clone()
         self.w = w.clone() if with_weight_quant else None
+        self.extra = []
+        if kind == "kgrouped":
+            # both operands are per-step activations: x (dY^T) and x2 (X^T)
+            x2 = extra
+            self.x2 = x2.clone()
+            M, N, T = inp.M, inp.N, inp.T
+            self.A = torch.empty((M, T), dtype=torch.uint8, device=dev)
+            self.SA = fg.empty_sfa(1, M, T, dev)
+            self.B = torch.empty((N, T), dtype=torch.uint8, device=dev)
+            self.SB = fg.empty_sfa(1, N, T, dev)
+            self.D = torch.empty((inp.G, M, N), dtype=torch.float32, device=dev)
+            self.extra = [self.x2]
+            return
         self.B = B.clone()
         self.SB = SB.clone()
-        self.extra = []
         if kind == "ffn":
             W2, SW2 = extra
             self.W2, self.SW2 = W2.clone(), SW2.clone()
@@ -372,7 +415,12 @@ class Step:
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
         extra = None
-        if kind == "ffn":
+        if kind == "kgrouped":
+            x, w = bf16(inp.a), None
+            extra = bf16(inp.b)
+            B = SB = None
+            self.ks = torch.from_numpy(inp.ks).to(dev)
+        elif kind == "ffn":
             # W1 [G][2I][H] in B/SB, W2 [G][H][I] alongside
             x, w = bf16(inp.a), bf16(inp.w1)
             B = torch.empty((inp.G, 2 * inp.I, inp.H), dtype=torch.uint8, device=dev)
@@ -408,9 +456,13 @@ class Step:
 
     def quant_acts(self, o):
         self.q_token(o.x, o.A, o.SA)
+        if self.kind == "kgrouped":
+            self.q_token(o.x2, o.B, o.SB)
 
     def gemm(self, o):
-        if self.kind == "ffn":
+        if self.kind == "kgrouped":
+            self.fg.fp8_k_grouped_gemm_nt_ue8m0(o.A, o.SA[0], o.B, o.SB[0], o.D, self.ks)
+        elif self.kind == "ffn":
             self.fg.fp8_moe_ffn_contiguous_ue8m0(o.A, o.SA, o.B, o.SB, o.W2, o.SW2, o.Hq, o.SH, o.D,
                                                  self.mi)
         elif self.kind == "dense":
@@ -421,7 +473,7 @@ class Step:
             self.g_masked(o.A, o.SA, o.B, o.SB, o.D, self.mm, self.expected_m)
 
     def launches_per_step(self):
-        return (3 if self.kind == "ffn" else 2) + (1 if self.with_wq else 0)
+        return (3 if self.kind in ("ffn", "kgrouped") else 2) + (1 if self.with_wq else 0)
 
     def run(self, i):
         o = self.sets[i % len(self.sets)]
@@ -442,9 +494,10 @@ def run_ours(args, rank, world, local_rank):
     inp = workloads.make(args.workload, seed=0)
     flops, alg_bytes = workloads.flops_and_bytes(kind, inp)
     rotate = args.l2 == "rotate"
-    ue8m0 = args.scales == "ue8m0" or kind == "ffn"  # the expert FFN uses power-of-two scales
-    if kind == "ffn" and args.with_weight_quant:
-        raise SystemExit("--with-weight-quant is not supported for the expert FFN workload")
+    # the expert FFN and the K-grouped GEMM use power-of-two scales
+    ue8m0 = args.scales == "ue8m0" or kind in ("ffn", "kgrouped")
+    if kind in ("ffn", "kgrouped") and args.with_weight_quant:
+        raise SystemExit("--with-weight-quant is not supported for the %s workload" % kind)
     step = Step(fg, torch, kind, inp, args.with_weight_quant,
                 ROTATE_MIN_BYTES if rotate else 0, ue8m0)
     R = len(step.sets)
@@ -553,6 +606,8 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         xh = step.sets[0].x.cpu().pin_memory()
+        # (K-grouped: both operands are the step's inputs)
+        x2h = step.sets[0].x2.cpu().pin_memory() if kind == "kgrouped" else None
         dh = [torch.empty(step.sets[0].D.shape, dtype=step.sets[0].D.dtype).pin_memory()
               for _ in range(2)]
         up, down = torch.cuda.Stream(), torch.cuda.Stream()
@@ -570,6 +625,8 @@ def run_ours(args, rank, world, local_rank):
                     if i >= R:
                         up.wait_event(done[i - R])
                     o.x.copy_(xh, non_blocking=True)
+                    if x2h is not None:
+                        o.x2.copy_(x2h, non_blocking=True)
                     uploaded = torch.cuda.Event()
                     uploaded.record(up)
                 comp.wait_event(uploaded)
@@ -590,7 +647,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e2e_ms = e2e_loop(K)
         barrier()
-        e2e = {"ms": e2e_ms, "h2d": xh.numel() * xh.element_size(),
+        e2e = {"ms": e2e_ms, "h2d": xh.numel() * xh.element_size() +
+                                    (x2h.numel() * x2h.element_size() if x2h is not None else 0),
                "d2h": dh[0].numel() * dh[0].element_size()}
 
     # max over ranks
@@ -643,6 +701,8 @@ def run_ours(args, rank, world, local_rank):
            "parallelism": "replicas" if world > 1 else "single GPU"}
     if kind == "ffn":
         cfg.update(H=inp.H, I=inp.I, G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
+    elif kind == "kgrouped":
+        cfg.update(M=inp.M, T=inp.T, G=inp.G, T_valid=int(inp.counts.sum()))
     elif kind == "dense":
         cfg["M"] = inp.M
     elif kind == "contiguous":
@@ -779,7 +839,7 @@ def run_reference(args, rank, world):
     threads = oracle.hardware_threads()
     per_step = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     cache = {}
-    ue8m0 = args.scales == "ue8m0" or kind == "ffn"
+    ue8m0 = args.scales == "ue8m0" or kind in ("ffn", "kgrouped")
     for _ in range(args.warmup):
         cpu_sample(inp, kind, per_step, threads, cache, ue8m0)
     vals, descs, secs = [], [], []

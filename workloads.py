@@ -25,6 +25,11 @@ inference shapes"):
                            workload's 8 experts and token counts; W1 [8][4096][7168]
                            (gate rows, then up rows) and W2 [8][7168][2048]
                            ~ N(0, 0.02)
+  kgrouped_8x4096x7168     K-grouped weight-gradient GEMM of the contiguous
+                           workload's experts: A = dY^T [4096][T] ~ N(0,1),
+                           B = X^T [7168][T] ~ N(0,1), the experts' token
+                           ranges (counts padded to 128, padding tokens zero)
+                           stacked along T
 
 Seeds: every tensor draws from its own ``numpy.random.default_rng(seed + i)``
 with i = 0 for A, 1 for B (the FFN's W1), 2 for the routing, 3 for masked_m
@@ -199,6 +204,34 @@ def ffn_contiguous(H: int, I: int, G: int = 8, seed: int = 0, a_std: float = 1.0
 
 
 @dataclasses.dataclass
+class KGroupedInputs:
+    a: np.ndarray       # bf16 bits [M][T] (the output gradient, transposed)
+    b: np.ndarray       # bf16 bits [N][T] (the activations, transposed)
+    ks: np.ndarray      # int32 [G] token counts, multiples of 128
+    counts: np.ndarray  # int64 [G] valid tokens per expert (the rest are zero)
+    M: int
+    N: int
+    T: int
+    G: int
+
+    @property
+    def K(self) -> int:
+        return self.T
+
+
+def k_grouped(M: int, N: int, G: int = 8, seed: int = 0) -> KGroupedInputs:
+    counts = zipf_top8_counts(seed)[:G].astype(np.int64)
+    m_indices, T = contiguous_layout(counts)
+    valid = m_indices >= 0
+    a = np.zeros((M, T), np.uint16)
+    b = np.zeros((N, T), np.uint16)
+    a[:, valid] = normal_bf16(np.random.default_rng(seed + 0), (M, int(valid.sum())), 1.0)
+    b[:, valid] = normal_bf16(np.random.default_rng(seed + 1), (N, int(valid.sum())), 1.0)
+    ks = np.array([-(-int(c) // ALIGN_M) * ALIGN_M for c in counts], np.int32)
+    return KGroupedInputs(a=a, b=b, ks=ks, counts=counts, M=M, N=N, T=int(T), G=G)
+
+
+@dataclasses.dataclass
 class DequantInputs:
     b: np.ndarray  # bf16 bits [N][K] (quantized once, then dequantized)
     N: int
@@ -232,6 +265,8 @@ WORKLOADS = {
     "dequant_7168x2048": ("dequant", dict(N=7168, K=2048)),
     # expert FFN (first GEMM + SwiGLU + requantization, second GEMM)
     "ffn_contiguous_8x7168x2048": ("ffn", dict(H=7168, I=2048, G=8)),
+    # K-grouped weight-gradient GEMM of the contiguous workload's experts
+    "kgrouped_8x4096x7168": ("kgrouped", dict(M=4096, N=7168, G=8)),
 }
 
 
@@ -245,6 +280,8 @@ def make(name: str, seed: int = 0):
         return dequant(seed=seed, **kw)
     if kind == "ffn":
         return ffn_contiguous(seed=seed, **kw)
+    if kind == "kgrouped":
+        return k_grouped(seed=seed, **kw)
     return masked(seed=seed, **kw)
 
 
@@ -256,6 +293,14 @@ def flops_and_bytes(kind: str, inp) -> tuple:
     128 elements) + B (1 B/elt) and its fp32 scales (one per 128x128 block) for
     every expert with at least one valid row + D (2 B/elt) over valid rows.
     """
+    if kind == "kgrouped":
+        # FLOPs over the valid tokens; bytes: both operands and their per-row
+        # scales over the padded token range, the fp32 output of every expert
+        M, N, T = inp.M, inp.N, inp.T
+        tv = int(inp.counts.sum())
+        flops = 2.0 * M * N * tv
+        byts = (M + N) * T + 4 * (M + N) * (T // 128) + 4 * inp.G * M * N
+        return flops, float(byts)
     if kind == "ffn":
         # both GEMMs; bytes: X and its scales, W1 and W2 with their block
         # scales for every expert with a token, h written and read back with
