@@ -276,8 +276,8 @@ fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const 
  * Tuning knob of the three _ue8m0 GEMMs (process-wide). width = 0: choose the
  * tile per shape (default). Otherwise always use the block-scaled kernel, thin
  * shapes included, with weight tiles of `width` rows: 128, 224 or 256 with
- * pair = 0 (one CTA per 128-token tile), or 224 with pair = 1 (two CTAs of a
- * cluster per pair of token tiles of one expert, tcgen05 cta_group::2).
+ * pair = 0 (one CTA per 128-token tile), or 224 or 192 with pair = 1 (two CTAs
+ * of a cluster per pair of token tiles of one expert, tcgen05 cta_group::2).
  * Other values: FG_ERR_INVALID_ARG.
  */
 fg_status fg_set_ue8m0_tile(int width, int pair);

@@ -324,7 +324,7 @@ def fp8_k_grouped_gemm_nt_ue8m0(A, sfa, B, sfb, D, ks, stream=None) -> None:
 
 def set_ue8m0_tile(width: int, pair: bool = False) -> None:
     """0 = automatic (default); else force weight tiles of `width` rows (128,
-    224 or 256 single-CTA, or 224 as a CTA pair)."""
+    224 or 256 single-CTA, or 224 or 192 as a CTA pair)."""
     _check(load_library().fg_set_ue8m0_tile(int(width), 1 if pair else 0))
 
 

@@ -431,6 +431,7 @@ using MxN128 = MxCfg<128, 5, 2, 1, false, 1>;
 using MxN224 = MxCfg<224, 4, 2, 1, false, 1>;
 using MxN256 = MxCfg<256, 3, 1, 2, false, 1>;
 using MxP224 = MxCfg<224, 3, 2, 1, true, 2>;  // CTA pairs, 256 x 224 tiles
+using MxP192 = MxCfg<192, 3, 2, 1, true, 2>;  // CTA pairs, 256 x 192 tiles (N = 11 x 192 = 2112 ...)
 // first GEMM of the expert FFN with the fused SwiGLU + requantization epilogue
 using MxFfnP = MxCfg<256, 3, 1, 1, true, 2, 1>;
 using MxFfnS = MxCfg<256, 4, 1, 1, false, 1, 1>;
@@ -599,9 +600,10 @@ MxPlan mx_plan(const Problem& pr, int sm_count, int expected_m) {
     token_tiles = per_expert * pr.G;
     pairs = (per_expert + 1) / 2 * pr.G;
   }
-  // relative cost of one tile's MMA work per SM, measured on B200
+  // relative cost of one tile's MMA work per SM, measured on B200 (pair 192 vs 224: 1.04-1.11
+  // on dense shapes of equal work per round)
   const struct { int bw; bool pair; double weight; } cand[] = {
-      {224, true, 1.0}, {224, false, 1.15}, {256, false, 1.4}, {128, false, 1.5}};
+      {224, true, 1.0}, {192, true, 1.07}, {224, false, 1.15}, {256, false, 1.4}, {128, false, 1.5}};
   MxPlan best{224, false};
   double best_cost = 1e300;
   for (const auto& c : cand) {
@@ -620,7 +622,10 @@ MxPlan mx_plan(const Problem& pr, int sm_count, int expected_m) {
 
 template <int FORM>
 fg_status dispatch_mx(const Problem& pr, MxPlan pl, const DeviceInfo& dev, int dev_id, cudaStream_t stream) {
-  if (pl.pair) return launch_mx<MxP224, FORM>(pr, dev, dev_id, stream);
+  if (pl.pair) {
+    if (pl.bw == 192) return launch_mx<MxP192, FORM>(pr, dev, dev_id, stream);
+    return launch_mx<MxP224, FORM>(pr, dev, dev_id, stream);
+  }
   switch (pl.bw) {
     case 128: return launch_mx<MxN128, FORM>(pr, dev, dev_id, stream);
     case 256: return launch_mx<MxN256, FORM>(pr, dev, dev_id, stream);
@@ -960,7 +965,8 @@ fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const 
 }
 
 fg_status fg_set_ue8m0_tile(int width, int pair) {
-  const bool ok = width == 0 || (pair ? width == 224 : (width == 128 || width == 224 || width == 256));
+  const bool ok = width == 0 || (pair ? (width == 224 || width == 192)
+                                      : (width == 128 || width == 224 || width == 256));
   if (!ok)
     return fail(FG_ERR_INVALID_ARG, "tile %d%s: 0 (automatic), 128, 224, 256, or 224 as a pair",
                 width, pair ? " (pair)" : "");

@@ -23,7 +23,7 @@ torch = pytest.importorskip("torch")
 
 SENTINEL = 0xFFFF
 # forced tiles: (weight rows, CTA pair); (0, False) = the automatic choice
-TILES = [(128, False), (224, False), (256, False), (224, True), (0, False)]
+TILES = [(128, False), (224, False), (256, False), (224, True), (192, True), (0, False)]
 
 
 @pytest.fixture(scope="module")

@@ -105,7 +105,7 @@ def test_ue8m0_gemm_validation_without_the_device(lib):
     assert lib.fp8_gemm_nt_ue8m0(ok, ok, ok, ok, ok, 0, 256, 256, None) == 0
     assert lib.fp8_grouped_gemm_contiguous_ue8m0(ok, ok, ok, ok, ok, ok, 0, 256, 256, 2, None) == 0
     # the tile knob takes 0, 128, 224 and 256 single-CTA and 224 as a pair
-    for w, pair in ((0, 0), (128, 0), (224, 0), (256, 0), (224, 1), (0, 1)):
+    for w, pair in ((0, 0), (128, 0), (224, 0), (256, 0), (224, 1), (192, 1), (0, 1)):
         assert lib.fg_set_ue8m0_tile(w, pair) == 0
     for w, pair in ((-1, 0), (64, 0), (192, 0), (512, 0), (128, 1), (256, 1)):
         assert lib.fg_set_ue8m0_tile(w, pair) == 1
