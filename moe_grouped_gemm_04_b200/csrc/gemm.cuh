@@ -13,26 +13,28 @@
 // section "swapAB与Mega MoE".
 //
 // CTA roles (one CTA per SM, persistent over output tiles):
-//   warp 0      TMA producer: per K block, lane 0 loads the weight tile, lane 1
-//               the token tile and lane 2 the token scales, each onto the
-//               stage's "full" barrier. (A thread's tensor copies complete one
-//               after another at a roughly fixed time per copy, so one thread
-//               per stream keeps three copies in flight per stage.)
+//   producer    TMA: per K block one thread loads the weight tile, one the
+//               token tile and one the token scales, each onto the stage's
+//               barrier. In the 8-warp form they are lane 0 of warps 0, 2 and
+//               3 (three lanes of one warp diverge, and a lane waiting for its
+//               stage to be released stalled the other two: the producer then
+//               ran barely one stage ahead of the MMA); in the 4-warp form
+//               lanes 0..2 of warp 0.
 //   warp 1      MMA issuer (converged warp, one elected lane issues): 4 x
 //               tcgen05.mma (K = 32 each) per K block into one of two TMEM
 //               partial buffers, then commits to the stage's "empty" barrier
 //               and the buffer's "tmem full" barrier.
-//   promotion warps (2..5, or 4..11 in the 8-warp form whose warps 2-3 idle
-//   so that warpgroup 0 holds the single-lane roles and can give registers
-//   to the promotion warpgroups): per K block read the partial from TMEM
+//   promotion warps (2..5, or 4..11 in the 8-warp form, where warpgroup 0
+//   holds the producer and MMA roles and gives registers to the promotion
+//   warpgroups): per K block read the partial from TMEM
 //               (tcgen05.ld), add partial * (sa * sb) into fp32 registers
 //               (sb, one value per 128 weight rows and K block, is read from
-//               global memory two K blocks ahead), release the TMEM buffer and
+//               global memory one stage ahead), release the TMEM buffer and
 //               the stage; after the last K block round to bf16 and store D.
 //               Normal form: a warp whose 32 token rows are all stored writes
-//               its slice through shared memory with tensor stores (16
-//               columns per round, two buffers per warp), so that the stores
-//               drain while the warp promotes the next tile.
+//               its slice in one pass into a swizzled shared-memory image and
+//               sends it with tensor stores, which drain while the warp
+//               promotes the next tile.
 // Two TMEM buffers let the MMA of block kb+1 run while block kb is promoted.
 //
 // Normal form: MMA M = 128 token rows, MMA N = BW weight rows (TMEM lane =
@@ -490,22 +492,29 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
   if (warp < C::PW_BASE) {
   if constexpr (C::REG_SPLIT) warpgroup_reg_dealloc<C::REG_LOW>();
-  if (warp == 0) {
+  // Producer streams: 0 = weight tiles, 1 = token tiles, 2 = token scales.
+  // With 8 promotion warps each stream has a warp of its own (warps 0, 2 and
+  // 3), so that one stream's barrier wait does not hold up the others (three
+  // lanes of one warp diverge, and a waiting lane stalls its warp); with 4
+  // they are lanes 0..2 of warp 0.
+  constexpr bool OWN_WARPS = C::PW_BASE == 4;
+  const int stream = OWN_WARPS ? (warp == 0 ? 0 : warp - 1) : lane;
+  if (warp != 1) {
     // ------------------------------------------------------------ producer
-    if (lane < 3) {
+    if (OWN_WARPS ? lane == 0 : (warp == 0 && lane < 3)) {
       uint32_t it = 0;
       for (int t = t_first; t < total; t += t_step) {
         const Tile w = resolve_tile<C, FORM>(p, table, t, pair_rank);
         if (!w.valid) continue;
         for (int kq = kb_first; kq < p.KB; kq += C::KPS * kb_step, ++it) {
-          if (lane < 2) {
+          if (stream < 2) {
             const int s = it % C::STAGES;
             if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1u) ^ 1u, ctl)) goto producer_done;
           } else {
             const int q = it % C::SAS;
             if (!mbar_wait(&sa_empty[q], ((it / C::SAS) & 1u) ^ 1u, ctl)) goto producer_done;
           }
-          issue_stage<C, FORM>(lane, p, w, kq, kb_step, it, sA, sB, sSA, full, sa_full, &tmA, &tmB,
+          issue_stage<C, FORM>(stream, p, w, kq, kb_step, it, sA, sB, sSA, full, sa_full, &tmA, &tmB,
                                &tmSA, pair_rank);
         }
       }
@@ -515,14 +524,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     producer_done:
       // Before the CTA exits, the last fill of every stage must have landed
       // and been released (its TMA bytes and the MMA commit's arrival).
-      if (lane == 0) {
+      if (stream == 0) {
         for (uint32_t s = 0; s < C::STAGES && s < it; ++s) {
           const uint32_t last = (it - 1 - s) / C::STAGES * C::STAGES + s;
           // (a pair's operand bytes complete on the leader's barrier)
           if (!C::PAIR || pair_rank == 0) drain_wait(&full[s], (last / C::STAGES) & 1u, kDrainLimitNs);
           drain_wait(&empty[s], (last / C::STAGES) & 1u, kDrainLimitNs);
         }
-      } else if (lane == 2) {
+      } else if (stream == 2) {
         for (uint32_t q = 0; q < C::SAS && q < it; ++q) {
           const uint32_t last = (it - 1 - q) / C::SAS * C::SAS + q;
           drain_wait(&sa_full[q], (last / C::SAS) & 1u, kDrainLimitNs);
@@ -582,7 +591,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     mma_done:
       if (it > 0 && lane == 0) drain_wait(&tfull[(it - 1) & 1], ((it - 1) >> 1) & 1u, kDrainLimitNs);
     }
-  }  // warps 2 .. PW_BASE - 1 (8-warp form) idle
+  }
   } else {
     // ------------------------------------------------------------ promotion + epilogue
     if constexpr (C::REG_SPLIT) warpgroup_reg_alloc<C::REG_HIGH>();
@@ -909,7 +918,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   }
 
   // ---------------------------------------------------------------- teardown
-  // Lane 0 of warps 0 and 1 ran their role alone: reconverge every warp
+  // Single lanes of warpgroup 0 ran their roles alone: reconverge every warp
   // before the CTA-wide barrier (a barrier reached by part of a warp does not
   // wait for the rest of the CTA).
   __syncwarp();
