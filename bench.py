@@ -37,6 +37,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -94,11 +95,17 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources with comments and whitespace removed, so
+    that a capture stays valid across comment-only edits."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_grouped_gemm_04_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+            text = f.read()
+        text = re.sub(rb"/\*.*?\*/", b" ", text, flags=re.S)
+        text = re.sub(rb"//[^\n]*", b" ", text)
+        text = b" ".join(text.split())
+        h.update(name.encode() + b"\0" + text)
     return h.hexdigest()[:16]
 
 

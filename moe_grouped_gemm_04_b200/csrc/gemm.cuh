@@ -138,7 +138,7 @@ struct GemmCfg {
   static constexpr int NUM_THREADS = (PW_BASE + PW) * 32;
   // the whole register file for the one CTA of an SM (allocation in steps of 8)
   static constexpr int MAX_REGS = (65536 / NUM_THREADS) / 8 * 8 > 255 ? 255 : (65536 / NUM_THREADS) / 8 * 8;
-  // 8 promotion warps: warpgroup 0 (producer, MMA, two idle warps) drops to
+  // 8 promotion warps: warpgroup 0 (the producer and MMA warps) drops to
   // REG_LOW registers and the two promotion warpgroups rise to REG_HIGH; the
   // shares add up to the launch allocation of MAX_REGS per thread.
   static constexpr bool REG_SPLIT = PW == 8;
