@@ -94,19 +94,26 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources with comments and whitespace removed, so
-    that a capture stays valid across comment-only edits."""
+def source_hash(files: dict) -> str:
+    """Hash of {file name: source bytes} with C/C++ comments and whitespace
+    removed, so that comment-only edits keep the hash."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "moe_grouped_gemm_04_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            text = f.read()
-        text = re.sub(rb"/\*.*?\*/", b" ", text, flags=re.S)
+    for name in sorted(files):
+        text = re.sub(rb"/\*.*?\*/", b" ", files[name], flags=re.S)
         text = re.sub(rb"//[^\n]*", b" ", text)
         text = b" ".join(text.split())
         h.update(name.encode() + b"\0" + text)
     return h.hexdigest()[:16]
+
+
+def kernel_source_hash() -> str:
+    """source_hash of the kernel sources (moe_grouped_gemm_04_b200/csrc)."""
+    csrc = os.path.join(ROOT, "moe_grouped_gemm_04_b200", "csrc")
+    files = {}
+    for name in os.listdir(csrc):
+        with open(os.path.join(csrc, name), "rb") as f:
+            files[name] = f.read()
+    return source_hash(files)
 
 
 def traffic_for(workload: str, ue8m0: bool = False):

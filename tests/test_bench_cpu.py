@@ -1,0 +1,42 @@
+"""Host logic of bench.py that needs no GPU: the kernel-source hash that keys
+the committed ncu traffic captures, and the kernel names the launch counts
+refer to."""
+import bench
+import workloads
+
+
+def test_source_hash_ignores_comments_and_whitespace():
+    code = b"__global__ void k(int* p) {\n  p[0] = 1;  // store\n}\n"
+    same = [
+        b"// leading comment\n__global__ void k(int* p) {\n  p[0] = 1;\n}\n",
+        b"__global__ void k(int* p) { /* block\n comment */ p[0] = 1; }",
+        b"__global__   void k(int* p)\n{\n\n    p[0] = 1;\n}\n",
+    ]
+    h = bench.source_hash({"a.cuh": code})
+    for s in same:
+        assert bench.source_hash({"a.cuh": s}) == h
+
+
+def test_source_hash_sees_code_and_file_changes():
+    code = b"__global__ void k(int* p) { p[0] = 1; }"
+    h = bench.source_hash({"a.cuh": code})
+    assert bench.source_hash({"a.cuh": code.replace(b"1", b"2")}) != h
+    assert bench.source_hash({"b.cuh": code}) != h
+    assert bench.source_hash({"a.cuh": code, "b.cuh": b"int x;"}) != h
+    # the order files are listed in does not matter
+    two = {"a.cuh": code, "b.cuh": b"int x;"}
+    assert bench.source_hash(dict(reversed(list(two.items())))) == bench.source_hash(two)
+
+
+def test_kernel_source_hash_is_stable():
+    assert bench.kernel_source_hash() == bench.kernel_source_hash()
+    assert len(bench.kernel_source_hash()) == 16
+
+
+def test_gemm_kernel_names():
+    d = workloads.DenseInputs(a=None, b=None, M=64, N=4096, K=7168)
+    assert bench.gemm_kernel_name("dense", d, False) == "fp8_gemm_kernel"
+    p = workloads.DenseInputs(a=None, b=None, M=4096, N=7168, K=2048)
+    assert bench.gemm_kernel_name("dense", p, True) == "fp8_gemm_mx_kernel"
+    # thin shapes take the promoted swapped kernel for power-of-two scales too
+    assert bench.gemm_kernel_name("dense", d, True) == "fp8_gemm_kernel"
