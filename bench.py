@@ -825,6 +825,114 @@ def run_dequant(args, rank, world, local_rank):
     }
 
 
+QUANT_METRIC = "FP8 activation quantization (bf16 -> e4m3 + per-token 1x128 scales) GB/s (device-timed)"
+
+
+def run_quant(args, rank, world, local_rank):
+    """The activation quantizer alone: bf16 activations -> e4m3 codes and
+    per-token scales (amax / 448, or powers of two with --scales ue8m0), on
+    operand sets whose total exceeds L2, used in turn, K launches replayed
+    from one CUDA graph between one pair of events."""
+    import torch
+
+    import moe_grouped_gemm_04_b200 as fg
+
+    torch.cuda.set_device(local_rank)
+    fg.load_library()
+    inp = workloads.make(args.workload, seed=0)
+    M, K = inp.M, inp.K
+    ue8m0 = args.scales == "ue8m0"
+    cast = fg.per_token_cast_to_fp8_ue8m0 if ue8m0 else fg.per_token_cast_to_fp8
+    _, alg_bytes = workloads.flops_and_bytes("quant", inp)
+    x0 = torch.from_numpy(np.ascontiguousarray(inp.a).view(np.int16)).cuda().view(torch.bfloat16)
+    per = int(alg_bytes)
+    R = max(2, -(-ROTATE_MIN_BYTES // per))
+    sets = [(x0.clone(), torch.empty((M, K), dtype=torch.uint8, device="cuda"),
+             fg.empty_sfa(1, M, K, "cuda")) for _ in range(R)]
+
+    def launch(i):
+        x, q, sc = sets[i % R]
+        cast(x, q, sc)
+
+    for i in range(max(args.warmup, R)):
+        launch(i)
+    torch.cuda.synchronize()
+    assert fg.get_device_status() == 0
+    steps = args.steps
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for i in range(steps):
+            launch(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    clocks = sampler.stop()
+    # the timed launches did the work: the last outputs equal a fresh call's
+    last = sets[(steps - 1) % R]
+    timed_q, timed_s = last[1].clone(), last[2][..., :M].clone()
+    last[1].fill_(0x7F)
+    last[2].fill_(float("nan"))
+    launch(steps - 1)
+    torch.cuda.synchronize()
+    assert torch.equal(timed_q, last[1]), "timed codes differ"
+    assert torch.equal(timed_s.view(torch.int32), last[2][..., :M].view(torch.int32)), "timed scales differ"
+    if world > 1:
+        import torch.distributed as dist
+        ms = max_over_ranks(dist, [ms], "cuda")[0]
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = quant_cpu_sample(inp, args.cpu_seconds, ue8m0)
+    return {
+        "metric": QUANT_METRIC, "value": world * gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3",
+        "data": "synthetic (seeded numpy)",
+        "config": {"workload": args.workload, "kind": "quant", "M": M, "K": K,
+                   "scales": "power-of-two (UE8M0)" if ue8m0 else "fp32 amax/448",
+                   "l2": "inputs larger than L2: %d operand sets of %.1f MB used in turn" % (R, per / 1e6),
+                   "launch": "K launches captured in one CUDA graph, replayed once untimed, then timed"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "per_token_cast_kernel", "kernel_ms": ms,
+                     "algorithmic_per_launch": {"bytes": alg_bytes},
+                     "peak_source": "%s HBM copy bandwidth" % peak_src},
+        "cpu_baseline": cpu, "gpu_launches": steps, "clocks": clocks, "e2e": None,
+    }
+
+
+def quant_cpu_sample(inp, target_s: float, ue8m0: bool = False):
+    """The oracle's activation quantizer on a bounded sample of rows."""
+    import oracle
+    threads = oracle.hardware_threads()
+    rows = 16
+    while True:
+        t0 = time.perf_counter()
+        oracle.per_token_cast(inp.a[:rows], threads=threads, ue8m0=ue8m0)
+        dt = time.perf_counter() - t0
+        if dt >= 0.3 * target_s or rows >= inp.M:
+            break
+        rows = min(inp.M, rows * 2)
+    byts = rows * inp.K * 3 + 4 * rows * (inp.K // 128)
+    return {"value": byts / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d rows x K=%d" % (rows, inp.M, inp.K), "seconds": dt}
+
+
 def dequant_cpu_sample(inp, target_s: float):
     """The oracle's dequantizer on a bounded sample of rows of the same weight."""
     import oracle
@@ -882,13 +990,20 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference" and workloads.WORKLOADS[args.workload][0] == "dequant":
+    kind = workloads.WORKLOADS[args.workload][0]
+    if args.impl == "reference" and kind in ("dequant", "quant"):
         out = None
         if rank == 0:
-            cpu = dequant_cpu_sample(workloads.make(args.workload, seed=0), min(args.cpu_seconds, 5.0))
-            out = {"impl": "reference", "metric": DEQUANT_METRIC, "value": cpu["value"], "unit": "GB/s",
+            inp = workloads.make(args.workload, seed=0)
+            if kind == "dequant":
+                cpu = dequant_cpu_sample(inp, min(args.cpu_seconds, 5.0))
+                metric, dtype = DEQUANT_METRIC, "f32->bf16"
+            else:
+                cpu = quant_cpu_sample(inp, min(args.cpu_seconds, 5.0), args.scales == "ue8m0")
+                metric, dtype = QUANT_METRIC, "bf16->e4m3"
+            out = {"impl": "reference", "metric": metric, "value": cpu["value"], "unit": "GB/s",
                    "n_gpus": world, "steps": 1, "warmup": 0, "higher_is_better": True,
-                   "scaling": "weak", "vs_baseline": None, "dtype": "f32->bf16",
+                   "scaling": "weak", "vs_baseline": None, "dtype": dtype,
                    "data": "synthetic (seeded numpy)", "config": {"workload": args.workload},
                    "cpu_baseline": cpu,
                    "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -905,8 +1020,10 @@ def main():
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                     device_id=torch.device("cuda", local_rank))
         try:
-            if workloads.WORKLOADS[args.workload][0] == "dequant":
+            if kind == "dequant":
                 out = run_dequant(args, rank, world, local_rank)
+            elif kind == "quant":
+                out = run_quant(args, rank, world, local_rank)
             else:
                 out = run_ours(args, rank, world, local_rank)
         finally:

@@ -40,3 +40,12 @@ def test_gemm_kernel_names():
     assert bench.gemm_kernel_name("dense", p, True) == "fp8_gemm_mx_kernel"
     # thin shapes take the promoted swapped kernel for power-of-two scales too
     assert bench.gemm_kernel_name("dense", d, True) == "fp8_gemm_kernel"
+
+
+def test_quantizer_cpu_sample_reports_bytes_per_second():
+    inp = workloads.quant(M=64, K=256, seed=1)
+    for ue8m0 in (False, True):
+        r = bench.quant_cpu_sample(inp, 0.01, ue8m0)
+        assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0 and r["cores"] >= 1
+        rows = int(r["sample"].split()[0])
+        assert 16 <= rows <= 64

@@ -129,6 +129,14 @@ def test_work_counts_grouped_count_valid_rows_and_used_experts():
     assert b == 67 * 256 + 4 * 67 * 2 + 2 * (128 * 256 + 4 * 1 * 2) + 2 * 67 * 128
 
 
+def test_quant_workload_is_the_prefill_activation():
+    q = workloads.make("quant_4096x7168")
+    d = workloads.dense(4096, 2112, 7168)
+    assert np.array_equal(q.a, d.a)
+    # bf16 read, e4m3 written, one fp32 scale per 128 elements written
+    assert workloads.flops_and_bytes("quant", q) == (0.0, 4096 * 7168 * 3 + 4 * 4096 * 56)
+
+
 def test_work_counts_dequant_ffn_and_k_grouped():
     q = workloads.DequantInputs(b=None, N=300, K=256)
     assert workloads.flops_and_bytes("dequant", q) == (0.0, 300 * 256 + 4 * 3 * 2 + 2 * 300 * 256)

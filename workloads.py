@@ -25,6 +25,8 @@ inference shapes"):
                            workload's 8 experts and token counts; W1 [8][4096][7168]
                            (gate rows, then up rows) and W2 [8][7168][2048]
                            ~ N(0, 0.02)
+  quant_4096x7168          the activation quantizer alone, on the activations
+                           of prefill_4096x2112x7168 (A ~ N(0,1))
   kgrouped_8x4096x7168     K-grouped weight-gradient GEMM of the contiguous
                            workload's experts: A = dY^T [4096][T] ~ N(0,1),
                            B = X^T [7168][T] ~ N(0,1), the experts' token
@@ -242,6 +244,18 @@ def dequant(N: int, K: int, seed: int = 0, b_std: float = 0.02) -> DequantInputs
     return DequantInputs(b=normal_bf16(np.random.default_rng(seed + 1), (N, K), b_std), N=N, K=K)
 
 
+@dataclasses.dataclass
+class QuantInputs:
+    a: np.ndarray  # bf16 bits [M][K]
+    M: int
+    K: int
+
+
+def quant(M: int, K: int, seed: int = 0, a_std: float = 1.0) -> QuantInputs:
+    """Activations alone: the same draw as a dense workload's A (no outliers)."""
+    return QuantInputs(a=normal_bf16(np.random.default_rng(seed + 0), (M, K), a_std), M=M, K=K)
+
+
 def masked(G: int, M_max: int, N: int, K: int, seed: int = 0,
            masked_m: Optional[np.ndarray] = None, a_std: float = 1.0,
            b_std: float = 0.02) -> MaskedInputs:
@@ -263,6 +277,8 @@ WORKLOADS = {
     "masked_32x256x4096x7168": ("masked", dict(G=32, M_max=256, N=4096, K=7168)),
     # weight dequantization (e4m3 + 128x128 scales -> bf16) of a prefill weight
     "dequant_7168x2048": ("dequant", dict(N=7168, K=2048)),
+    # activation quantization (bf16 -> e4m3 + per-token scales) of a prefill input
+    "quant_4096x7168": ("quant", dict(M=4096, K=7168)),
     # expert FFN (first GEMM + SwiGLU + requantization, second GEMM)
     "ffn_contiguous_8x7168x2048": ("ffn", dict(H=7168, I=2048, G=8)),
     # K-grouped weight-gradient GEMM of the contiguous workload's experts
@@ -278,6 +294,8 @@ def make(name: str, seed: int = 0):
         return contiguous(seed=seed, **kw)
     if kind == "dequant":
         return dequant(seed=seed, **kw)
+    if kind == "quant":
+        return quant(seed=seed, **kw)
     if kind == "ffn":
         return ffn_contiguous(seed=seed, **kw)
     if kind == "kgrouped":
@@ -287,7 +305,7 @@ def make(name: str, seed: int = 0):
 
 def flops_and_bytes(kind: str, inp) -> tuple:
     """Algorithmic FLOPs and HBM bytes of one GEMM call (valid rows only), or of
-    one weight dequantization (bytes only).
+    one weight dequantization or activation quantization (bytes only).
 
     FLOPs = 2 * M_valid * N * K. Bytes = A (1 B/elt) + its fp32 scales (one per
     128 elements) + B (1 B/elt) and its fp32 scales (one per 128x128 block) for
@@ -301,6 +319,8 @@ def flops_and_bytes(kind: str, inp) -> tuple:
         flops = 2.0 * M * N * tv
         byts = (M + N) * T + 4 * (M + N) * (T // 128) + 4 * inp.G * M * N
         return flops, float(byts)
+    if kind == "quant":  # bf16 read; codes and one fp32 scale per 128 elements written
+        return 0.0, float(3 * inp.M * inp.K + 4 * inp.M * (inp.K // 128))
     if kind == "ffn":
         # both GEMMs; bytes: X and its scales, W1 and W2 with their block
         # scales for every expert with a token, h written and read back with
