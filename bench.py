@@ -741,6 +741,33 @@ def run_ours(args, rank, world, local_rank):
 DEQUANT_METRIC = "FP8 weight dequantization (e4m3 + 128x128 scales -> bf16) GB/s (device-timed)"
 
 
+def time_graph_launches(launch, steps: int, local_rank: int, world: int):
+    """launch(0 .. steps-1) captured in one CUDA graph, replayed once untimed
+    (upload), then timed between one pair of CUDA events while the clocks are
+    sampled. Returns (ms per launch, clock summary)."""
+    import torch
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for i in range(steps):
+            launch(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    return ms, sampler.stop()
+
+
 def run_dequant(args, rank, world, local_rank):
     """The weight dequantizer alone: codes and block scales (quantized once on
     the GPU) -> bf16, on operand sets whose total exceeds L2, used in turn,
@@ -771,26 +798,7 @@ def run_dequant(args, rank, world, local_rank):
         launch(i)
     torch.cuda.synchronize()
     steps = args.steps
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    time.sleep(0.3)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, capture_error_mode="thread_local"):
-        for i in range(steps):
-            launch(i)
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    del g
-    clocks = sampler.stop()
+    ms, clocks = time_graph_launches(launch, steps, local_rank, world)
     # the timed launches did the work: the last output equals a fresh call
     last = sets[(steps - 1) % R]
     timed_x = last[2].clone()
@@ -859,26 +867,7 @@ def run_quant(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert fg.get_device_status() == 0
     steps = args.steps
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    time.sleep(0.3)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, capture_error_mode="thread_local"):
-        for i in range(steps):
-            launch(i)
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    del g
-    clocks = sampler.stop()
+    ms, clocks = time_graph_launches(launch, steps, local_rank, world)
     # the timed launches did the work: the last outputs equal a fresh call's
     last = sets[(steps - 1) % R]
     timed_q, timed_s = last[1].clone(), last[2][..., :M].clone()
