@@ -1,9 +1,11 @@
-// CPU oracle for the FP8 block-scaled GEMM and its two quantizers.
+// CPU oracle for the FP8 block-scaled GEMM, its quantizers and dequantizer,
+// the K-grouped GEMM and the expert FFN's activation.
 //
 // TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or
 // load this file or the library built from it: only tests/, the smoke check
-// in __graft_entry__.py and the CPU-baseline leg of bench.py use it. It shares
-// no code, header, table or constant generator with the CUDA library.
+// in __graft_entry__.py and bench.py's CPU legs (the CPU baseline and the
+// reference arm) use it. It shares no code, header, table or constant
+// generator with the CUDA library.
 //
 // What it computes (all plain definitions, written out without blocking,
 // fusion or reordering beyond what the definition states):
@@ -34,6 +36,8 @@
 //    only the two scale multiplies and the outer sum over K blocks round in
 //    fp64. The result is kept in fp64, not rounded to bf16.
 //
+//  * Weight dequantization (the review's quantize / dequantize / GEMM trio):
+//    x = bf16(fp32(dec(q) * s)) per element with the block's scale s.
 //  * The K-grouped GEMM of FP8 training's expert weight gradients (the
 //    animattoys.com page, section "為現代 AI 計算而造", names FP8 training
 //    among DeepGEMM's uses; the DeepSeek-V3 review's quantize / dequantize /
