@@ -80,8 +80,9 @@ def parse_args():
                          "(steps back to back) or by flushing L2 before every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample (a sample takes at "
+                         "least 0.85 of it)")
     return ap.parse_args()
 
 
@@ -192,6 +193,23 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------- CPU legs
 
+# a CPU sample stops growing once it takes this fraction of the target time
+SAMPLE_STOP = 0.85
+
+
+def repeat_for(fn, target_s: float):
+    """Calls fn() until at least target_s seconds have passed; returns
+    (calls, seconds)."""
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        fn()
+        calls += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            return calls, dt
+
+
 def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict, ue8m0: bool = False):
     """Oracle on a bounded sample of the workload: quantize the sampled A rows
     and compute their outputs against all N columns (weights are quantized
@@ -233,23 +251,22 @@ def cpu_sample(inp, kind: str, target_s: float, threads: int, cache: dict, ue8m0
             qb, sb = weights(int(e))
             oracle.gemm_nt(qa[sub], sa[sub], qb, sb, threads=threads)
         dt = time.perf_counter() - t0
-        if dt >= 0.5 * target_s or len(take) >= len(order):
+        if dt >= SAMPLE_STOP * target_s or len(take) >= len(order):
             break
-        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9))
+        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.05))
     cache["rows"] = rows
     done = len(take)
     passes = 1
-    if done >= len(order) and dt < 0.5 * target_s:
-        # the whole workload is smaller than the target: repeat it
-        passes = max(1, int(target_s / max(dt, 1e-3)))
-        t0 = time.perf_counter()
-        for _ in range(passes):
+    if done >= len(order) and dt < SAMPLE_STOP * target_s:
+        # the whole workload is smaller than the target: repeat it until the
+        # target time has passed
+        def one_pass():
             qa, sa = oracle.per_token_cast(a_rows, threads=threads, ue8m0=ue8m0)
             for e in np.unique(experts):
                 sub = np.nonzero(experts == e)[0]
                 qb, sb = weights(int(e))
                 oracle.gemm_nt(qa[sub], sa[sub], qb, sb, threads=threads)
-        dt = time.perf_counter() - t0
+        passes, dt = repeat_for(one_pass, target_s)
     flops = 2.0 * done * N * K * passes
     desc = "%d of %d valid A rows x all %d columns, K=%d (activation quantization + GEMM)" % (
         done, len(order), N, K)
@@ -290,9 +307,9 @@ def ffn_cpu_sample(inp, target_s: float, threads: int, cache: dict):
             hq, sh = oracle.per_token_cast(h, threads=threads, ue8m0=True)
             oracle.gemm_nt(hq, sh, w2q, sw2, threads=threads)
         dt = time.perf_counter() - t0
-        if dt >= 0.5 * target_s or len(take) >= len(order):
+        if dt >= SAMPLE_STOP * target_s or len(take) >= len(order):
             break
-        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9))
+        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.05))
     cache["rows"] = rows
     flops = 6.0 * len(take) * H * I
     desc = ("%d of %d valid rows through the whole expert FFN (quantization, first GEMM, "
@@ -317,9 +334,9 @@ def kgrouped_cpu_sample(inp, target_s: float, threads: int, cache: dict):
         qa, sa = oracle.per_token_cast(inp.a[take], threads=threads, ue8m0=True)
         oracle.k_grouped(qa, sa, qb, sb, inp.ks, threads=threads)
         dt = time.perf_counter() - t0
-        if dt >= 0.5 * target_s or len(take) >= inp.M:
+        if dt >= SAMPLE_STOP * target_s or len(take) >= inp.M:
             break
-        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9))
+        rows = max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.05))
     cache["rows"] = rows
     flops = 2.0 * len(take) * inp.N * tv
     desc = ("%d of %d A rows x all %d B rows over all %d experts' tokens (T=%d, quantization "
@@ -914,12 +931,16 @@ def quant_cpu_sample(inp, target_s: float, ue8m0: bool = False):
         t0 = time.perf_counter()
         oracle.per_token_cast(inp.a[:rows], threads=threads, ue8m0=ue8m0)
         dt = time.perf_counter() - t0
-        if dt >= 0.3 * target_s or rows >= inp.M:
+        if dt >= SAMPLE_STOP * target_s or rows >= inp.M:
             break
         rows = min(inp.M, rows * 2)
-    byts = rows * inp.K * 3 + 4 * rows * (inp.K // 128)
+    passes = 1
+    if dt < SAMPLE_STOP * target_s:
+        passes, dt = repeat_for(
+            lambda: oracle.per_token_cast(inp.a[:rows], threads=threads, ue8m0=ue8m0), target_s)
+    byts = passes * (rows * inp.K * 3 + 4 * rows * (inp.K // 128))
     return {"value": byts / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": "%d of %d rows x K=%d" % (rows, inp.M, inp.K), "seconds": dt}
+            "sample": "%d of %d rows x K=%d, %d passes" % (rows, inp.M, inp.K, passes), "seconds": dt}
 
 
 def dequant_cpu_sample(inp, target_s: float):
@@ -932,12 +953,16 @@ def dequant_cpu_sample(inp, target_s: float):
         t0 = time.perf_counter()
         oracle.per_block_dequant(q[:rows], s[:-(-rows // 128)], threads=threads)
         dt = time.perf_counter() - t0
-        if dt >= 0.3 * target_s or rows >= inp.N:
+        if dt >= SAMPLE_STOP * target_s or rows >= inp.N:
             break
         rows = min(inp.N, rows * 2)
-    byts = rows * inp.K * 3 + 4 * (-(-rows // 128)) * (inp.K // 128)
+    passes = 1
+    if dt < SAMPLE_STOP * target_s:
+        passes, dt = repeat_for(
+            lambda: oracle.per_block_dequant(q[:rows], s[:-(-rows // 128)], threads=threads), target_s)
+    byts = passes * (rows * inp.K * 3 + 4 * (-(-rows // 128)) * (inp.K // 128))
     return {"value": byts / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": "%d of %d rows x K=%d" % (rows, inp.N, inp.K), "seconds": dt}
+            "sample": "%d of %d rows x K=%d, %d passes" % (rows, inp.N, inp.K, passes), "seconds": dt}
 
 
 def run_reference(args, rank, world):
