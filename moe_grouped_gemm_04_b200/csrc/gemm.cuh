@@ -547,6 +547,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     if (pair_rank == 0) {  // a pair's MMAs are issued by its leader
       constexpr uint32_t idesc = mma_idesc_e4m3(C::MMA_M, C::MMA_N);
       uint32_t it = 0;
+      // the next iteration's TMEM buffer / operand stage were seen free /
+      // full by a non-blocking peek made while this iteration's MMAs ran
+      bool empty_seen = false, full_seen = false;
       for (int t = t_first; t < total; t += t_step) {
         const Tile w = resolve_tile<C, FORM>(p, table, t, pair_rank);
         if (!w.valid) continue;
@@ -555,9 +558,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           const uint32_t ph = (it / C::STAGES) & 1u;
           const int b = it & 1;
           const uint32_t tph = (it >> 1) & 1u;
-          if (!warp_wait(&tempty[b], tph ^ 1u, ctl, lane)) goto mma_done;
+          if (!empty_seen && !warp_wait(&tempty[b], tph ^ 1u, ctl, lane)) goto mma_done;
           tc_fence_after();
-          if (!warp_wait(&full[s], ph, ctl, lane)) goto mma_done;
+          if (!full_seen && !warp_wait(&full[s], ph, ctl, lane)) goto mma_done;
           tc_fence_after();
           if (elect_one()) {
 #pragma unroll
@@ -585,6 +588,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
               mma_commit(&empty[s]);
               mma_commit(&tfull[b]);
             }
+          }
+          {
+            // peek at the next iteration's buffer and stage while these MMAs
+            // run: a phase seen complete here needs no blocking wait (phases
+            // of both barriers advance at most one ahead of this warp)
+            const uint32_t nx = it + 1;
+            int r = 0;
+            if (lane == 0) {
+              r = mbar_test_wait(&tempty[nx & 1], ((nx >> 1) & 1u) ^ 1u) ? 1 : 0;
+              r |= mbar_test_wait(&full[nx % C::STAGES], (nx / C::STAGES) & 1u) ? 2 : 0;
+            }
+            r = __shfl_sync(0xffffffffu, r, 0);
+            empty_seen = (r & 1) != 0;
+            full_seen = (r & 2) != 0;
           }
         }
       }
