@@ -9,8 +9,11 @@ GEMM (dense, contiguous-grouped or masked-grouped, per the workload). Weights
 are quantized once before timing, as inference stores them (pass
 --with-weight-quant to quantize them inside every step as well).
 
-The default workload is decode_64x4096x7168 (the swapped-product decode
-shape). Inputs are resident in HBM when the timed region starts. By default
+The default workload is contiguous_8x4096x7168 (MoE grouped GEMM in the
+contiguous layout: 8 experts with the top-8-of-256 Zipf routing of 4096
+tokens, N=4096, K=7168), the largest single-GPU configuration, with fp32
+scales amax/448 (the promoted GEMM). Inputs are resident in HBM when the
+timed region starts. By default
 the step's operands (activations, quantized weights, scales, output) exist in
 several copies whose total is three times the 126 MB L2, used in turn, so that
 no step finds its inputs in L2; the K timed steps run back to back between one
@@ -60,6 +63,10 @@ SENTINEL_BF16 = 0x7FC1  # a bf16 NaN pattern the kernels never produce
 ROTATE_MIN_BYTES = 3 * (126 << 20)  # operand sets in turn: three times the 126 MB L2
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 rated figures (vendor datasheet, dense): the second denominator of
+# every roofline fraction, beside the measured one
+RATED_FP8_TFLOPS = 4500.0
+RATED_HBM_GBS = 8000.0
 
 
 def parse_args():
@@ -67,7 +74,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode_64x4096x7168", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="contiguous_8x4096x7168", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--with-weight-quant", action="store_true")
     ap.add_argument("--scales", default="fp32", choices=["fp32", "ue8m0"],
@@ -514,6 +521,50 @@ class Step:
         self.gemm(o)
 
 
+def workload_config(kind: str, inp) -> dict:
+    """The workload's sizes as they appear in the JSON line's `config` (the same
+    keys in both arms, so the two lines describe the same problem)."""
+    cfg = {"N": inp.N, "K": inp.K}
+    if kind == "ffn":
+        cfg = {"H": inp.H, "I": inp.I, "G": inp.G, "M_total": inp.M_total,
+               "M_valid": int(inp.counts.sum())}
+    elif kind == "kgrouped":
+        cfg.update(M=inp.M, T=inp.T, G=inp.G, T_valid=int(inp.counts.sum()))
+    elif kind == "dense":
+        cfg["M"] = inp.M
+    elif kind == "contiguous":
+        cfg.update(G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
+    elif kind == "masked":
+        cfg.update(G=inp.G, M_max=inp.M_max, M_valid=int(inp.masked_m.sum()))
+    return cfg
+
+
+def step_config(args, kind: str, inp, world: int, ue8m0: bool) -> dict:
+    """The JSON line's `config`: what problem one step solves. Both arms build
+    it with this function, so their lines carry the same config; how a step
+    was timed goes into the separate `method` object."""
+    return {"workload": args.workload, "kind": kind, **workload_config(kind, inp),
+            "weights": "quantized inside every step" if args.with_weight_quant
+                       else "quantized once before timing",
+            "scales": ("power-of-two (UE8M0) scales, block-scaled tensor-core GEMM" if ue8m0 else
+                       "fp32 scales amax/448, promoted per 128-wide K block"),
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
+def peaks_used(peaks: dict, source: str) -> dict:
+    """The denominators a roofline fraction was taken against, with where they
+    came from, so that the fraction can be recomputed."""
+    d = {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+         "fp8_tflops": FP8_OVER_BF16 * peaks["bf16_tflops"],
+         "fp8_rule": "%.1f x the bf16 burst figure" % FP8_OVER_BF16,
+         "source": "MEASURED_PEAKS.json" if source == "measured" else "recipe fallback",
+         "rated_fp8_tflops": RATED_FP8_TFLOPS, "rated_hbm_gbs": RATED_HBM_GBS}
+    clk = peaks.get("clocks_under_load") or {}
+    if clk.get("sm_mhz_median") is not None:
+        d["sm_mhz_median_when_measured"] = clk["sm_mhz_median"]
+    return d
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -631,9 +682,10 @@ def run_ours(args, rank, world, local_rank):
     # output back. As in a serving loop the steps are pipelined on three
     # streams (upload, compute, download), so the upload of step i+1 and the
     # download of step i-1 overlap the compute of step i; each step uses its
-    # own operand set, whose previous use must have finished before the upload
-    # overwrites it. Timed between events on the compute stream, which waits
-    # for the last download before the closing event.
+    # own operand set, whose previous use (compute and read-back) must have
+    # finished before the upload overwrites it. Timed between events on the
+    # compute stream, which waits for the last download before the closing
+    # event.
     e2e = None
     if not args.no_e2e:
         xh = step.sets[0].x.cpu().pin_memory()
@@ -643,31 +695,37 @@ def run_ours(args, rank, world, local_rank):
               for _ in range(2)]
         up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
+        # events are created once and re-recorded: set i % R's upload,
+        # compute-done and download-done events (a wait sees the most recent
+        # record)
+        up_ev = [torch.cuda.Event() for _ in range(R)]
+        done_ev = [torch.cuda.Event() for _ in range(R)]
+        dl_ev = [torch.cuda.Event() for _ in range(R)]
+
         def e2e_loop(n):
             comp = torch.cuda.current_stream()
             e0, e1 = ev(), ev()
             e0.record(comp)
             up.wait_event(e0)
             down.wait_event(e0)
-            done = []
             for i in range(n):
-                o = step.sets[i % R]
+                j = i % R
+                o = step.sets[j]
                 with torch.cuda.stream(up):
                     if i >= R:
-                        up.wait_event(done[i - R])
+                        # the set's previous step has been computed and read back
+                        up.wait_event(dl_ev[j])
                     o.x.copy_(xh, non_blocking=True)
                     if x2h is not None:
                         o.x2.copy_(x2h, non_blocking=True)
-                    uploaded = torch.cuda.Event()
-                    uploaded.record(up)
-                comp.wait_event(uploaded)
+                    up_ev[j].record(up)
+                comp.wait_event(up_ev[j])
                 step.run(i)
-                d = torch.cuda.Event()
-                d.record(comp)
-                done.append(d)
+                done_ev[j].record(comp)
                 with torch.cuda.stream(down):
-                    down.wait_event(d)
+                    down.wait_event(done_ev[j])
                     dh[i % 2].copy_(o.D, non_blocking=True)
+                    dl_ev[j].record(down)
             comp.wait_stream(down)
             e1.record(comp)
             torch.cuda.synchronize()
@@ -696,20 +754,23 @@ def run_ours(args, rank, world, local_rank):
         peak = FP8_OVER_BF16 * peaks["bf16_tflops"]
         achieved = flops / (gms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak}
+                "frac": achieved / peak, "peak_rated": RATED_FP8_TFLOPS,
+                "frac_rated": achieved / RATED_FP8_TFLOPS}
         peak_note = "FP8 = %.1f x %s bf16 burst %.1f TFLOP/s (%s)" % (
             FP8_OVER_BF16, peak_src, peaks["bf16_tflops"], "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
     else:
         peak = peaks["hbm_gbs"]
         achieved = alg_bytes / (gms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak}
+                "frac": achieved / peak, "peak_rated": RATED_HBM_GBS,
+                "frac_rated": achieved / RATED_HBM_GBS}
         peak_note = "%s HBM copy bandwidth (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
     roof["traffic"] = traffic_for(args.workload, ue8m0)
     roof["kernel"] = gemm_kernel_name(kind, inp, ue8m0)
     roof["algorithmic_per_launch"] = {"flops": flops, "bytes": alg_bytes}
     roof["kernel_ms"] = gms
     roof["peak_source"] = peak_note
+    roof["peaks_used"] = peaks_used(peaks, peak_src)
 
     cpu = None
     if not args.no_cpu_baseline:
@@ -720,31 +781,19 @@ def run_ours(args, rank, world, local_rank):
                "sample": desc, "seconds": secs}
 
     value = world * flops / (ms * 1e-3) / 1e12
-    cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K,
-           "l2": ("inputs larger than L2: %d operand sets of %.1f MB used in turn, steps back to back"
-                  % (R, step.set_bytes / 1e6)) if rotate else
-                 "flushed before every timed step (256 MiB write + 256 MiB read, outside the step events)",
-           "launch": ("the K timed steps captured in one CUDA graph, replayed once untimed, "
-                      "then once between the events") if use_graph else "eager launches from Python",
-           "weights": "quantized inside every step" if args.with_weight_quant else "quantized once before timing",
-           "scales": ("power-of-two (UE8M0) scales, block-scaled tensor-core GEMM" if ue8m0 else
-                      "fp32 scales amax/448, promoted per 128-wide K block"),
-           "parallelism": "replicas" if world > 1 else "single GPU"}
-    if kind == "ffn":
-        cfg.update(H=inp.H, I=inp.I, G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
-    elif kind == "kgrouped":
-        cfg.update(M=inp.M, T=inp.T, G=inp.G, T_valid=int(inp.counts.sum()))
-    elif kind == "dense":
-        cfg["M"] = inp.M
-    elif kind == "contiguous":
-        cfg.update(G=inp.G, M_total=inp.M_total, M_valid=int(inp.counts.sum()))
-    else:
-        cfg.update(G=inp.G, M_max=inp.M_max, M_valid=int(inp.masked_m.sum()))
+    cfg = step_config(args, kind, inp, world, ue8m0)
+    method = {
+        "l2": ("inputs larger than L2: %d operand sets of %.1f MB used in turn, steps back to back"
+               % (R, step.set_bytes / 1e6)) if rotate else
+              "flushed before every timed step (256 MiB write + 256 MiB read, outside the step events)",
+        "launch": ("the K timed steps captured in one CUDA graph, replayed once untimed, "
+                   "then once between the events") if use_graph else "eager launches from Python",
+        "timing": "CUDA events on the launching stream, max over ranks"}
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic (seeded numpy, random weights)",
-        "config": cfg, "roofline": roof, "cpu_baseline": cpu,
+        "config": cfg, "method": method, "roofline": roof, "cpu_baseline": cpu,
         "gpu_launches": step.launches_per_step() * K,
         "clocks": clocks,
     }
@@ -986,13 +1035,15 @@ def run_reference(args, rank, world):
         secs.append(s)
     value = float(np.mean(vals)) / 1e12
     ms = float(np.mean(secs)) * 1e3
-    cfg = {"workload": args.workload, "kind": kind, "N": inp.N, "K": inp.K,
-           "scales": "power-of-two (UE8M0)" if ue8m0 else "fp32 amax/448"}
+    cfg = step_config(args, kind, inp, world, ue8m0)
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy)",
         "config": cfg,
+        "method": {"timing": "host wall clock (perf_counter) around each step's oracle calls; "
+                             "each step is a bounded sample of the workload",
+                   "threads": threads},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": descs[-1] if descs else ""},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

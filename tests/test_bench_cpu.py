@@ -49,3 +49,37 @@ def test_quantizer_cpu_sample_reports_bytes_per_second():
         assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0 and r["cores"] >= 1
         rows = int(r["sample"].split()[0])
         assert 16 <= rows <= 64
+
+
+def test_both_arms_describe_the_same_problem():
+    """The reference arm and the GPU arm build `config` with one function: the
+    same keys and values for the same workload and options."""
+    import argparse
+    args = argparse.Namespace(workload="contiguous_8x4096x7168", with_weight_quant=False)
+    inp = workloads.contiguous(N=256, K=256, counts=[130, 0, 5], seed=3)
+    a = bench.step_config(args, "contiguous", inp, 1, False)
+    b = bench.step_config(args, "contiguous", inp, 1, False)
+    assert a == b
+    assert a["M_total"] == inp.M_total and a["M_valid"] == 135 and a["G"] == 3
+    assert "l2" not in a and "launch" not in a  # how a step is timed lives in `method`
+    d = workloads.DenseInputs(a=None, b=None, M=64, N=4096, K=7168)
+    assert bench.step_config(args, "dense", d, 1, False)["M"] == 64
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    import sys
+    old = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        args = bench.parse_args()
+    finally:
+        sys.argv = old
+    assert args.workload == "contiguous_8x4096x7168" and args.scales == "fp32"
+
+
+def test_peaks_used_records_both_denominators():
+    d = bench.peaks_used({"hbm_gbs": 6549.1, "bf16_tflops": 1654.5,
+                         "clocks_under_load": {"sm_mhz_median": 1192.0}}, "measured")
+    assert d["fp8_tflops"] == 2 * 1654.5 and d["rated_fp8_tflops"] == 4500.0
+    assert d["rated_hbm_gbs"] == 8000.0 and d["sm_mhz_median_when_measured"] == 1192.0
+    assert d["source"] == "MEASURED_PEAKS.json"
