@@ -77,6 +77,7 @@ typedef enum {
 #define FG_DEVICE_BAD_MASKED_M 2   /* masked_m[e] < 0 or > M_max (clamped) */
 #define FG_DEVICE_BAD_M_INDEX 3    /* m_indices entry >= G (tile skipped) */
 #define FG_DEVICE_BAD_K_GROUP 4    /* ks entry < 0, not a multiple of 128, or sum > T (truncated) */
+#define FG_DEVICE_BAD_SCALE 5      /* a block-scaled _ue8m0 GEMM read a scale that is not a power of two */
 
 /* Row stride (in floats) of the MN-major activation-scale layout. */
 int fg_sfa_stride(int M);
@@ -190,8 +191,13 @@ fg_status fp8_grouped_gemm_masked(const uint8_t* A, const float* sfa, const uint
  * fp8_grouped_gemm_contiguous and fp8_grouped_gemm_masked; additionally every
  * sfa and sfb entry that is read must be a power of two in the fp32 normal
  * range (what per_token_cast_to_fp8_ue8m0 / per_block_cast_to_fp8_ue8m0
- * write). The kernel keeps only each scale's exponent field: a scale that is
- * not a power of two acts as the power of two at or below it, zero as 2^-127.
+ * write), or zero (which acts as 2^-127). The block-scaled kernel keeps only
+ * each scale's exponent field; it checks every weight scale it reads and the
+ * token scales of every row it stores, and a scale with a sign or mantissa
+ * bit set, or an infinite or NaN scale, sets FG_DEVICE_BAD_SCALE: the call's
+ * output is then not the product of the given scales and must be discarded.
+ * (The promoted kernel that thin shapes use applies any fp32 scale exactly
+ * and checks nothing.)
  *
  * For token tiles of 128 rows (or pairs of them of one expert, computed by
  * the two CTAs of a cluster) the scales are applied inside the tensor core (tcgen05.mma
@@ -286,6 +292,12 @@ fg_status fg_set_ue8m0_tile(int width, int pair);
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns FG_OK when it was clear, FG_ERR_DEVICE otherwise
  * (the detail is in fg_last_error and *code, which may be NULL).
+ * There is one status word per device, shared by every stream and every call
+ * of this library on that device: it holds the first FG_DEVICE_* code any
+ * kernel recorded since it was last cleared. Only `stream` is synchronised,
+ * so a call still running on another stream may set the word after it was
+ * read; to attribute a status to one call, run that call alone (or
+ * synchronise the device) before this read.
  */
 fg_status fg_get_device_status(cudaStream_t stream, int* code);
 

@@ -205,15 +205,23 @@ using CfgSwap32S4 = GemmCfg<32, 128, true, 4, 4, 4, 2>;
 using CfgSwap64S4 = GemmCfg<64, 128, true, 3, 4, 4, 2>;
 
 struct KernelInfo {
-  bool attr_set = false;
+  std::atomic<bool> attr_set{false};  // published after max_clusters (release)
   int max_clusters = 0;  // max co-resident clusters (split-K and pair configs)
 };
 
+// One-time set-up of a kernel on a device, safe when several host threads
+// make their first call at once: double-checked under g_mu, and the flag is
+// published only after every field it guards has been written.
 template <class C, int FORM>
 fg_status kernel_info(int dev, KernelInfo** out) {
   static KernelInfo info[kMaxDevices];
   KernelInfo& k = info[dev];
-  if (!k.attr_set) {
+  if (k.attr_set.load(std::memory_order_acquire)) {
+    *out = &k;
+    return FG_OK;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!k.attr_set.load(std::memory_order_relaxed)) {
     cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<C, FORM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::smem_bytes(FORM));
@@ -246,7 +254,7 @@ fg_status kernel_info(int dev, KernelInfo** out) {
       if (n < 1) return fail(FG_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", C::CLUSTER);
       k.max_clusters = n;
     }
-    k.attr_set = true;
+    k.attr_set.store(true, std::memory_order_release);
   }
   *out = &k;
   return FG_OK;
@@ -451,9 +459,14 @@ struct FfnOut {
 // clusters (the persistent grid's size).
 template <class C, int FORM>
 fg_status mx_kernel_attr(int dev, int* max_clusters) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices];  // (zero-initialised: false)
   static int clusters[kMaxDevices] = {};
-  if (!done[dev]) {
+  if (done[dev].load(std::memory_order_acquire)) {
+    *max_clusters = clusters[dev];
+    return FG_OK;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);  // (see kernel_info)
+  if (!done[dev].load(std::memory_order_relaxed)) {
     cudaError_t e = cudaFuncSetAttribute(fp8_gemm_mx_kernel<C, FORM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::smem_bytes(FORM));
@@ -476,7 +489,7 @@ fg_status mx_kernel_attr(int dev, int* max_clusters) {
       if (n < 1) return fail(FG_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", C::CLUSTER);
       clusters[dev] = n;
     }
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
   }
   *max_clusters = clusters[dev];
   return FG_OK;
@@ -989,6 +1002,7 @@ fg_status fg_get_device_status(cudaStream_t stream, int* code) {
                      : v == FG_DEVICE_BAD_MASKED_M ? "masked_m outside [0, M_max]"
                      : v == FG_DEVICE_BAD_M_INDEX  ? "m_indices entry >= G"
                      : v == FG_DEVICE_BAD_K_GROUP  ? "ks entry negative, not a multiple of 128, or past T"
+                     : v == FG_DEVICE_BAD_SCALE    ? "a scale of a block-scaled (_ue8m0) GEMM is not a power of two"
                                                    : "unknown device status";
   return fail(FG_ERR_DEVICE, "device status %d: %s", v, what);
 }

@@ -180,6 +180,13 @@ __device__ __forceinline__ int sw64_offset(int r, int c) { return r * 64 + ((c ^
 // UE8M0 byte of an fp32 power of two: its biased exponent.
 __device__ __forceinline__ uint32_t ue8m0_byte(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
+// A scale this kernel cannot apply exactly: not +0 or a positive power of two
+// (sign bit or mantissa bits set), or an infinity / NaN (exponent field 255).
+__device__ __forceinline__ bool not_pow2_scale(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x807FFFFFu) != 0u || (u >> 23) == 0xFFu;
+}
+
 // Tables of the grouped layouts, built by warp 0 before the main loops.
 // Contiguous: table[mt] = expert of token tile mt (from its first row; -1 for
 // padding tiles); with pairs also units[u] = first token tile of pair unit u
@@ -635,6 +642,25 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1)
           jb[g][r1] = C::EPI == 1 ? g : ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
+      // rows of this lane (lane + 32 r1) whose outputs are stored: only their
+      // token scales must be powers of two (rows past M arrive as zeros;
+      // masked rows past masked_m and contiguous rows of another expert or
+      // padding hold whatever the caller left there)
+      uint32_t rows_ok = 0xFu;
+      if constexpr (FORM == kFormMasked) {
+        int mv = __ldg(p.masked_m + w.e);
+        mv = mv < 0 ? 0 : (mv > p.M ? p.M : mv);
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1)
+          if (w.mt * C::BT + 32 * r1 + lane >= mv) rows_ok &= ~(1u << r1);
+      } else if constexpr (FORM == kFormContig) {
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1) {
+          const int m = w.mt * C::BT + 32 * r1 + lane;
+          if (m >= p.M || __ldg(p.m_indices + m) != w.e) rows_ok &= ~(1u << r1);
+        }
+      }
+      bool bad_scale = false;
       const int KQ = (w.nkb + 3) >> 2;  // quads of the tile
       for (int qi = 0; qi < KQ; ++qi, rr.next(), sq.next()) {
         // the quad's scales have landed, and the slot's previous quad has
@@ -653,7 +679,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         for (int k = 0; k < 4; ++k) {
           if (k < nk) {
 #pragma unroll
-            for (int r1 = 0; r1 < 4; ++r1) wa[r1] |= ue8m0_byte(raw[k * 128 + 32 * r1 + lane]) << (8 * k);
+            for (int r1 = 0; r1 < 4; ++r1) {
+              const float sa = raw[k * 128 + 32 * r1 + lane];
+              bad_scale |= ((rows_ok >> r1) & 1u) && not_pow2_scale(sa);
+              wa[r1] |= ue8m0_byte(sa) << (8 * k);
+            }
 #pragma unroll
             for (int g = 0; g < C::SFB_GROUPS; ++g)
 #pragma unroll
@@ -661,9 +691,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
                 if constexpr (C::EPI == 2) {
                   // per-row weight scale of tile row 128 g + 32 r1 + lane
                   const int n = 128 * g + 32 * r1 + lane;
-                  wb[g][r1] |= (n < C::BW ? ue8m0_byte(raw[C::RAW_A / 4 + k * C::BW + n]) : 127u) << (8 * k);
+                  const float sb = n < C::BW ? raw[C::RAW_A / 4 + k * C::BW + n] : 1.0f;
+                  bad_scale |= not_pow2_scale(sb);
+                  wb[g][r1] |= (n < C::BW ? ue8m0_byte(sb) : 127u) << (8 * k);
                 } else {
-                  wb[g][r1] |= ue8m0_byte(raw[C::RAW_A / 4 + k * C::NBT + jb[g][r1]]) << (8 * k);
+                  // (blocks past the weight's last one arrive as zeros)
+                  const float sb = raw[C::RAW_A / 4 + k * C::NBT + jb[g][r1]];
+                  bad_scale |= not_pow2_scale(sb);
+                  wb[g][r1] |= ue8m0_byte(sb) << (8 * k);
                 }
               }
           }
@@ -690,6 +725,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             mbar_arrive(&sf_full[sq.slot]);
         }
       }
+      // a scale the block-scaled MMA would round: the call's result is wrong
+      if (__any_sync(0xffffffffu, bad_scale) && lane == 0)
+        raise_status(p.status, 5 /* FG_DEVICE_BAD_SCALE */);
     }
   convert_done:;
   } else if (C::EPI == 1 && warp >= C::EPI_BASE) {

@@ -51,14 +51,16 @@ __device__ __forceinline__ uint2 quantize8(uint4 w, float inv) {
 // UE8M0 = true: s = the smallest power of two at or above amax_c / 448 (from
 // the fp32 bits of the quotient: 2^E if its mantissa field is zero, else
 // 2^(E+1)), inv = 1 / s exactly (biased exponent 254 - e), so that x * inv
-// equals x / s.
+// equals x / s. A slice holding an infinity has s = +inf and inv = 0, which
+// is x / s as well: finite elements give (signed) zero codes, infinities NaN.
+// (For finite bf16 input E stays far below 254: amax / 448 < 2^120.)
 template <bool UE8M0>
 __device__ __forceinline__ void group_scale(float amx, float& scale, float& inv) {
   if constexpr (UE8M0) {
     const uint32_t u = __float_as_uint(__fdiv_rn(amx, kFp8Max));
     const uint32_t e = ((u >> 23) & 0xFFu) + ((u & 0x007FFFFFu) != 0 ? 1u : 0u);
-    scale = __uint_as_float(e << 23);
-    inv = __uint_as_float((254u - e) << 23);
+    scale = __uint_as_float((e > 255u ? 255u : e) << 23);
+    inv = e >= 255u ? 0.0f : __uint_as_float((254u - e) << 23);
   } else {
     scale = __fdiv_rn(amx, kFp8Max);
     inv = __fdiv_rn(kFp8Max, amx);

@@ -268,7 +268,8 @@ def moe_ffn_contiguous(xq, sx, w1q, sw1, w2q, sw2, m_indices, threads: int = 0):
     bf16, h = swiglu(gate, up), h quantized per token per 128 channels with
     power-of-two scales, the second grouped GEMM. Returns (gu_bits [M][2I],
     hq [M][I], sh [M][I/128], y fp64 [M][H]); rows with m_indices < 0 are
-    computed as the grouped GEMM defines them (zero) and ignored by callers."""
+    undefined, as in the grouped GEMM (NaN values, NaN codes 0x7F), and are
+    ignored by callers."""
     I = w1q.shape[1] // 2
     gu = f64_to_bf16(grouped_contiguous(xq, sx, w1q, sw1, m_indices, threads))
     h = swiglu(gu[:, :I], gu[:, I:])

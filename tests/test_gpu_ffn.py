@@ -159,10 +159,10 @@ def test_ffn_masked_parity(fg, masked_m, M_max, H, I, expected):
         assert np.all(hq[e, v:] == SENT8)
 
 
-def test_ffn_contiguous_deepseek_expert_shape_sampled(fg):
+def test_ffn_contiguous_deepseek_expert_shape(fg):
     """An expert shape of the MoE layers (H = 7168, I = 2048) on the
-    contiguous workload's token counts: GU and Y on sampled outputs, the
-    requantization bit-exact on sampled rows."""
+    contiguous workload's token counts: every valid output of GU and Y, and the
+    requantization of every valid row bit for bit."""
     inp = workloads.make("contiguous_8x4096x7168")
     H, I = 7168, 2048
     mi = inp.m_indices
@@ -170,16 +170,11 @@ def test_ffn_contiguous_deepseek_expert_shape_sampled(fg):
     xq, sx = oracle.per_token_cast(inp.a, ue8m0=True)
     w1q, sw1, w2q, sw2 = _weights(rng, inp.G, H, I)
     gu, hq, sh, y = run_contiguous(fg, xq, sx, w1q, sw1, w2q, sw2, mi)
-    valid_rows = np.nonzero(mi >= 0)[0]
-    P = 8000
-    r = valid_rows[rng.integers(0, valid_rows.size, P)]
-    e = mi[r].astype(np.int64)
-    n1 = rng.integers(0, 2 * I, P)
-    ref1 = oracle.gemm_points(xq, sx, w1q, sw1, r, e, n1)
-    check_gemm(bf16_bits_to_f64(gu[r, n1]), ref1, "ffn GEMM1 full")
-    rows = valid_rows[rng.integers(0, valid_rows.size, 64)]
-    _check_requant(gu[rows], hq[rows], sh[rows], I, "ffn full")
-    n2 = rng.integers(0, H, P)
-    ref2 = oracle.gemm_points(hq, sh, w2q, sw2, r, e, n2)
-    check_gemm(bf16_bits_to_f64(y[r, n2]), ref2, "ffn GEMM2 full")
-    assert np.all(y[mi < 0] == SENT16)
+    valid = mi >= 0
+    ref1 = oracle.grouped_contiguous(xq, sx, w1q, sw1, mi)
+    check_gemm(bf16_bits_to_f64(gu[valid]), ref1[valid], "ffn GEMM1 full")
+    del ref1
+    _check_requant(gu[valid], hq[valid], sh[valid], I, "ffn full")
+    ref2 = oracle.grouped_contiguous(hq * valid[:, None], sh, w2q, sw2, mi)
+    check_gemm(bf16_bits_to_f64(y[valid]), ref2[valid], "ffn GEMM2 full")
+    assert np.all(y[~valid] == SENT16)

@@ -3,8 +3,8 @@ oracle through the C ABI.
 
 Operands are quantized by the oracle on the CPU and uploaded, so these tests
 isolate the GEMM kernels; the whole-path tests at the end quantize on the GPU
-too. Small cases are compared element by element over every valid output;
-full-size cases on sampled outputs the oracle computes one by one. The bar is
+too. Every case, full-size workloads included, is compared element by element
+over every valid output. The bar is
 |gpu - ref| <= 2^-7 |ref| + 1e-3 rms(ref) per element and a global
 1 - 2 sum(xy)/sum(x^2+y^2) < 1e-3; integer cases with power-of-two scales must
 be exact.
@@ -115,25 +115,16 @@ def test_dense_split_k_parity_and_determinism(fg, M, N, K):
     check_gemm(bf16_bits_to_f64(a), ref, "split-K %dx%dx%d" % (M, N, K))
 
 
-def _sampled_check(fg, got_bits, qa, sa, qb, sb, rows, experts, cols, what):
-    ref = oracle.gemm_points(qa, sa, qb, sb, rows, experts, cols)
-    return check_gemm(bf16_bits_to_f64(got_bits), ref, what)
-
-
 @pytest.mark.parametrize("name", ["decode_64x4096x7168", "prefill_4096x7168x2048",
                                   "prefill_4096x2112x7168"])
-def test_dense_full_size_sampled(fg, name):
+def test_dense_full_size(fg, name):
+    """Every output of the full-size dense shapes (the swapped split-K decode
+    shape and both prefill shapes, one with a ragged N) against the oracle."""
     inp = workloads.make(name)
     qa, sa, qb, sb = quantize_dense(inp)
     got = run_dense(fg, qa, sa, qb, sb)
-    rng = np.random.default_rng(99)
-    P = 20000
-    r = rng.integers(0, inp.M, P)
-    n = rng.integers(0, inp.N, P)
-    # include the last rows / columns (ragged tails)
-    r[:64] = inp.M - 1
-    n[64:128] = inp.N - 1
-    _sampled_check(fg, got[r, n], qa, sa, qb, sb, r, np.zeros(P, np.int64), n, name)
+    ref = oracle.gemm_nt(qa, sa, qb, sb)
+    check_gemm(bf16_bits_to_f64(got), ref, name)
 
 
 # ------------------------------------------------------------------ contiguous
@@ -188,19 +179,17 @@ def test_contiguous_padding_tiles_and_odd_runs(fg):
     assert np.all(got[~valid] == SENTINEL), "padding rows must stay unwritten"
 
 
-def test_contiguous_full_size_sampled(fg):
+def test_contiguous_full_size(fg):
+    """Every valid output of the 8-expert contiguous workload against the
+    oracle; padding rows stay unwritten."""
     inp = workloads.make("contiguous_8x4096x7168")
     qa, sa = oracle.per_token_cast(inp.a)
     qb, sb = oracle.per_block_cast(inp.b)
     got = run_contiguous(fg, qa, sa, qb, sb, inp.m_indices)
-    valid_rows = np.nonzero(inp.m_indices >= 0)[0]
-    rng = np.random.default_rng(7)
-    P = 20000
-    r = valid_rows[rng.integers(0, valid_rows.size, P)]
-    n = rng.integers(0, inp.N, P)
-    e = inp.m_indices[r].astype(np.int64)
-    _sampled_check(fg, got[r, n], qa, sa, qb, sb, r, e, n, "contiguous full")
-    assert np.all(got[inp.m_indices < 0] == SENTINEL)
+    ref = oracle.grouped_contiguous(qa, sa, qb, sb, inp.m_indices)
+    valid = inp.m_indices >= 0
+    check_gemm(bf16_bits_to_f64(got[valid]), ref[valid], "contiguous full")
+    assert np.all(got[~valid] == SENTINEL)
 
 
 # ------------------------------------------------------------------ masked
@@ -241,7 +230,9 @@ def test_masked_parity_small(fg, masked_m, M_max, N, K, expected):
         assert np.all(got[e, mv:] == SENTINEL), "rows past masked_m must stay unwritten"
 
 
-def test_masked_full_size_sampled(fg):
+def test_masked_full_size(fg):
+    """Every valid output of the 32-expert masked workload against the oracle;
+    A rows past masked_m hold e4m3 NaN codes and their D rows stay unwritten."""
     inp = workloads.make("masked_32x256x4096x7168")
     qa, sa = oracle.per_token_cast(inp.a)
     qb, sb = oracle.per_block_cast(inp.b)
@@ -250,21 +241,10 @@ def test_masked_full_size_sampled(fg):
         qa_nan[e, mv:] = 0x7F
     got, status = run_masked(fg, qa_nan, sa, qb, sb, inp.masked_m, 128)
     assert status == 0
-    rows, experts = [], []
-    for e, mv in enumerate(inp.masked_m):
-        rows += [e * inp.M_max + m for m in range(mv)]
-        experts += [e] * int(mv)
-        assert np.all(got[e, mv:] == SENTINEL)
-    rows = np.array(rows)
-    experts = np.array(experts)
-    rng = np.random.default_rng(3)
-    P = 20000
-    pick = rng.integers(0, rows.size, P)
-    r, e = rows[pick], experts[pick]
-    n = rng.integers(0, inp.N, P)
-    flat = got.reshape(-1, inp.N)
-    _sampled_check(fg, flat[r, n], qa.reshape(-1, inp.K), sa.reshape(-1, inp.K // 128), qb, sb,
-                   r, e, n, "masked full")
+    ref = oracle.grouped_masked(qa, sa, qb, sb, inp.masked_m)
+    valid = np.arange(inp.M_max)[None, :] < np.asarray(inp.masked_m)[:, None]
+    check_gemm(bf16_bits_to_f64(got[valid]), ref[valid], "masked full")
+    assert np.all(got[~valid] == SENTINEL)
 
 
 def test_masked_bad_count_sets_device_status(fg):

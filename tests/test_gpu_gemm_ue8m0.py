@@ -120,18 +120,13 @@ def test_dense_parity_small(fg, width, M, N, K):
 
 @pytest.mark.parametrize("name", ["prefill_4096x7168x2048", "prefill_4096x2112x7168",
                                   "decode_64x4096x7168"])
-def test_dense_full_size_sampled(fg, name):
+def test_dense_full_size(fg, name):
+    """Every output of the full-size dense shapes against the oracle."""
     inp = workloads.make(name)
     qa, sa, qb, sb = quantize_dense(inp)
     got = run_dense(fg, qa, sa, qb, sb)
-    rng = np.random.default_rng(98)
-    P = 20000
-    r = rng.integers(0, inp.M, P)
-    n = rng.integers(0, inp.N, P)
-    r[:64] = inp.M - 1
-    n[64:128] = inp.N - 1
-    ref = oracle.gemm_points(qa, sa, qb, sb, r, np.zeros(P, np.int64), n)
-    check_gemm(bf16_bits_to_f64(got[r, n]), ref, "ue8m0 " + name)
+    ref = oracle.gemm_nt(qa, sa, qb, sb)
+    check_gemm(bf16_bits_to_f64(got), ref, "ue8m0 " + name)
 
 
 # ------------------------------------------------------------------ grouped forms
@@ -187,20 +182,16 @@ def test_contiguous_padding_tiles_and_odd_runs(fg, width):
     assert np.all(got[~valid] == SENTINEL), "padding rows must stay unwritten"
 
 
-def test_contiguous_full_size_sampled(fg):
+def test_contiguous_full_size(fg):
+    """Every valid output of the 8-expert contiguous workload."""
     inp = workloads.make("contiguous_8x4096x7168")
     qa, sa = oracle.per_token_cast(inp.a, ue8m0=True)
     qb, sb = oracle.per_block_cast(inp.b, ue8m0=True)
     got = run_contiguous(fg, qa, sa, qb, sb, inp.m_indices)
-    valid_rows = np.nonzero(inp.m_indices >= 0)[0]
-    rng = np.random.default_rng(8)
-    P = 20000
-    r = valid_rows[rng.integers(0, valid_rows.size, P)]
-    n = rng.integers(0, inp.N, P)
-    e = inp.m_indices[r].astype(np.int64)
-    ref = oracle.gemm_points(qa, sa, qb, sb, r, e, n)
-    check_gemm(bf16_bits_to_f64(got[r, n]), ref, "ue8m0 contiguous full")
-    assert np.all(got[inp.m_indices < 0] == SENTINEL)
+    ref = oracle.grouped_contiguous(qa, sa, qb, sb, inp.m_indices)
+    valid = inp.m_indices >= 0
+    check_gemm(bf16_bits_to_f64(got[valid]), ref[valid], "ue8m0 contiguous full")
+    assert np.all(got[~valid] == SENTINEL)
 
 
 def run_masked(fg, qa, sa, qb, sb, masked_m, expected_m):
@@ -237,33 +228,24 @@ def test_masked_parity_small(fg, width, masked_m, M_max, N, K, expected):
         assert np.all(got[e, mv:] == SENTINEL), "rows past masked_m must stay unwritten"
 
 
-def test_masked_full_size_sampled(fg):
+def test_masked_full_size(fg):
+    """Every valid output of the 32-expert masked workload."""
     inp = workloads.make("masked_32x256x4096x7168")
     qa, sa = oracle.per_token_cast(inp.a, ue8m0=True)
     qb, sb = oracle.per_block_cast(inp.b, ue8m0=True)
     got, status = run_masked(fg, qa, sa, qb, sb, inp.masked_m, 128)
     assert status == 0
-    rows, experts = [], []
-    for e, mv in enumerate(inp.masked_m):
-        rows += [e * inp.M_max + m for m in range(mv)]
-        experts += [e] * int(mv)
-        assert np.all(got[e, mv:] == SENTINEL)
-    rows = np.array(rows)
-    experts = np.array(experts)
-    rng = np.random.default_rng(4)
-    P = 20000
-    pick = rng.integers(0, rows.size, P)
-    r, e = rows[pick], experts[pick]
-    n = rng.integers(0, inp.N, P)
-    ref = oracle.gemm_points(qa.reshape(-1, inp.K), sa.reshape(-1, inp.K // 128), qb, sb, r, e, n)
-    check_gemm(bf16_bits_to_f64(got.reshape(-1, inp.N)[r, n]), ref, "ue8m0 masked full")
+    ref = oracle.grouped_masked(qa, sa, qb, sb, inp.masked_m)
+    valid = np.arange(inp.M_max)[None, :] < np.asarray(inp.masked_m)[:, None]
+    check_gemm(bf16_bits_to_f64(got[valid]), ref[valid], "ue8m0 masked full")
+    assert np.all(got[~valid] == SENTINEL)
 
 
 # ------------------------------------------------------------------ whole path
 
 def test_whole_path_prefill_gpu_quantized(fg):
     """bf16 in -> GPU UE8M0 quantizers -> block-scaled GEMM, against the
-    oracle's UE8M0 quantizers and GEMM on sampled outputs."""
+    oracle's UE8M0 quantizers and GEMM on every output."""
     inp = workloads.make("prefill_4096x7168x2048")
     M, N, K = inp.M, inp.N, inp.K
     x = bf16_tensor(inp.a)
@@ -279,10 +261,88 @@ def test_whole_path_prefill_gpu_quantized(fg):
     torch.cuda.synchronize()
     assert fg.get_device_status() == 0
     qa, sa, qb, sb = quantize_dense(inp)
-    rng = np.random.default_rng(5)
-    P = 20000
-    r = rng.integers(0, M, P)
-    n = rng.integers(0, N, P)
-    ref = oracle.gemm_points(qa, sa, qb, sb, r, np.zeros(P, np.int64), n)
-    got = tensor_bf16_bits(D)
-    check_gemm(bf16_bits_to_f64(got[r, n]), ref, "ue8m0 whole path prefill")
+    ref = oracle.gemm_nt(qa, sa, qb, sb)
+    check_gemm(bf16_bits_to_f64(tensor_bf16_bits(D)), ref, "ue8m0 whole path prefill")
+
+
+# ------------------------------------------------------------------ scale check
+
+FG_DEVICE_BAD_SCALE = 5
+
+
+def _dense_ue8m0_status(fg, qa, sa, qb, sb):
+    M, K = qa.shape
+    D = _d_tensor((M, qb.shape[0]))
+    fg.fp8_gemm_nt_ue8m0(to_torch(qa), to_torch(sa_to_mn_major(sa)), to_torch(qb),
+                         to_torch(np.ascontiguousarray(sb, np.float32)), D)
+    torch.cuda.synchronize()
+    return fg.get_device_status()
+
+
+@pytest.mark.parametrize("which", ["token", "weight", "fp32 quantizer"])
+def test_non_power_of_two_scale_is_reported(fg, which):
+    """The block-scaled kernel keeps only a scale's exponent, so a scale with
+    mantissa bits (one token scale, one weight-block scale, or the amax/448
+    scales of the fp32 quantizers) cannot be applied: the call reports
+    FG_DEVICE_BAD_SCALE instead of returning a silently rounded product."""
+    inp = workloads.dense(256, 256, 512, seed=5)
+    ue8m0 = which != "fp32 quantizer"
+    qa, sa = oracle.per_token_cast(inp.a, ue8m0=ue8m0)
+    qb, sb = oracle.per_block_cast(inp.b, ue8m0=ue8m0)
+    sa, sb = sa.copy(), sb.copy()
+    if which == "token":
+        sa[17, 2] *= np.float32(1.5)
+    elif which == "weight":
+        sb[1, 3] *= np.float32(1.25)
+    assert _dense_ue8m0_status(fg, qa, sa, qb, sb) == FG_DEVICE_BAD_SCALE
+    assert fg.get_device_status() == 0  # the read cleared it
+    # the unmodified power-of-two scales pass the check
+    qa, sa = oracle.per_token_cast(inp.a, ue8m0=True)
+    qb, sb = oracle.per_block_cast(inp.b, ue8m0=True)
+    assert _dense_ue8m0_status(fg, qa, sa, qb, sb) == 0
+
+
+def test_zero_and_negative_scales(fg):
+    """Zero is accepted (it acts as 2^-127); a negative power of two is not a
+    scale the kernel can apply (only the exponent field is used)."""
+    inp = workloads.dense(256, 256, 256, seed=6)
+    qa, sa = oracle.per_token_cast(inp.a, ue8m0=True)
+    qb, sb = oracle.per_block_cast(inp.b, ue8m0=True)
+    sa = sa.copy()
+    sa[3, 1] = 0.0
+    assert _dense_ue8m0_status(fg, qa, sa, qb, sb) == 0
+    sa[3, 1] = -0.5
+    assert _dense_ue8m0_status(fg, qa, sa, qb, sb) == FG_DEVICE_BAD_SCALE
+
+
+def test_scales_of_rows_never_stored_are_not_checked(fg):
+    """Only the token scales of stored rows must be powers of two: masked rows
+    past masked_m and contiguous padding rows may hold any scale."""
+    G, M_max, N, K = 3, 256, 256, 256
+    mm = np.array([200, 0, 131], np.int32)
+    mi = workloads.masked(G, M_max, N, K, seed=9, masked_m=mm)
+    qa, sa = oracle.per_token_cast(mi.a, ue8m0=True)
+    qb, sb = oracle.per_block_cast(mi.b, ue8m0=True)
+    sa = sa.copy()
+    for e in range(G):
+        sa[e, mm[e]:, :] = np.float32(1.5)
+    got, status = run_masked(fg, qa, sa, qb, sb, mm, 128)
+    assert status == 0
+    ref = oracle.grouped_masked(qa, sa, qb, sb, mm)
+    for e in range(G):
+        if mm[e]:
+            check_gemm(bf16_bits_to_f64(got[e, :mm[e]]), ref[e, :mm[e]], "masked expert %d" % e)
+    # ... and the same scale on a stored row is reported
+    sa[0, 5, 0] = np.float32(1.5)
+    _, status = run_masked(fg, qa, sa, qb, sb, mm, 128)
+    assert status == FG_DEVICE_BAD_SCALE
+
+    ci = workloads.contiguous(N, K, counts=np.array([130, 5]), seed=10)
+    qa, sa = oracle.per_token_cast(ci.a, ue8m0=True)
+    qb, sb = oracle.per_block_cast(ci.b, ue8m0=True)
+    sa = sa.copy()
+    sa[ci.m_indices < 0, :] = np.float32(3.0)
+    got = run_contiguous(fg, qa, sa, qb, sb, ci.m_indices)  # asserts a clear status
+    valid = ci.m_indices >= 0
+    ref = oracle.grouped_contiguous(qa, sa, qb, sb, ci.m_indices)
+    check_gemm(bf16_bits_to_f64(got[valid]), ref[valid], "contiguous padding scales")

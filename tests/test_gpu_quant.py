@@ -115,6 +115,36 @@ def test_per_token_zero_padding_rows(fg):
     assert np.array_equal(q[0], qr) and np.array_equal(sa.view(np.uint32), sr.view(np.uint32))
 
 
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_slices_with_infinities_and_nan_bit_exact(fg, ue8m0):
+    """Infinities give the slice an infinite scale and zero codes (NaN for the
+    infinities themselves); NaN elements map to 0x7F without raising the
+    amax. Codes and scale bits equal the oracle's, per token and per block."""
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((130, 384), dtype=np.float32)
+    bits = workloads.bf16_bits(x)
+    bits[0, 7], bits[0, 9] = 0x7F80, 0xFF80      # +inf, -inf in slice (0, 0)
+    bits[0, 11], bits[5, 200] = 0x7FC0, 0x7FC0   # NaN with and without an inf
+    bits[129, 300] = 0xFF80                      # -inf in the N-tail block
+    sfx = "_ue8m0" if ue8m0 else ""
+    xt = bf16_tensor(bits[None])
+    q = torch.empty((1, 130, 384), dtype=torch.uint8, device="cuda")
+    s = torch.full((1, 3, fg.sfa_stride(130)), -1.0, dtype=torch.float32, device="cuda")
+    getattr(fg, "per_token_cast_to_fp8" + sfx)(xt, q, s)
+    qb = torch.empty((1, 130, 384), dtype=torch.uint8, device="cuda")
+    sb = fg.empty_sfb(1, 130, 384, "cuda")
+    getattr(fg, "per_block_cast_to_fp8" + sfx)(xt, qb, sb)
+    torch.cuda.synchronize()
+    qr, sr = oracle.per_token_cast(bits, ue8m0=ue8m0)
+    assert np.array_equal(q.cpu().numpy()[0], qr)
+    got_s = sa_from_mn_major(s.cpu().numpy(), 130)[0]
+    assert np.array_equal(got_s.view(np.uint32), sr.view(np.uint32))
+    assert np.isposinf(got_s[0, 0])
+    qbr, sbr = oracle.per_block_cast(bits, ue8m0=ue8m0)
+    assert np.array_equal(qb.cpu().numpy()[0], qbr)
+    assert np.array_equal(sb.cpu().numpy()[0].view(np.uint32), sbr.view(np.uint32))
+
+
 def test_quantizer_argument_errors(fg):
     x = torch.zeros((4, 100), dtype=torch.bfloat16, device="cuda")
     q = torch.zeros((4, 100), dtype=torch.uint8, device="cuda")

@@ -147,6 +147,39 @@ def test_per_token_invariants():
     assert np.all(q[5, 128:256] == 0)
 
 
+def test_slices_with_infinities_and_nan():
+    """A slice holding +-inf has amax = inf, so its scale is +inf in both modes
+    and every element maps to x / inf: finite elements to a zero code with
+    their own sign, infinities (inf / inf) and NaN to the NaN code 0x7F. NaN
+    elements do not raise the amax; a slice of NaN and finite values quantizes
+    like its finite values."""
+    x = np.zeros((2, 256), np.float32)
+    x[0, :128] = np.linspace(-3.0, 3.0, 128, dtype=np.float32)
+    x[0, 7], x[0, 9], x[0, 11] = np.inf, -np.inf, np.nan
+    x[1, :128] = np.linspace(-1.0, 1.0, 128, dtype=np.float32)
+    x[1, 40] = np.nan
+    x[:, 128:] = np.linspace(0.5, 2.0, 128, dtype=np.float32)
+    bits = workloads.bf16_bits(np.nan_to_num(x, nan=0.0, posinf=0.0, neginf=0.0))
+    bits[0, 7], bits[0, 9], bits[0, 11], bits[1, 40] = 0x7F80, 0xFF80, 0x7FC0, 0x7FC0
+    finite = workloads.bf16_to_f32(bits)
+    for ue8m0 in (False, True):
+        q, s = oracle.per_token_cast(bits, ue8m0=ue8m0)
+        assert np.isposinf(s[0, 0])
+        expect = np.where(np.signbit(finite[0, :128]), 0x80, 0x00).astype(np.uint8)
+        expect[[7, 9, 11]] = 0x7F
+        assert np.array_equal(q[0, :128], expect)
+        # the NaN element alone is 0x7F; the rest quantizes as without it
+        clean = bits[1:2, :128].copy()
+        clean[0, 40] = 0
+        qc, sc = oracle.per_token_cast(clean, ue8m0=ue8m0)
+        assert s[1, 0] == sc[0, 0] and q[1, 40] == 0x7F
+        rest = np.arange(128) != 40
+        assert np.array_equal(q[1, :128][rest], qc[0][rest])
+        # the other slices are untouched
+        q2, s2 = oracle.per_token_cast(bits[:, 128:], ue8m0=ue8m0)
+        assert np.array_equal(q[:, 128:], q2) and np.array_equal(s[:, 1:], s2)
+
+
 def test_per_token_power_of_two_slices_are_exact():
     K = 256
     j = np.arange(-14, 2)                          # 16 powers of two, max 2
