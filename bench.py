@@ -364,9 +364,18 @@ def max_over_ranks(dist, values, device):
 
 # ---------------------------------------------------------------------- GPU leg
 
+def ffn_one_launch(inp) -> bool:
+    """The library's automatic choice of the expert FFN's form for a contiguous
+    batch: one launch when an expert's rows (M_total / G) are at most 128."""
+    return inp.M_total // inp.G <= 128
+
+
 def gemm_kernel_name(kind: str, inp, ue8m0: bool) -> str:
     """The GEMM kernel a step launches (the library's choice for the shape)."""
     if kind == "ffn":
+        if ffn_one_launch(inp):
+            return ("fp8_gemm_mx_kernel (both expert GEMMs in one launch: first GEMM with fused "
+                    "SwiGLU + requantization, then second GEMM)")
         return "fp8_gemm_mx_kernel x2 (first GEMM with fused SwiGLU + requantization, second GEMM)"
     if kind == "kgrouped":
         return "fp8_gemm_mx_kernel (K-grouped, fp32 output)"
@@ -407,6 +416,8 @@ class OperandSet:
             self.Hq = torch.empty((M, I), dtype=torch.uint8, device=dev)
             self.SH = fg.empty_sfa(1, M, I, dev)
             self.D = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+            # the one-kernel FFN's ready counters (cleared by every call)
+            self.WS = fg.empty_ffn_workspace(fg.FG_LAYOUT_CONTIGUOUS, M, inp.G, dev)
             self.extra = [self.W2, self.SW2, self.Hq, self.SH]
             return
         if kind == "dense":
@@ -502,7 +513,7 @@ class Step:
             self.fg.fp8_k_grouped_gemm_nt_ue8m0(o.A, o.SA[0], o.B, o.SB[0], o.D, self.ks)
         elif self.kind == "ffn":
             self.fg.fp8_moe_ffn_contiguous_ue8m0(o.A, o.SA, o.B, o.SB, o.W2, o.SW2, o.Hq, o.SH, o.D,
-                                                 self.mi)
+                                                 self.mi, ws=o.WS)
         elif self.kind == "dense":
             self.g_dense(o.A, o.SA, o.B, o.SB, o.D)
         elif self.kind == "contiguous":
@@ -511,7 +522,14 @@ class Step:
             self.g_masked(o.A, o.SA, o.B, o.SB, o.D, self.mm, self.expected_m)
 
     def launches_per_step(self):
-        return (3 if self.kind in ("ffn", "kgrouped") else 2) + (1 if self.with_wq else 0)
+        """Kernels of this library per step: the activation quantizer and the
+        GEMM; the FFN's two GEMMs are two kernels, or one in its one-launch
+        form (whose counter reset is a memset, not a kernel); K-grouped: two
+        quantizers and the GEMM."""
+        n = 3 if self.kind == "kgrouped" else 2
+        if self.kind == "ffn" and not ffn_one_launch(self.inp):
+            n = 3
+        return n + (1 if self.with_wq else 0)
 
     def run(self, i):
         o = self.sets[i % len(self.sets)]

@@ -229,9 +229,17 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
  *   Hq, sfh = per_token_cast_to_fp8_ue8m0(h)
  *   Y  = bf16(Hq W2_e^T)           (second grouped GEMM; W2_e is H x I)
  * the single-GPU part of the "Mega MoE" kernel, which fuses both expert GEMMs
- * with the SwiGLU activation ("DeepGEMM" overview, section "swapAB与Mega MoE").
- * The SwiGLU and the requantization run in the first GEMM's epilogue (no bf16
- * intermediate goes to memory); the second GEMM is fp8_grouped_gemm_*_ue8m0.
+ * with the SwiGLU activation in one kernel ("DeepGEMM" overview, section
+ * "swapAB与Mega MoE"). The first GEMM's tiles run the SwiGLU and the
+ * requantization in their epilogue (no bf16 intermediate goes to memory).
+ * For decode-sized batches (at most 128 expected rows per expert) one
+ * persistent launch computes both GEMMs: the first GEMM's tiles count up a
+ * ready counter per 128-token tile once its quantized activations are
+ * written; the second GEMM's tiles come after them in every CTA's work list
+ * and wait (bounded) for their token tile's counter, so the second GEMM starts
+ * on finished token tiles while the first GEMM's last tiles still run, with no
+ * second launch. Larger batches run the two GEMMs as two launches, which is
+ * faster there (see fg_set_ffn_mode).
  * Scales must be powers of two (as for the _ue8m0 GEMMs).
  * Contiguous: X e4m3 [M_total][H], sfx MN-major [H/128][stride(M_total)],
  *   m_indices int32 [M_total] (contract of fp8_grouped_gemm_contiguous);
@@ -242,18 +250,33 @@ fg_status fp8_grouped_gemm_masked_ue8m0(const uint8_t* A, const float* sfa, cons
  * sfw2 [G][H/128][I/128]. GU: optional (NULL = not written) bf16 [rows][2I]
  * output of the first GEMM (gate columns, then up columns), which the SwiGLU
  * backward pass needs. Hq, sfh and Y (and GU) are written on valid rows only.
+ * ws: device workspace of at least fg_moe_ffn_workspace_bytes(layout, M, G)
+ *   bytes (M = M_total or M_max), 16-byte aligned, owned by the caller, for
+ *   the ready counters of the one-launch form (required for both forms); the
+ *   call clears the counters it uses (cudaMemsetAsync on `stream`) before its
+ *   kernel, so the workspace needs no initialisation, and two calls in flight
+ *   at once must not share it. Smaller: FG_ERR_INVALID_ARG.
  * H % 128 == 0, I % 128 == 0, G >= 1; other limits as for the grouped GEMMs.
  */
+#define FG_LAYOUT_CONTIGUOUS 0
+#define FG_LAYOUT_MASKED 1
+/* Form of the expert FFN (process-wide): 0 = automatic (one launch when the
+ * expected rows per expert, expected_m or M_total / G, are at most 128, else
+ * two launches), 1 = always one launch, 2 = always two launches. Other
+ * values: FG_ERR_INVALID_ARG. */
+fg_status fg_set_ffn_mode(int mode);
+/* Workspace bytes of the expert FFN (0 for invalid arguments). */
+size_t fg_moe_ffn_workspace_bytes(int layout, int M, int G);
 fg_status fp8_moe_ffn_contiguous_ue8m0(const uint8_t* X, const float* sfx, const uint8_t* W1,
                                       const float* sfw1, const uint8_t* W2, const float* sfw2,
                                       uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
                                       const int32_t* m_indices, int M_total, int H, int I, int G,
-                                      cudaStream_t stream);
+                                      void* ws, size_t ws_bytes, cudaStream_t stream);
 fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uint8_t* W1,
                                   const float* sfw1, const uint8_t* W2, const float* sfw2,
                                   uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
                                   const int32_t* masked_m, int G, int M_max, int H, int I,
-                                  int expected_m, cudaStream_t stream);
+                                  int expected_m, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * K-grouped GEMM with power-of-two scales, for the weight gradients of MoE

@@ -39,7 +39,8 @@ EXPORTED = (
     "per_token_cast_to_fp8_ue8m0", "per_block_cast_to_fp8_ue8m0", "fp8_gemm_nt",
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
     "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
-    "fg_set_ue8m0_tile", "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
+    "fg_set_ue8m0_tile", "fg_set_ffn_mode", "fg_moe_ffn_workspace_bytes", "fp8_moe_ffn_contiguous_ue8m0",
+    "fp8_moe_ffn_masked_ue8m0",
     "fp8_k_grouped_gemm_nt_ue8m0",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
@@ -79,8 +80,12 @@ def load_library() -> ctypes.CDLL:
     lib.fp8_grouped_gemm_contiguous_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fp8_grouped_gemm_masked_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
     lib.fg_set_ue8m0_tile.argtypes = [I, I]
-    lib.fp8_moe_ffn_contiguous_ue8m0.argtypes = [P] * 11 + [I, I, I, I, P]
-    lib.fp8_moe_ffn_masked_ue8m0.argtypes = [P] * 11 + [I, I, I, I, I, P]
+    Z = ctypes.c_size_t
+    lib.fg_set_ffn_mode.argtypes = [I]
+    lib.fg_moe_ffn_workspace_bytes.argtypes = [I, I, I]
+    lib.fg_moe_ffn_workspace_bytes.restype = Z
+    lib.fp8_moe_ffn_contiguous_ue8m0.argtypes = [P] * 11 + [I, I, I, I, P, Z, P]
+    lib.fp8_moe_ffn_masked_ue8m0.argtypes = [P] * 11 + [I, I, I, I, I, P, Z, P]
     lib.fp8_k_grouped_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
@@ -93,7 +98,7 @@ def load_library() -> ctypes.CDLL:
               "fp8_gemm_nt",
               "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked",
               "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0",
-              "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile",
+              "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile", "fg_set_ffn_mode",
               "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
               "fp8_k_grouped_gemm_nt_ue8m0",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
@@ -279,32 +284,59 @@ def fp8_grouped_gemm_masked_ue8m0(A: torch.Tensor, sfa: torch.Tensor, B: torch.T
                  expected_m, stream)
 
 
+FG_LAYOUT_CONTIGUOUS = 0
+FG_LAYOUT_MASKED = 1
+
+
+def set_ffn_mode(mode: int) -> None:
+    """Expert FFN form: 0 automatic, 1 one launch, 2 two launches."""
+    _check(load_library().fg_set_ffn_mode(int(mode)))
+
+
+def moe_ffn_workspace_bytes(layout: int, M: int, G: int) -> int:
+    """Bytes of the workspace the expert FFN needs (M = M_total or M_max)."""
+    return int(load_library().fg_moe_ffn_workspace_bytes(layout, M, G))
+
+
+def empty_ffn_workspace(layout: int, M: int, G: int, device="cuda"):
+    """A workspace for the expert FFN (its contents need no initialisation)."""
+    n = max(moe_ffn_workspace_bytes(layout, M, G), 256)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
 def fp8_moe_ffn_contiguous_ue8m0(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, m_indices, GU=None,
-                                 stream=None) -> None:
+                                 ws=None, stream=None) -> None:
     """Expert FFN (contiguous layout): X uint8 [M_total][H], W1 uint8 [G][2I][H],
     W2 uint8 [G][H][I] -> Hq uint8 [M_total][I], sfh [I/128][stride], Y bf16
-    [M_total][H] (and GU bf16 [M_total][2I] if given)."""
+    [M_total][H] (and GU bf16 [M_total][2I] if given). ws: the workspace (a
+    torch tensor; one is allocated when it is not given)."""
     M_total, H = X.shape
     G, I2, _ = W1.shape
     if m_indices.dtype != torch.int32 or m_indices.numel() != M_total:
         raise FP8GemmError(FG_ERR_INVALID_ARG, "m_indices must be int32 [M_total]")
+    if ws is None:
+        ws = empty_ffn_workspace(FG_LAYOUT_CONTIGUOUS, M_total, G, X.device)
     _check(load_library().fp8_moe_ffn_contiguous_ue8m0(
         _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
-        _ptr(GU), _ptr(Y), _ptr(m_indices), M_total, H, I2 // 2, G, _stream(stream)))
+        _ptr(GU), _ptr(Y), _ptr(m_indices), M_total, H, I2 // 2, G, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def fp8_moe_ffn_masked_ue8m0(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, masked_m, expected_m,
-                             GU=None, stream=None) -> None:
+                             GU=None, ws=None, stream=None) -> None:
     """Expert FFN (masked layout): X uint8 [G][M_max][H] -> Hq [G][M_max][I],
-    sfh [G][I/128][stride], Y bf16 [G][M_max][H] (and GU [G][M_max][2I])."""
+    sfh [G][I/128][stride], Y bf16 [G][M_max][H] (and GU [G][M_max][2I]).
+    ws as for the contiguous form."""
     G, M_max, H = X.shape
     I2 = W1.shape[1]
     if masked_m.dtype != torch.int32 or masked_m.numel() != G:
         raise FP8GemmError(FG_ERR_INVALID_ARG, "masked_m must be int32 [G]")
+    if ws is None:
+        ws = empty_ffn_workspace(FG_LAYOUT_MASKED, M_max, G, X.device)
     _check(load_library().fp8_moe_ffn_masked_ue8m0(
         _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
-        _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m),
-        _stream(stream)))
+        _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def fp8_k_grouped_gemm_nt_ue8m0(A, sfa, B, sfb, D, ks, stream=None) -> None:

@@ -94,6 +94,15 @@ struct GemmParams {
   // (device) and the fp32 output [G][M][N]
   const int32_t* ks;
   float* d32;
+  // one-kernel expert FFN (both GEMMs in one persistent launch): the second
+  // GEMM's weight rows (H), K blocks (I / 128), weight-block rows and tiles,
+  // its weight-block scales, and the per-token-tile ready counters in global
+  // scratch (zero at launch; the first GEMM's epilogue warps count up, the
+  // second GEMM's loads of a token tile wait for ready_target)
+  int N2, KB2, NB2, num_nt2;
+  const float* sfb2;
+  int* ready;
+  int ready_target;
 };
 
 template <int BT_, int BW_, bool SWAP_, int STAGES_, int PW_, int SPLIT_, int KPS_ = 2,
@@ -211,6 +220,8 @@ struct Tile {
   int nt;     // weight tile
   int kb0;    // first K block (block-scaled kernel; K-grouped: the expert's first token block)
   int nkb;    // K blocks of the tile
+  int phase;  // one-kernel expert FFN: 0 = first GEMM (+ SwiGLU, requant), 1 = second GEMM
+  int owned;  // one-kernel expert FFN: the token tile's rows belong to this tile's expert
 };
 
 template <class C, int FORM>

@@ -99,7 +99,12 @@ namespace fg {
 
 template <int BW_, int STAGES_, int ACC_, int EPQ_, bool PAIR_, int KPS_, int EPI_ = 0>
 struct MxCfg {
-  static constexpr int EPI = EPI_;        // 0: bf16 D; 1: SwiGLU + UE8M0 requantization; 2: K-grouped, fp32 D
+  // 0: bf16 D; 1: SwiGLU + UE8M0 requantization; 2: K-grouped, fp32 D;
+  // 3: the whole expert FFN in one launch (first-GEMM tiles with the EPI = 1
+  // epilogue, then second-GEMM tiles with a bf16 epilogue)
+  static constexpr int EPI = EPI_;
+  static constexpr bool FFN = EPI == 1 || EPI == 3;  // tiles of 128 gate + 128 up weight rows
+  static constexpr bool FUSED = EPI == 3;
   static constexpr int BT = 128;          // token rows per CTA tile
   static constexpr int BW = BW_;          // weight rows per tile (MMA N)
   static constexpr bool SWAP = false;     // tile helpers of gemm.cuh: tokens on the lanes
@@ -114,10 +119,12 @@ struct MxCfg {
   static constexpr int EPQ = EPQ_;        // epilogue warps per TMEM lane quadrant
   static_assert(BW % 32 == 0 && BW >= 32 && BW <= 256, "tcgen05 N, 32-column chunks");
   static_assert(!PAIR || B_ROWS % 16 == 0, "pair: half tiles of whole 8-row swizzle atoms");
-  static_assert(EPI != 1 || (BW == 256 && ACC == 1 && EPQ == 1),
+  static_assert(!FFN || (BW == 256 && ACC == 1 && EPQ == 1),
                 "fused FFN epilogue: 128 gate + 128 up columns, one accumulator, one warp per quadrant");
   // weight rows per tensor load: the fused FFN tile is two 128-row blocks
-  static constexpr int B_BOX = EPI == 1 ? 128 : B_ROWS;
+  // (the second GEMM's tiles of the one-kernel FFN load 128 consecutive rows
+  // per box as well)
+  static constexpr int B_BOX = FFN ? 128 : B_ROWS;
   static constexpr int B_LOADS = B_ROWS / B_BOX;
   static constexpr int EW = 4 * EPQ;      // epilogue warps
   static constexpr int ECOLS = BW / EPQ;  // accumulator columns per epilogue warp
@@ -131,14 +138,25 @@ struct MxCfg {
   static constexpr int SFS = 3;           // scale slots (quads in flight)
   // staged fp32 scales of a quad: 4 x 128 token scales (one TMA box), then
   // 4 x NBT weight-block scales ([k][j]: K block 4q + k, block nb0 + j)
-  static constexpr int NBT = EPI == 1 ? 2 : SFB_GROUPS + 1;
+  // one-kernel FFN: the second GEMM's tiles are BW2 = 224 weight rows wide
+  // with two accumulators (the tile's K loop is short, so its epilogue must
+  // overlap the next tile's MMAs); tensor memory: the first GEMM's 256-column
+  // accumulator at column 0, the second GEMM's two at 0 and BW2, then the
+  // scale slots. Staged weight-block scales: 2 for the first GEMM (gate, up),
+  // up to 3 for a 224-row tile of the second.
+  static constexpr int BW2 = FUSED ? 224 : BW;
+  static constexpr int B_ROWS2 = PAIR ? BW2 / 2 : BW2;
+  static constexpr int ACCB = FUSED ? 2 : ACC;  // accumulator barrier pairs
+  static constexpr int SF_BASE = FUSED ? 2 * BW2 : ACC * BW;
+  static_assert(!FUSED || (2 * BW2 >= BW && B_ROWS2 % 16 == 0 && B_ROWS2 <= 256), "second-GEMM tiles");
+  static constexpr int NBT = FUSED ? 3 : (FFN ? 2 : SFB_GROUPS + 1);
   static constexpr int RAW_A = 4 * 512;
   // K-grouped: per-row weight scales, BW rows x 4 K blocks (one TMA box)
   static constexpr int RAW_B = EPI == 2 ? 4 * BW * 4 : 128;
   static constexpr int RAW_BYTES = RAW_A + (RAW_B + 127) / 128 * 128;
   static constexpr int RAWS = 2;          // staged-scale ring
   static_assert(EPI == 2 || 4 * NBT * 4 <= RAW_BYTES - RAW_A, "staged weight-block scales");
-  static constexpr int TMEM_USED = ACC * BW + SFS * SF_COLS;
+  static constexpr int TMEM_USED = SF_BASE + SFS * SF_COLS;
   static_assert(TMEM_USED <= 512, "TMEM has 512 columns");
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
                                    : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
@@ -155,8 +173,8 @@ struct MxCfg {
   static constexpr int OFF_SF = OFF_B + STAGES * STAGE_B;
   static constexpr int OFF_RAW = OFF_SF + SFS * SF_BYTES;  // 128-byte aligned
   static constexpr int OFF_EPI = (OFF_RAW + RAWS * RAW_BYTES + 1023) / 1024 * 1024;
-  static constexpr int OFF_BAR = OFF_EPI + (EPI == 1 ? 0 : EW * EPI_RING * BOX_BYTES);  // (the fused FFN stages no D)
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * SFS + 2 * RAWS + 2 * ACC;
+  static constexpr int OFF_BAR = OFF_EPI + (FFN ? 0 : EW * EPI_RING * BOX_BYTES);  // (the FFN epilogues stage nothing)
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * SFS + 2 * RAWS + 2 * ACCB;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TABLE = (OFF_MISC + 16 + 15) / 16 * 16;
   // grouped layouts: token-tile table; contiguous pairs: + the pair-unit table
@@ -273,7 +291,9 @@ __device__ void mx_build_table(const GemmParams& p, int* table, int* num_units, 
       }
       int rows = (mm + C::BT - 1) / C::BT;  // token tiles
       if (C::PAIR) rows = (rows + 1) / 2;    // ... or tile pairs
-      const int cnt = rows * p.num_nt;
+      // (one-kernel FFN: the prefix counts token tiles or pairs; both GEMMs'
+      // tiles are laid over them)
+      const int cnt = C::FUSED ? rows : rows * p.num_nt;
       table[e + 1] = cnt;
       local += cnt;
     }
@@ -292,8 +312,16 @@ __device__ void mx_build_table(const GemmParams& p, int* table, int* num_units, 
   }
 }
 
+// One-kernel FFN: token tiles (contiguous, single CTAs), pair units
+// (contiguous pairs) or the masked prefix's tiles / pairs.
+template <class C, int FORM>
+__device__ __forceinline__ int mx_ffn_units(const GemmParams& p, const int* table, int num_units) {
+  return FORM == kFormMasked ? table[p.G] : (C::PAIR ? num_units : p.num_mt);
+}
+
 template <class C, int FORM>
 __device__ __forceinline__ int mx_total(const GemmParams& p, const int* table, int num_units) {
+  if (C::FUSED) return mx_ffn_units<C, FORM>(p, table, num_units) * (p.num_nt + p.num_nt2);
   if (FORM == kFormMasked) return table[p.G];
   if (FORM == kFormKGrouped) return p.G * (C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
   if (FORM == kFormContig && C::PAIR) return num_units * p.num_nt;
@@ -301,12 +329,50 @@ __device__ __forceinline__ int mx_total(const GemmParams& p, const int* table, i
 }
 
 // Work item t of this CTA (rank = its place in the pair; 0 without pairs).
+// One-kernel FFN: items [0, t1) are the first GEMM's tiles, unit by unit (the
+// num_nt tiles of a token tile or pair unit are consecutive), then the second
+// GEMM's in the same order; `owned` says whether this CTA's token tile is the
+// unit's own (a contiguous odd run's partner tile belongs to another expert
+// or lies past the last tile; a masked pair's second tile may lie past M_max).
 template <class C, int FORM>
-__device__ __forceinline__ Tile mx_resolve(const GemmParams& p, const int* table, int t, int rank) {
+__device__ __forceinline__ Tile mx_resolve(const GemmParams& p, const int* table, int t, int rank,
+                                           int t1 = 0) {
   Tile w;
   w.valid = 1;
   w.kb0 = 0;
   w.nkb = p.KB;
+  w.phase = 0;
+  w.owned = 1;
+  if constexpr (C::FUSED) {
+    w.phase = t >= t1 ? 1 : 0;
+    const int local = w.phase ? t - t1 : t;
+    const int nts = w.phase ? p.num_nt2 : p.num_nt;
+    const int u = local / nts;
+    w.nt = local % nts;
+    w.nkb = w.phase ? p.KB2 : p.KB;
+    if (FORM == kFormMasked) {
+      int lo = 0, hi = p.G;  // table[lo] <= u < table[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (table[mid] <= u) lo = mid; else hi = mid;
+      }
+      const int li = u - table[lo];
+      w.e = lo;
+      w.mt = C::PAIR ? 2 * li + rank : li;
+      w.owned = w.mt < p.num_mt;
+    } else if (C::PAIR) {
+      const int mt0 = table[kTableMax + u];
+      w.e = table[mt0];
+      w.mt = mt0 + rank;
+      w.owned = w.mt < p.num_mt && table[w.mt] == w.e;
+    } else {
+      w.mt = u;
+      w.e = table[u];
+      w.valid = w.e >= 0;
+      w.owned = w.valid;
+    }
+    return w;
+  }
   if (FORM == kFormKGrouped) {
     const int per = (C::PAIR ? (p.num_mt + 1) / 2 : p.num_mt) * p.num_nt;
     w.e = t / per;
@@ -343,6 +409,34 @@ __device__ __forceinline__ Tile mx_resolve(const GemmParams& p, const int* table
   return w;
 }
 
+// Accumulator of a CTA's next tile: the tiles take the accumulators in turn
+// (ACC of them); the one-kernel FFN's first-GEMM tiles always use the
+// 256-column accumulator 0, its second-GEMM tiles alternate between two
+// 224-column ones starting with 0 (so the first of them waits for the last
+// first-GEMM tile's epilogue, whose columns the second one overlaps).
+// uses(b) counts the tiles accumulator b has held (its barriers' parity);
+// k1 counts the second-GEMM tiles seen.
+template <class C>
+struct AccTurn {
+  static_assert(C::ACCB == 1 || C::ACCB == 2, "one or two accumulators");
+  uint32_t u0 = 0, u1 = 0;  // tiles accumulator 0 / 1 has held (its barriers' parity)
+  uint32_t tiles = 0, k1 = 0;
+  __device__ __forceinline__ int next(const Tile& w) const {
+    if constexpr (C::FUSED) return w.phase ? static_cast<int>(k1 & 1u) : 0;
+    return static_cast<int>(tiles % C::ACC);
+  }
+  __device__ __forceinline__ uint32_t uses(int b) const { return b ? u1 : u0; }
+  __device__ __forceinline__ void done(const Tile& w, int b) {
+    if (b) ++u1; else ++u0;
+    ++tiles;
+    if (C::FUSED && w.phase) ++k1;
+  }
+  // first tensor-memory column of accumulator b for tile w
+  __device__ __forceinline__ static uint32_t column(const Tile& w, int b) {
+    return static_cast<uint32_t>(C::FUSED ? (w.phase ? b * C::BW2 : 0) : b * C::BW);
+  }
+};
+
 // Position in a ring of N slots, advanced one use at a time: slot index and
 // the parity of the slot's current phase.
 template <int N>
@@ -360,7 +454,9 @@ template <class C, int FORM>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                       const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
+                       const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmA2,
+                       const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmSA2,
+                       const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem + C::OFF_A;
@@ -374,7 +470,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   uint64_t* sa_full = sf_empty + C::SFS;    // a quad's fp32 scales have landed
   uint64_t* sa_empty = sa_full + C::RAWS;   // ... and the converter has read them
   uint64_t* tfull = sa_empty + C::RAWS;     // an accumulator holds a finished tile
-  uint64_t* tempty = tfull + C::ACC;        // ... and has been read by the epilogue
+  uint64_t* tempty = tfull + C::ACCB;       // ... and has been read by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* table = reinterpret_cast<int*>(smem + C::OFF_TABLE);
@@ -400,7 +496,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       mbar_init(&sa_full[r], C::EPI == 2 ? 1 : 2);
       mbar_init(&sa_empty[r], 1);  // the converter
     }
-    for (int b = 0; b < C::ACC; ++b) {
+    for (int b = 0; b < C::ACCB; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::CLUSTER * C::EW);  // one arrival per epilogue warp (of both CTAs)
     }
@@ -410,7 +506,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmSA);
     if (C::EPI == 2) tma_prefetch_desc(&tmSB);
-    if (C::EPI != 1) tma_prefetch_desc(&tmD);
+    if (!C::FFN) tma_prefetch_desc(&tmD);
+    if (C::FUSED) {
+      // the second GEMM's operands: the quantized activations, W2 and sfh
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+      tma_prefetch_desc(&tmSA2);
+    }
   }
   if constexpr (!C::PAIR) {
     if (warp == 1) {
@@ -440,9 +542,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_sf = tmem_base + static_cast<uint32_t>(C::ACC * C::BW);
+  const uint32_t tmem_sf = tmem_base + static_cast<uint32_t>(C::SF_BASE);
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   const int total = mx_total<C, FORM>(p, table, *num_units);
+  // one-kernel FFN: the first GEMM's items come first
+  const int t1 = C::FUSED ? mx_ffn_units<C, FORM>(p, table, *num_units) * p.num_nt : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -450,19 +554,35 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       Ring<C::STAGES> st;
       uint32_t fills = 0;
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+        const Tile w = mx_resolve<C, FORM>(p, table, t, rank, t1);
         if (!w.valid) continue;
         // fused FFN: gate block nt*128.. and up block I + nt*128.. of the
         // expert's 2I rows (a pair's CTAs load one block each)
         // (K-grouped: B is one matrix whose K range the experts share)
-        const int b_base = FORM == kFormKGrouped ? 0 : w.e * p.N;
-        const int row = lane == 0 ? (C::EPI == 1 ? b_base + (C::PAIR ? rank : 0) * p.I + w.nt * 128
-                                                 : b_base + w.nt * C::BW + rank * C::B_ROWS)
+        // (one-kernel FFN, second GEMM: BW consecutive rows of the expert's
+        // W2 and the tile's rows of the quantized activations)
+        const bool ffn_tile = C::EPI == 1 || (C::FUSED && w.phase == 0);
+        const bool second = C::FUSED && w.phase == 1;
+        const int b_base = FORM == kFormKGrouped ? 0 : w.e * (second ? p.N2 : p.N);
+        const int row = lane == 0 ? (ffn_tile ? b_base + (C::PAIR ? rank : 0) * p.I + w.nt * 128
+                                   : second ? b_base + w.nt * C::BW2 + rank * C::B_ROWS2
+                                            : b_base + w.nt * C::BW + rank * C::B_ROWS)
                                   : (FORM == kFormMasked ? w.e * p.M : 0) + w.mt * C::BT;
-        const CUtensorMap* map = lane == 0 ? &tmB : &tmA;
-        const uint32_t bytes = lane == 0 ? C::B_BYTES : C::A_BYTES;
-        const int loads = lane == 0 ? C::B_LOADS : 1;  // tensor loads per K block
-        const int load_step = C::EPI == 1 ? p.I : 0;   // rows between them
+        const CUtensorMap* map = lane == 0 ? (second ? &tmB2 : &tmB) : (second ? &tmA2 : &tmA);
+        // K block j of a stage sits at j * stride; `bytes` of it are loaded
+        // (the second GEMM's B_ROWS2-row weight tiles leave the rest unused)
+        const uint32_t stride = lane == 0 ? C::B_BYTES : C::A_BYTES;
+        const uint32_t bytes = lane == 0 ? (second ? C::B_ROWS2 * 128 : C::B_BYTES) : C::A_BYTES;
+        const int loads = lane == 0 && !second ? C::B_LOADS : 1;  // tensor loads per K block
+        const int load_step = ffn_tile ? p.I : C::B_BOX;         // rows between them
+        if (second && lane == 1 && w.owned) {
+          // the tile's quantized activations are complete (every first-GEMM
+          // tile of this token tile has published its rows)
+          const int ri = (FORM == kFormMasked ? w.e * p.num_mt : 0) + w.mt;
+          if (!wait_counter(p.ready + ri, p.ready_target, abort_flag, p.status, p.timeout_ns))
+            goto producer_done;
+          fence_proxy_async_global();  // the tensor loads below read them
+        }
         for (int kb0 = 0; kb0 < w.nkb; kb0 += C::KPS, st.next(), ++fills) {
           if (!mbar_wait(&empty[st.slot], st.phase ^ 1u, ctl)) goto producer_done;
           const int nk = min(C::KPS, w.nkb - kb0);
@@ -474,13 +594,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             const uint32_t bar = mapa_shared(smem_u32(&full[st.slot]), 0);
             for (int j = 0; j < nk; ++j)
               for (int h = 0; h < loads; ++h)
-                tma_load_2d_pair(dst + j * bytes + h * C::B_BOX * 128, map, bar, kx + j * 128,
+                tma_load_2d_pair(dst + j * stride + h * C::B_BOX * 128, map, bar, kx + j * 128,
                                  row + h * load_step);
           } else {
             mbar_arrive_expect_tx(&full[st.slot], nk * bytes);
             for (int j = 0; j < nk; ++j)
               for (int h = 0; h < loads; ++h)
-                tma_load_2d(dst + j * bytes + h * C::B_BOX * 128, map, &full[st.slot], kx + j * 128,
+                tma_load_2d(dst + j * stride + h * C::B_BOX * 128, map, &full[st.slot], kx + j * 128,
                             row + h * load_step);
           }
         }
@@ -500,18 +620,29 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       Ring<C::RAWS> rr;
       uint32_t fills = 0;
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+        const Tile w = mx_resolve<C, FORM>(p, table, t, rank, t1);
         if (!w.valid) continue;
         // weight blocks the tile's rows touch (clamped: rows past N are never stored)
-        const int nb0 = (w.nt * C::BW) >> 7;
-        const float* sfb_e = p.sfb + static_cast<int64_t>(w.e) * p.NB * p.KB;
+        const bool ffn_tile = C::EPI == 1 || (C::FUSED && w.phase == 0);
+        const bool second = C::FUSED && w.phase == 1;
+        const int NB = second ? p.NB2 : p.NB;
+        const int KB = second ? p.KB2 : p.KB;
+        const int nb0 = (w.nt * (second ? C::BW2 : C::BW)) >> 7;
+        const float* sfb_e = (second ? p.sfb2 : p.sfb) + static_cast<int64_t>(w.e) * NB * KB;
+        if (second && w.owned) {
+          // the tile's token scales are written by the first GEMM's epilogue
+          const int ri = (FORM == kFormMasked ? w.e * p.num_mt : 0) + w.mt;
+          if (!wait_counter(p.ready + ri, p.ready_target, abort_flag, p.status, p.timeout_ns))
+            goto scales_done;
+          fence_proxy_async_global();
+        }
         const int KQ = (w.nkb + 3) >> 2;  // quads of the tile
         for (int qi = 0; qi < KQ; ++qi, rr.next(), ++fills) {
           if (!mbar_wait(&sa_empty[rr.slot], rr.phase ^ 1u, ctl)) goto scales_done;
           uint8_t* raw = sRAW + rr.slot * C::RAW_BYTES;
           // 4 K blocks of token scales; rows past M read as zero, K blocks past
           // the tile's last one are never used
-          const int ky = (FORM == kFormMasked ? w.e * p.KB : 0) + w.kb0 + 4 * qi;
+          const int ky = (FORM == kFormMasked ? w.e * KB : 0) + w.kb0 + 4 * qi;
           if constexpr (C::EPI == 2) {
             // per-row weight scales: BW rows x 4 K blocks beside them
             mbar_arrive_expect_tx(&sa_full[rr.slot], C::RAW_A + C::RAW_B);
@@ -520,15 +651,16 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             continue;
           }
           mbar_arrive_expect_tx(&sa_full[rr.slot], C::RAW_A);
-          tma_load_2d(raw, &tmSA, &sa_full[rr.slot], w.mt * C::BT, ky);
+          tma_load_2d(raw, second ? &tmSA2 : &tmSA, &sa_full[rr.slot], w.mt * C::BT, ky);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int kb = w.kb0 + min(4 * qi + k, w.nkb - 1);
 #pragma unroll
             for (int j = 0; j < C::NBT; ++j) {
-              // fused FFN: the gate block nt and the up block I/128 + nt
-              const int nb = C::EPI == 1 ? (j == 0 ? w.nt : (p.I >> 7) + w.nt) : min(nb0 + j, p.NB - 1);
-              cp_async_4(raw + C::RAW_A + 4 * (k * C::NBT + j), sfb_e + static_cast<int64_t>(nb) * p.KB + kb);
+              // fused FFN: the gate block nt and the up block I/128 + nt (a
+              // third staged block, where the config has one, repeats it)
+              const int nb = ffn_tile ? (j == 0 ? w.nt : (p.I >> 7) + w.nt) : min(nb0 + j, NB - 1);
+              cp_async_4(raw + C::RAW_A + 4 * (k * C::NBT + j), sfb_e + static_cast<int64_t>(nb) * KB + kb);
             }
           }
           cp_async_mbar_arrive(&sa_full[rr.slot]);
@@ -547,18 +679,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     // instructions, the same lane every time (copies and the MMAs that read
     // them must come from one thread).
     if (rank == 0) {  // a pair's MMAs are issued by its leader
-      constexpr uint32_t idesc = mma_idesc_e4m3_bs(C::MMA_M, C::BW);
+      constexpr uint32_t idesc1 = mma_idesc_e4m3_bs(C::MMA_M, C::BW);
+      constexpr uint32_t idesc2 = mma_idesc_e4m3_bs(C::MMA_M, C::BW2);  // (one-kernel FFN, second GEMM)
       Ring<C::STAGES> st;
       Ring<C::SFS> sq;
-      uint32_t tc = 0;
+      AccTurn<C> acc;
+      int last_b = 0;
       bool ready = false;  // the current stage's "full" phase was seen complete by a peek
       for (int t = t_first; t < total; t += t_step) {
-        const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+        const Tile w = mx_resolve<C, FORM>(p, table, t, rank, t1);
         if (!w.valid || w.nkb == 0) continue;  // (an expert without tokens: no MMA)
-        const int b = tc % C::ACC;
-        if (!warp_wait(&tempty[b], ((tc / C::ACC) & 1u) ^ 1u, ctl, lane)) goto mma_done;
+        const int b = acc.next(w);
+        if (!warp_wait(&tempty[b], (acc.uses(b) & 1u) ^ 1u, ctl, lane)) goto mma_done;
         tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::BW);
+        const uint32_t d = tmem_base + AccTurn<C>::column(w, b);
+        const uint32_t idesc = C::FUSED && w.phase ? idesc2 : idesc1;
         for (int kb0 = 0; kb0 < w.nkb; kb0 += C::KPS, st.next()) {
           if (!ready && !warp_wait(&full[st.slot], st.phase, ctl, lane)) goto mma_done;
           tc_fence_after();
@@ -622,26 +757,30 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           if constexpr (C::PAIR) mma_commit_pair(&tfull[b]);
           else mma_commit(&tfull[b]);
         }
-        ++tc;
+        acc.done(w, b);
+        last_b = b;
       }
     mma_done:
-      if (tc > 0 && lane == 0) drain_wait(&tfull[(tc - 1) % C::ACC], ((tc - 1) / C::ACC) & 1u, kDrainLimitNs);
+      if (acc.tiles > 0 && lane == 0)
+        drain_wait(&tfull[last_b], (acc.uses(last_b) - 1) & 1u, kDrainLimitNs);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale converter
     Ring<C::RAWS> rr;
     Ring<C::SFS> sq;
     for (int t = t_first; t < total; t += t_step) {
-      const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+      const Tile w = mx_resolve<C, FORM>(p, table, t, rank, t1);
       if (!w.valid) continue;
       // staged weight-block index of this lane's weight rows lane + 32 r1 + 128 g
-      const int n0 = w.nt * C::BW;
+      // (a first-GEMM FFN tile: group 0 = the gate block, 1 = the up block)
+      const bool ffn_tile = C::EPI == 1 || (C::FUSED && w.phase == 0);
+      const int n0 = w.nt * (C::FUSED && w.phase ? C::BW2 : C::BW);
       int jb[C::SFB_GROUPS][4];
 #pragma unroll
       for (int g = 0; g < C::SFB_GROUPS; ++g)
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1)
-          jb[g][r1] = C::EPI == 1 ? g : ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
+          jb[g][r1] = ffn_tile ? g : ((n0 + 128 * g + 32 * r1 + lane) >> 7) - (n0 >> 7);
       // rows of this lane (lane + 32 r1) whose outputs are stored: only their
       // token scales must be powers of two (rows past M arrive as zeros;
       // masked rows past masked_m and contiguous rows of another expert or
@@ -730,15 +869,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         raise_status(p.status, 5 /* FG_DEVICE_BAD_SCALE */);
     }
   convert_done:;
-  } else if (C::EPI == 1 && warp >= C::EPI_BASE) {
+  } else if (C::FFN && warp >= C::EPI_BASE) {
     // ------------------------------------------------------------ fused FFN epilogue
     const int quad = warp & 3;          // TMEM lanes this warp may access (one warp per quadrant)
     const int row = quad * 32 + lane;   // token row of this CTA's tile
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     const int IB = p.I >> 7;
-    uint32_t tc = 0;
+    AccTurn<C> acc;
     for (int t = t_first; t < total; t += t_step) {
-      const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+      const Tile w = mx_resolve<C, FORM>(p, table, t, rank, t1);
       if (!w.valid) continue;
       int m_valid = p.M;
       if (FORM == kFormMasked) {
@@ -749,8 +888,42 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ok = m < m_valid;
       if (FORM == kFormContig) ok = ok && __ldg(p.m_indices + m) == w.e;
       const int64_t grow = (FORM == kFormMasked ? static_cast<int64_t>(w.e) * p.M : 0) + m;
-      if (!warp_wait(&tfull[0], tc & 1u, ctl, lane)) goto ffn_done;
+      const int b = acc.next(w);
+      if (!warp_wait(&tfull[b], acc.uses(b) & 1u, ctl, lane)) goto ffn_done;
       tc_fence_after();
+      if (C::FUSED && w.phase == 1) {
+        // one-kernel FFN, second GEMM: the row's BW2 accumulator columns as
+        // packed bf16, the accumulator released (the next tile's MMAs run in
+        // the other one meanwhile), then Y written directly
+        constexpr int YW = C::BW2 / 2;  // packed pairs
+        uint32_t yp[YW];
+        const uint32_t a0 = tmem_base + t_lane + AccTurn<C>::column(w, b);
+#pragma unroll
+        for (int c = 0; c < C::BW2 / 32; ++c) {
+          uint32_t r0[32];
+          tmem_ld32_issue(a0 + static_cast<uint32_t>(32 * c), r0);
+          tmem_wait_ld32(r0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            yp[16 * c + j] = pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (C::PAIR && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+          else mbar_arrive(&tempty[b]);
+        }
+        if (ok) {
+          const int x0 = w.nt * C::BW2;  // columns past H (a last, partial tile) are not stored
+          uint16_t* ydst = p.D + grow * p.N2 + x0;
+#pragma unroll
+          for (int j = 0; j < YW; j += 4)
+            if (x0 + 2 * j < p.N2)
+              *reinterpret_cast<uint4*>(ydst + 2 * j) = make_uint4(yp[j], yp[j + 1], yp[j + 2], yp[j + 3]);
+        }
+        acc.done(w, b);
+        continue;
+      }
       // gate and up values as packed bf16 pairs (the activation takes them in
       // bf16): all 256 columns are read first, so that the accumulator goes
       // back to the MMA before the activation arithmetic
@@ -771,8 +944,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (C::PAIR && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[0]), 0));
-        else mbar_arrive(&tempty[0]);
+        if (C::PAIR && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+        else mbar_arrive(&tempty[b]);
       }
       if (p.gu != nullptr && ok) {
         // bf16 gate at columns nt*128.., up at I + nt*128..
@@ -783,17 +956,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           *reinterpret_cast<uint4*>(gdst + p.I + 2 * j) = make_uint4(upk[j], upk[j + 1], upk[j + 2], upk[j + 3]);
         }
       }
-      // h = bf16(silu(gate) * up), kept as packed bf16 pairs, and its amax
-      uint32_t hp[64];
-      float amax = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float h0 = round_bf16(__fmul_rn(silu_fixed(bf16_lo(gp[j])), bf16_lo(upk[j])));
-        const float h1 = round_bf16(__fmul_rn(silu_fixed(bf16_hi(gp[j])), bf16_hi(upk[j])));
-        amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
-        hp[j] = pack_bf16x2(h0, h1);
-      }
       if (ok) {
+        // h = bf16(silu(gate) * up), kept as packed bf16 pairs, and its amax;
+        // only for rows that are stored (padding rows are zeros, on which the
+        // IEEE division of silu runs its slow path: a warp of them took twice
+        // as long as a warp of tokens and held up the next tile)
+        uint32_t hp[64];
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float h0 = round_bf16(__fmul_rn(silu_fixed(bf16_lo(gp[j])), bf16_lo(upk[j])));
+          const float h1 = round_bf16(__fmul_rn(silu_fixed(bf16_hi(gp[j])), bf16_hi(upk[j])));
+          amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
+          hp[j] = pack_bf16x2(h0, h1);
+        }
         // the per-token power-of-two quantization of per_token_cast_to_fp8_ue8m0
         float scale, inv;
         group_scale<true>(fmaxf(amax, kAmaxFloor), scale, inv);
@@ -811,7 +987,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         }
         p.sfh[static_cast<int64_t>((FORM == kFormMasked ? w.e * IB : 0) + w.nt) * p.sfh_stride + m] = scale;
       }
-      ++tc;
+      if constexpr (C::FUSED) {
+        if (w.owned) {
+          // publish this warp's rows of the token tile to the second GEMM's
+          // tensor loads (other CTAs): the lanes' stores, ordered before the
+          // async proxy's later reads, then, after the warp barrier (which
+          // orders every lane's stores before lane 0's next operations), one
+          // count per warp with release semantics at GPU scope; the reader
+          // acquires the count and fences its own proxy before loading.
+          fence_proxy_async_global();
+          __syncwarp();
+          if (lane == 0)
+            red_release_gpu_add(p.ready + (FORM == kFormMasked ? w.e * p.num_mt : 0) + w.mt, 1);
+        }
+      }
+      acc.done(w, b);
     }
   ffn_done:;
   } else if (warp >= C::EPI_BASE) {
@@ -824,7 +1014,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     uint8_t* ring = smem + C::OFF_EPI + ew * C::EPI_RING * C::BOX_BYTES;
     uint32_t tc = 0, boxes = 0;
     for (int t = t_first; t < total; t += t_step) {
-      const Tile w = mx_resolve<C, FORM>(p, table, t, rank);
+      const Tile w = mx_resolve<C, FORM>(p, table, t, rank, t1);
       if (!w.valid) continue;
       int m_valid = p.M;
       if (FORM == kFormMasked) {

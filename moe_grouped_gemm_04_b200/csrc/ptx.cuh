@@ -122,6 +122,49 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// ---------------------------------------------------------------- cross-CTA hand-off
+
+// Orders this thread's generic-proxy global writes and reads with its later
+// (or, on the writing side, another thread's later) async-proxy accesses to
+// global memory, e.g. tensor loads of data written with ordinary stores.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// counter += v with release semantics at GPU scope: writes that happen
+// before it (this thread's, and other threads' ordered before it by a
+// barrier) are visible to a thread that acquires the new value.
+__device__ __forceinline__ void red_release_gpu_add(int* counter, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(counter), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *counter >= target (acquire, GPU scope), bounded like
+// mbar_wait: gives up when another role of the CTA aborted or after
+// `limit_ns`, then records FG_DEVICE_WAIT_TIMEOUT and sets the abort flag.
+__device__ __forceinline__ bool wait_counter(const int* counter, int target, volatile int* abort_flag,
+                                             int* status, uint64_t limit_ns) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = wait_clock();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (wait_clock() - t0 > wait_cycles(limit_ns)) {
+        atomicCAS(status, 0, 1 /* FG_DEVICE_WAIT_TIMEOUT */);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA / cp.async
 
 // 4-byte asynchronous copy global -> shared (L1-allocating).

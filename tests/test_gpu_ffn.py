@@ -32,7 +32,16 @@ def fg():
         pytest.skip("no CUDA device")
     import moe_grouped_gemm_04_b200 as m
     m.load_library()
-    return m
+    yield m
+    m.set_ffn_mode(0)
+
+
+@pytest.fixture(params=[1, 2], ids=["one-launch", "two-launches"])
+def mode(request, fg):
+    """Both forms of the FFN: one persistent launch, and two launches."""
+    fg.set_ffn_mode(request.param)
+    yield request.param
+    fg.set_ffn_mode(0)
 
 
 def _filled(shape, value, dtype):
@@ -82,7 +91,7 @@ def oracle_stride(M):
 
 @pytest.mark.parametrize("counts,H,I", [([130, 0, 200], 256, 256), ([1], 128, 128),
                                         ([300, 77, 128, 5], 512, 384)])
-def test_ffn_contiguous_parity(fg, counts, H, I):
+def test_ffn_contiguous_parity(fg, mode, counts, H, I):
     rng = np.random.default_rng(sum(counts) + H + I)
     G = len(counts)
     # groups stacked along M, each padded to 128 rows
@@ -131,7 +140,7 @@ def run_masked(fg, xq, sx, w1q, sw1, w2q, sw2, mm, expected_m):
     ([256, 3, 0, 200], 256, 256, 256, 200),    # CTA pairs (expected rows > 128)
     ([130, 1], 192, 384, 128, 130),            # pairs whose second tile lies past M_max
 ])
-def test_ffn_masked_parity(fg, masked_m, M_max, H, I, expected):
+def test_ffn_masked_parity(fg, mode, masked_m, M_max, H, I, expected):
     rng = np.random.default_rng(M_max + H + I)
     G = len(masked_m)
     mm = np.array(masked_m, np.int32)
@@ -159,7 +168,7 @@ def test_ffn_masked_parity(fg, masked_m, M_max, H, I, expected):
         assert np.all(hq[e, v:] == SENT8)
 
 
-def test_ffn_contiguous_deepseek_expert_shape(fg):
+def test_ffn_contiguous_deepseek_expert_shape(fg, mode):
     """An expert shape of the MoE layers (H = 7168, I = 2048) on the
     contiguous workload's token counts: every valid output of GU and Y, and the
     requantization of every valid row bit for bit."""
@@ -178,3 +187,64 @@ def test_ffn_contiguous_deepseek_expert_shape(fg):
     ref2 = oracle.grouped_contiguous(hq * valid[:, None], sh, w2q, sw2, mi)
     check_gemm(bf16_bits_to_f64(y[valid]), ref2[valid], "ffn GEMM2 full")
     assert np.all(y[~valid] == SENT16)
+
+
+def test_ffn_workspace_needs_no_initialisation(fg):
+    fg.set_ffn_mode(1)  # the one-launch form reads the counters
+    """The one-kernel FFN's second GEMM waits on ready counters in the
+    workspace, which each call clears itself: a workspace holding garbage
+    (counters that would read as complete) gives the same bits as a fresh
+    one, and calls in a row reusing it do too."""
+    counts = [300, 77, 128, 5]                    # odd runs: pair partners of other experts
+    H, I = 256, 384
+    rng = np.random.default_rng(77)
+    G = len(counts)
+    blocks = [-(-c // 128) * 128 for c in counts]
+    M = sum(blocks)
+    mi = np.full(M, -1, np.int32)
+    r = 0
+    for e, (c, b) in enumerate(zip(counts, blocks)):
+        mi[r:r + c] = e
+        r += b
+    x = np.zeros((M, H), np.uint16)
+    valid = mi >= 0
+    x[valid] = workloads.bf16_bits(rng.standard_normal((int(valid.sum()), H)).astype(np.float32))
+    xq, sx = oracle.per_token_cast(x, ue8m0=True)
+    w1q, sw1, w2q, sw2 = _weights(rng, G, H, I)
+    args = [to_torch(xq), to_torch(sa_to_mn_major(sx)), to_torch(w1q), to_torch(sw1),
+            to_torch(w2q), to_torch(sw2)]
+    mit = to_torch(mi)
+    ws = fg.empty_ffn_workspace(fg.FG_LAYOUT_CONTIGUOUS, M, G)
+    outs = []
+    for fill in (0x00, 0x7F, 0x7F, 0xFF):
+        ws.fill_(fill)
+        Hq = _filled((M, I), SENT8, np.uint8)
+        SH = _filled((I // 128, oracle_stride(M)), np.nan, np.float32)
+        Y = _bf16((M, H))
+        fg.fp8_moe_ffn_contiguous_ue8m0(*args, Hq, SH, Y, mit, ws=ws)
+        torch.cuda.synchronize()
+        assert fg.get_device_status() == 0
+        outs.append((tensor_bf16_bits(Y), Hq.cpu().numpy(), SH.cpu().numpy()))
+    for y, hq, sh in outs[1:]:
+        assert np.array_equal(y, outs[0][0]) and np.array_equal(hq, outs[0][1])
+        assert np.array_equal(sh.view(np.uint32), outs[0][2].view(np.uint32))
+    _, _, _, yo = oracle.moe_ffn_contiguous(xq, sx, w1q, sw1, w2q, sw2, mi)
+    check_gemm(bf16_bits_to_f64(outs[0][0][valid]), yo[valid], "ffn end to end, reused workspace")
+    fg.set_ffn_mode(0)
+
+
+def test_ffn_workspace_too_small(fg):
+    xq = torch.zeros((256, 128), dtype=torch.uint8, device="cuda")
+    sx = torch.ones((1, 256), dtype=torch.float32, device="cuda")
+    w1 = torch.zeros((1, 256, 128), dtype=torch.uint8, device="cuda")
+    sw1 = torch.ones((1, 2, 1), dtype=torch.float32, device="cuda")
+    w2 = torch.zeros((1, 128, 128), dtype=torch.uint8, device="cuda")
+    sw2 = torch.ones((1, 1, 1), dtype=torch.float32, device="cuda")
+    Hq = torch.zeros((256, 128), dtype=torch.uint8, device="cuda")
+    sh = torch.zeros((1, 256), dtype=torch.float32, device="cuda")
+    Y = torch.zeros((256, 128), dtype=torch.bfloat16, device="cuda")
+    mi = torch.zeros(256, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fg.FP8GemmError) as ei:
+        fg.fp8_moe_ffn_contiguous_ue8m0(xq, sx, w1, sw1, w2, sw2, Hq, sh, Y, mi, ws=ws)
+    assert ei.value.status == fg.FG_ERR_INVALID_ARG

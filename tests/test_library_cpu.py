@@ -116,22 +116,49 @@ def test_ffn_validation_without_the_device(lib):
     P = ctypes.c_void_p
     ok = P(FAKE)
     args = [ok] * 11
+    ws = [ok, 1 << 20]  # workspace and its size
     # I and H must be positive multiples of 128; M_total a multiple of 128
-    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 100, 2, None) == 1
-    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 200, 128, 2, None) == 1
-    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 100, 256, 128, 2, None) == 1
-    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 128, 0, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 100, 2, *ws, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 200, 128, 2, *ws, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 100, 256, 128, 2, *ws, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 128, 0, *ws, None) == 1
     bad = list(args)
     bad[6] = P(MISALIGNED)  # Hq
-    assert lib.fp8_moe_ffn_contiguous_ue8m0(*bad, 256, 256, 128, 2, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*bad, 256, 256, 128, 2, *ws, None) == 1
     margs = list(args)
     margs[10] = None  # masked_m
-    assert lib.fp8_moe_ffn_masked_ue8m0(*margs, 2, 64, 256, 128, 32, None) == 1
-    assert lib.fp8_moe_ffn_masked_ue8m0(*args, 2, 0, 256, 128, 32, None) == 1
+    assert lib.fp8_moe_ffn_masked_ue8m0(*margs, 2, 64, 256, 128, 32, *ws, None) == 1
+    assert lib.fp8_moe_ffn_masked_ue8m0(*args, 2, 0, 256, 128, 32, *ws, None) == 1
+    # the workspace: present, aligned and at least fg_moe_ffn_workspace_bytes
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 128, 2, None, 1 << 20, None) == 1
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 128, 2, P(MISALIGNED), 1 << 20, None) == 1
+    need = lib.fg_moe_ffn_workspace_bytes(0, 256, 2)
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*args, 256, 256, 128, 2, ok, need - 1, None) == 1
+    assert lib.fp8_moe_ffn_masked_ue8m0(*args, 2, 64, 256, 128, 32, ok,
+                                        lib.fg_moe_ffn_workspace_bytes(1, 64, 2) - 1, None) == 1
     # an empty contiguous problem is a no-op success; GU may be NULL
     nogu = list(args)
     nogu[8] = None
-    assert lib.fp8_moe_ffn_contiguous_ue8m0(*nogu, 0, 256, 128, 2, None) == 0
+    assert lib.fp8_moe_ffn_contiguous_ue8m0(*nogu, 0, 256, 128, 2, *ws, None) == 0
+
+
+def test_ffn_mode_knob(lib):
+    for m in (0, 1, 2):
+        assert lib.fg_set_ffn_mode(m) == 0
+    for m in (-1, 3):
+        assert lib.fg_set_ffn_mode(m) == 1
+    assert lib.fg_set_ffn_mode(0) == 0
+
+
+def test_ffn_workspace_bytes(lib):
+    """One int counter per 128-token tile (masked: per expert and tile of its
+    slab), rounded up to 256 bytes; 0 for invalid arguments."""
+    assert lib.fg_moe_ffn_workspace_bytes(0, 13952, 8) == 512          # 109 tiles: 436 bytes
+    assert lib.fg_moe_ffn_workspace_bytes(0, 128 * 100, 8) == 512      # 100 tiles
+    assert lib.fg_moe_ffn_workspace_bytes(1, 256, 32) == 256           # 32 x 2 tiles
+    assert lib.fg_moe_ffn_workspace_bytes(1, 200, 100) == 1024         # 100 x 2 tiles
+    assert lib.fg_moe_ffn_workspace_bytes(2, 256, 8) == 0
+    assert lib.fg_moe_ffn_workspace_bytes(0, 256, 0) == 0
 
 
 def test_k_grouped_validation_without_the_device(lib):
