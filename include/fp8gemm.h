@@ -279,6 +279,36 @@ fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uin
                                   int expected_m, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * The masked expert FFN above in its one-launch form, for callers that must
+ * not allocate device memory: it takes no workspace. This entry point has no
+ * counterpart in the pages; it exists for code that is handed its input and
+ * output buffers but cannot obtain more device memory - for example a serving
+ * runtime that reserves all of the GPU's memory for its weights and KV cache
+ * when it starts and hands each operator fixed buffers, or a plugin that runs
+ * inside another framework's memory manager and is given no allocator - so
+ * that a workspace would otherwise have to be carved out of someone else's
+ * buffers.
+ * Its ready counters live in a fixed array of this library's own device
+ * memory (16 KB, 4096 counters; every GPU that loads the library holds it
+ * until the process exits). The call allocates and frees nothing; it clears
+ * the counters it uses (cudaMemsetAsync on `stream`) before its kernel.
+ * Limit: G * ceil(M_max / 128) <= 4096 token tiles; larger problems return
+ * FG_ERR_UNSUPPORTED (use fp8_moe_ffn_masked_ue8m0 with a workspace).
+ * The first call on a device looks up the array's device address there
+ * (once, cached); make that first call before capturing any stream.
+ * All calls share the one array per device: calls whose kernels can overlap
+ * on the GPU (on different streams) race on it and give wrong results;
+ * calls in order on one stream are safe.
+ * Arguments, layouts, results and other errors: those of
+ * fp8_moe_ffn_masked_ue8m0 (always the one-launch form).
+ */
+fg_status fp8_moe_ffn_masked_ue8m0_noalloc(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                          const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                          uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                          const int32_t* masked_m, int G, int M_max, int H, int I,
+                                          int expected_m, cudaStream_t stream);
+
+/*
  * K-grouped GEMM with power-of-two scales, for the weight gradients of MoE
  * experts in FP8 training (dW_e = dY_e^T X_e: the contraction runs over the
  * tokens routed to each expert). The experts' token ranges are stacked along

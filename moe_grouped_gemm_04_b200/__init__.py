@@ -40,7 +40,7 @@ EXPORTED = (
     "fp8_grouped_gemm_contiguous", "fp8_grouped_gemm_masked", "per_block_dequant_to_bf16",
     "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
     "fg_set_ue8m0_tile", "fg_set_ffn_mode", "fg_moe_ffn_workspace_bytes", "fp8_moe_ffn_contiguous_ue8m0",
-    "fp8_moe_ffn_masked_ue8m0",
+    "fp8_moe_ffn_masked_ue8m0", "fp8_moe_ffn_masked_ue8m0_noalloc",
     "fp8_k_grouped_gemm_nt_ue8m0",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
@@ -86,6 +86,7 @@ def load_library() -> ctypes.CDLL:
     lib.fg_moe_ffn_workspace_bytes.restype = Z
     lib.fp8_moe_ffn_contiguous_ue8m0.argtypes = [P] * 11 + [I, I, I, I, P, Z, P]
     lib.fp8_moe_ffn_masked_ue8m0.argtypes = [P] * 11 + [I, I, I, I, I, P, Z, P]
+    lib.fp8_moe_ffn_masked_ue8m0_noalloc.argtypes = [P] * 11 + [I, I, I, I, I, P]
     lib.fp8_k_grouped_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
@@ -100,6 +101,7 @@ def load_library() -> ctypes.CDLL:
               "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0",
               "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile", "fg_set_ffn_mode",
               "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
+              "fp8_moe_ffn_masked_ue8m0_noalloc",
               "fp8_k_grouped_gemm_nt_ue8m0",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
@@ -337,6 +339,20 @@ def fp8_moe_ffn_masked_ue8m0(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, masked_m, e
         _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
         _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def fp8_moe_ffn_masked_ue8m0_noalloc(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, masked_m, expected_m,
+                                     GU=None, stream=None) -> None:
+    """The masked expert FFN for callers that may not allocate device memory:
+    no workspace (the library's own fixed scratch holds the ready counters;
+    G * ceil(M_max / 128) <= 4096; calls that overlap on the GPU race on it)."""
+    G, M_max, H = X.shape
+    I2 = W1.shape[1]
+    if masked_m.dtype != torch.int32 or masked_m.numel() != G:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "masked_m must be int32 [G]")
+    _check(load_library().fp8_moe_ffn_masked_ue8m0_noalloc(
+        _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
+        _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m), _stream(stream)))
 
 
 def fp8_k_grouped_gemm_nt_ue8m0(A, sfa, B, sfb, D, ks, stream=None) -> None:

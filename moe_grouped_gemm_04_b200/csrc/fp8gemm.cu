@@ -902,6 +902,83 @@ fg_status run_per_block(const uint16_t* x, uint8_t* q, float* sfb, int num_group
   return FG_OK;
 }
 
+// ---------------------------------------------------------------- FFN without allocation
+
+// Ready counters of fp8_moe_ffn_masked_ue8m0_noalloc, for callers that are
+// given device buffers for their inputs and outputs but may not allocate any
+// further device memory. The array is this library's own: every GPU that
+// loads the library holds it (16 KB) until the process exits. In host code
+// `g_ffn_scratch` names a host-side stand-in, not device memory: kernels are
+// given the device address looked up below.
+constexpr size_t kFfnScratchCounters = 4096;
+static __device__ __align__(256) int g_ffn_scratch[kFfnScratchCounters];
+
+std::mutex g_scratch_mu;
+int* g_scratch_dev[kMaxDevices] = {};
+
+// Device address of g_ffn_scratch on the current device `dev`, looked up on
+// the first call for that device (cudaGetSymbolAddress, with `dev` current)
+// and cached.
+fg_status ffn_scratch(int dev, int** out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_dev[dev] == nullptr) {
+    int* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress((void**)&ptr, g_ffn_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(FFN scratch)");
+    g_scratch_dev[dev] = ptr;
+  }
+  *out = g_scratch_dev[dev];
+  return FG_OK;
+}
+
+fg_status run_ffn_masked_noalloc(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                 const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                 uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                 const int32_t* masked_m, int G, int M_max, int H, int I,
+                                 int expected_m, cudaStream_t stream) {
+  if (G < 1) return fail(FG_ERR_INVALID_ARG, "G=%d must be >= 1", G);
+  if (H <= 0 || H % 128 != 0) return fail(FG_ERR_INVALID_ARG, "H=%d must be a positive multiple of 128", H);
+  if (I <= 0 || I % 128 != 0) return fail(FG_ERR_INVALID_ARG, "I=%d must be a positive multiple of 128", I);
+  if (M_max < 1) return fail(FG_ERR_INVALID_ARG, "M_max=%d must be >= 1", M_max);
+  FG_TRY(check_ptr(masked_m, "masked_m"));
+  if (G + 1 > kTableMax) return fail(FG_ERR_UNSUPPORTED, "G %d exceeds %d experts", G, kTableMax - 1);
+  const size_t need = ffn_ready_count(kFormMasked, M_max, G);
+  if (need > kFfnScratchCounters)
+    return fail(FG_ERR_UNSUPPORTED,
+                "fp8_moe_ffn_masked_ue8m0_noalloc: G * ceil(M_max / 128) = %zu token tiles exceed the "
+                "%zu of its fixed scratch (use fp8_moe_ffn_masked_ue8m0 with a workspace)",
+                need, kFfnScratchCounters);
+  if (expected_m <= 0) expected_m = M_max;
+  FG_TRY(check_ptr(X, "X"));
+  FG_TRY(check_ptr(sfx, "sfx"));
+  FG_TRY(check_ptr(W1, "W1"));
+  FG_TRY(check_ptr(sfw1, "sfw1"));
+  FG_TRY(check_ptr(W2, "W2"));
+  FG_TRY(check_ptr(sfw2, "sfw2"));
+  FG_TRY(check_ptr(Hq, "Hq"));
+  FG_TRY(check_ptr(sfh, "sfh"));
+  FG_TRY(check_ptr(Y, "Y"));
+  if (GU) FG_TRY(check_ptr(GU, "GU"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  int* ready = nullptr;
+  FG_TRY(ffn_scratch(dev_id, &ready));
+  // the array keeps the previous call's counts: clear the ones this call uses
+  const cudaError_t e = cudaMemsetAsync(ready, 0, need * sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(FFN scratch)");
+  FfnOut out{Hq, sfh, GU, I};
+  out.W2 = W2;
+  out.sfw2 = sfw2;
+  out.Y = Y;
+  out.H = H;
+  out.ready = ready;
+  Problem p1{kFormMasked, X, sfx, W1, sfw1, nullptr, nullptr, masked_m, M_max, 2 * I, H, G, G};
+  return expected_m > 128 ? launch_mx<MxFfn1P, kFormMasked>(p1, *dev, dev_id, stream, &out)
+                          : launch_mx<MxFfn1S, kFormMasked>(p1, *dev, dev_id, stream, &out);
+}
+
 }  // namespace
 }  // namespace fg
 
@@ -1046,6 +1123,15 @@ fg_status fp8_moe_ffn_masked_ue8m0(const uint8_t* X, const float* sfx, const uin
                                   int expected_m, void* ws, size_t ws_bytes, cudaStream_t stream) {
   return run_ffn(kFormMasked, X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, GU, Y, nullptr, masked_m, M_max,
                  H, I, G, expected_m, ws, ws_bytes, stream);
+}
+
+fg_status fp8_moe_ffn_masked_ue8m0_noalloc(const uint8_t* X, const float* sfx, const uint8_t* W1,
+                                          const float* sfw1, const uint8_t* W2, const float* sfw2,
+                                          uint8_t* Hq, float* sfh, uint16_t* GU, uint16_t* Y,
+                                          const int32_t* masked_m, int G, int M_max, int H, int I,
+                                          int expected_m, cudaStream_t stream) {
+  return run_ffn_masked_noalloc(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, GU, Y, masked_m, G, M_max, H, I,
+                                expected_m, stream);
 }
 
 fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
