@@ -78,6 +78,7 @@ typedef enum {
 #define FG_DEVICE_BAD_M_INDEX 3    /* m_indices entry >= G (tile skipped) */
 #define FG_DEVICE_BAD_K_GROUP 4    /* ks entry < 0, not a multiple of 128, or sum > T (truncated) */
 #define FG_DEVICE_BAD_SCALE 5      /* a block-scaled _ue8m0 GEMM read a scale that is not a power of two */
+#define FG_DEVICE_EP_OVERFLOW 6    /* a local expert received more than M_max rows (the rest dropped) */
 
 /* Row stride (in floats) of the MN-major activation-scale layout. */
 int fg_sfa_stride(int M);
@@ -330,6 +331,56 @@ fg_status fp8_moe_ffn_masked_ue8m0_noalloc(const uint8_t* X, const float* sfx, c
 fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
                                      const float* sfb, float* D, const int32_t* ks, int G, int M,
                                      int N, int T, cudaStream_t stream);
+
+/*
+ * Expert-parallel dispatch into the masked layout and the combine after it,
+ * around an all-to-all exchange that the caller performs (NCCL over
+ * NVLink); the masked layout is the one the grouped GEMM shares with the
+ * communication library ("DeepGEMM" overview, section "约300行JIT核心",
+ * paragraph on MoE layouts; the transfer over NVLink: section "swapAB与Mega
+ * MoE"). E experts over W GPUs, G = E / W local experts per GPU: GPU d holds
+ * experts [d * G, (d + 1) * G). A "pair" is (token t, choice j), p = t * k + j,
+ * with expert topk_idx[p]. All arrays are device arrays owned by the caller.
+ *
+ * ep_dispatch_layout: counts[E] = pairs of each expert; send_pos[T * k] = the
+ *   pair's row in the send buffer, in which pairs are ordered by expert, and
+ *   within an expert by p (so GPU d's pairs are the contiguous rows
+ *   [sum of counts of experts < d * G, + its experts' counts)). A negative
+ *   expert is a dropped choice (send_pos = -1); an expert >= E too, and it
+ *   sets FG_DEVICE_BAD_M_INDEX. T >= 0, k >= 1, E >= 1.
+ * ep_dispatch_pack: copies token row t of q (e4m3 [T][K]) and its K / 128
+ *   scales (MN-major sfa [K/128][stride(T)], what per_token_cast_to_fp8
+ *   writes) to row send_pos[p] of send_q [P][K] and send_s [P][K/128] for
+ *   every pair with send_pos >= 0 (P = counts summed, at most T * k).
+ * ep_dispatch_unpack_masked: the R received rows (recv_q [R][K], recv_s
+ *   [R][K/128]) come source GPU by source GPU, each source's rows local expert
+ *   by local expert, recv_counts[s * G + g] of them (int32, device) - the
+ *   segments the sources' layouts put in front of this GPU. Row i of (s, g)
+ *   goes to slot (rows of expert g from sources before s) + i of the masked
+ *   layout A [G][M_max][K], sfa [G][K/128][stride(M_max)]; masked_m[g] = rows
+ *   of g (capped at M_max: rows past it are dropped, recv_slot = -1 and
+ *   FG_DEVICE_EP_OVERFLOW); recv_slot[r] = g * M_max + slot. W * G <= 4096.
+ * ep_combine_gather: out[r] = D row recv_slot[r] (bf16 [.][N] -> [R][N], zero
+ *   for dropped rows): the masked GEMM's outputs back in receive order, to be
+ *   sent back to their sources. N % 8 == 0.
+ * ep_combine_reduce: with y [P][N] the rows returned in send order,
+ *   out[t][n] = bf16(sum over j = 0..k-1 of topk_w[t][j] * y[send_pos[t*k+j]][n]),
+ *   each term an fp32 fused multiply-add in j order, rounded to nearest even
+ *   once; choices with send_pos < 0 add nothing. N % 8 == 0.
+ * Errors: FG_ERR_INVALID_ARG for sizes and null or misaligned pointers.
+ */
+fg_status ep_dispatch_layout(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
+                             int32_t* send_pos, cudaStream_t stream);
+fg_status ep_dispatch_pack(const uint8_t* q, const float* sfa, const int32_t* send_pos, int T, int k,
+                           int K, uint8_t* send_q, float* send_s, cudaStream_t stream);
+fg_status ep_dispatch_unpack_masked(const uint8_t* recv_q, const float* recv_s,
+                                    const int32_t* recv_counts, int W, int G, int R, int M_max,
+                                    int K, uint8_t* A, float* sfa, int32_t* masked_m,
+                                    int32_t* recv_slot, cudaStream_t stream);
+fg_status ep_combine_gather(const uint16_t* D, const int32_t* recv_slot, int R, int N, uint16_t* out,
+                            cudaStream_t stream);
+fg_status ep_combine_reduce(const uint16_t* y, const int32_t* send_pos, const float* topk_w, int T, int k,
+                            int N, uint16_t* out, cudaStream_t stream);
 
 /*
  * Tuning knob of the three _ue8m0 GEMMs (process-wide). width = 0: choose the

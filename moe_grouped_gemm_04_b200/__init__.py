@@ -41,6 +41,8 @@ EXPORTED = (
     "fp8_gemm_nt_ue8m0", "fp8_grouped_gemm_contiguous_ue8m0", "fp8_grouped_gemm_masked_ue8m0",
     "fg_set_ue8m0_tile", "fg_set_ffn_mode", "fg_moe_ffn_workspace_bytes", "fp8_moe_ffn_contiguous_ue8m0",
     "fp8_moe_ffn_masked_ue8m0", "fp8_moe_ffn_masked_ue8m0_noalloc",
+    "ep_dispatch_layout", "ep_dispatch_pack", "ep_dispatch_unpack_masked", "ep_combine_gather",
+    "ep_combine_reduce",
     "fp8_k_grouped_gemm_nt_ue8m0",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
 )
@@ -87,6 +89,11 @@ def load_library() -> ctypes.CDLL:
     lib.fp8_moe_ffn_contiguous_ue8m0.argtypes = [P] * 11 + [I, I, I, I, P, Z, P]
     lib.fp8_moe_ffn_masked_ue8m0.argtypes = [P] * 11 + [I, I, I, I, I, P, Z, P]
     lib.fp8_moe_ffn_masked_ue8m0_noalloc.argtypes = [P] * 11 + [I, I, I, I, I, P]
+    lib.ep_dispatch_layout.argtypes = [P, I, I, I, P, P, P]
+    lib.ep_dispatch_pack.argtypes = [P, P, P, I, I, I, P, P, P]
+    lib.ep_dispatch_unpack_masked.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
+    lib.ep_combine_gather.argtypes = [P, P, I, I, P, P]
+    lib.ep_combine_reduce.argtypes = [P, P, P, I, I, I, P, P]
     lib.fp8_k_grouped_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
     lib.fg_selftest_wait_timeout.argtypes = [I, P]
@@ -102,6 +109,8 @@ def load_library() -> ctypes.CDLL:
               "fp8_grouped_gemm_masked_ue8m0", "fg_set_ue8m0_tile", "fg_set_ffn_mode",
               "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
               "fp8_moe_ffn_masked_ue8m0_noalloc",
+              "ep_dispatch_layout", "ep_dispatch_pack", "ep_dispatch_unpack_masked",
+              "ep_combine_gather", "ep_combine_reduce",
               "fp8_k_grouped_gemm_nt_ue8m0",
               "fg_get_device_status", "fg_selftest_wait_timeout"):
         getattr(lib, f).restype = I
@@ -353,6 +362,50 @@ def fp8_moe_ffn_masked_ue8m0_noalloc(X, sfx, W1, sfw1, W2, sfw2, Hq, sfh, Y, mas
     _check(load_library().fp8_moe_ffn_masked_ue8m0_noalloc(
         _ptr(X), _ptr(sfx), _ptr(W1), _ptr(sfw1), _ptr(W2), _ptr(sfw2), _ptr(Hq), _ptr(sfh),
         _ptr(GU), _ptr(Y), _ptr(masked_m), G, M_max, H, I2 // 2, int(expected_m), _stream(stream)))
+
+
+def ep_dispatch_layout(topk_idx, E, counts, send_pos, stream=None) -> None:
+    """topk_idx int32 [T][k] -> counts int32 [E], send_pos int32 [T][k]."""
+    T, k = topk_idx.shape
+    _check(load_library().ep_dispatch_layout(_ptr(topk_idx), T, k, int(E), _ptr(counts),
+                                             _ptr(send_pos), _stream(stream)))
+
+
+def ep_dispatch_pack(q, sfa, send_pos, send_q, send_s, stream=None) -> None:
+    """q uint8 [T][K], sfa MN-major [K/128][stride(T)], send_pos [T][k] ->
+    send_q uint8 [P][K], send_s fp32 [P][K/128]."""
+    T, K = q.shape
+    k = send_pos.shape[1]
+    _check(load_library().ep_dispatch_pack(_ptr(q), _ptr(sfa), _ptr(send_pos), T, k, K, _ptr(send_q),
+                                           _ptr(send_s), _stream(stream)))
+
+
+def ep_dispatch_unpack_masked(recv_q, recv_s, recv_counts, A, sfa, masked_m, recv_slot,
+                              stream=None) -> None:
+    """Received rows (source by source, local expert by local expert;
+    recv_counts int32 [W][G]) -> masked layout A [G][M_max][K], sfa
+    [G][K/128][stride(M_max)], masked_m [G], recv_slot [R]."""
+    W, G = recv_counts.shape
+    R = recv_q.shape[0]
+    _, M_max, K = A.shape
+    _check(load_library().ep_dispatch_unpack_masked(
+        _ptr(recv_q), _ptr(recv_s), _ptr(recv_counts), W, G, R, M_max, K, _ptr(A), _ptr(sfa),
+        _ptr(masked_m), _ptr(recv_slot), _stream(stream)))
+
+
+def ep_combine_gather(D, recv_slot, out, stream=None) -> None:
+    """out [R][N] = rows recv_slot of D (bf16 [G][M_max][N]; zero where -1)."""
+    R, N = out.shape
+    _check(load_library().ep_combine_gather(_ptr(D), _ptr(recv_slot), R, N, _ptr(out),
+                                            _stream(stream)))
+
+
+def ep_combine_reduce(y, send_pos, topk_w, out, stream=None) -> None:
+    """out [T][N] = bf16(sum_j topk_w[t][j] * y[send_pos[t][j]]) (fp32, j in order)."""
+    T, k = send_pos.shape
+    N = out.shape[1]
+    _check(load_library().ep_combine_reduce(_ptr(y), _ptr(send_pos), _ptr(topk_w), T, k, N, _ptr(out),
+                                            _stream(stream)))
 
 
 def fp8_k_grouped_gemm_nt_ue8m0(A, sfa, B, sfb, D, ks, stream=None) -> None:

@@ -15,6 +15,7 @@
 
 #include "fp8gemm.h"
 #include "gemm.cuh"
+#include "ep.cuh"
 #include "gemm_mx.cuh"
 #include "quant.cuh"
 
@@ -1134,6 +1135,100 @@ fg_status fp8_moe_ffn_masked_ue8m0_noalloc(const uint8_t* X, const float* sfx, c
                                 expected_m, stream);
 }
 
+// ---------------------------------------------------------------- expert-parallel dispatch / combine
+
+fg_status ep_dispatch_layout(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
+                             int32_t* send_pos, cudaStream_t stream) {
+  if (T < 0 || k < 1 || E < 1) return fail(FG_ERR_INVALID_ARG, "T=%d k=%d E=%d", T, k, E);
+  FG_TRY(check_ptr(counts, "counts"));
+  if (T == 0) {
+    const cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream);
+    return e == cudaSuccess ? FG_OK : cuda_fail(e, "cudaMemsetAsync(counts)");
+  }
+  FG_TRY(check_ptr(topk_idx, "topk_idx"));
+  FG_TRY(check_ptr(send_pos, "send_pos"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  const int P = T * k;
+  cudaError_t e = launch_pdl(ep_count_kernel, dim3(E), dim3(kEpBlock), stream, topk_idx, P, E, counts,
+                             send_pos, dev->status);
+  if (e != cudaSuccess) return cuda_fail(e, "ep_count_kernel launch");
+  e = launch_pdl(ep_position_kernel, dim3(E), dim3(kEpBlock), stream, topk_idx, P,
+                 static_cast<const int32_t*>(counts), send_pos);
+  return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_position_kernel launch");
+}
+
+fg_status ep_dispatch_pack(const uint8_t* q, const float* sfa, const int32_t* send_pos, int T, int k,
+                           int K, uint8_t* send_q, float* send_s, cudaStream_t stream) {
+  if (T < 0 || k < 1) return fail(FG_ERR_INVALID_ARG, "T=%d k=%d", T, k);
+  if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
+  if (T == 0) return FG_OK;
+  FG_TRY(check_ptr(q, "q"));
+  FG_TRY(check_ptr(sfa, "sfa"));
+  FG_TRY(check_ptr(send_pos, "send_pos"));
+  FG_TRY(check_ptr(send_q, "send_q"));
+  FG_TRY(check_ptr(send_s, "send_s"));
+  const int P = T * k;
+  const int per = kEpBlock / 32;
+  const cudaError_t e = launch_pdl(ep_pack_kernel, dim3((P + per - 1) / per), dim3(kEpBlock), stream, q,
+                                   sfa, sfa_stride(T), send_pos, P, k, K, send_q, send_s);
+  return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_pack_kernel launch");
+}
+
+fg_status ep_dispatch_unpack_masked(const uint8_t* recv_q, const float* recv_s,
+                                    const int32_t* recv_counts, int W, int G, int R, int M_max,
+                                    int K, uint8_t* A, float* sfa, int32_t* masked_m,
+                                    int32_t* recv_slot, cudaStream_t stream) {
+  if (W < 1 || G < 1 || R < 0 || M_max < 1)
+    return fail(FG_ERR_INVALID_ARG, "W=%d G=%d R=%d M_max=%d", W, G, R, M_max);
+  if (static_cast<int64_t>(W) * G > kEpMaxTable)
+    return fail(FG_ERR_UNSUPPORTED, "W * G = %lld exceeds %d", static_cast<long long>(W) * G, kEpMaxTable);
+  if (K <= 0 || K % 128 != 0) return fail(FG_ERR_INVALID_ARG, "K=%d must be a positive multiple of 128", K);
+  FG_TRY(check_ptr(recv_counts, "recv_counts"));
+  FG_TRY(check_ptr(A, "A"));
+  FG_TRY(check_ptr(sfa, "sfa"));
+  FG_TRY(check_ptr(masked_m, "masked_m"));
+  if (R > 0) {
+    FG_TRY(check_ptr(recv_q, "recv_q"));
+    FG_TRY(check_ptr(recv_s, "recv_s"));
+    FG_TRY(check_ptr(recv_slot, "recv_slot"));
+  }
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  const int per = kEpBlock / 32;
+  const int blocks = R > 0 ? (R + per - 1) / per : 1;  // (block 0 writes masked_m)
+  const cudaError_t e = launch_pdl(ep_unpack_kernel, dim3(blocks), dim3(kEpBlock), stream, recv_q, recv_s,
+                                   recv_counts, W, G, R, M_max, K, A, sfa, masked_m, recv_slot,
+                                   dev->status);
+  return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_unpack_kernel launch");
+}
+
+fg_status ep_combine_gather(const uint16_t* D, const int32_t* recv_slot, int R, int N, uint16_t* out,
+                            cudaStream_t stream) {
+  if (R < 0 || N <= 0 || N % 8 != 0) return fail(FG_ERR_INVALID_ARG, "R=%d N=%d (N %% 8 == 0)", R, N);
+  if (R == 0) return FG_OK;
+  FG_TRY(check_ptr(D, "D"));
+  FG_TRY(check_ptr(recv_slot, "recv_slot"));
+  FG_TRY(check_ptr(out, "out"));
+  const int per = kEpBlock / 32;
+  const cudaError_t e = launch_pdl(ep_gather_kernel, dim3((R + per - 1) / per), dim3(kEpBlock), stream, D,
+                                   recv_slot, R, N, out);
+  return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_gather_kernel launch");
+}
+
+fg_status ep_combine_reduce(const uint16_t* y, const int32_t* send_pos, const float* topk_w, int T, int k,
+                            int N, uint16_t* out, cudaStream_t stream) {
+  if (T < 0 || k < 1 || N <= 0 || N % 8 != 0) return fail(FG_ERR_INVALID_ARG, "T=%d k=%d N=%d", T, k, N);
+  if (T == 0) return FG_OK;
+  FG_TRY(check_ptr(y, "y"));
+  FG_TRY(check_ptr(send_pos, "send_pos"));
+  FG_TRY(check_ptr(topk_w, "topk_w"));
+  FG_TRY(check_ptr(out, "out"));
+  const cudaError_t e = launch_pdl(ep_combine_kernel, dim3(T), dim3(kEpBlock), stream, y, send_pos, topk_w,
+                                   k, N, out);
+  return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_combine_kernel launch");
+}
+
 fg_status fp8_k_grouped_gemm_nt_ue8m0(const uint8_t* A, const float* sfa, const uint8_t* B,
                                      const float* sfb, float* D, const int32_t* ks, int G, int M,
                                      int N, int T, cudaStream_t stream) {
@@ -1188,6 +1283,7 @@ fg_status fg_get_device_status(cudaStream_t stream, int* code) {
                      : v == FG_DEVICE_BAD_M_INDEX  ? "m_indices entry >= G"
                      : v == FG_DEVICE_BAD_K_GROUP  ? "ks entry negative, not a multiple of 128, or past T"
                      : v == FG_DEVICE_BAD_SCALE    ? "a scale of a block-scaled (_ue8m0) GEMM is not a power of two"
+                     : v == FG_DEVICE_EP_OVERFLOW  ? "a local expert received more than M_max rows"
                                                    : "unknown device status";
   return fail(FG_ERR_DEVICE, "device status %d: %s", v, what);
 }

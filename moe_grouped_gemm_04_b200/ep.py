@@ -1,0 +1,136 @@
+"""Expert-parallel MoE layer around the masked grouped GEMM.
+
+The masked layout ([G][M_max][K] per GPU with a per-expert valid-row count on
+the device) is the one the grouped GEMM shares with the communication library
+that moves tokens between the GPUs of an expert-parallel group ("DeepGEMM"
+overview, section "约300行JIT核心", paragraph on MoE layouts); the tokens
+travel over NVLink to the GPUs that hold their experts and the results travel
+back (same page, section "swapAB与Mega MoE").
+
+One call of `expert_parallel_masked_moe` on every rank of the group:
+
+  1. quantizes the rank's tokens per token per 128 channels (the library's
+     quantizer: the rows travel as e4m3 codes with their scales, half the
+     bytes of bf16);
+  2. orders the (token, choice) pairs by expert (`ep_dispatch_layout`) and
+     copies the rows into that order (`ep_dispatch_pack`), so that the pairs
+     for rank d are one contiguous segment (rank d holds experts
+     [d * G, (d + 1) * G));
+  3. exchanges the per-expert counts, then the rows and their scales, with
+     all-to-all collectives (NCCL over NVLink on GPUs);
+  4. places the received rows into the masked layout and counts them per
+     local expert on the device (`ep_dispatch_unpack_masked`);
+  5. runs the masked grouped GEMM against the rank's expert weights;
+  6. gathers the output rows back into receive order (`ep_combine_gather`),
+     sends them back, and sums each token's choices weighted by the router
+     (`ep_combine_reduce`: fp32, choices in order, one bf16 rounding).
+
+Every step on the data runs in the library's CUDA kernels; this module only
+allocates the buffers (torch device memory) and orders the kernels and the
+collectives. The split sizes of the row exchange are read back to the host
+(one synchronisation per call), as NCCL's all-to-all takes them on the host.
+bf16 rows are exchanged as their bit patterns. No tensor-map or bulk
+copy in this path reads another GPU's memory: the collectives copy the rows
+into this GPU's memory before any kernel reads them.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+import torch.distributed as dist
+
+from . import (FG_ERR_INVALID_ARG, FP8GemmError, empty_sfa, ep_combine_gather, ep_combine_reduce,
+               ep_dispatch_layout, ep_dispatch_pack, ep_dispatch_unpack_masked,
+               fp8_grouped_gemm_masked, per_token_cast_to_fp8)
+
+
+class _LibraryOps:
+    """The library calls the layer is made of (each a CUDA kernel)."""
+    quantize = staticmethod(per_token_cast_to_fp8)
+    layout = staticmethod(ep_dispatch_layout)
+    pack = staticmethod(ep_dispatch_pack)
+    unpack = staticmethod(ep_dispatch_unpack_masked)
+    gemm = staticmethod(fp8_grouped_gemm_masked)
+    gather = staticmethod(ep_combine_gather)
+    combine = staticmethod(ep_combine_reduce)
+
+
+_ops = _LibraryOps
+
+
+def _as_bits(t: torch.Tensor) -> torch.Tensor:
+    """bf16 rows (an even number of columns) as int32 pairs of bit patterns,
+    a type every collective backend moves."""
+    return t.view(torch.int32) if t.dtype == torch.bfloat16 else t
+
+
+def expert_parallel_masked_moe(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+                               w_local: torch.Tensor, sfb_local: torch.Tensor, num_experts: int,
+                               M_max: int, group=None,
+                               expected_m: Optional[int] = None) -> torch.Tensor:
+    """Routed expert GEMM over an expert-parallel group.
+
+    x: bf16 [T][K] (this rank's tokens); topk_idx: int32 [T][k] global expert
+    ids (negative = no expert); topk_w: fp32 [T][k] router weights; w_local:
+    e4m3 [G][N][K] and sfb_local fp32 [G][ceil(N/128)][K/128], the weights of
+    this rank's G = num_experts / world_size experts, quantized per 128 x 128
+    block; M_max: rows per local expert in the masked layout (more are
+    dropped, FG_DEVICE_EP_OVERFLOW). Returns bf16 [T][N]:
+    out[t] = sum_j topk_w[t][j] * bf16((x_t quantized) W_{topk_idx[t][j]}^T).
+    """
+    W = dist.get_world_size(group)
+    if num_experts % W != 0:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "num_experts %d is not a multiple of the group size %d"
+                           % (num_experts, W))
+    G = num_experts // W
+    T, K = x.shape
+    k = topk_idx.shape[1]
+    N = w_local.shape[1]
+    if w_local.shape[0] != G:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "w_local holds %d experts, this rank owns %d"
+                           % (w_local.shape[0], G))
+    dev = x.device
+    KB = K // 128
+
+    # 1-2: quantize, order the pairs by expert, pack the rows
+    q = torch.empty((T, K), dtype=torch.uint8, device=dev)
+    s = empty_sfa(1, T, K, dev)
+    _ops.quantize(x, q, s)
+    counts = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    send_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    _ops.layout(topk_idx, num_experts, counts, send_pos)
+
+    # 3: counts, then rows and scales
+    recv_counts = torch.empty((W, G), dtype=torch.int32, device=dev)
+    dist.all_to_all_single(recv_counts.view(-1), counts, group=group)
+    send_sizes = [int(v) for v in counts.view(W, G).sum(dim=1).tolist()]
+    recv_sizes = [int(v) for v in recv_counts.sum(dim=1).tolist()]
+    P, R = sum(send_sizes), sum(recv_sizes)
+    send_q = torch.empty((P, K), dtype=torch.uint8, device=dev)
+    send_s = torch.empty((P, KB), dtype=torch.float32, device=dev)
+    _ops.pack(q, s[0], send_pos, send_q, send_s)
+    recv_q = torch.empty((R, K), dtype=torch.uint8, device=dev)
+    recv_s = torch.empty((R, KB), dtype=torch.float32, device=dev)
+    dist.all_to_all_single(recv_q, send_q, recv_sizes, send_sizes, group=group)
+    dist.all_to_all_single(recv_s, send_s, recv_sizes, send_sizes, group=group)
+
+    # 4-5: masked layout, grouped GEMM with the local experts
+    A = torch.empty((G, M_max, K), dtype=torch.uint8, device=dev)
+    sfa = empty_sfa(G, M_max, K, dev)
+    masked_m = torch.empty(G, dtype=torch.int32, device=dev)
+    recv_slot = torch.empty(R, dtype=torch.int32, device=dev)
+    _ops.unpack(recv_q, recv_s, recv_counts, A, sfa, masked_m, recv_slot)
+    D = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=dev)
+    if expected_m is None:
+        expected_m = max(1, min(M_max, -(-R // G)))
+    _ops.gemm(A, sfa, w_local, sfb_local, D, masked_m, expected_m)
+
+    # 6: back to the sources, weighted sum of each token's choices
+    y_recv = torch.empty((R, N), dtype=torch.bfloat16, device=dev)
+    _ops.gather(D, recv_slot, y_recv)
+    y_send = torch.empty((P, N), dtype=torch.bfloat16, device=dev)
+    dist.all_to_all_single(_as_bits(y_send), _as_bits(y_recv), send_sizes, recv_sizes, group=group)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    _ops.combine(y_send, send_pos, topk_w, out)
+    return out
