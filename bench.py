@@ -31,6 +31,11 @@ of consecutive steps pipelined on three streams, as a serving loop would);
 `--scales ue8m0` quantizes with power-of-two scales and runs the block-scaled
 GEMM entry points (the oracle then uses the same power-of-two quantizers).
 
+`--workload peak_fp8_mma_16384` measures the FP8 tensor-core rate itself: one
+CTA per SM issues the GEMMs' MMA instruction back to back from operands that
+stay in shared memory (no loads, no promotion), and the accumulators are
+checked exactly; it is the in-library ceiling of the tensor-bound lines.
+
 Multi-GPU (torchrun, one process per GPU): the path does not shard across
 GPUs within one call, so every rank runs an independent replica (weak
 scaling); the timed region is bracketed by a barrier and the reported time is
@@ -1032,6 +1037,82 @@ def dequant_cpu_sample(inp, target_s: float):
             "sample": "%d of %d rows x K=%d, %d passes" % (rows, inp.N, inp.K, passes), "seconds": dt}
 
 
+PEAK_METRIC = ("FP8 tensor-core rate (tcgen05.mma kind::f8f6f4, M=128 N=256 K=32, operands resident "
+               "in shared memory) TFLOP/s (device-timed)")
+
+
+def peak_expected(iters: int) -> np.ndarray:
+    """The accumulator every CTA of the tensor-core rate kernel ends with
+    (the formula its C-ABI declaration states): small integers, exact."""
+    m = np.arange(128)[:, None]
+    n = np.arange(256)[:, None]
+    j = np.arange(16)[None, :]
+    a = (2 * m + 3 * j) % 5 - 2
+    b = (3 * n + 2 * j + n // 16) % 5 - 2
+    return (8.0 * iters) * (a.astype(np.float64) @ b.T.astype(np.float64))
+
+
+def run_peak(args, rank, world, local_rank):
+    """The FP8 tensor-core rate: one CTA per SM issuing the GEMMs' MMA
+    instruction back to back from resident operands, K launches replayed
+    from one CUDA graph between one pair of events. The ceiling of every
+    tensor-bound line, measured with this library's own instruction stream."""
+    import torch
+
+    import moe_grouped_gemm_04_b200 as fg
+
+    torch.cuda.set_device(local_rank)
+    fg.load_library()
+    inp = workloads.make(args.workload)
+    iters = inp.iters
+    ctas = fg.fp8_mma_peak_ctas()
+    out = torch.empty((ctas, 128, 256), dtype=torch.float32, device="cuda")
+
+    def launch(i):
+        fg.fp8_mma_peak(iters, out)
+
+    for i in range(max(args.warmup, 3)):
+        launch(i)
+    torch.cuda.synchronize()
+    assert fg.get_device_status() == 0
+    out.fill_(float("nan"))
+    steps = args.steps
+    ms, clocks = time_graph_launches(launch, steps, local_rank, world)
+    assert fg.get_device_status() == 0
+    # every MMA ran: each CTA holds the exact accumulator
+    got = out.cpu().numpy()
+    assert np.array_equal(got, np.broadcast_to(peak_expected(iters).astype(np.float32), got.shape)), \
+        "tensor-core rate kernel: accumulator differs"
+    if world > 1:
+        import torch.distributed as dist
+        ms = max_over_ranks(dist, [ms], "cuda")[0]
+    if rank != 0:
+        return None
+    flops = 2.0 * 128 * 256 * 128 * iters * ctas
+    tflops = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    anchor = FP8_OVER_BF16 * peaks["bf16_tflops"]
+    return {
+        "metric": PEAK_METRIC, "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "data": "operands generated in shared memory by the kernel (small integers)",
+        "config": {"workload": args.workload, "kind": "peak", "ctas": ctas, "iters": iters,
+                   "mma": "128x256x32 kind::f8f6f4, fp32 accumulator in tensor memory",
+                   "l2": "no memory operands (nothing to flush)",
+                   "launch": "K launches captured in one CUDA graph, replayed once untimed, then timed"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": anchor, "unit": "TFLOP/s",
+                     "frac": tflops / anchor, "peak_rated": RATED_FP8_TFLOPS,
+                     "frac_rated": tflops / RATED_FP8_TFLOPS, "traffic": None,
+                     "kernel": "fp8_mma_peak_kernel", "kernel_ms": ms,
+                     "algorithmic_per_launch": {"flops": flops, "bytes": 0.0},
+                     "peak_source": "FP8 = %.1f x %s bf16 burst %.1f TFLOP/s" % (
+                         FP8_OVER_BF16, peak_src, peaks["bf16_tflops"]),
+                     "peaks_used": peaks_used(peaks, peak_src)},
+        "cpu_baseline": None, "gpu_launches": steps, "clocks": clocks, "e2e": None,
+    }
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm, on rank 0 only."""
     if rank != 0:
@@ -1074,7 +1155,13 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     kind = workloads.WORKLOADS[args.workload][0]
-    if args.impl == "reference" and kind in ("dequant", "quant"):
+    if args.impl == "reference" and kind == "peak":
+        out = None
+        if rank == 0:
+            out = {"impl": "reference", "metric": PEAK_METRIC,
+                   "unavailable": "the tensor-core rate workload measures the GPU itself; the oracle "
+                                  "has no counterpart"}
+    elif args.impl == "reference" and kind in ("dequant", "quant"):
         out = None
         if rank == 0:
             inp = workloads.make(args.workload, seed=0)
@@ -1107,6 +1194,8 @@ def main():
                 out = run_dequant(args, rank, world, local_rank)
             elif kind == "quant":
                 out = run_quant(args, rank, world, local_rank)
+            elif kind == "peak":
+                out = run_peak(args, rank, world, local_rank)
             else:
                 out = run_ours(args, rank, world, local_rank)
         finally:

@@ -412,6 +412,29 @@ fg_status fg_get_device_status(cudaStream_t stream, int* code);
  */
 fg_status fg_selftest_wait_timeout(int timeout_us, cudaStream_t stream);
 
+/*
+ * Tensor-core rate (a measurement aid, not a step of the method): the FP8
+ * tensor-core instruction every GEMM here issues (tcgen05.mma kind::f8f6f4,
+ * M = 128, N = 256, K = 32), run back to back from operands that stay in
+ * shared memory, with nothing loaded or promoted, so that the time of a
+ * launch gives the rate the tensor cores sustain at the clock of the moment.
+ * The GEMMs are judged by their FP8 TFLOPS ("DeepGEMM" overview, section
+ * "约300行JIT核心"); this gives the ceiling of that figure on this GPU.
+ *
+ * One CTA on each of the fg_fp8_mma_peak_ctas() SMs; each runs `iters` K
+ * blocks of 128 (1 <= iters <= 32768), i.e. 2 * 128 * 256 * 128 * iters
+ * FLOPs per CTA. The operands are generated in the kernel from small
+ * integers, so the result is exact and shows that every MMA ran:
+ *   out[c][m][n] = iters * 8 * sum_{j<16} A(m, j) * B(n, j),
+ *   A(m, j) = (2m + 3j) mod 5 - 2,  B(n, j) = (3n + 2j + floor(n/16)) mod 5 - 2,
+ * for every CTA c < fg_fp8_mma_peak_ctas(), m < 128, n < 256.
+ * out: device fp32 [fg_fp8_mma_peak_ctas()][128][256], caller-owned.
+ * Errors: FG_ERR_INVALID_ARG (iters out of range, null out),
+ * FG_ERR_UNSUPPORTED / FG_ERR_CUDA as for the GEMMs.
+ */
+int fg_fp8_mma_peak_ctas(void); /* SM count of the current device; 0 if it is not usable */
+fg_status fg_fp8_mma_peak(int iters, float* out, cudaStream_t stream);
+
 const char* fg_status_string(fg_status s);
 const char* fg_last_error(void);
 

@@ -45,6 +45,7 @@ EXPORTED = (
     "ep_combine_reduce",
     "fp8_k_grouped_gemm_nt_ue8m0",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
+    "fg_fp8_mma_peak_ctas", "fg_fp8_mma_peak",
 )
 
 
@@ -101,6 +102,9 @@ def load_library() -> ctypes.CDLL:
     lib.fg_status_string.restype = ctypes.c_char_p
     lib.fg_last_error.argtypes = []
     lib.fg_last_error.restype = ctypes.c_char_p
+    lib.fg_fp8_mma_peak_ctas.argtypes = []
+    lib.fg_fp8_mma_peak_ctas.restype = I
+    lib.fg_fp8_mma_peak.argtypes = [I, P, P]
     for f in ("per_token_cast_to_fp8", "per_block_cast_to_fp8", "per_token_cast_to_fp8_ue8m0",
               "per_block_cast_to_fp8_ue8m0", "per_block_dequant_to_bf16",
               "fp8_gemm_nt",
@@ -112,7 +116,7 @@ def load_library() -> ctypes.CDLL:
               "ep_dispatch_layout", "ep_dispatch_pack", "ep_dispatch_unpack_masked",
               "ep_combine_gather", "ep_combine_reduce",
               "fp8_k_grouped_gemm_nt_ue8m0",
-              "fg_get_device_status", "fg_selftest_wait_timeout"):
+              "fg_get_device_status", "fg_selftest_wait_timeout", "fg_fp8_mma_peak"):
         getattr(lib, f).restype = I
     _lib = lib
     return lib
@@ -440,3 +444,22 @@ def get_device_status(stream=None) -> int:
 
 def selftest_wait_timeout(timeout_us: int, stream=None) -> None:
     _check(load_library().fg_selftest_wait_timeout(int(timeout_us), _stream(stream)))
+
+
+def fp8_mma_peak_ctas() -> int:
+    """CTAs of one fp8_mma_peak launch (the SM count of the current device)."""
+    n = load_library().fg_fp8_mma_peak_ctas()
+    if n <= 0:
+        raise FP8GemmError(FG_ERR_UNSUPPORTED, load_library().fg_last_error().decode())
+    return int(n)
+
+
+def fp8_mma_peak(iters: int, out, stream=None) -> None:
+    """The tensor-core rate kernel: `iters` K blocks of FP8 MMAs (M = 128,
+    N = 256, K = 128 each) per CTA; out: fp32 [fp8_mma_peak_ctas()][128][256]
+    on the device receives each CTA's exact integer accumulator."""
+    ctas = fp8_mma_peak_ctas()
+    if tuple(out.shape) != (ctas, 128, 256) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "out must be contiguous fp32 [%d][128][256]" % ctas)
+    _check(load_library().fg_fp8_mma_peak(int(iters), _ptr(out), _stream(stream)))
+

@@ -16,6 +16,7 @@
 #include "fp8gemm.h"
 #include "gemm.cuh"
 #include "ep.cuh"
+#include "peak.cuh"
 #include "gemm_mx.cuh"
 #include "quant.cuh"
 
@@ -1311,5 +1312,39 @@ const char* fg_status_string(fg_status s) {
 }
 
 const char* fg_last_error(void) { return g_last_error.c_str(); }
+
+// ---------------------------------------------------------------- tensor-core rate
+
+int fg_fp8_mma_peak_ctas(void) {
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev) != FG_OK) return 0;
+  return dev->sm_count;
+}
+
+fg_status fg_fp8_mma_peak(int iters, float* out, cudaStream_t stream) {
+  if (iters < 1 || iters > kPeakMaxIters)
+    return fail(FG_ERR_INVALID_ARG, "iters=%d must be in [1, %d]", iters, kPeakMaxIters);
+  FG_TRY(check_ptr(out, "out"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  int d = 0;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static std::atomic<bool> attr_set[kMaxDevices];
+  if (!attr_set[d].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!attr_set[d].load(std::memory_order_relaxed)) {
+      e = cudaFuncSetAttribute(fp8_mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kPeakSmem + 1024);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      attr_set[d].store(true, std::memory_order_release);
+    }
+  }
+  fp8_mma_peak_kernel<<<dev->sm_count, 128, kPeakSmem + 1024, stream>>>(iters, out, dev->status,
+                                                                      wait_limit_ns());
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_mma_peak_kernel launch");
+  return FG_OK;
+}
 
 }  // extern "C"

@@ -1,6 +1,8 @@
 """Host logic of bench.py that needs no GPU: the kernel-source hash that keys
 the committed ncu traffic captures, and the kernel names the launch counts
 refer to."""
+import numpy as np
+
 import bench
 import workloads
 
@@ -83,3 +85,35 @@ def test_peaks_used_records_both_denominators():
     assert d["fp8_tflops"] == 2 * 1654.5 and d["rated_fp8_tflops"] == 4500.0
     assert d["rated_hbm_gbs"] == 8000.0 and d["sm_mhz_median_when_measured"] == 1192.0
     assert d["source"] == "MEASURED_PEAKS.json"
+
+
+def test_peak_expected_matches_the_declared_sums():
+    """The tensor-core rate kernel's check value against the declaration's
+    definition summed element by element over one 128-wide K block."""
+    import bench
+    iters = 3
+    want = np.zeros((128, 256))
+    for m in (0, 1, 17, 127):
+        for n in (0, 5, 16, 255):
+            s = 0
+            for k in range(128):
+                j = k % 16
+                s += ((2 * m + 3 * j) % 5 - 2) * ((3 * n + 2 * j + n // 16) % 5 - 2)
+            want[m, n] = iters * s
+            assert bench.peak_expected(iters)[m, n] == want[m, n]
+    assert np.abs(bench.peak_expected(32768)).max() < 2 ** 24  # exact in fp32
+
+
+def test_peak_reference_arm_is_unavailable(capsys):
+    import json
+    import sys
+
+    import bench
+    argv = sys.argv
+    sys.argv = ["bench.py", "--impl", "reference", "--workload", "peak_fp8_mma_16384"]
+    try:
+        bench.main()
+    finally:
+        sys.argv = argv
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and "unavailable" in line

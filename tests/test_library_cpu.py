@@ -85,6 +85,10 @@ def test_validation_rejects_without_touching_the_device(lib):
     assert lib.per_block_dequant_to_bf16(ok, ok, ok, 0, 64, 128, None) == 1
     assert lib.per_block_dequant_to_bf16(ok, ok, ok, 1, 0, 128, None) == 1
     assert lib.per_block_dequant_to_bf16(ok, ok, P(MISALIGNED), 1, 64, 128, None) == 1
+    # tensor-core rate kernel: launch length and output pointer
+    assert lib.fg_fp8_mma_peak(0, ok, None) == 1
+    assert lib.fg_fp8_mma_peak(32769, ok, None) == 1
+    assert lib.fg_fp8_mma_peak(16, None, None) == 1
     # empty problems are a no-op success
     assert lib.fp8_gemm_nt(ok, ok, ok, ok, ok, 0, 256, 256, None) == 0
     assert lib.per_token_cast_to_fp8(ok, ok, ok, 1, 0, 128, None) == 0

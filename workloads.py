@@ -27,6 +27,9 @@ inference shapes"):
                            ~ N(0, 0.02)
   quant_4096x7168          the activation quantizer alone, on the activations
                            of prefill_4096x2112x7168 (A ~ N(0,1))
+  peak_fp8_mma_16384       no inputs: the FP8 tensor-core rate, 16384 K blocks
+                           of MMAs (128 x 256 x 128 each) per CTA from operands
+                           the kernel generates in shared memory
   kgrouped_8x4096x7168     K-grouped weight-gradient GEMM of the contiguous
                            workload's experts: A = dY^T [4096][T] ~ N(0,1),
                            B = X^T [7168][T] ~ N(0,1), the experts' token
@@ -245,6 +248,11 @@ def dequant(N: int, K: int, seed: int = 0, b_std: float = 0.02) -> DequantInputs
 
 
 @dataclasses.dataclass
+class PeakInputs:
+    iters: int  # K blocks per CTA and launch
+
+
+@dataclasses.dataclass
 class QuantInputs:
     a: np.ndarray  # bf16 bits [M][K]
     M: int
@@ -283,6 +291,8 @@ WORKLOADS = {
     "ffn_contiguous_8x7168x2048": ("ffn", dict(H=7168, I=2048, G=8)),
     # K-grouped weight-gradient GEMM of the contiguous workload's experts
     "kgrouped_8x4096x7168": ("kgrouped", dict(M=4096, N=7168, G=8)),
+    # the FP8 tensor-core rate (operands generated in shared memory)
+    "peak_fp8_mma_16384": ("peak", dict(iters=16384)),
 }
 
 
@@ -300,6 +310,8 @@ def make(name: str, seed: int = 0):
         return ffn_contiguous(seed=seed, **kw)
     if kind == "kgrouped":
         return k_grouped(seed=seed, **kw)
+    if kind == "peak":
+        return PeakInputs(**kw)
     return masked(seed=seed, **kw)
 
 
