@@ -574,6 +574,16 @@ def step_config(args, kind: str, inp, world: int, ue8m0: bool) -> dict:
             "parallelism": "replicas" if world > 1 else "single GPU"}
 
 
+def fp8_mma_rate():
+    """The FP8 tensor-core rate this library's own MMA loop reached on this
+    pool (workload peak_fp8_mma_16384), from its committed record, or None."""
+    path = os.path.join(ROOT, "profiles", "fp8_mma_rate.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        return json.load(f).get("tflops")
+
+
 def peaks_used(peaks: dict, source: str) -> dict:
     """The denominators a roofline fraction was taken against, with where they
     came from, so that the fraction can be recomputed."""
@@ -582,6 +592,9 @@ def peaks_used(peaks: dict, source: str) -> dict:
          "fp8_rule": "%.1f x the bf16 burst figure" % FP8_OVER_BF16,
          "source": "MEASURED_PEAKS.json" if source == "measured" else "recipe fallback",
          "rated_fp8_tflops": RATED_FP8_TFLOPS, "rated_hbm_gbs": RATED_HBM_GBS}
+    rate = fp8_mma_rate()
+    if rate:
+        d["fp8_mma_in_library_tflops"] = rate
     clk = peaks.get("clocks_under_load") or {}
     if clk.get("sm_mhz_median") is not None:
         d["sm_mhz_median_when_measured"] = clk["sm_mhz_median"]
@@ -779,6 +792,9 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_rated": RATED_FP8_TFLOPS,
                 "frac_rated": achieved / RATED_FP8_TFLOPS}
+        if fp8_mma_rate():
+            roof["peak_in_library"] = fp8_mma_rate()
+            roof["frac_in_library"] = achieved / fp8_mma_rate()
         peak_note = "FP8 = %.1f x %s bf16 burst %.1f TFLOP/s (%s)" % (
             FP8_OVER_BF16, peak_src, peaks["bf16_tflops"], "MEASURED_PEAKS.json" if peak_src == "measured" else "recipe fallback")
     else:

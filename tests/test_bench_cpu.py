@@ -85,6 +85,8 @@ def test_peaks_used_records_both_denominators():
     assert d["fp8_tflops"] == 2 * 1654.5 and d["rated_fp8_tflops"] == 4500.0
     assert d["rated_hbm_gbs"] == 8000.0 and d["sm_mhz_median_when_measured"] == 1192.0
     assert d["source"] == "MEASURED_PEAKS.json"
+    # the committed in-library tensor-core rate rides along as a third denominator
+    assert d["fp8_mma_in_library_tflops"] == bench.fp8_mma_rate() > 0
 
 
 def test_peak_expected_matches_the_declared_sums():
