@@ -875,9 +875,10 @@ fg_status run_per_token(const uint16_t* x, uint8_t* q, float* sfa, int num_group
   FG_TRY(device_info(&dev));
   const int64_t slices = static_cast<int64_t>(num_groups) * M * (K / 128);
   if (slices >= (int64_t(1) << 31)) return fail(FG_ERR_UNSUPPORTED, "too many 128-element slices");
-  // one pass for small inputs (latency); up to QUNROLL slice pairs per warp
-  // and pass for large ones (several loads in flight per thread)
-  const int64_t blocks_needed = (slices * 16 + 255) / 256;
+  // one warp per work item of QROW_ITEM slices of a row, up to 8 blocks of
+  // 256 threads per SM (grid-stride beyond that)
+  const int64_t items = static_cast<int64_t>(num_groups) * M * ((K / 128 + QROW_ITEM - 1) / QROW_ITEM);
+  const int64_t blocks_needed = (items * 32 + 255) / 256;
   const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, int64_t(dev->sm_count) * 8));
   const cudaError_t e = launch_pdl(ue8m0 ? per_token_cast_kernel<true> : per_token_cast_kernel<false>, dim3(grid), dim3(256), stream, x, q, sfa,
                                    num_groups, M, K, sfa_stride(M));

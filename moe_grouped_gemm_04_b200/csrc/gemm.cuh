@@ -605,14 +605,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             // run: a phase seen complete here needs no blocking wait (phases
             // of both barriers advance at most one ahead of this warp)
             const uint32_t nx = it + 1;
-            int r = 0;
-            if (lane == 0) {
-              r = mbar_test_wait(&tempty[nx & 1], ((nx >> 1) & 1u) ^ 1u) ? 1 : 0;
-              r |= mbar_test_wait(&full[nx % C::STAGES], (nx / C::STAGES) & 1u) ? 2 : 0;
-            }
-            r = __shfl_sync(0xffffffffu, r, 0);
-            empty_seen = (r & 1) != 0;
-            full_seen = (r & 2) != 0;
+            empty_seen = __all_sync(0xffffffffu, mbar_test_wait(&tempty[nx & 1], ((nx >> 1) & 1u) ^ 1u));
+            full_seen = __all_sync(0xffffffffu, mbar_test_wait(&full[nx % C::STAGES], (nx / C::STAGES) & 1u));
           }
         }
       }

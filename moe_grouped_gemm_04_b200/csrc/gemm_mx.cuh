@@ -745,8 +745,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           {
             Ring<C::STAGES> nx = st;
             nx.next();
-            const int r = lane == 0 ? (mbar_test_wait(&full[nx.slot], nx.phase) ? 1 : 0) : 0;
-            ready = __shfl_sync(0xffffffffu, r, 0) != 0;
+            ready = __all_sync(0xffffffffu, mbar_test_wait(&full[nx.slot], nx.phase));
           }
           if (elect_one()) {
             if constexpr (C::PAIR) mma_commit_pair(&empty[st.slot]);  // both CTAs' stage

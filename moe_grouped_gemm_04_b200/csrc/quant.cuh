@@ -1,7 +1,7 @@
 // FP8 quantizers: per-token (1x128) activation scaling and per-block (128x128)
 // weight scaling. Both are HBM-bound streams: 2 bytes read and 1 byte written
-// per element plus one fp32 scale per group. Loads and stores are 16-byte
-// and 8-byte vectors; the amax reduction is a warp shuffle (per token) or a
+// per element plus one fp32 scale per group. Loads are 16-byte vectors,
+// code stores 16-byte (per token) or 8-byte (per block) vectors; the amax reduction is a warp shuffle (per token) or a
 // warp shuffle plus a shared-memory step (per block).
 //
 // Arithmetic (must match the oracle bit for bit):
@@ -78,14 +78,17 @@ __device__ __forceinline__ float amax8(uint4 w) {
   return m;
 }
 
-// One 128-element slice per 16 consecutive threads (8 elements each).
-// Slices are enumerated with the token index fastest so that consecutive
-// slices write consecutive scale entries of the MN-major layout. A warp
-// covers two adjacent slices and takes QUNROLL such pairs a grid stride apart,
-// issuing all their loads before using any, so that several 16-byte loads per
-// thread are in flight. The host keeps the slice count below 2^31 (32-bit
-// index arithmetic).
-constexpr int QUNROLL = 4;
+// One 128-element slice per 8 consecutive threads (16 elements, two 16-byte
+// loads each), so that a warp covers 4 adjacent slices of one token row per
+// step. A work item is QROW_STEPS such steps of one row (8 slices, 2 KB of
+// bf16); warps take items grid-stride, so the only index arithmetic is one
+// division per item, and all of an item's loads are issued before any is
+// used (4 x 16 bytes in flight per thread). Small inputs still spread over
+// many warps (a 64-token row set is 64 x 7 items for K = 7168). The codes of
+// a slice leave as one 16-byte store per thread; its scale as one 4-byte
+// store into the MN-major layout.
+constexpr int QROW_STEPS = 2;  // warp steps (4 slices each) per work item
+constexpr int QROW_ITEM = 4 * QROW_STEPS;  // slices per work item
 
 template <bool UE8M0>
 __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __restrict__ x,
@@ -96,39 +99,47 @@ __global__ void __launch_bounds__(256) per_token_cast_kernel(const uint16_t* __r
   // before touching memory
   grid_launch_dependents();
   grid_dependency_wait();
-  const uint32_t KB = static_cast<uint32_t>(K / 128);
-  const uint32_t slices = static_cast<uint32_t>(G) * KB * static_cast<uint32_t>(M);
-  const int sub = threadIdx.x & 15;
-  const uint32_t half = (threadIdx.x >> 4) & 1;  // which slice of the warp's pair
-  // the loop bound is uniform across a warp (the shuffles below need every
-  // lane); each warp takes the slice pairs base, base + step, ...
-  const uint32_t base0 = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 2;
-  const uint32_t step = ((gridDim.x * blockDim.x) >> 5) * 2;
-  for (uint32_t b0 = base0; b0 < slices; b0 += QUNROLL * step) {
-    uint4 w[QUNROLL];
-    int64_t off[QUNROLL];
-    uint32_t m[QUNROLL], gk[QUNROLL];
-    bool ok[QUNROLL];
+  const int KB = K / 128;
+  const int chunks = (KB + QROW_ITEM - 1) / QROW_ITEM;
+  const int64_t items = static_cast<int64_t>(G) * M * chunks;
+  const int lane = threadIdx.x & 31;
+  const int grp = lane >> 3;  // slice of the warp step
+  const int sub = lane & 7;   // 16 elements of the slice
+  const int64_t first = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t step = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  // the loop bound is uniform across a warp (the shuffles below need every lane)
+  for (int64_t it = first; it < items; it += step) {
+    const int64_t r = it / chunks;  // g * M + m
+    const int kb0 = static_cast<int>(it % chunks) * QROW_ITEM;
+    const int g = static_cast<int>(r / M), m = static_cast<int>(r % M);
+    const uint16_t* xr = x + r * K;
+    uint8_t* qr = q + r * K;
+    uint4 lo[QROW_STEPS], hi[QROW_STEPS];
 #pragma unroll
-    for (int u = 0; u < QUNROLL; ++u) {
-      const uint32_t s = b0 + u * step + half;
-      ok[u] = s < slices;
-      m[u] = s % static_cast<uint32_t>(M);
-      gk[u] = s / static_cast<uint32_t>(M);  // g * KB + kb
-      const uint32_t g = gk[u] / KB, kb = gk[u] % KB;
-      off[u] = (static_cast<int64_t>(g) * M + m[u]) * K + kb * 128 + sub * 8;
-      w[u] = ok[u] ? __ldg(reinterpret_cast<const uint4*>(x + off[u])) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < QROW_STEPS; ++u) {
+      const int kb = kb0 + u * 4 + grp;
+      if (kb < KB) {
+        const uint4* src = reinterpret_cast<const uint4*>(xr + kb * 128 + sub * 16);
+        lo[u] = __ldg(src);
+        hi[u] = __ldg(src + 1);
+      } else {
+        lo[u] = make_uint4(0, 0, 0, 0);
+        hi[u] = lo[u];
+      }
     }
 #pragma unroll
-    for (int u = 0; u < QUNROLL; ++u) {
-      float a = amax8(w[u]);
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-      if (ok[u]) {
+    for (int u = 0; u < QROW_STEPS; ++u) {
+      const int kb = kb0 + u * 4 + grp;
+      float a = fmaxf(amax8(lo[u]), amax8(hi[u]));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      if (kb < KB) {
         float scale, inv;
         group_scale<UE8M0>(fmaxf(a, kAmaxFloor), scale, inv);
-        *reinterpret_cast<uint2*>(q + off[u]) = quantize8(w[u], inv);
-        if (sub == 0) sfa[static_cast<int64_t>(gk[u]) * stride + m[u]] = scale;
+        const uint2 c0 = quantize8(lo[u], inv), c1 = quantize8(hi[u], inv);
+        *reinterpret_cast<uint4*>(qr + kb * 128 + sub * 16) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+        if (sub == 0) sfa[(static_cast<int64_t>(g) * KB + kb) * stride + m] = scale;
       }
     }
   }
