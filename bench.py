@@ -31,6 +31,11 @@ of consecutive steps pipelined on three streams, as a serving loop would);
 `--scales ue8m0` quantizes with power-of-two scales and runs the block-scaled
 GEMM entry points (the oracle then uses the same power-of-two quantizers).
 
+The default run (the contiguous workload) also times the other named GEMM
+configurations (decode, both prefill shapes, the masked layout) the same way,
+device-timed only, and lists them under `other_configs` in the same JSON line;
+`--no-other-configs` skips them.
+
 `--workload peak_fp8_mma_16384` measures the FP8 tensor-core rate itself: one
 CTA per SM issues the GEMMs' MMA instruction back to back from operands that
 stay in shared memory (no loads, no promotion), and the accumulators are
@@ -62,6 +67,13 @@ if ROOT not in sys.path:
 
 import workloads  # noqa: E402
 
+DEFAULT_WORKLOAD = "contiguous_8x4096x7168"
+# the other GEMM configurations the method's measurements name (decode, the two
+# prefill shapes, the masked layout), timed in the default run as well
+OTHER_CONFIGS = ("decode_64x4096x7168", "prefill_4096x7168x2048", "prefill_4096x2112x7168",
+                 "masked_32x256x4096x7168")
+
+
 METRIC = "FP8 block-scaled GEMM TFLOPS (device-timed) and % of B200 FP8/HBM roofline"
 L2_FLUSH_BYTES = 256 << 20
 SENTINEL_BF16 = 0x7FC1  # a bf16 NaN pattern the kernels never produce
@@ -79,7 +91,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="contiguous_8x4096x7168", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--with-weight-quant", action="store_true")
     ap.add_argument("--scales", default="fp32", choices=["fp32", "ue8m0"],
@@ -92,6 +104,10 @@ def parse_args():
                          "(steps back to back) or by flushing L2 before every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="the default run also times the other named GEMM configurations "
+                         "(device-timed, no CPU baseline or e2e) and lists them under "
+                         "other_configs; this skips them")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample (a sample takes at "
                          "least 0.85 of it)")
@@ -1129,6 +1145,29 @@ def run_peak(args, rank, world, local_rank):
     }
 
 
+def run_other_configs(args, rank, world, local_rank):
+    """Each of OTHER_CONFIGS through run_ours with the same steps, warm-up and
+    scales, device-timed only; rank 0 gets one summary per configuration."""
+    import argparse as _ap
+
+    import torch
+    res = []
+    for w in OTHER_CONFIGS:
+        a = _ap.Namespace(**vars(args))
+        a.workload, a.no_cpu_baseline, a.no_e2e = w, True, True
+        r = run_ours(a, rank, world, local_rank)
+        torch.cuda.empty_cache()
+        if r is not None:
+            roof = r["roofline"]
+            res.append({"workload": w, "value": r["value"], "unit": r["unit"],
+                        "ms_per_step": r["ms_per_step"], "kernel_ms": roof["kernel_ms"],
+                        "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                                          "frac_rated", "frac_in_library", "traffic")
+                                     if k in roof},
+                        "clocks": r.get("clocks")})
+    return res
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm, on rank 0 only."""
     if rank != 0:
@@ -1214,6 +1253,10 @@ def main():
                 out = run_peak(args, rank, world, local_rank)
             else:
                 out = run_ours(args, rank, world, local_rank)
+                if args.workload == DEFAULT_WORKLOAD and not args.no_other_configs:
+                    others = run_other_configs(args, rank, world, local_rank)
+                    if out is not None:
+                        out["other_configs"] = others
         finally:
             if world > 1:
                 import torch.distributed as dist

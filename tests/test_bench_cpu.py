@@ -119,3 +119,27 @@ def test_peak_reference_arm_is_unavailable(capsys):
         sys.argv = argv
     line = json.loads(capsys.readouterr().out.strip())
     assert line["impl"] == "reference" and "unavailable" in line
+
+
+def test_other_configs_run_each_named_config_device_timed_only(monkeypatch):
+    """The default run's extra configurations: every one of OTHER_CONFIGS in
+    order, without the CPU baseline or the end-to-end leg, summarised from the
+    same fields a full line carries."""
+    import argparse
+    seen = []
+
+    def fake_run_ours(a, rank, world, local_rank):
+        seen.append((a.workload, a.no_cpu_baseline, a.no_e2e, a.steps))
+        return {"value": 1.0, "unit": "TFLOP/s", "ms_per_step": 0.5, "clocks": {"sm_mhz": 1965.0},
+                "roofline": {"bound": "tensor", "achieved": 2.0, "peak": 3.0, "unit": "TFLOP/s",
+                             "frac": 0.6, "frac_rated": 0.4, "kernel_ms": 0.4, "traffic": None,
+                             "kernel": "k"}}
+    monkeypatch.setattr(bench, "run_ours", fake_run_ours)
+    args = argparse.Namespace(workload=bench.DEFAULT_WORKLOAD, no_cpu_baseline=False, no_e2e=False, steps=7)
+    res = bench.run_other_configs(args, 0, 1, 0)
+    assert [s[0] for s in seen] == list(bench.OTHER_CONFIGS)
+    assert all(s[1] and s[2] and s[3] == 7 for s in seen)
+    assert args.workload == bench.DEFAULT_WORKLOAD and not args.no_e2e  # the caller's args untouched
+    assert [r["workload"] for r in res] == list(bench.OTHER_CONFIGS)
+    assert res[0]["kernel_ms"] == 0.4 and res[0]["roofline"]["frac"] == 0.6
+    assert "kernel" not in res[0]["roofline"]
