@@ -54,7 +54,10 @@ def gpu_per_block(fg, bits: np.ndarray):
 
 
 @pytest.mark.parametrize("G,M,K", [(1, 1, 128), (1, 63, 512), (1, 130, 384), (3, 80, 256),
-                                   (1, 64, 7168), (2, 257, 1024)])
+                                   (1, 64, 7168), (2, 257, 1024),
+                                   # rows of 9 and 15 slices: a full work item of 8
+                                   # slices, then a partial one
+                                   (1, 5, 1152), (2, 3, 1920)])
 def test_per_token_bit_exact(fg, G, M, K):
     rng = np.random.default_rng(M * 1000 + K + G)
     x = _special_rows(rng.standard_normal((G, M, K), dtype=np.float32))
