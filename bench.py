@@ -1069,6 +1069,122 @@ def dequant_cpu_sample(inp, target_s: float):
             "sample": "%d of %d rows x K=%d, %d passes" % (rows, inp.N, inp.K, passes), "seconds": dt}
 
 
+EP_METRIC = ("Expert-parallel MoE layer (quantize, dispatch into the masked layout, masked FP8 GEMM, "
+             "combine) TFLOP/s (device-timed)")
+
+
+def run_ep(args, rank, world, local_rank):
+    """The expert-parallel layer (moe_grouped_gemm_04_b200.ep) over the ranks
+    of this run (one rank: its all-to-alls are local copies through NCCL),
+    each step timed between CUDA events around one layer call (the layer
+    reads its split sizes back to the host once, so steps are not captured
+    in a graph); the masked GEMM of the layer timed alone on the layout the
+    layer dispatched, K launches in one CUDA graph, for the roofline."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import moe_grouped_gemm_04_b200 as fg
+    import moe_grouped_gemm_04_b200.ep as ep
+
+    torch.cuda.set_device(local_rank)
+    fg.load_library()
+    created = False
+    if not dist.is_initialized():
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        created = True
+    try:
+        inp = workloads.make(args.workload, seed=rank)
+        E, k, N, K, M_max = inp.E, inp.k, inp.N, inp.K, inp.M_max
+        G = E // world
+        dev = "cuda"
+        x = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).to(dev).view(torch.bfloat16)
+        topk = torch.from_numpy(inp.topk).to(dev)
+        topk_w = torch.from_numpy(inp.topk_w).to(dev)
+        wb = torch.from_numpy(np.ascontiguousarray(inp.w[rank * G:(rank + 1) * G]).view(np.int16)).to(dev)
+        wq = torch.empty((G, N, K), dtype=torch.uint8, device=dev)
+        ws = fg.empty_sfb(G, N, K, dev)
+        fg.per_block_cast_to_fp8(wb.view(torch.bfloat16), wq, ws)
+        del wb
+
+        def step():
+            return ep.expert_parallel_masked_moe(x, topk, topk_w, wq, ws, E, M_max)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        assert fg.get_device_status() == 0
+        sampler = ClockSampler(local_rank)
+        sampler.start()
+        time.sleep(0.3)
+        dist.barrier()
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for e0, e1 in pairs:
+            e0.record()
+            step()
+            e1.record()
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in pairs]))
+        # the layer's GEMM alone, on the layout this rank's dispatch produced
+        h = ep.ep_dispatch(x, topk, E, M_max)
+        D = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=dev)
+        em = max(1, min(M_max, -(-h.received // G)))
+        gms, _ = time_graph_launches(lambda i: fg.fp8_grouped_gemm_masked(h.A, h.sfa, wq, ws, D, h.masked_m, em),
+                                     args.steps, local_rank, 1)
+        clocks = sampler.stop()
+        assert fg.get_device_status() == 0
+        mm = h.masked_m.cpu().numpy()
+        rows = int(mm.sum())
+        if world > 1:
+            ms, gms = max_over_ranks(dist, [ms, gms], "cuda")
+            rows_all = torch.tensor([float(rows)], device=dev)
+            dist.all_reduce(rows_all)
+            rows_total = int(rows_all.item())
+        else:
+            rows_total = rows
+    finally:
+        if created:
+            dist.destroy_process_group()
+    if rank != 0:
+        return None
+    flops = 2.0 * rows_total * N * K          # every rank's GEMM rows
+    gemm_flops = 2.0 * rows * N * K           # this rank's GEMM (the roofline's kernel)
+    experts = int((mm > 0).sum())
+    gemm_bytes = float(experts * (N * K + 4 * (-(-N // 128)) * (K // 128)) + rows * (K + 4 * (K // 128))
+                       + 2 * rows * N)
+    peaks, peak_src = load_peaks()
+    gbs = gemm_bytes / (gms * 1e-3) / 1e9
+    return {
+        "metric": EP_METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "data": "synthetic (seeded numpy, random weights and uniform top-%d routing)" % k,
+        "config": {"workload": args.workload, "kind": "ep", "experts": E, "experts_per_rank": G,
+                   "tokens_per_rank": inp.T, "topk": k, "N": N, "K": K, "M_max": M_max,
+                   "rows_this_rank": rows, "scales": "fp32 amax/448 (promoted masked GEMM)",
+                   "exchange": "NCCL all_to_all_single (%d rank%s)" % (world, "" if world == 1 else "s"),
+                   "timing": "CUDA events around each layer call (one host read of the split sizes per call)",
+                   "l2": "inputs larger than L2: the rank's expert weights (%.0f MB)" % (G * N * K / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "peak_rated": RATED_HBM_GBS,
+                     "frac_rated": gbs / RATED_HBM_GBS, "traffic": None,
+                     "kernel": "fp8_gemm_kernel (masked form)", "kernel_ms": gms,
+                     "algorithmic_per_launch": {"flops": gemm_flops, "bytes": gemm_bytes},
+                     "peak_source": "%s HBM copy bandwidth" % peak_src},
+        # per layer call: quantizer, pair count and position, pack, unpack, masked
+        # GEMM, gather, combine (NCCL's own copy kernels not counted)
+        "cpu_baseline": None, "gpu_launches": 8 * args.steps, "clocks": clocks, "e2e": None,
+    }
+
+
 PEAK_METRIC = ("FP8 tensor-core rate (tcgen05.mma kind::f8f6f4, M=128 N=256 K=32, operands resident "
                "in shared memory) TFLOP/s (device-timed)")
 
@@ -1210,7 +1326,13 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     kind = workloads.WORKLOADS[args.workload][0]
-    if args.impl == "reference" and kind == "peak":
+    if args.impl == "reference" and kind == "ep":
+        out = None
+        if rank == 0:
+            out = {"impl": "reference", "metric": EP_METRIC,
+                   "unavailable": "the oracle has no all-to-all exchange; its masked GEMM is the "
+                                  "masked_32x256x4096x7168 reference line"}
+    elif args.impl == "reference" and kind == "peak":
         out = None
         if rank == 0:
             out = {"impl": "reference", "metric": PEAK_METRIC,
@@ -1251,6 +1373,8 @@ def main():
                 out = run_quant(args, rank, world, local_rank)
             elif kind == "peak":
                 out = run_peak(args, rank, world, local_rank)
+            elif kind == "ep":
+                out = run_ep(args, rank, world, local_rank)
             else:
                 out = run_ours(args, rank, world, local_rank)
                 if args.workload == DEFAULT_WORKLOAD and not args.no_other_configs:

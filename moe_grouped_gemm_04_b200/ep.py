@@ -7,7 +7,8 @@ overview, section "约300行JIT核心", paragraph on MoE layouts); the tokens
 travel over NVLink to the GPUs that hold their experts and the results travel
 back (same page, section "swapAB与Mega MoE").
 
-One call of `expert_parallel_masked_moe` on every rank of the group:
+One call of `expert_parallel_masked_moe` on every rank of the group (or its
+parts: `ep_dispatch` for steps 1-4, the masked GEMM, `ep_combine` for step 6):
 
   1. quantizes the rank's tokens per token per 128 channels (the library's
      quantizer: the rows travel as e4m3 codes with their scales, half the
@@ -65,20 +66,29 @@ def _as_bits(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.int32) if t.dtype == torch.bfloat16 else t
 
 
-def expert_parallel_masked_moe(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
-                               w_local: torch.Tensor, sfb_local: torch.Tensor, num_experts: int,
-                               M_max: int, group=None,
-                               expected_m: Optional[int] = None) -> torch.Tensor:
-    """Routed expert GEMM over an expert-parallel group.
+class EpDispatch:
+    """What ep_dispatch hands to the masked GEMM and to ep_combine: the masked
+    layout of this rank's experts (A [G][M_max][K] e4m3, sfa in the MN-major
+    layout, masked_m [G] on the device) and the bookkeeping of the exchange
+    (each received row's slot in the layout, each own pair's position in the
+    send order, and the split sizes of both all-to-alls)."""
 
-    x: bf16 [T][K] (this rank's tokens); topk_idx: int32 [T][k] global expert
-    ids (negative = no expert); topk_w: fp32 [T][k] router weights; w_local:
-    e4m3 [G][N][K] and sfb_local fp32 [G][ceil(N/128)][K/128], the weights of
-    this rank's G = num_experts / world_size experts, quantized per 128 x 128
-    block; M_max: rows per local expert in the masked layout (more are
-    dropped, FG_DEVICE_EP_OVERFLOW). Returns bf16 [T][N]:
-    out[t] = sum_j topk_w[t][j] * bf16((x_t quantized) W_{topk_idx[t][j]}^T).
-    """
+    def __init__(self, A, sfa, masked_m, recv_slot, send_pos, send_sizes, recv_sizes, num_experts):
+        self.A, self.sfa, self.masked_m = A, sfa, masked_m
+        self.recv_slot, self.send_pos = recv_slot, send_pos
+        self.send_sizes, self.recv_sizes = send_sizes, recv_sizes
+        self.num_experts = num_experts
+
+    @property
+    def received(self) -> int:
+        return sum(self.recv_sizes)
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, M_max: int,
+                group=None) -> EpDispatch:
+    """Steps 1-4 of the layer: quantize this rank's tokens, order the pairs by
+    expert, exchange counts, rows and scales, and place the received rows into
+    the masked layout of this rank's G = num_experts / world_size experts."""
     W = dist.get_world_size(group)
     if num_experts % W != 0:
         raise FP8GemmError(FG_ERR_INVALID_ARG, "num_experts %d is not a multiple of the group size %d"
@@ -86,14 +96,9 @@ def expert_parallel_masked_moe(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: 
     G = num_experts // W
     T, K = x.shape
     k = topk_idx.shape[1]
-    N = w_local.shape[1]
-    if w_local.shape[0] != G:
-        raise FP8GemmError(FG_ERR_INVALID_ARG, "w_local holds %d experts, this rank owns %d"
-                           % (w_local.shape[0], G))
     dev = x.device
     KB = K // 128
 
-    # 1-2: quantize, order the pairs by expert, pack the rows
     q = torch.empty((T, K), dtype=torch.uint8, device=dev)
     s = empty_sfa(1, T, K, dev)
     _ops.quantize(x, q, s)
@@ -101,7 +106,6 @@ def expert_parallel_masked_moe(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: 
     send_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
     _ops.layout(topk_idx, num_experts, counts, send_pos)
 
-    # 3: counts, then rows and scales
     recv_counts = torch.empty((W, G), dtype=torch.int32, device=dev)
     dist.all_to_all_single(recv_counts.view(-1), counts, group=group)
     send_sizes = [int(v) for v in counts.view(W, G).sum(dim=1).tolist()]
@@ -115,22 +119,55 @@ def expert_parallel_masked_moe(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: 
     dist.all_to_all_single(recv_q, send_q, recv_sizes, send_sizes, group=group)
     dist.all_to_all_single(recv_s, send_s, recv_sizes, send_sizes, group=group)
 
-    # 4-5: masked layout, grouped GEMM with the local experts
     A = torch.empty((G, M_max, K), dtype=torch.uint8, device=dev)
     sfa = empty_sfa(G, M_max, K, dev)
     masked_m = torch.empty(G, dtype=torch.int32, device=dev)
     recv_slot = torch.empty(R, dtype=torch.int32, device=dev)
     _ops.unpack(recv_q, recv_s, recv_counts, A, sfa, masked_m, recv_slot)
-    D = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=dev)
-    if expected_m is None:
-        expected_m = max(1, min(M_max, -(-R // G)))
-    _ops.gemm(A, sfa, w_local, sfb_local, D, masked_m, expected_m)
+    return EpDispatch(A, sfa, masked_m, recv_slot, send_pos, send_sizes, recv_sizes, num_experts)
 
-    # 6: back to the sources, weighted sum of each token's choices
-    y_recv = torch.empty((R, N), dtype=torch.bfloat16, device=dev)
-    _ops.gather(D, recv_slot, y_recv)
-    y_send = torch.empty((P, N), dtype=torch.bfloat16, device=dev)
-    dist.all_to_all_single(_as_bits(y_send), _as_bits(y_recv), send_sizes, recv_sizes, group=group)
+
+def ep_combine(D: torch.Tensor, h: EpDispatch, topk_w: torch.Tensor, group=None) -> torch.Tensor:
+    """Step 6: gather the GEMM's output rows into receive order, send them back
+    to their source ranks, and sum each token's choices weighted by the router
+    (fp32, choices in order, one bf16 rounding). D: bf16 [G][M_max][N]."""
+    dev = D.device
+    N = D.shape[2]
+    T = h.send_pos.shape[0]
+    y_recv = torch.empty((h.received, N), dtype=torch.bfloat16, device=dev)
+    _ops.gather(D, h.recv_slot, y_recv)
+    y_send = torch.empty((sum(h.send_sizes), N), dtype=torch.bfloat16, device=dev)
+    dist.all_to_all_single(_as_bits(y_send), _as_bits(y_recv), h.send_sizes, h.recv_sizes, group=group)
     out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
-    _ops.combine(y_send, send_pos, topk_w, out)
+    _ops.combine(y_send, h.send_pos, topk_w, out)
     return out
+
+
+def expert_parallel_masked_moe(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+                               w_local: torch.Tensor, sfb_local: torch.Tensor, num_experts: int,
+                               M_max: int, group=None,
+                               expected_m: Optional[int] = None) -> torch.Tensor:
+    """Routed expert GEMM over an expert-parallel group: ep_dispatch, the masked
+    grouped GEMM with this rank's experts, ep_combine.
+
+    x: bf16 [T][K] (this rank's tokens); topk_idx: int32 [T][k] global expert
+    ids (negative = no expert); topk_w: fp32 [T][k] router weights; w_local:
+    e4m3 [G][N][K] and sfb_local fp32 [G][ceil(N/128)][K/128], the weights of
+    this rank's G = num_experts / world_size experts, quantized per 128 x 128
+    block; M_max: rows per local expert in the masked layout (more are
+    dropped, FG_DEVICE_EP_OVERFLOW). Returns bf16 [T][N]:
+    out[t] = sum_j topk_w[t][j] * bf16((x_t quantized) W_{topk_idx[t][j]}^T).
+    """
+    W = dist.get_world_size(group)
+    G = num_experts // W if num_experts % W == 0 else -1
+    if G > 0 and w_local.shape[0] != G:
+        raise FP8GemmError(FG_ERR_INVALID_ARG, "w_local holds %d experts, this rank owns %d"
+                           % (w_local.shape[0], G))
+    h = ep_dispatch(x, topk_idx, num_experts, M_max, group)
+    G = h.A.shape[0]
+    N = w_local.shape[1]
+    D = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=x.device)
+    if expected_m is None:
+        expected_m = max(1, min(M_max, -(-h.received // G)))
+    _ops.gemm(h.A, h.sfa, w_local, sfb_local, D, h.masked_m, expected_m)
+    return ep_combine(D, h, topk_w, group)

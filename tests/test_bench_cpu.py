@@ -143,3 +143,16 @@ def test_other_configs_run_each_named_config_device_timed_only(monkeypatch):
     assert [r["workload"] for r in res] == list(bench.OTHER_CONFIGS)
     assert res[0]["kernel_ms"] == 0.4 and res[0]["roofline"]["frac"] == 0.6
     assert "kernel" not in res[0]["roofline"]
+
+
+def test_ep_reference_arm_is_unavailable(capsys):
+    import json
+    import sys
+    argv = sys.argv
+    sys.argv = ["bench.py", "--impl", "reference", "--workload", "ep_32x512x8_4096x7168"]
+    try:
+        bench.main()
+    finally:
+        sys.argv = argv
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and "unavailable" in line

@@ -152,3 +152,19 @@ def test_work_counts_dequant_ffn_and_k_grouped():
     f, b = workloads.flops_and_bytes("kgrouped", k)
     assert f == 2 * 64 * 96 * 300
     assert b == (64 + 96) * 384 + 4 * (64 + 96) * 3 + 4 * 2 * 64 * 96
+
+
+def test_expert_parallel_inputs():
+    """The expert-parallel workload's routing: k distinct experts per token
+    (uniform Gumbel-top-k), router weights summing to one per token, and a
+    seed that reproduces it; small sizes stand in for the bench's."""
+    a = workloads.expert_parallel(T=64, E=16, k=4, N=128, K=256, M_max=64, seed=3)
+    b = workloads.expert_parallel(T=64, E=16, k=4, N=128, K=256, M_max=64, seed=3)
+    assert np.array_equal(a.topk, b.topk) and np.array_equal(a.x, b.x)
+    assert a.topk.shape == (64, 4) and a.topk.dtype == np.int32
+    assert all(len(set(r)) == 4 for r in a.topk.tolist())
+    assert a.topk.min() >= 0 and a.topk.max() < 16
+    assert np.allclose(a.topk_w.sum(axis=1), 1.0, atol=1e-6) and (a.topk_w > 0).all()
+    assert a.counts.sum() == 64 * 4 and a.w.shape == (16, 128, 256)
+    c = workloads.expert_parallel(T=64, E=16, k=4, N=128, K=256, M_max=64, seed=4)
+    assert not np.array_equal(a.topk, c.topk)

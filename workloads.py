@@ -27,6 +27,12 @@ inference shapes"):
                            ~ N(0, 0.02)
   quant_4096x7168          the activation quantizer alone, on the activations
                            of prefill_4096x2112x7168 (A ~ N(0,1))
+  ep_32x512x8_4096x7168    expert-parallel layer (dispatch, masked GEMM, combine):
+                           32 experts, 512 tokens ~ N(0,1) with K = 7168, each
+                           routed to 8 distinct experts drawn uniformly
+                           (Gumbel-top-k on equal weights), router weights
+                           U(0,1) normalised per token, expert weights
+                           [32][4096][7168] ~ N(0, 0.02), capacity M_max = 256
   peak_fp8_mma_16384       no inputs: the FP8 tensor-core rate, 16384 K blocks
                            of MMAs (128 x 256 x 128 each) per CTA from operands
                            the kernel generates in shared memory
@@ -248,6 +254,36 @@ def dequant(N: int, K: int, seed: int = 0, b_std: float = 0.02) -> DequantInputs
 
 
 @dataclasses.dataclass
+class EpInputs:
+    x: np.ndarray      # bf16 bits [T][K]
+    topk: np.ndarray   # int32 [T][k] expert ids
+    topk_w: np.ndarray  # fp32 [T][k] router weights
+    w: np.ndarray      # bf16 bits [E][N][K]
+    T: int
+    E: int
+    k: int
+    N: int
+    K: int
+    M_max: int
+
+    @property
+    def counts(self) -> np.ndarray:
+        return np.bincount(self.topk.ravel(), minlength=self.E).astype(np.int64)
+
+
+def expert_parallel(T: int, E: int, k: int, N: int, K: int, M_max: int, seed: int = 0,
+                    a_std: float = 1.0, b_std: float = 0.02) -> EpInputs:
+    x = normal_bf16(np.random.default_rng(seed + 0), (T, K), a_std)
+    w = normal_bf16(np.random.default_rng(seed + 1), (E, N, K), b_std)
+    rng = np.random.default_rng(seed + 2)
+    g = rng.gumbel(size=(T, E))
+    topk = np.argpartition(-g, k - 1, axis=1)[:, :k].astype(np.int32)
+    wt = rng.random((T, k)).astype(np.float32)
+    wt /= wt.sum(axis=1, keepdims=True)
+    return EpInputs(x=x, topk=topk, topk_w=wt, w=w, T=T, E=E, k=k, N=N, K=K, M_max=M_max)
+
+
+@dataclasses.dataclass
 class PeakInputs:
     iters: int  # K blocks per CTA and launch
 
@@ -293,6 +329,8 @@ WORKLOADS = {
     "kgrouped_8x4096x7168": ("kgrouped", dict(M=4096, N=7168, G=8)),
     # the FP8 tensor-core rate (operands generated in shared memory)
     "peak_fp8_mma_16384": ("peak", dict(iters=16384)),
+    # the expert-parallel layer around the masked GEMM
+    "ep_32x512x8_4096x7168": ("ep", dict(T=512, E=32, k=8, N=4096, K=7168, M_max=256)),
 }
 
 
@@ -312,6 +350,8 @@ def make(name: str, seed: int = 0):
         return k_grouped(seed=seed, **kw)
     if kind == "peak":
         return PeakInputs(**kw)
+    if kind == "ep":
+        return expert_parallel(seed=seed, **kw)
     return masked(seed=seed, **kw)
 
 
