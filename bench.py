@@ -1114,29 +1114,37 @@ def run_ep(args, rank, world, local_rank):
         fg.per_block_cast_to_fp8(wb.view(torch.bfloat16), wq, ws)
         del wb
 
-        def step():
-            return ep.expert_parallel_masked_moe(x, topk, topk_w, wq, ws, E, M_max)
+        # a fixed capacity of every pair a rank has (T * k rows per destination:
+        # nothing can be dropped), so the layer never reads counts back
+        cap = inp.T * k
 
-        for _ in range(max(args.warmup, 3)):
-            step()
-        torch.cuda.synchronize()
-        assert fg.get_device_status() == 0
+        def step(capacity):
+            return ep.expert_parallel_masked_moe(x, topk, topk_w, wq, ws, E, M_max, capacity=capacity)
+
+        def timed_steps(capacity):
+            for _ in range(max(args.warmup, 3)):
+                step(capacity)
+            torch.cuda.synchronize()
+            assert fg.get_device_status() == 0
+            dist.barrier()
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)]
+            for e0, e1 in pairs:
+                e0.record()
+                step(capacity)
+                e1.record()
+            torch.cuda.synchronize()
+            return float(np.mean([a.elapsed_time(b) for a, b in pairs]))
+
         sampler = ClockSampler(local_rank)
         sampler.start()
         time.sleep(0.3)
-        dist.barrier()
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(args.steps)]
-        for e0, e1 in pairs:
-            e0.record()
-            step()
-            e1.record()
-        torch.cuda.synchronize()
-        ms = float(np.mean([a.elapsed_time(b) for a, b in pairs]))
+        ms = timed_steps(cap)
+        ms_exact = timed_steps(None)
         # the layer's GEMM alone, on the layout this rank's dispatch produced
-        h = ep.ep_dispatch(x, topk, E, M_max)
+        h = ep.ep_dispatch(x, topk, E, M_max, capacity=cap)
         D = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=dev)
-        em = max(1, min(M_max, -(-h.received // G)))
+        em = max(1, min(M_max, -(-inp.T * k // G)))
         gms, _ = time_graph_launches(lambda i: fg.fp8_grouped_gemm_masked(h.A, h.sfa, wq, ws, D, h.masked_m, em),
                                      args.steps, local_rank, 1)
         clocks = sampler.stop()
@@ -1144,7 +1152,7 @@ def run_ep(args, rank, world, local_rank):
         mm = h.masked_m.cpu().numpy()
         rows = int(mm.sum())
         if world > 1:
-            ms, gms = max_over_ranks(dist, [ms, gms], "cuda")
+            ms, gms, ms_exact = max_over_ranks(dist, [ms, gms, ms_exact], "cuda")
             rows_all = torch.tensor([float(rows)], device=dev)
             dist.all_reduce(rows_all)
             rows_total = int(rows_all.item())
@@ -1170,8 +1178,10 @@ def run_ep(args, rank, world, local_rank):
         "config": {"workload": args.workload, "kind": "ep", "experts": E, "experts_per_rank": G,
                    "tokens_per_rank": inp.T, "topk": k, "N": N, "K": K, "M_max": M_max,
                    "rows_this_rank": rows, "scales": "fp32 amax/448 (promoted masked GEMM)",
-                   "exchange": "NCCL all_to_all_single (%d rank%s)" % (world, "" if world == 1 else "s"),
-                   "timing": "CUDA events around each layer call (one host read of the split sizes per call)",
+                   "exchange": "NCCL all_to_all_single (%d rank%s), fixed capacity of %d rows per "
+                               "destination (no host read of the counts)" % (world, "" if world == 1 else "s", cap),
+                   "exact_splits_ms_per_step": ms_exact,
+                   "timing": "CUDA events around each layer call, eager launches",
                    "l2": "inputs larger than L2: the rank's expert weights (%.0f MB)" % (G * N * K / 1e6)},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "peak_rated": RATED_HBM_GBS,
@@ -1179,9 +1189,9 @@ def run_ep(args, rank, world, local_rank):
                      "kernel": "fp8_gemm_kernel (masked form)", "kernel_ms": gms,
                      "algorithmic_per_launch": {"flops": gemm_flops, "bytes": gemm_bytes},
                      "peak_source": "%s HBM copy bandwidth" % peak_src},
-        # per layer call: quantizer, pair count and position, pack, unpack, masked
-        # GEMM, gather, combine (NCCL's own copy kernels not counted)
-        "cpu_baseline": None, "gpu_launches": 8 * args.steps, "clocks": clocks, "e2e": None,
+        # per layer call: quantizer, pair count, position and capacity, pack,
+        # unpack, masked GEMM, gather, combine (NCCL's own copy kernels not counted)
+        "cpu_baseline": None, "gpu_launches": 9 * args.steps, "clocks": clocks, "e2e": None,
     }
 
 

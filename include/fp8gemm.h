@@ -379,6 +379,36 @@ fg_status ep_dispatch_unpack_masked(const uint8_t* recv_q, const float* recv_s,
                                     int32_t* recv_slot, cudaStream_t stream);
 fg_status ep_combine_gather(const uint16_t* D, const int32_t* recv_slot, int R, int N, uint16_t* out,
                             cudaStream_t stream);
+
+/*
+ * The same dispatch with a fixed capacity of C rows per destination GPU, so
+ * that every exchange has equal, host-known split sizes (C rows to and from
+ * every GPU) and no count has to be read back to the host before it: the
+ * whole layer then runs without a host synchronisation. Not a step the pages
+ * name; it trades exchange bytes (W * C rows each way) for that.
+ * ep_dispatch_layout_capacity: as ep_dispatch_layout, with W GPUs of
+ *   G = E / W experts each (E % W == 0), but send_pos[p] = d * C + (the
+ *   pair's position among destination d's pairs, ordered by expert, then by
+ *   p), d = expert / G; a pair whose position would be C or more is dropped
+ *   (send_pos = -1, FG_DEVICE_EP_OVERFLOW), and counts[e] counts only the
+ *   pairs of expert e that are sent (what the receivers must expect). The send buffers of
+ *   ep_dispatch_pack then need W * C rows (rows a destination does not fill
+ *   are left as they were and never read).
+ * ep_dispatch_unpack_masked_capacity: as ep_dispatch_unpack_masked for a
+ *   receive buffer of W * C rows in which source s's rows start at row s * C
+ *   (local expert by local expert, recv_counts[s * G + g] of them); the rows
+ *   after a source's last one get recv_slot = -1. recv_slot holds W * C
+ *   entries; counts that put more than C rows in a segment set
+ *   FG_DEVICE_EP_OVERFLOW. ep_combine_gather and ep_combine_reduce are used
+ *   unchanged with R = W * C and these send_pos.
+ * C >= 1, W * C < 2^31; other errors as above.
+ */
+fg_status ep_dispatch_layout_capacity(const int32_t* topk_idx, int T, int k, int E, int W, int C,
+                                      int32_t* counts, int32_t* send_pos, cudaStream_t stream);
+fg_status ep_dispatch_unpack_masked_capacity(const uint8_t* recv_q, const float* recv_s,
+                                             const int32_t* recv_counts, int W, int G, int C, int M_max,
+                                             int K, uint8_t* A, float* sfa, int32_t* masked_m,
+                                             int32_t* recv_slot, cudaStream_t stream);
 fg_status ep_combine_reduce(const uint16_t* y, const int32_t* send_pos, const float* topk_w, int T, int k,
                             int N, uint16_t* out, cudaStream_t stream);
 

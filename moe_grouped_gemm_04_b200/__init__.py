@@ -42,7 +42,7 @@ EXPORTED = (
     "fg_set_ue8m0_tile", "fg_set_ffn_mode", "fg_moe_ffn_workspace_bytes", "fp8_moe_ffn_contiguous_ue8m0",
     "fp8_moe_ffn_masked_ue8m0", "fp8_moe_ffn_masked_ue8m0_noalloc",
     "ep_dispatch_layout", "ep_dispatch_pack", "ep_dispatch_unpack_masked", "ep_combine_gather",
-    "ep_combine_reduce",
+    "ep_combine_reduce", "ep_dispatch_layout_capacity", "ep_dispatch_unpack_masked_capacity",
     "fp8_k_grouped_gemm_nt_ue8m0",
     "fg_get_device_status", "fg_selftest_wait_timeout", "fg_status_string", "fg_last_error",
     "fg_fp8_mma_peak_ctas", "fg_fp8_mma_peak",
@@ -94,6 +94,8 @@ def load_library() -> ctypes.CDLL:
     lib.ep_dispatch_pack.argtypes = [P, P, P, I, I, I, P, P, P]
     lib.ep_dispatch_unpack_masked.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.ep_combine_gather.argtypes = [P, P, I, I, P, P]
+    lib.ep_dispatch_layout_capacity.argtypes = [P, I, I, I, I, I, P, P, P]
+    lib.ep_dispatch_unpack_masked_capacity.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.ep_combine_reduce.argtypes = [P, P, P, I, I, I, P, P]
     lib.fp8_k_grouped_gemm_nt_ue8m0.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
     lib.fg_get_device_status.argtypes = [P, ctypes.POINTER(I)]
@@ -114,7 +116,8 @@ def load_library() -> ctypes.CDLL:
               "fp8_moe_ffn_contiguous_ue8m0", "fp8_moe_ffn_masked_ue8m0",
               "fp8_moe_ffn_masked_ue8m0_noalloc",
               "ep_dispatch_layout", "ep_dispatch_pack", "ep_dispatch_unpack_masked",
-              "ep_combine_gather", "ep_combine_reduce",
+              "ep_combine_gather", "ep_combine_reduce", "ep_dispatch_layout_capacity",
+              "ep_dispatch_unpack_masked_capacity",
               "fp8_k_grouped_gemm_nt_ue8m0",
               "fg_get_device_status", "fg_selftest_wait_timeout", "fg_fp8_mma_peak"):
         getattr(lib, f).restype = I
@@ -394,6 +397,25 @@ def ep_dispatch_unpack_masked(recv_q, recv_s, recv_counts, A, sfa, masked_m, rec
     _, M_max, K = A.shape
     _check(load_library().ep_dispatch_unpack_masked(
         _ptr(recv_q), _ptr(recv_s), _ptr(recv_counts), W, G, R, M_max, K, _ptr(A), _ptr(sfa),
+        _ptr(masked_m), _ptr(recv_slot), _stream(stream)))
+
+
+def ep_dispatch_layout_capacity(topk_idx, E, W, C, counts, send_pos, stream=None) -> None:
+    """As ep_dispatch_layout with C send rows per destination GPU (W GPUs of
+    E / W experts): send_pos = d * C + position within destination d's rows."""
+    T, k = topk_idx.shape
+    _check(load_library().ep_dispatch_layout_capacity(_ptr(topk_idx), T, k, int(E), int(W), int(C),
+                                                      _ptr(counts), _ptr(send_pos), _stream(stream)))
+
+
+def ep_dispatch_unpack_masked_capacity(recv_q, recv_s, recv_counts, C, A, sfa, masked_m, recv_slot,
+                                       stream=None) -> None:
+    """As ep_dispatch_unpack_masked for W * C received rows, source s's from
+    row s * C; recv_slot [W * C]."""
+    W, G = recv_counts.shape
+    _, M_max, K = A.shape
+    _check(load_library().ep_dispatch_unpack_masked_capacity(
+        _ptr(recv_q), _ptr(recv_s), _ptr(recv_counts), W, G, int(C), M_max, K, _ptr(A), _ptr(sfa),
         _ptr(masked_m), _ptr(recv_slot), _stream(stream)))
 
 

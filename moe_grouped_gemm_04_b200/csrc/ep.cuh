@@ -90,27 +90,60 @@ __global__ void __launch_bounds__(kEpBlock) ep_count_kernel(const int32_t* topk,
 
 // send_pos of expert e's pairs: (pairs of experts before e) + the pair's rank
 // among expert e's pairs in (t, j) order. Block e handles expert e.
+// Fixed capacity (C > 0, G experts per destination GPU): the send buffer
+// holds C rows per destination, so the position is (e / G) * C + (pairs of
+// the destination's experts before e) + the rank; a pair that would land at
+// C or beyond in its destination's segment is dropped (send_pos = -1,
+// FG_DEVICE_EP_OVERFLOW).
 __global__ void __launch_bounds__(kEpBlock) ep_position_kernel(const int32_t* topk, int P,
-                                                               const int32_t* counts,
-                                                               int32_t* send_pos) {
+                                                               const int32_t* counts, int G, int C,
+                                                               int32_t* send_pos, int* status) {
   grid_dependency_wait();
   __shared__ int scratch[kEpBlock / 32];
   __shared__ int base_s;
   const int e = blockIdx.x;
+  const int first = C > 0 ? e / G * G : 0;  // first expert of e's segment
   if (threadIdx.x == 0) {
     int b = 0;
-    for (int x = 0; x < e; ++x) b += counts[x];
+    for (int x = first; x < e; ++x) b += counts[x];
     base_s = b;
   }
   __syncthreads();
   int run = base_s;
+  bool over = false;
   for (int p0 = 0; p0 < P; p0 += kEpBlock) {
     const int p = p0 + threadIdx.x;
     const int mine = p < P && topk[p] == e ? 1 : 0;
     int total;
     const int ex = block_excl_scan(mine, scratch, &total);
-    if (mine) send_pos[p] = run + ex;
+    if (mine) {
+      const int i = run + ex;  // position within the segment (C > 0) or the buffer
+      if (C > 0 && i >= C) {
+        send_pos[p] = -1;
+        over = true;
+      } else {
+        send_pos[p] = C > 0 ? (e / G) * C + i : i;
+      }
+    }
     run += total;
+  }
+  if (over) raise_status(status, 6 /* FG_DEVICE_EP_OVERFLOW */);
+}
+
+// Fixed capacity: counts[e] becomes the pairs of expert e that are sent,
+// i.e. those below C in their destination's rows (the receivers size their
+// segments by these counts). One thread per destination, after the position
+// kernel has read the full counts.
+__global__ void __launch_bounds__(kEpBlock) ep_cap_counts_kernel(int32_t* counts, int E, int G, int C) {
+  grid_dependency_wait();
+  for (int d = threadIdx.x; d < E / G; d += kEpBlock) {
+    int run = 0;
+    for (int e = d * G; e < (d + 1) * G; ++e) {
+      const int c = counts[e];
+      const int room = C - run;
+      counts[e] = room <= 0 ? 0 : (c < room ? c : room);
+      run += c;
+    }
   }
 }
 
@@ -138,13 +171,16 @@ __global__ void __launch_bounds__(kEpBlock) ep_pack_kernel(const uint8_t* q, con
 }
 
 // Receive order -> masked layout. recv_counts[s * G + g] = rows source s sent
-// for local expert g; the R received rows come source by source, expert by
-// expert. Row r of (s, g) at index i lands in slot (rows of g from sources
-// before s) + i of expert g; slots past M_max are dropped (recv_slot = -1,
-// FG_DEVICE_EP_OVERFLOW). Every block builds the prefix tables in shared
-// memory; one warp per received row; block 0 writes masked_m.
+// for local expert g; the received rows come source by source, expert by
+// expert: packed one after another (C = 0, R rows in all), or source s's rows
+// from row s * C of a buffer of C rows per source (C > 0, R = W * C, the rows
+// after a source's last one unused: recv_slot = -1). Row r of (s, g) at index
+// i lands in slot (rows of g from sources before s) + i of expert g; slots
+// past M_max are dropped (recv_slot = -1, FG_DEVICE_EP_OVERFLOW). Every block
+// builds the prefix tables in shared memory; one warp per received row; block
+// 0 writes masked_m.
 __global__ void __launch_bounds__(kEpBlock) ep_unpack_kernel(
-    const uint8_t* recv_q, const float* recv_s, const int32_t* recv_counts, int W, int G, int R,
+    const uint8_t* recv_q, const float* recv_s, const int32_t* recv_counts, int W, int G, int C, int R,
     int M_max, int K, uint8_t* A, float* sfa, int32_t* masked_m, int32_t* recv_slot, int* status) {
   grid_dependency_wait();
   __shared__ int off[kEpMaxTable + 1];  // receive-order start of (s, g), flattened s * G + g
@@ -152,11 +188,17 @@ __global__ void __launch_bounds__(kEpBlock) ep_unpack_kernel(
   const int SG = W * G;
   if (threadIdx.x == 0) {
     int run = 0;
+    bool over = false;
     for (int x = 0; x < SG; ++x) {
+      if (C > 0 && x % G == 0) run = (x / G) * C;  // each source's segment starts on its own
       off[x] = run;
       run += recv_counts[x];
+      // (a segment never holds more than C rows; counts that say otherwise
+      // are reported, and the rows past the segment are never read)
+      if (C > 0 && x % G == G - 1 && run > (x / G + 1) * C) over = true;
     }
-    off[SG] = run;
+    off[SG] = C > 0 ? W * C : run;
+    if (over && blockIdx.x == 0) raise_status(status, 6 /* FG_DEVICE_EP_OVERFLOW */);
   }
   for (int g = threadIdx.x; g < G; g += kEpBlock) {
     int run = 0;
@@ -180,7 +222,8 @@ __global__ void __launch_bounds__(kEpBlock) ep_unpack_kernel(
   }
   const int g = lo % G;
   const int slot = eoff[lo] + (r - off[lo]);
-  if (slot >= M_max) {
+  // (the unused rows after a source's last one in a fixed-capacity buffer)
+  if (r - off[lo] >= recv_counts[lo] || slot >= M_max) {
     if (lane == 0) recv_slot[r] = -1;
     return;
   }

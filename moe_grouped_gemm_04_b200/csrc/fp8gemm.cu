@@ -1156,8 +1156,35 @@ fg_status ep_dispatch_layout(const int32_t* topk_idx, int T, int k, int E, int32
                              send_pos, dev->status);
   if (e != cudaSuccess) return cuda_fail(e, "ep_count_kernel launch");
   e = launch_pdl(ep_position_kernel, dim3(E), dim3(kEpBlock), stream, topk_idx, P,
-                 static_cast<const int32_t*>(counts), send_pos);
+                 static_cast<const int32_t*>(counts), 1, 0, send_pos, dev->status);
   return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_position_kernel launch");
+}
+
+fg_status ep_dispatch_layout_capacity(const int32_t* topk_idx, int T, int k, int E, int W, int C,
+                                      int32_t* counts, int32_t* send_pos, cudaStream_t stream) {
+  if (T < 0 || k < 1 || E < 1 || W < 1 || C < 1)
+    return fail(FG_ERR_INVALID_ARG, "T=%d k=%d E=%d W=%d C=%d", T, k, E, W, C);
+  if (E % W != 0) return fail(FG_ERR_INVALID_ARG, "E=%d is not a multiple of W=%d", E, W);
+  if (static_cast<int64_t>(W) * C > INT32_MAX)
+    return fail(FG_ERR_UNSUPPORTED, "W * C = %lld rows", static_cast<long long>(W) * C);
+  FG_TRY(check_ptr(counts, "counts"));
+  if (T == 0) {
+    const cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream);
+    return e == cudaSuccess ? FG_OK : cuda_fail(e, "cudaMemsetAsync(counts)");
+  }
+  FG_TRY(check_ptr(topk_idx, "topk_idx"));
+  FG_TRY(check_ptr(send_pos, "send_pos"));
+  DeviceInfo* dev = nullptr;
+  FG_TRY(device_info(&dev));
+  const int P = T * k;
+  cudaError_t e = launch_pdl(ep_count_kernel, dim3(E), dim3(kEpBlock), stream, topk_idx, P, E, counts,
+                             send_pos, dev->status);
+  if (e != cudaSuccess) return cuda_fail(e, "ep_count_kernel launch");
+  e = launch_pdl(ep_position_kernel, dim3(E), dim3(kEpBlock), stream, topk_idx, P,
+                 static_cast<const int32_t*>(counts), E / W, C, send_pos, dev->status);
+  if (e != cudaSuccess) return cuda_fail(e, "ep_position_kernel launch");
+  e = launch_pdl(ep_cap_counts_kernel, dim3(1), dim3(kEpBlock), stream, counts, E, E / W, C);
+  return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_cap_counts_kernel launch");
 }
 
 fg_status ep_dispatch_pack(const uint8_t* q, const float* sfa, const int32_t* send_pos, int T, int k,
@@ -1177,10 +1204,9 @@ fg_status ep_dispatch_pack(const uint8_t* q, const float* sfa, const int32_t* se
   return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_pack_kernel launch");
 }
 
-fg_status ep_dispatch_unpack_masked(const uint8_t* recv_q, const float* recv_s,
-                                    const int32_t* recv_counts, int W, int G, int R, int M_max,
-                                    int K, uint8_t* A, float* sfa, int32_t* masked_m,
-                                    int32_t* recv_slot, cudaStream_t stream) {
+static fg_status run_unpack(const uint8_t* recv_q, const float* recv_s, const int32_t* recv_counts, int W, int G,
+                     int C, int R, int M_max, int K, uint8_t* A, float* sfa, int32_t* masked_m,
+                     int32_t* recv_slot, cudaStream_t stream) {
   if (W < 1 || G < 1 || R < 0 || M_max < 1)
     return fail(FG_ERR_INVALID_ARG, "W=%d G=%d R=%d M_max=%d", W, G, R, M_max);
   if (static_cast<int64_t>(W) * G > kEpMaxTable)
@@ -1200,9 +1226,27 @@ fg_status ep_dispatch_unpack_masked(const uint8_t* recv_q, const float* recv_s,
   const int per = kEpBlock / 32;
   const int blocks = R > 0 ? (R + per - 1) / per : 1;  // (block 0 writes masked_m)
   const cudaError_t e = launch_pdl(ep_unpack_kernel, dim3(blocks), dim3(kEpBlock), stream, recv_q, recv_s,
-                                   recv_counts, W, G, R, M_max, K, A, sfa, masked_m, recv_slot,
+                                   recv_counts, W, G, C, R, M_max, K, A, sfa, masked_m, recv_slot,
                                    dev->status);
   return e == cudaSuccess ? FG_OK : cuda_fail(e, "ep_unpack_kernel launch");
+}
+
+fg_status ep_dispatch_unpack_masked(const uint8_t* recv_q, const float* recv_s,
+                                    const int32_t* recv_counts, int W, int G, int R, int M_max,
+                                    int K, uint8_t* A, float* sfa, int32_t* masked_m,
+                                    int32_t* recv_slot, cudaStream_t stream) {
+  return run_unpack(recv_q, recv_s, recv_counts, W, G, 0, R, M_max, K, A, sfa, masked_m, recv_slot, stream);
+}
+
+fg_status ep_dispatch_unpack_masked_capacity(const uint8_t* recv_q, const float* recv_s,
+                                             const int32_t* recv_counts, int W, int G, int C, int M_max,
+                                             int K, uint8_t* A, float* sfa, int32_t* masked_m,
+                                             int32_t* recv_slot, cudaStream_t stream) {
+  if (C < 1) return fail(FG_ERR_INVALID_ARG, "C=%d must be >= 1", C);
+  if (static_cast<int64_t>(W) * C > INT32_MAX)
+    return fail(FG_ERR_UNSUPPORTED, "W * C = %lld rows", static_cast<long long>(W) * C);
+  return run_unpack(recv_q, recv_s, recv_counts, W, G, C, W * C, M_max, K, A, sfa, masked_m, recv_slot,
+                    stream);
 }
 
 fg_status ep_combine_gather(const uint16_t* D, const int32_t* recv_slot, int R, int N, uint16_t* out,

@@ -34,6 +34,45 @@ def layout_ref(topk: np.ndarray, E: int):
     return counts, pos.reshape(topk.shape)
 
 
+def layout_capacity_ref(topk: np.ndarray, E: int, W: int, C: int):
+    """counts[E] of the pairs sent and send_pos with C rows per destination:
+    d * C + the pair's position among destination d's pairs (by expert,
+    stably by p), -1 for pairs with no expert and for pairs at position C or
+    beyond (which the counts leave out)."""
+    counts, pos = layout_ref(topk, E)
+    G = E // W
+    prefix = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    e = topk.reshape(-1).astype(np.int64)
+    out = np.full(e.size, -1, np.int32)
+    sent = np.zeros(E, np.int32)
+    flat = pos.reshape(-1)
+    for p in range(e.size):
+        if flat[p] < 0:
+            continue
+        d = int(e[p]) // G
+        i = int(flat[p]) - int(prefix[d * G])  # position within destination d's pairs
+        if i < C:
+            out[p] = d * C + i
+            sent[e[p]] += 1
+    return sent, out.reshape(topk.shape)
+
+
+def unpack_capacity_ref(recv_q, recv_s, recv_counts, C, M_max):
+    """unpack_ref for a W * C-row receive buffer, source s's rows from s * C."""
+    W, G = recv_counts.shape
+    K = recv_q.shape[1]
+    rows = np.concatenate([recv_q[s * C:s * C + int(recv_counts[s].sum())] for s in range(W)])
+    srows = np.concatenate([recv_s[s * C:s * C + int(recv_counts[s].sum())] for s in range(W)])
+    A, sa, mm, slot_packed = unpack_ref(rows, srows, recv_counts, M_max)
+    slot = np.full(W * C, -1, np.int32)
+    r = 0
+    for s in range(W):
+        n = int(recv_counts[s].sum())
+        slot[s * C:s * C + n] = slot_packed[r:r + n]
+        r += n
+    return A, sa, mm, slot
+
+
 def unpack_ref(recv_q, recv_s, recv_counts, M_max):
     """Masked layout from the received rows (source by source, expert by
     expert): A [G][M_max][K], sa [G][M_max][KB] (logical), masked_m [G],
@@ -109,6 +148,22 @@ class CpuOps:
     def unpack(recv_q, recv_s, recv_counts, A, sfa, masked_m, recv_slot):
         M_max = A.shape[1]
         a, sa, mm, slot = unpack_ref(_np(recv_q), _np(recv_s), _np(recv_counts), M_max)
+        A.copy_(torch.from_numpy(a))
+        sfa.zero_()
+        sfa[:, :, :M_max] = torch.from_numpy(np.ascontiguousarray(sa.transpose(0, 2, 1)))
+        masked_m.copy_(torch.from_numpy(mm))
+        recv_slot.copy_(torch.from_numpy(slot))
+
+    @staticmethod
+    def layout_capacity(topk, E, W, C, counts, send_pos):
+        c, p = layout_capacity_ref(_np(topk), E, W, C)
+        counts.copy_(torch.from_numpy(c))
+        send_pos.copy_(torch.from_numpy(p))
+
+    @staticmethod
+    def unpack_capacity(recv_q, recv_s, recv_counts, C, A, sfa, masked_m, recv_slot):
+        M_max = A.shape[1]
+        a, sa, mm, slot = unpack_capacity_ref(_np(recv_q), _np(recv_s), _np(recv_counts), C, M_max)
         A.copy_(torch.from_numpy(a))
         sfa.zero_()
         sfa[:, :, :M_max] = torch.from_numpy(np.ascontiguousarray(sa.transpose(0, 2, 1)))

@@ -48,7 +48,7 @@ def _case(rank):
     return x, topk, wt, wq, ws
 
 
-def _rank_main(rank, world, port, out_path):
+def _rank_main(rank, world, port, out_path, capacity=None):
     import datetime
 
     import torch.distributed as dist
@@ -68,23 +68,31 @@ def _rank_main(rank, world, port, out_path):
         out = ep.expert_parallel_masked_moe(
             xt, torch.from_numpy(topk), torch.from_numpy(wt),
             torch.from_numpy(np.ascontiguousarray(wq[rank * G:(rank + 1) * G])),
-            torch.from_numpy(np.ascontiguousarray(ws[rank * G:(rank + 1) * G])), E, M_max)
+            torch.from_numpy(np.ascontiguousarray(ws[rank * G:(rank + 1) * G])), E, M_max,
+            capacity=capacity)
         np.save(out_path % rank, out.view(torch.int16).numpy().view(np.uint16))
     finally:
         dist.destroy_process_group()
 
 
-def test_dispatch_gemm_combine_on_two_ranks(tmp_path):
+@pytest.mark.parametrize("capacity", [None, 40, 9])  # 9: some pairs beyond a destination's rows
+def test_dispatch_gemm_combine_on_two_ranks(tmp_path, capacity):
+    """Exact splits (capacity None) and the fixed-capacity exchange; with a
+    capacity smaller than a destination's pairs the pairs past it are
+    dropped, and the output is that of the routing without them."""
     import torch.multiprocessing as mp
 
     import ep_reference
     world = 2
     out = str(tmp_path / "rank%d.npy")
-    mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True,
+    mp.start_processes(_rank_main, args=(world, _free_port(), out, capacity), nprocs=world, join=True,
                        start_method="spawn")
     for rank in range(world):
         x, topk, wt, wq, ws = _case(rank)
         got = np.load(out % rank)
+        if capacity is not None:
+            _, pos = ep_reference.layout_capacity_ref(topk, E, world, capacity)
+            topk = np.where(pos < 0, -1, topk).astype(np.int32)
         want = ep_reference.expected_output(x, topk, wt, wq, ws)
         assert got.shape == want.shape
         assert np.array_equal(got, want), "rank %d: %d outputs differ" % (rank, int((got != want).sum()))
@@ -98,3 +106,16 @@ def test_layout_reference_orders_pairs_by_expert():
     counts, pos = ep_reference.layout_ref(topk, 4)
     assert counts.tolist() == [3, 1, 2, 0]
     assert pos.tolist() == [[4, 0], [1, -1], [5, 3], [-1, 2]]
+
+
+def test_capacity_layout_reference():
+    """Fixed capacity: destination d's pairs from row d * C in expert order;
+    pairs at position C or beyond in their destination's rows are dropped."""
+    import ep_reference
+    topk = np.array([[2, 0], [0, -1], [2, 1], [3, 0]], np.int32)  # E = 4, W = 2: G = 2
+    counts, pos = ep_reference.layout_capacity_ref(topk, 4, 2, 3)
+    assert counts.tolist() == [3, 0, 2, 1]  # the pairs sent
+    # destination 0 (experts 0, 1): pairs (0,1) (1,0) (3,1) of expert 0, then (2,1) of expert 1
+    #   -> positions 0, 1, 2, 3; 3 >= C is dropped
+    # destination 1 (experts 2, 3): (0,0) (2,0) of expert 2, (3,0) of expert 3 -> rows 3, 4, 5
+    assert pos.tolist() == [[3, 0], [1, -1], [4, -1], [5, 2]]

@@ -67,6 +67,48 @@ def test_layout_and_pack(fg):
     assert np.array_equal(send_s.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
 
 
+@pytest.mark.parametrize("C", [300, 37])  # 37: destinations with more pairs drop the rest
+def test_layout_capacity(fg, C):
+    rng = np.random.default_rng(11)
+    T, k, E, W = 300, 4, 16, 4
+    topk = _topk(rng, T, k, E)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    pos = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    fg.ep_dispatch_layout_capacity(to_torch(topk), E, W, C, counts, pos)
+    torch.cuda.synchronize()
+    c_ref, p_ref = ep_reference.layout_capacity_ref(topk, E, W, C)
+    dropped = bool(((p_ref < 0) & (topk >= 0)).any())
+    assert fg.get_device_status() == (6 if dropped else 0)  # FG_DEVICE_EP_OVERFLOW
+    assert dropped == (C == 37)
+    assert np.array_equal(counts.cpu().numpy(), c_ref)
+    assert np.array_equal(pos.cpu().numpy(), p_ref)
+
+
+def test_unpack_capacity_skips_the_unused_rows(fg):
+    rng = np.random.default_rng(12)
+    W, G, K, C, M_max = 3, 4, 256, 30, 64
+    recv_counts = rng.integers(0, 8, (W, G)).astype(np.int32)
+    recv_counts[2] = 0  # a source that sent nothing
+    recv_q = rng.integers(0, 0x7E, (W * C, K)).astype(np.uint8)
+    recv_s = rng.random((W * C, K // 128)).astype(np.float32)
+    A = torch.full((G, M_max, K), 0x7F, dtype=torch.uint8, device="cuda")
+    sfa = torch.full((G, K // 128, fg.sfa_stride(M_max)), float("nan"), device="cuda")
+    mm = torch.empty(G, dtype=torch.int32, device="cuda")
+    slot = torch.empty(W * C, dtype=torch.int32, device="cuda")
+    fg.ep_dispatch_unpack_masked_capacity(to_torch(recv_q), to_torch(recv_s), to_torch(recv_counts), C, A,
+                                          sfa, mm, slot)
+    torch.cuda.synchronize()
+    assert fg.get_device_status() == 0
+    a_ref, sa_ref, mm_ref, slot_ref = ep_reference.unpack_capacity_ref(recv_q, recv_s, recv_counts, C, M_max)
+    assert np.array_equal(mm.cpu().numpy(), mm_ref)
+    assert np.array_equal(slot.cpu().numpy(), slot_ref)
+    An, sn = A.cpu().numpy(), sfa.cpu().numpy()
+    for g in range(G):
+        v = mm_ref[g]
+        assert np.array_equal(An[g, :v], a_ref[g, :v])
+        assert np.array_equal(sn[g, :, :v].T.view(np.uint32), sa_ref[g, :v].view(np.uint32))
+
+
 def test_layout_expert_out_of_range(fg):
     topk = np.array([[0, 7], [3, 1]], np.int32)  # 7 >= E
     counts = torch.empty(4, dtype=torch.int32, device="cuda")
@@ -141,9 +183,11 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_expert_parallel_layer_on_one_gpu(fg):
+@pytest.mark.parametrize("capacity", [None, 300, 40])  # 40: some pairs dropped
+def test_expert_parallel_layer_on_one_gpu(fg, capacity):
     """The whole layer through NCCL collectives on a one-GPU group: its output
-    against the oracle's per-choice GEMM rows and combine."""
+    against the oracle's per-choice GEMM rows and combine (with a fixed
+    capacity, of the routing without the pairs it drops)."""
     import datetime
 
     import torch.distributed as dist
@@ -164,12 +208,16 @@ def test_expert_parallel_layer_on_one_gpu(fg):
     try:
         out = ep.expert_parallel_masked_moe(
             to_torch(x.view(np.int16)).view(torch.bfloat16), to_torch(topk), to_torch(wt), to_torch(wq),
-            to_torch(np.ascontiguousarray(ws, np.float32)), E, M_max)
+            to_torch(np.ascontiguousarray(ws, np.float32)), E, M_max, capacity=capacity)
         torch.cuda.synchronize()
-        assert fg.get_device_status() == 0
+        assert fg.get_device_status() == (6 if capacity == 40 else 0)
     finally:
         if created:
             dist.destroy_process_group()
+    if capacity is not None:
+        _, pos = ep_reference.layout_capacity_ref(topk, E, 1, capacity)
+        assert ((pos < 0) & (topk >= 0)).any() == (capacity == 40)
+        topk = np.where(pos < 0, -1, topk).astype(np.int32)
     got = bf16_bits_to_f64(tensor_bf16_bits(out))
     want = bf16_bits_to_f64(ep_reference.expected_output(x, topk, wt, wq, ws))
     check_gemm(got, want, "expert-parallel layer")
