@@ -22,6 +22,10 @@
 //     receive order (ep_gather_rows), exchanged back, and on the source GPU
 //     out[t] = bf16(sum_j w[t][j] * y[pair (t, j)]) in fp32, j ascending
 //     (ep_combine).
+// With a fixed capacity of C rows per destination, segment d starts at row
+// d * C of the send buffer and source s's rows at row s * C of the receive
+// buffer (equal exchange sizes, known on the host); pairs past C in their
+// destination's segment are dropped, and the counts record the pairs sent.
 #pragma once
 
 #include <cstdint>
