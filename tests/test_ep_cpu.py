@@ -1,4 +1,4 @@
-"""The expert-parallel layer's exchange protocol on two gloo CPU ranks.
+"""The expert-parallel layer's exchange protocol on two and four gloo CPU ranks.
 
 Each rank runs moe_grouped_gemm_04_b200.ep.expert_parallel_masked_moe with
 its own tokens and router choices (uneven counts, dropped choices, experts
@@ -19,7 +19,7 @@ TESTS = os.path.dirname(os.path.abspath(__file__))
 
 torch = pytest.importorskip("torch")
 
-E, K, N, k, M_max = 4, 256, 128, 2, 64
+E, K, N, k, M_max = 4, 256, 128, 2, 160  # M_max above any expert's rows (four ranks send up to ~110 to expert 1)
 
 
 def _free_port():
@@ -75,15 +75,15 @@ def _rank_main(rank, world, port, out_path, capacity=None):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("capacity", [None, 40, 9])  # 9: some pairs beyond a destination's rows
-def test_dispatch_gemm_combine_on_two_ranks(tmp_path, capacity):
-    """Exact splits (capacity None) and the fixed-capacity exchange; with a
-    capacity smaller than a destination's pairs the pairs past it are
-    dropped, and the output is that of the routing without them."""
+@pytest.mark.parametrize("world,capacity", [(2, None), (2, 40), (2, 9), (4, None), (4, 9)])
+def test_dispatch_gemm_combine_on_gloo_ranks(tmp_path, world, capacity):
+    """Exact splits (capacity None) and the fixed-capacity exchange (9 rows:
+    some destinations have more pairs, which are dropped, and the output is
+    that of the routing without them), on two ranks of two experts and four
+    ranks of one."""
     import torch.multiprocessing as mp
 
     import ep_reference
-    world = 2
     out = str(tmp_path / "rank%d.npy")
     mp.start_processes(_rank_main, args=(world, _free_port(), out, capacity), nprocs=world, join=True,
                        start_method="spawn")
