@@ -44,10 +44,16 @@ CTA per SM issues the GEMMs' MMA instruction back to back from operands that
 stay in shared memory (no loads, no promotion), and the accumulators are
 checked exactly; it is the in-library ceiling of the tensor-bound lines.
 
-Multi-GPU (torchrun, one process per GPU): the path does not shard across
-GPUs within one call, so every rank runs an independent replica (weak
+`--workload ep_32x512x8_4096x7168` times the expert-parallel layer
+(quantize, dispatch into the masked layout, masked GEMM, combine) per call,
+with NCCL's all-to-all over the ranks of the run, and its masked GEMM alone
+for the roofline.
+
+Multi-GPU (torchrun, one process per GPU): the GEMM path does not shard
+across GPUs within one call, so every rank runs an independent replica (weak
 scaling); the timed region is bracketed by a barrier and the reported time is
-the max over ranks.
+the max over ranks. The expert-parallel workload exchanges tokens between the
+ranks.
 """
 from __future__ import annotations
 
